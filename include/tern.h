@@ -1,0 +1,189 @@
+/*
+ * tern.h -- ternary-g128 weight-only matrix multiply for NVIDIA B200 (sm_100a).
+ *
+ * The number format.  Each weight is a ternary value t in {-1, 0, +1}; every
+ * 128 consecutive weights along K share one FP16 scale s_g, and the weight is
+ * w = s_g * t.  ("Bonsai 27B ternary / 1-bit quantization", ThakiCloud blog,
+ * section "How compression works": w_i = s_g * t_i with one FP16 scale per
+ * 128-weight group; "Ternary-Bonsai-27B" model summary, aitrends.kr, section
+ * "Technical features": the group scale is applied inside the matrix multiply
+ * and the kernels consume the packed 2-bit slots directly, without an FP16
+ * copy of the weights.)
+ *
+ * The storage ("2-bit slots": "Ternary quantization: 27B in 7 GB", devnsb
+ * blog, section "Limits") is this library's own contract; the pages do not
+ * fix a byte layout.  For a weight matrix W with N rows and K columns
+ * (K contiguous), G = K / 128:
+ *
+ *   slots   uint8 [N][K/4]   weight (n,k) is the 2-bit code c = t + 1
+ *                            (0 -> -1, 1 -> 0, 2 -> +1; 3 is invalid) in byte
+ *                            n*K/4 + k/4, bits 2*(k%4) .. 2*(k%4)+1
+ *                            (least significant pair first);
+ *   scales  fp16  [N][G]     weight (n,k) uses scales[n][k/128].
+ *
+ * Bytes: K*N/4 + 2*K*N/128, i.e. 2.125 bits per weight (the ideal for this
+ * format, log2(3) + 16/128 ~= 1.71, needs a non-power-of-two packing).
+ *
+ * The products.  y[M][N] = x[M][K] * W^T: fp16 activations, fp32
+ * accumulation, fp16 output (round to nearest even).  y is overwritten.
+ *
+ * Conventions for every entry point:
+ *   - All buffers are DEVICE memory owned by the caller; the library keeps no
+ *     pointer after a call returns and allocates no device memory.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream).  Work is enqueued asynchronously on it.
+ *   - Argument errors are detected on the host before anything is launched
+ *     and returned synchronously; nothing is written in that case.
+ *   - A launch failure returns TERN_ERR_CUDA; tern_last_error() has the text.
+ *     Errors raised while kernels run surface on the caller's next
+ *     synchronisation, as for any CUDA work.
+ *   - K must be a positive multiple of 128; M and N must be >= 1.
+ *   - x, slots, codes and y must be 16-byte aligned; scales 16-byte aligned.
+ *     (Allocations from cudaMalloc / PyTorch are 256-byte aligned.)
+ *   - An invalid slot value (3) in tern_gemv / tern_gemm contributes an
+ *     unspecified finite value for that weight; it never faults.  Validation
+ *     is the job of tern_pack_g128.
+ *   - Thread safety: calls on different streams may run concurrently.
+ *     tern_set_option changes process-wide state and is meant for tests and
+ *     benchmarks only.
+ */
+#ifndef TERN_H
+#define TERN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum tern_status {
+    TERN_OK = 0,
+    TERN_ERR_INVALID_ARG = 1, /* null pointer, negative or zero count, bad option */
+    TERN_ERR_ALIGN = 2,       /* a pointer is not aligned as documented */
+    TERN_ERR_SHAPE = 3,       /* K not a positive multiple of 128, M or N < 1, too large */
+    TERN_ERR_WORKSPACE = 4,   /* workspace smaller than tern_workspace_bytes() */
+    TERN_ERR_CUDA = 5,        /* a CUDA runtime call or launch failed */
+    TERN_ERR_TIMEOUT = 6,     /* a bounded on-device wait gave up (see tern_gemm) */
+    TERN_ERR_DEVICE = 7       /* current device is not compute capability 10.0 */
+} tern_status;
+
+/* Library version, e.g. 100 for 0.1.0. */
+int tern_version(void);
+
+/* Static text for a status code ("ok", "invalid argument", ...). */
+const char *tern_status_string(int status);
+
+/* Text of the most recent error raised on the calling host thread ("" if
+ * none).  Valid until the next library call on that thread. */
+const char *tern_last_error(void);
+
+/* Size in bytes of the slot buffer / scale buffer of an N x K matrix;
+ * 0 if N < 1 or K is not a positive multiple of 128. */
+size_t tern_slots_bytes(int64_t N, int64_t K);
+size_t tern_scales_bytes(int64_t N, int64_t K);
+
+/* Workspace needed by tern_gemv / tern_gemm / tern_gemv_grouped for this
+ * shape.  The current kernels need none and return 0; a caller that passes a
+ * workspace anyway is fine.  A non-zero value would be stated here. */
+size_t tern_workspace_bytes(int64_t M, int64_t N, int64_t K);
+
+/*
+ * tern_pack_g128 -- build the slot layout from ternary values.
+ *   codes      int8 [N][K], each value in {-1, 0, +1}          (device, read)
+ *   scales_in  fp16 [N][K/128] as raw 16-bit patterns           (device, read)
+ *   slots_out  uint8 [N][K/4]                                  (device, written)
+ *   scales_out fp16 [N][K/128], a bit-exact copy of scales_in   (device, written;
+ *              may equal scales_in, then nothing is copied)
+ *   invalid_count  optional device int32: atomically incremented by the
+ *              number of codes outside {-1,0,+1}; such a code is stored as
+ *              slot value 3.  NULL to skip counting.
+ * Alignment: codes and slots_out 16 bytes; scales 2 bytes.  Any N >= 1.
+ * Result is bit-exact and independent of launch configuration.
+ */
+tern_status tern_pack_g128(const int8_t *codes, const uint16_t *scales_in, int64_t N, int64_t K,
+                           uint8_t *slots_out, uint16_t *scales_out, int32_t *invalid_count,
+                           void *stream);
+
+/*
+ * tern_unpack_g128 -- inverse of the slot layout.
+ *   slots      uint8 [N][K/4]  (device, read)
+ *   codes_out  int8  [N][K]    (device, written): t = c - 1; slot value 3 is
+ *              written as the sentinel 2.
+ * Alignment: 16 bytes for both.
+ */
+tern_status tern_unpack_g128(const uint8_t *slots, int64_t N, int64_t K, int8_t *codes_out,
+                             void *stream);
+
+/*
+ * tern_gemv -- decode matrix-vector product, M = 1:  y[n] = sum_k x[k] * w[n][k].
+ *   x       fp16 [K]        (device, read)
+ *   slots   uint8 [N][K/4]  (device, read)
+ *   scales  fp16 [N][K/128] (device, read)
+ *   y       fp16 [N]        (device, written)
+ *   workspace / ws_bytes: may be NULL / 0 (see tern_workspace_bytes).
+ * Bandwidth-bound: the weights are streamed from HBM once, unpacked in
+ * registers and never written back in any other precision.
+ */
+tern_status tern_gemv(const uint16_t *x, const uint8_t *slots, const uint16_t *scales, uint16_t *y,
+                      int64_t N, int64_t K, void *workspace, size_t ws_bytes, void *stream);
+
+/*
+ * tern_gemm -- y[M][N] = x[M][K] * W^T for any M >= 1.
+ *   x  fp16 [M][K] row-major (device, read);  y  fp16 [M][N] row-major (device, written).
+ * M <= 8 (speculative-verify batches) runs the same bandwidth-bound kernel as
+ * tern_gemv, reading the weights once for all rows.  Larger M runs the
+ * tensor-core prefill kernel, which unpacks weight tiles on chip to s*t
+ * (exact in fp16) and accumulates in fp32.
+ */
+tern_status tern_gemm(const uint16_t *x, const uint8_t *slots, const uint16_t *scales, uint16_t *y,
+                      int64_t M, int64_t N, int64_t K, void *workspace, size_t ws_bytes,
+                      void *stream);
+
+/* One matrix of a grouped product (all fields describe device buffers as in
+ * tern_gemm; every descriptor of one call has the same M). */
+typedef struct tern_gemv_desc {
+    const uint16_t *x;      /* fp16 [M][K] */
+    const uint8_t *slots;   /* uint8 [N][K/4] */
+    const uint16_t *scales; /* fp16 [N][K/128] */
+    uint16_t *y;            /* fp16 [M][N] */
+    int64_t N;
+    int64_t K;
+} tern_gemv_desc;
+
+/* Largest number of descriptors accepted by tern_gemv_grouped. */
+#define TERN_MAX_GROUP 16
+
+/*
+ * tern_gemv_grouped -- up to TERN_MAX_GROUP independent products with the same
+ * M (1..8) in ONE kernel launch, e.g. the q/k/v projections of a layer, or
+ * all seven projections of one synthetic decode layer.  Descriptors are read
+ * on the host during the call (the array need not outlive it).  Outputs must
+ * not overlap inputs or each other.
+ */
+tern_status tern_gemv_grouped(const tern_gemv_desc *descs, int32_t count, int64_t M, void *workspace,
+                              size_t ws_bytes, void *stream);
+
+/*
+ * Process-wide tuning knobs, for tests and benchmarks.  Value 0 restores the
+ * built-in heuristic.  Not thread-safe.
+ *   TERN_OPT_GEMV_KSPLIT   warps sharing one 16-row tile along K (1,2,4,8)
+ *   TERN_OPT_GEMV_CLUSTER  CTAs sharing one tile along K through a thread
+ *                          block cluster and distributed shared memory (1,2,4,8)
+ *   TERN_OPT_GEMV_CTAS     cap on resident CTAs per SM used for the grid
+ *   TERN_OPT_GEMM_PATH     1 = force the bandwidth kernel (M<=8 chunks),
+ *                          2 = force the tensor-core kernel
+ */
+enum {
+    TERN_OPT_GEMV_KSPLIT = 1,
+    TERN_OPT_GEMV_CLUSTER = 2,
+    TERN_OPT_GEMV_CTAS = 3,
+    TERN_OPT_GEMM_PATH = 4
+};
+tern_status tern_set_option(int option, int64_t value);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TERN_H */

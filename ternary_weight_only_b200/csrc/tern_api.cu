@@ -1,0 +1,233 @@
+// C entry points of libtern: argument checks on the host, then dispatch to
+// the kernels.  Nothing here allocates device memory.
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "tern_internal.cuh"
+
+namespace tern {
+
+Options g_opt;
+
+namespace {
+thread_local char t_err[512] = "";
+std::mutex g_dev_mu;
+DeviceInfo g_dev_cache[64];
+bool g_dev_valid[64];
+}  // namespace
+
+void clear_error() { t_err[0] = '\0'; }
+
+tern_status fail(tern_status st, const char *fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    std::vsnprintf(t_err, sizeof(t_err), fmt, ap);
+    va_end(ap);
+    return st;
+}
+
+tern_status cuda_fail(cudaError_t e, const char *what) {
+    if (e == cudaSuccess) return TERN_OK;
+    return fail(TERN_ERR_CUDA, "%s: %s (%s)", what, cudaGetErrorName(e), cudaGetErrorString(e));
+}
+
+tern_status current_device(DeviceInfo *out) {
+    int dev = -1;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    if (dev < 0 || dev >= 64) return fail(TERN_ERR_DEVICE, "device ordinal %d out of range", dev);
+    std::lock_guard<std::mutex> lock(g_dev_mu);
+    if (!g_dev_valid[dev]) {
+        DeviceInfo d;
+        d.device = dev;
+        e = cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev);
+        if (e == cudaSuccess) e = cudaDeviceGetAttribute(&d.major, cudaDevAttrComputeCapabilityMajor, dev);
+        if (e == cudaSuccess) e = cudaDeviceGetAttribute(&d.minor, cudaDevAttrComputeCapabilityMinor, dev);
+        int smem = 0;
+        if (e == cudaSuccess) e = cudaDeviceGetAttribute(&smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute");
+        d.max_smem_optin = static_cast<size_t>(smem);
+        g_dev_cache[dev] = d;
+        g_dev_valid[dev] = true;
+    }
+    *out = g_dev_cache[dev];
+    if (out->major != 10 || out->minor != 0)
+        return fail(TERN_ERR_DEVICE, "device %d is sm_%d%d; this library is built for sm_100a", dev,
+                    out->major, out->minor);
+    return TERN_OK;
+}
+
+}  // namespace tern
+
+using namespace tern;
+
+namespace {
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+tern_status check_nk(int64_t N, int64_t K) {
+    if (N < 1) return fail(TERN_ERR_SHAPE, "N must be >= 1 (got %lld)", static_cast<long long>(N));
+    if (K < kGroup || K % kGroup != 0)
+        return fail(TERN_ERR_SHAPE, "K must be a positive multiple of 128 (got %lld)",
+                    static_cast<long long>(K));
+    if (N > (int64_t(1) << 31) - 1 || K > (int64_t(1) << 30))
+        return fail(TERN_ERR_SHAPE, "N or K too large (N=%lld, K=%lld)", static_cast<long long>(N),
+                    static_cast<long long>(K));
+    if (N * K > (int64_t(1) << 46))
+        return fail(TERN_ERR_SHAPE, "N*K too large");
+    return TERN_OK;
+}
+
+tern_status check_mat(const void *x, const void *slots, const void *scales, const void *y) {
+    if (!x || !slots || !scales || !y) return fail(TERN_ERR_INVALID_ARG, "null buffer pointer");
+    if (!aligned16(x)) return fail(TERN_ERR_ALIGN, "x is not 16-byte aligned");
+    if (!aligned16(slots)) return fail(TERN_ERR_ALIGN, "slots is not 16-byte aligned");
+    if (!aligned16(scales)) return fail(TERN_ERR_ALIGN, "scales is not 16-byte aligned");
+    if (!aligned16(y)) return fail(TERN_ERR_ALIGN, "y is not 16-byte aligned");
+    return TERN_OK;
+}
+
+MatDesc mat(const uint16_t *x, const uint8_t *slots, const uint16_t *scales, uint16_t *y, int64_t N,
+            int64_t K) {
+    MatDesc d;
+    d.x = reinterpret_cast<const __half *>(x);
+    d.slots = slots;
+    d.scales = reinterpret_cast<const __half *>(scales);
+    d.y = reinterpret_cast<__half *>(y);
+    d.N = static_cast<int>(N);
+    d.K = static_cast<int>(K);
+    return d;
+}
+
+}  // namespace
+
+extern "C" {
+
+int tern_version(void) { return 100; }
+
+const char *tern_status_string(int status) {
+    switch (status) {
+        case TERN_OK: return "ok";
+        case TERN_ERR_INVALID_ARG: return "invalid argument";
+        case TERN_ERR_ALIGN: return "misaligned pointer";
+        case TERN_ERR_SHAPE: return "unsupported shape";
+        case TERN_ERR_WORKSPACE: return "workspace too small";
+        case TERN_ERR_CUDA: return "CUDA error";
+        case TERN_ERR_TIMEOUT: return "device wait timed out";
+        case TERN_ERR_DEVICE: return "unsupported device";
+        default: return "unknown status";
+    }
+}
+
+const char *tern_last_error(void) { return t_err; }
+
+size_t tern_slots_bytes(int64_t N, int64_t K) {
+    if (N < 1 || K < kGroup || K % kGroup != 0) return 0;
+    return static_cast<size_t>(N) * static_cast<size_t>(K / 4);
+}
+
+size_t tern_scales_bytes(int64_t N, int64_t K) {
+    if (N < 1 || K < kGroup || K % kGroup != 0) return 0;
+    return static_cast<size_t>(N) * static_cast<size_t>(K / kGroup) * 2;
+}
+
+size_t tern_workspace_bytes(int64_t M, int64_t N, int64_t K) {
+    (void)M;
+    (void)N;
+    (void)K;
+    return 0;
+}
+
+tern_status tern_pack_g128(const int8_t *codes, const uint16_t *scales_in, int64_t N, int64_t K,
+                           uint8_t *slots_out, uint16_t *scales_out, int32_t *invalid_count,
+                           void *stream) {
+    clear_error();
+    tern_status st = check_nk(N, K);
+    if (st != TERN_OK) return st;
+    if (!codes || !scales_in || !slots_out || !scales_out)
+        return fail(TERN_ERR_INVALID_ARG, "null buffer pointer");
+    if (!aligned16(codes)) return fail(TERN_ERR_ALIGN, "codes is not 16-byte aligned");
+    if (!aligned16(slots_out)) return fail(TERN_ERR_ALIGN, "slots_out is not 16-byte aligned");
+    if ((reinterpret_cast<uintptr_t>(scales_in) | reinterpret_cast<uintptr_t>(scales_out)) & 1u)
+        return fail(TERN_ERR_ALIGN, "scales are not 2-byte aligned");
+    if ((reinterpret_cast<uintptr_t>(invalid_count) & 3u) != 0)
+        return fail(TERN_ERR_ALIGN, "invalid_count is not 4-byte aligned");
+    return launch_pack(codes, scales_in, N, K, slots_out, scales_out, invalid_count,
+                       static_cast<cudaStream_t>(stream));
+}
+
+tern_status tern_unpack_g128(const uint8_t *slots, int64_t N, int64_t K, int8_t *codes_out,
+                             void *stream) {
+    clear_error();
+    tern_status st = check_nk(N, K);
+    if (st != TERN_OK) return st;
+    if (!slots || !codes_out) return fail(TERN_ERR_INVALID_ARG, "null buffer pointer");
+    if (!aligned16(slots) || !aligned16(codes_out))
+        return fail(TERN_ERR_ALIGN, "slots and codes_out must be 16-byte aligned");
+    return launch_unpack(slots, N, K, codes_out, static_cast<cudaStream_t>(stream));
+}
+
+tern_status tern_gemm(const uint16_t *x, const uint8_t *slots, const uint16_t *scales, uint16_t *y,
+                      int64_t M, int64_t N, int64_t K, void *workspace, size_t ws_bytes,
+                      void *stream) {
+    clear_error();
+    (void)workspace;
+    (void)ws_bytes;
+    if (M < 1) return fail(TERN_ERR_SHAPE, "M must be >= 1 (got %lld)", static_cast<long long>(M));
+    if (M > (int64_t(1) << 24)) return fail(TERN_ERR_SHAPE, "M too large");
+    tern_status st = check_nk(N, K);
+    if (st != TERN_OK) return st;
+    st = check_mat(x, slots, scales, y);
+    if (st != TERN_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    // Bandwidth kernel, eight token rows per launch (weights re-read per chunk).
+    for (int64_t m0 = 0; m0 < M; m0 += 8) {
+        const int mc = static_cast<int>(M - m0 < 8 ? M - m0 : 8);
+        MatDesc d = mat(x + m0 * K, slots, scales, y + m0 * N, N, K);
+        st = launch_gemv_mma(&d, 1, mc, s);
+        if (st != TERN_OK) return st;
+    }
+    return TERN_OK;
+}
+
+tern_status tern_gemv(const uint16_t *x, const uint8_t *slots, const uint16_t *scales, uint16_t *y,
+                      int64_t N, int64_t K, void *workspace, size_t ws_bytes, void *stream) {
+    return tern_gemm(x, slots, scales, y, 1, N, K, workspace, ws_bytes, stream);
+}
+
+tern_status tern_gemv_grouped(const tern_gemv_desc *descs, int32_t count, int64_t M,
+                              void *workspace, size_t ws_bytes, void *stream) {
+    clear_error();
+    (void)workspace;
+    (void)ws_bytes;
+    if (!descs) return fail(TERN_ERR_INVALID_ARG, "descs is NULL");
+    if (count < 1 || count > TERN_MAX_GROUP)
+        return fail(TERN_ERR_INVALID_ARG, "count must be 1..%d (got %d)", TERN_MAX_GROUP, count);
+    if (M < 1 || M > 8) return fail(TERN_ERR_SHAPE, "grouped product takes M in 1..8 (got %lld)",
+                                    static_cast<long long>(M));
+    MatDesc d[TERN_MAX_GROUP];
+    for (int i = 0; i < count; i++) {
+        tern_status st = check_nk(descs[i].N, descs[i].K);
+        if (st != TERN_OK) return st;
+        st = check_mat(descs[i].x, descs[i].slots, descs[i].scales, descs[i].y);
+        if (st != TERN_OK) return st;
+        d[i] = mat(descs[i].x, descs[i].slots, descs[i].scales, descs[i].y, descs[i].N, descs[i].K);
+    }
+    return launch_gemv_mma(d, count, static_cast<int>(M), static_cast<cudaStream_t>(stream));
+}
+
+tern_status tern_set_option(int option, int64_t value) {
+    clear_error();
+    if (value < 0 || value > 1024) return fail(TERN_ERR_INVALID_ARG, "option value %lld", static_cast<long long>(value));
+    switch (option) {
+        case TERN_OPT_GEMV_KSPLIT: g_opt.gemv_ksplit = static_cast<int>(value); return TERN_OK;
+        case TERN_OPT_GEMV_CLUSTER: g_opt.gemv_cluster = static_cast<int>(value); return TERN_OK;
+        case TERN_OPT_GEMV_CTAS: g_opt.gemv_ctas = static_cast<int>(value); return TERN_OK;
+        case TERN_OPT_GEMM_PATH: g_opt.gemm_path = static_cast<int>(value); return TERN_OK;
+        default: return fail(TERN_ERR_INVALID_ARG, "unknown option %d", option);
+    }
+}
+
+}  // extern "C"

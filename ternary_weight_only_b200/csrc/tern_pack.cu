@@ -1,0 +1,124 @@
+// Slot packing and unpacking for the ternary-g128 format.
+//
+// The format: t in {-1,0,+1} per weight and one fp16 scale per 128 weights
+// along K ("Bonsai 27B ternary / 1-bit quantization", ThakiCloud blog,
+// section "How compression works"), stored in 2-bit slots ("Ternary
+// quantization: 27B in 7 GB", devnsb blog, section "Limits").  The byte
+// layout (code c = t + 1, four codes per byte, least significant pair first)
+// is the one documented in tern.h.
+//
+// Both kernels are plain streaming kernels: every thread turns 16 consecutive
+// int8 codes (one 16-byte load) into one 32-bit slot word, so code j of the
+// chunk lands at bit 2j of the word -- byte j/4, bit pair j%4.
+#include "tern_internal.cuh"
+
+namespace tern {
+namespace {
+
+constexpr int kPackThreads = 256;
+
+__device__ __forceinline__ uint32_t code_of(int t, int &bad) {
+    // t in {-1,0,1} -> t + 1; anything else -> 3 (invalid)
+    const bool ok = (t >= -1) && (t <= 1);
+    bad += ok ? 0 : 1;
+    return ok ? static_cast<uint32_t>(t + 1) : 3u;
+}
+
+__global__ void __launch_bounds__(kPackThreads) pack_kernel(const int4 *__restrict__ codes,
+                                                            uint32_t *__restrict__ slots,
+                                                            int64_t nchunks,
+                                                            const uint16_t *__restrict__ sc_in,
+                                                            uint16_t *__restrict__ sc_out,
+                                                            int64_t nscales,
+                                                            int32_t *invalid_count) {
+    int bad = 0;
+    const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+    for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < nchunks;
+         i += stride) {
+        const int4 v = codes[i];
+        const uint32_t w4[4] = {static_cast<uint32_t>(v.x), static_cast<uint32_t>(v.y),
+                                static_cast<uint32_t>(v.z), static_cast<uint32_t>(v.w)};
+        uint32_t out = 0;
+#pragma unroll
+        for (int b = 0; b < 4; b++) {
+#pragma unroll
+            for (int j = 0; j < 4; j++) {
+                const int t = static_cast<int8_t>((w4[b] >> (8 * j)) & 0xFF);
+                out |= code_of(t, bad) << (2 * (4 * b + j));
+            }
+        }
+        slots[i] = out;
+    }
+    if (sc_out != nullptr) {
+        for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < nscales;
+             i += stride)
+            sc_out[i] = sc_in[i];
+    }
+    if (invalid_count != nullptr) {
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) bad += __shfl_xor_sync(0xffffffffu, bad, o);
+        if ((threadIdx.x & 31) == 0 && bad != 0) atomicAdd(invalid_count, bad);
+    }
+}
+
+__global__ void __launch_bounds__(kPackThreads) unpack_kernel(const uint32_t *__restrict__ slots,
+                                                              int4 *__restrict__ codes,
+                                                              int64_t nchunks) {
+    const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+    for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < nchunks;
+         i += stride) {
+        const uint32_t w = slots[i];
+        uint32_t o[4];
+#pragma unroll
+        for (int b = 0; b < 4; b++) {
+            uint32_t word = 0;
+#pragma unroll
+            for (int j = 0; j < 4; j++) {
+                const uint32_t c = (w >> (2 * (4 * b + j))) & 3u;
+                // c - 1 for c in {0,1,2}; the sentinel 2 for the invalid code 3
+                const int t = (c == 3u) ? 2 : static_cast<int>(c) - 1;
+                word |= (static_cast<uint32_t>(t) & 0xFFu) << (8 * j);
+            }
+            o[b] = word;
+        }
+        codes[i] = make_int4(static_cast<int>(o[0]), static_cast<int>(o[1]),
+                             static_cast<int>(o[2]), static_cast<int>(o[3]));
+    }
+}
+
+int grid_for(int64_t work, int sms) {
+    const int64_t want = (work + kPackThreads - 1) / kPackThreads;
+    const int64_t cap = static_cast<int64_t>(sms) * 8;
+    return static_cast<int>(want < 1 ? 1 : (want > cap ? cap : want));
+}
+
+}  // namespace
+
+tern_status launch_pack(const int8_t *codes, const uint16_t *scales_in, int64_t N, int64_t K,
+                        uint8_t *slots, uint16_t *scales_out, int32_t *invalid_count,
+                        cudaStream_t stream) {
+    DeviceInfo dev;
+    tern_status st = current_device(&dev);
+    if (st != TERN_OK) return st;
+    const int64_t nchunks = N * K / 16;
+    const int64_t nscales = N * (K / kGroup);
+    const uint16_t *sin = scales_in;
+    uint16_t *sout = (scales_in == scales_out) ? nullptr : scales_out;
+    pack_kernel<<<grid_for(nchunks, dev.sms), kPackThreads, 0, stream>>>(
+        reinterpret_cast<const int4 *>(codes), reinterpret_cast<uint32_t *>(slots), nchunks, sin,
+        sout, nscales, invalid_count);
+    return cuda_fail(cudaGetLastError(), "pack kernel launch");
+}
+
+tern_status launch_unpack(const uint8_t *slots, int64_t N, int64_t K, int8_t *codes,
+                          cudaStream_t stream) {
+    DeviceInfo dev;
+    tern_status st = current_device(&dev);
+    if (st != TERN_OK) return st;
+    const int64_t nchunks = N * K / 16;
+    unpack_kernel<<<grid_for(nchunks, dev.sms), kPackThreads, 0, stream>>>(
+        reinterpret_cast<const uint32_t *>(slots), reinterpret_cast<int4 *>(codes), nchunks);
+    return cuda_fail(cudaGetLastError(), "unpack kernel launch");
+}
+
+}  // namespace tern

@@ -1,0 +1,180 @@
+"""Python binding of libtern (include/tern.h): argument marshalling only.
+
+Every function here has the name of the C entry point it calls and takes
+PyTorch CUDA tensors; PyTorch supplies device memory and the current stream.
+All arithmetic runs in the CUDA kernels of libtern.so.  If the library is
+missing this module raises on import: there is no fallback path.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Sequence
+
+import torch
+
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libtern.so")
+if not os.path.exists(_LIB_PATH):
+    raise ImportError(
+        f"libtern.so not found at {_LIB_PATH}; build it with "
+        "`python -m ternary_weight_only_b200.build` (nvcc, sm_100a)")
+_L = ctypes.CDLL(_LIB_PATH)
+
+TERN_OK = 0
+TERN_ERR_INVALID_ARG = 1
+TERN_ERR_ALIGN = 2
+TERN_ERR_SHAPE = 3
+TERN_ERR_WORKSPACE = 4
+TERN_ERR_CUDA = 5
+TERN_ERR_TIMEOUT = 6
+TERN_ERR_DEVICE = 7
+
+TERN_OPT_GEMV_KSPLIT = 1
+TERN_OPT_GEMV_CLUSTER = 2
+TERN_OPT_GEMV_CTAS = 3
+TERN_OPT_GEMM_PATH = 4
+TERN_MAX_GROUP = 16
+
+_i64, _vp, _sz, _i32, _int = ctypes.c_int64, ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int32, ctypes.c_int
+
+
+class tern_gemv_desc(ctypes.Structure):
+    _fields_ = [("x", _vp), ("slots", _vp), ("scales", _vp), ("y", _vp), ("N", _i64), ("K", _i64)]
+
+
+_SIGS = {
+    "tern_version": ([], _int),
+    "tern_status_string": ([_int], ctypes.c_char_p),
+    "tern_last_error": ([], ctypes.c_char_p),
+    "tern_slots_bytes": ([_i64, _i64], _sz),
+    "tern_scales_bytes": ([_i64, _i64], _sz),
+    "tern_workspace_bytes": ([_i64, _i64, _i64], _sz),
+    "tern_pack_g128": ([_vp, _vp, _i64, _i64, _vp, _vp, _vp, _vp], _int),
+    "tern_unpack_g128": ([_vp, _i64, _i64, _vp, _vp], _int),
+    "tern_gemv": ([_vp, _vp, _vp, _vp, _i64, _i64, _vp, _sz, _vp], _int),
+    "tern_gemm": ([_vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp, _sz, _vp], _int),
+    "tern_gemv_grouped": ([ctypes.POINTER(tern_gemv_desc), _i32, _i64, _vp, _sz, _vp], _int),
+    "tern_set_option": ([_int, _i64], _int),
+}
+for _name, (_args, _res) in _SIGS.items():
+    _f = getattr(_L, _name)
+    _f.argtypes = _args
+    _f.restype = _res
+
+lib = _L  # raw C-ABI access (pointers and sizes), used by the tests
+
+
+class TernError(RuntimeError):
+    def __init__(self, status: int, fn: str):
+        self.status = status
+        detail = _L.tern_last_error().decode(errors="replace")
+        super().__init__(f"{fn}: {_L.tern_status_string(status).decode()} ({status}): {detail}")
+
+
+def _check(st: int, fn: str):
+    if st != TERN_OK:
+        raise TernError(st, fn)
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream
+    return int(stream)
+
+
+def _dev(t: torch.Tensor, name: str, dtype=None) -> int:
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t.data_ptr()
+
+
+def tern_version() -> int:
+    return _L.tern_version()
+
+
+def tern_slots_bytes(N: int, K: int) -> int:
+    return _L.tern_slots_bytes(N, K)
+
+
+def tern_scales_bytes(N: int, K: int) -> int:
+    return _L.tern_scales_bytes(N, K)
+
+
+def tern_workspace_bytes(M: int, N: int, K: int) -> int:
+    return _L.tern_workspace_bytes(M, N, K)
+
+
+def tern_set_option(option: int, value: int):
+    _check(_L.tern_set_option(option, value), "tern_set_option")
+
+
+def tern_pack_g128(codes: torch.Tensor, scales: torch.Tensor, slots_out: Optional[torch.Tensor] = None,
+                   scales_out: Optional[torch.Tensor] = None,
+                   invalid_count: Optional[torch.Tensor] = None, stream=None):
+    """codes int8 [N,K], scales fp16 [N,K/128] -> (slots uint8 [N,K/4], scales fp16 [N,K/128])."""
+    N, K = codes.shape
+    if slots_out is None:
+        slots_out = torch.empty((N, K // 4), dtype=torch.uint8, device=codes.device)
+    if scales_out is None:
+        scales_out = torch.empty_like(scales)
+    ic = 0 if invalid_count is None else _dev(invalid_count, "invalid_count", torch.int32)
+    _check(_L.tern_pack_g128(_dev(codes, "codes", torch.int8), _dev(scales, "scales", torch.float16),
+                             N, K, _dev(slots_out, "slots_out", torch.uint8),
+                             _dev(scales_out, "scales_out", torch.float16), ic or None,
+                             _stream(stream)), "tern_pack_g128")
+    return slots_out, scales_out
+
+
+def tern_unpack_g128(slots: torch.Tensor, K: int, codes_out: Optional[torch.Tensor] = None, stream=None):
+    N = slots.shape[0]
+    if codes_out is None:
+        codes_out = torch.empty((N, K), dtype=torch.int8, device=slots.device)
+    _check(_L.tern_unpack_g128(_dev(slots, "slots", torch.uint8), N, K,
+                               _dev(codes_out, "codes_out", torch.int8), _stream(stream)),
+           "tern_unpack_g128")
+    return codes_out
+
+
+def tern_gemv(x: torch.Tensor, slots: torch.Tensor, scales: torch.Tensor,
+              y: Optional[torch.Tensor] = None, stream=None):
+    """x fp16 [K] -> y fp16 [N]."""
+    N = slots.shape[0]
+    K = x.shape[-1]
+    if y is None:
+        y = torch.empty((N,), dtype=torch.float16, device=x.device)
+    _check(_L.tern_gemv(_dev(x, "x", torch.float16), _dev(slots, "slots", torch.uint8),
+                        _dev(scales, "scales", torch.float16), _dev(y, "y", torch.float16), N, K,
+                        None, 0, _stream(stream)), "tern_gemv")
+    return y
+
+
+def tern_gemm(x: torch.Tensor, slots: torch.Tensor, scales: torch.Tensor,
+              y: Optional[torch.Tensor] = None, stream=None):
+    """x fp16 [M,K] -> y fp16 [M,N]."""
+    M, K = x.shape
+    N = slots.shape[0]
+    if y is None:
+        y = torch.empty((M, N), dtype=torch.float16, device=x.device)
+    _check(_L.tern_gemm(_dev(x, "x", torch.float16), _dev(slots, "slots", torch.uint8),
+                        _dev(scales, "scales", torch.float16), _dev(y, "y", torch.float16), M, N, K,
+                        None, 0, _stream(stream)), "tern_gemm")
+    return y
+
+
+def tern_gemv_grouped(mats: Sequence, M: int, stream=None):
+    """mats: sequence of (x [M,K], slots [N,K/4], scales [N,K/128], y [M,N]) CUDA tensors."""
+    arr = (tern_gemv_desc * len(mats))()
+    for i, (x, s, sc, y) in enumerate(mats):
+        arr[i].x = _dev(x, "x", torch.float16)
+        arr[i].slots = _dev(s, "slots", torch.uint8)
+        arr[i].scales = _dev(sc, "scales", torch.float16)
+        arr[i].y = _dev(y, "y", torch.float16)
+        arr[i].N = s.shape[0]
+        arr[i].K = x.shape[-1]
+    _check(_L.tern_gemv_grouped(arr, len(mats), M, None, 0, _stream(stream)), "tern_gemv_grouped")

@@ -1,0 +1,127 @@
+"""The C ABI without a GPU: the library loads, exports every entry point that
+include/tern.h declares, and rejects bad arguments on the host before any
+launch."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "tern.h")
+
+
+def _declared():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(tern_[a-z0-9_]+)\s*\(", src)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from ternary_weight_only_b200 import build
+    build.build()
+    from ternary_weight_only_b200 import tern
+    return tern.lib
+
+
+def test_header_declares_the_boundary():
+    names = _declared()
+    for n in ["tern_pack_g128", "tern_unpack_g128", "tern_gemv", "tern_gemm",
+              "tern_gemv_grouped", "tern_workspace_bytes", "tern_slots_bytes",
+              "tern_scales_bytes", "tern_status_string", "tern_last_error", "tern_set_option",
+              "tern_version"]:
+        assert n in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    from ternary_weight_only_b200 import build
+    out = subprocess.run(["nm", "-D", "--defined-only", build.LIB], capture_output=True,
+                         text=True, check=True).stdout
+    exported = set(line.split()[-1] for line in out.splitlines() if line.strip())
+    for name in _declared():
+        assert name in exported, name
+        assert hasattr(lib, name)
+
+
+def test_sizes(lib):
+    assert lib.tern_slots_bytes(256, 512) == 256 * 128
+    assert lib.tern_scales_bytes(256, 512) == 256 * 4 * 2
+    assert lib.tern_slots_bytes(151936, 5120) + lib.tern_scales_bytes(151936, 5120) == \
+        151936 * 5120 * 17 // 64
+    for bad in [(0, 128), (4, 0), (4, 100), (-1, 128), (4, -128)]:
+        assert lib.tern_slots_bytes(*bad) == 0 and lib.tern_scales_bytes(*bad) == 0
+    assert lib.tern_workspace_bytes(1, 1024, 5120) == 0
+    assert lib.tern_version() >= 100
+
+
+def test_status_strings(lib):
+    for st in range(8):
+        assert lib.tern_status_string(st)
+    assert lib.tern_status_string(99) == b"unknown status"
+
+
+A = 1 << 20  # a fake 16-byte-aligned address: never dereferenced, checks fail first
+
+
+@pytest.mark.parametrize("args,status", [
+    ((None, A, A, A, 8, 128, None, 0, None), 1),          # null x
+    ((A, A, A, A, 8, 100, None, 0, None), 3),             # K % 128
+    ((A, A, A, A, 0, 128, None, 0, None), 3),             # N = 0
+    ((A + 2, A, A, A, 8, 128, None, 0, None), 2),         # misaligned x
+    ((A, A + 4, A, A, 8, 128, None, 0, None), 2),         # misaligned slots
+    ((A, A, A + 2, A, 8, 128, None, 0, None), 2),         # misaligned scales
+    ((A, A, A, A + 8, 8, 128, None, 0, None), 2),         # misaligned y
+])
+def test_gemv_rejects(lib, args, status):
+    assert lib.tern_gemv(*args) == status
+    assert lib.tern_last_error()
+
+
+def test_gemm_rejects(lib):
+    assert lib.tern_gemm(A, A, A, A, 0, 8, 128, None, 0, None) == 3
+    assert lib.tern_gemm(A, A, A, A, 4, 8, 130, None, 0, None) == 3
+    assert lib.tern_gemm(A, A, A, None, 4, 8, 128, None, 0, None) == 1
+
+
+def test_pack_rejects(lib):
+    assert lib.tern_pack_g128(None, A, 4, 128, A, A, None, None) == 1
+    assert lib.tern_pack_g128(A, A, 4, 96, A, A, None, None) == 3
+    assert lib.tern_pack_g128(A + 1, A, 4, 128, A, A, None, None) == 2
+    assert lib.tern_pack_g128(A, A + 1, 4, 128, A, A, None, None) == 2
+    assert lib.tern_pack_g128(A, A, 4, 128, A, A, A + 2, None) == 2
+    assert lib.tern_unpack_g128(A, 4, 128, A + 3, None) == 2
+    assert lib.tern_unpack_g128(A, 4, 127, A, None) == 3
+
+
+def test_grouped_rejects(lib):
+    from ternary_weight_only_b200 import tern
+    arr = (tern.tern_gemv_desc * 2)()
+    for d in arr:
+        d.x, d.slots, d.scales, d.y, d.N, d.K = A, A, A, A, 16, 256
+    assert lib.tern_gemv_grouped(None, 1, 1, None, 0, None) == 1
+    assert lib.tern_gemv_grouped(arr, 0, 1, None, 0, None) == 1
+    assert lib.tern_gemv_grouped(arr, 17, 1, None, 0, None) == 1
+    assert lib.tern_gemv_grouped(arr, 2, 9, None, 0, None) == 3
+    arr[1].K = 200
+    assert lib.tern_gemv_grouped(arr, 2, 1, None, 0, None) == 3
+    arr[1].K = 256
+    arr[1].y = A + 2
+    assert lib.tern_gemv_grouped(arr, 2, 1, None, 0, None) == 2
+
+
+def test_options(lib):
+    assert lib.tern_set_option(99, 1) == 1
+    assert lib.tern_set_option(1, -1) == 1
+    assert lib.tern_set_option(1, 0) == 0
+
+
+def test_valid_call_without_gpu_reports_cuda_error(lib):
+    """With no usable device a well-formed call fails cleanly with a status."""
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    st = lib.tern_gemv(A, A, A, A, 16, 256, None, 0, None)
+    assert st in (5, 7)
+    assert lib.tern_last_error()

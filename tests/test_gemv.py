@@ -1,0 +1,202 @@
+"""GPU bandwidth kernel (M = 1..8) against the fp64 oracle, element by element.
+
+Tolerance: |y - y_ref| <= 2e-3 * sum_k |x_k w_k| + 1e-5 (helpers.check_close).
+"""
+import os
+
+import numpy as np
+import pytest
+import torch
+
+from helpers import check_close, np_inputs
+
+pytestmark = pytest.mark.gpu
+NCPU = os.cpu_count() or 1
+
+
+@pytest.fixture(scope="module")
+def T():
+    from ternary_weight_only_b200 import build
+    build.build()
+    from ternary_weight_only_b200 import tern
+    yield tern
+    for o in (1, 2, 3, 4):
+        tern.tern_set_option(o, 0)
+
+
+def run_case(T, orc, x, codes, scales, what="", threads=None):
+    """Pack with the oracle (host), run the GPU product on those slots, compare."""
+    xn, cn, sn = np_inputs(x, codes, scales)
+    slots, sc, bad, _ = orc.pack(cn, sn)
+    assert bad == 0
+    yd = T.tern_gemm(x.cuda(), torch.from_numpy(slots).cuda(), scales.cuda())
+    torch.cuda.synchronize()
+    y_ref, bound = orc.matmul(xn, slots, sc, threads=threads or NCPU)
+    return check_close(yd, y_ref, bound, what)
+
+
+def test_tiny_gemv(T, orc):
+    from ternary_weight_only_b200 import synth
+    x, codes, scales = synth.tiny_gemv()
+    xn, cn, sn = np_inputs(x, codes, scales)
+    slots, sc, _, _ = orc.pack(cn, sn)
+    y = T.tern_gemv(x[0].cuda(), torch.from_numpy(slots).cuda(), scales.cuda())
+    torch.cuda.synchronize()
+    y_ref, bound = orc.matmul(xn, slots, sc)
+    check_close(y.view(1, -1), y_ref, bound, "tiny")
+
+
+@pytest.mark.parametrize("i", range(7))
+def test_decode_layer_projection(T, orc, i):
+    from ternary_weight_only_b200 import synth
+    x, codes, scales = synth.decode_proj(i)
+    run_case(T, orc, x, codes, scales, synth.LAYER_PROJ[i][0])
+
+
+@pytest.mark.parametrize("M", [2, 4, 8])
+@pytest.mark.parametrize("i", range(7))
+def test_verify_batch(T, orc, i, M):
+    from ternary_weight_only_b200 import synth
+    x, codes, scales = synth.decode_proj(i, M=M)
+    run_case(T, orc, x, codes, scales, f"{synth.LAYER_PROJ[i][0]} M={M}")
+
+
+@pytest.mark.parametrize("M,K,N", [
+    (1, 128, 1), (1, 128, 17), (3, 256, 5), (8, 384, 33), (5, 640, 100), (1, 1152, 129),
+    (2, 2048, 250), (7, 128, 16), (1, 4096, 1000), (6, 17408, 40), (8, 17408, 300),
+    (4, 25600, 64),
+])
+def test_ragged(T, orc, M, K, N):
+    from ternary_weight_only_b200 import synth
+    x, codes, scales = synth.case(M, K, N, seed=M * 1000 + K + N, codes="sparse", outlier_p=0.01)
+    run_case(T, orc, x, codes, scales, f"M={M} K={K} N={N}")
+
+
+@pytest.mark.parametrize("ks", [1, 2, 4, 8])
+@pytest.mark.parametrize("cl", [1, 2, 4])
+def test_split_options(T, orc, ks, cl):
+    from ternary_weight_only_b200 import synth
+    x, codes, scales = synth.case(3, 2048, 200, seed=ks * 10 + cl, codes="sparse")
+    T.tern_set_option(T.TERN_OPT_GEMV_KSPLIT, ks)
+    T.tern_set_option(T.TERN_OPT_GEMV_CLUSTER, cl)
+    try:
+        run_case(T, orc, x, codes, scales, f"ks={ks} cl={cl}")
+        x1, c1, s1 = synth.case(1, 5120, 1024, seed=ks * 10 + cl + 1, codes="sparse")
+        run_case(T, orc, x1, c1, s1, f"M=1 ks={ks} cl={cl}")
+    finally:
+        T.tern_set_option(T.TERN_OPT_GEMV_KSPLIT, 0)
+        T.tern_set_option(T.TERN_OPT_GEMV_CLUSTER, 0)
+
+
+def test_grid_cap(T, orc):
+    """Few resident CTAs: every CTA walks many tiles."""
+    from ternary_weight_only_b200 import synth
+    x, codes, scales = synth.case(1, 1024, 4000, seed=3, codes="sparse")
+    T.tern_set_option(T.TERN_OPT_GEMV_CTAS, 1)
+    try:
+        run_case(T, orc, x, codes, scales, "one CTA per SM")
+    finally:
+        T.tern_set_option(T.TERN_OPT_GEMV_CTAS, 0)
+
+
+def test_exact_special_cases(T, orc):
+    """Zero codes give exactly 0; a single non-zero per row gives s*t*x within
+    fp16 output rounding; all +1 codes with unit scales give row sums."""
+    from ternary_weight_only_b200 import synth
+    M, K, N = 4, 1024, 48
+    x, codes, scales = synth.case(M, K, N, seed=41)
+    z = torch.zeros_like(codes)
+    slots, _ = T.tern_pack_g128(z.cuda(), scales.cuda())
+    y = T.tern_gemm(x.cuda(), slots, scales.cuda())
+    torch.cuda.synchronize()
+    assert torch.all(y == 0)
+    one = torch.zeros_like(codes)
+    for n in range(N):
+        one[n, (n * 37 + 5) % K] = 1 if n % 2 else -1
+    run_case(T, orc, x, one, scales, "single non-zero")
+    ones = torch.ones_like(codes)
+    unit = torch.ones_like(scales)
+    xs = (torch.randn(M, K) * 0.05).half()  # keep row sums inside fp16 range
+    run_case(T, orc, xs, ones, unit, "row sums")
+
+
+def test_adversarial_accumulation(T, orc):
+    """Same-sign terms: x all +1 or with x20 outliers, codes all +1 in a group."""
+    M, K, N = 8, 2048, 64
+    codes = torch.ones((N, K), dtype=torch.int8)
+    codes[N // 2:, 128:] = -1
+    scales = torch.full((N, K // 128), 0.0499).half()
+    x = torch.ones((M, K)).half()
+    x[1::2, ::3] = 20.0
+    run_case(T, orc, x, codes, scales, "same sign")
+
+
+def test_negative_and_zero_scales(T, orc):
+    from ternary_weight_only_b200 import synth
+    x, codes, scales = synth.case(2, 768, 90, seed=43)
+    scales = scales.clone()
+    scales[::3] = -scales[::3]
+    scales[1::5] = 0
+    run_case(T, orc, x, codes, scales, "signed scales")
+
+
+def test_invalid_slot_value_is_finite(T):
+    slots = torch.full((32, 64), 0xFF, dtype=torch.uint8, device="cuda")  # every code 3
+    scales = torch.full((32, 2), 0.01).half().cuda()
+    x = torch.randn(1, 256).half().cuda()
+    y = T.tern_gemm(x, slots, scales)
+    torch.cuda.synchronize()
+    assert torch.isfinite(y.float()).all()
+
+
+def test_grouped_layer(T, orc):
+    """All seven projections of one decode layer in one launch."""
+    from ternary_weight_only_b200 import synth
+    for M in (1, 4):
+        mats, refs = [], []
+        for i in range(7):
+            x, codes, scales = synth.decode_proj(i, M=M)
+            xn, cn, sn = np_inputs(x, codes, scales)
+            slots, sc, _, _ = orc.pack(cn, sn)
+            N = codes.shape[0]
+            y = torch.full((M, N), float("nan"), dtype=torch.float16, device="cuda")
+            mats.append((x.cuda(), torch.from_numpy(slots).cuda(), scales.cuda(), y))
+            refs.append((xn, slots, sc))
+        T.tern_gemv_grouped(mats, M)
+        torch.cuda.synchronize()
+        for i, ((xn, slots, sc), m) in enumerate(zip(refs, mats)):
+            y_ref, bound = orc.matmul(xn, slots, sc, threads=NCPU)
+            check_close(m[3], y_ref, bound, f"grouped {synth.LAYER_PROJ[i][0]} M={M}")
+
+
+def test_head_full(T, orc):
+    """The 5120 -> 151936 output head at full size, every output checked."""
+    from ternary_weight_only_b200 import synth
+    N, K = 151936, 5120
+    g = synth.gen(4999, "cuda")
+    codes = synth.codes_sparse(N, K, g, device="cuda")
+    scales = synth.scales_uniform(N, K, g, device="cuda")
+    x = synth.activations(1, K, g, device="cuda")
+    slots, sc = T.tern_pack_g128(codes, scales)
+    y = T.tern_gemm(x, slots, sc)
+    torch.cuda.synchronize()
+    xn, cn, sn = np_inputs(x.cpu(), codes.cpu(), scales.cpu())
+    ref_slots, ref_sc, _, _ = orc.pack(cn, sn)
+    assert np.array_equal(ref_slots, slots.cpu().numpy())
+    y_ref, bound = orc.matmul(xn, ref_slots, ref_sc, threads=NCPU)
+    check_close(y, y_ref, bound, "head")
+
+
+def test_stream_argument(T, orc):
+    from ternary_weight_only_b200 import synth
+    x, codes, scales = synth.case(1, 512, 256, seed=8)
+    xn, cn, sn = np_inputs(x, codes, scales)
+    slots, sc, _, _ = orc.pack(cn, sn)
+    s = torch.cuda.Stream()
+    xd, sd, scd = x.cuda(), torch.from_numpy(slots).cuda(), scales.cuda()
+    torch.cuda.synchronize()
+    with torch.cuda.stream(s):
+        y = T.tern_gemm(xd, sd, scd)
+    s.synchronize()
+    y_ref, bound = orc.matmul(xn, slots, sc)
+    check_close(y, y_ref, bound, "side stream")
