@@ -150,11 +150,12 @@ def max_over_ranks(v, ws):
 class DecodeModel:
     """The synthetic 64-layer decode weight set, packed on the GPU."""
 
-    def __init__(self, T, device="cuda"):
+    def __init__(self, T, device="cuda", n_layers=synth.N_LAYERS):
         self.T = T
+        self.n_layers = n_layers
         self.layers = []  # per layer: list of (name, K, N, slots, scales)
         self.x_all = None
-        for l in range(synth.N_LAYERS):
+        for l in range(n_layers):
             g = synth.gen(4000 + l, device)
             mats = []
             for name, K, N in synth.LAYER_PROJ:
@@ -164,7 +165,7 @@ class DecodeModel:
                 del codes
                 mats.append((name, K, N, slots, sc))
             self.layers.append(mats)
-        g = synth.gen(4000 + synth.N_LAYERS, device)
+        g = synth.gen(4000 + synth.N_LAYERS, device)  # head seed independent of n_layers
         _, K, N = synth.HEAD
         codes = synth.codes_sparse(N, K, g, device=device)
         scales = synth.scales_uniform(N, K, g, device=device)
@@ -173,14 +174,14 @@ class DecodeModel:
         torch.cuda.synchronize()
         # Inputs: per layer x_h (q,k,v,gate,up), x_o (o), x_d (down); head input.
         per_layer = 5120 + 6144 + 17408
-        self.x_all = torch.empty(synth.N_LAYERS * per_layer + 5120, dtype=torch.float16, device=device)
+        self.x_all = torch.empty(n_layers * per_layer + 5120, dtype=torch.float16, device=device)
         g = synth.gen(5000, device)
         self.x_all.copy_(torch.randn(self.x_all.numel(), generator=g, device=device).half())
         yn = sum(N for _, _, N in synth.LAYER_PROJ)
-        self.y_all = torch.empty(synth.N_LAYERS * yn + synth.HEAD[2], dtype=torch.float16, device=device)
+        self.y_all = torch.empty(n_layers * yn + synth.HEAD[2], dtype=torch.float16, device=device)
         self.groups = []
         xo = yo = 0
-        for l in range(synth.N_LAYERS):
+        for l in range(n_layers):
             xh = self.x_all[xo:xo + 5120]
             xop = self.x_all[xo + 5120:xo + 5120 + 6144]
             xd = self.x_all[xo + 5120 + 6144:xo + per_layer]
@@ -201,7 +202,9 @@ class DecodeModel:
         _, K, N, slots, sc = self.head
         T.tern_gemv(self.head_io[0], slots, sc, self.head_io[1])
 
-    launches_per_step = synth.N_LAYERS + 1
+    @property
+    def launches_per_step(self):
+        return self.n_layers + 1
 
 
 def cuda_time(fn, iters, stream=None):
@@ -358,8 +361,8 @@ def run_reference(args):
 def traffic_from_profile():
     """Per-launch DRAM bytes of the dominant kernel from the committed ncu
     summary, only if the kernel source is unchanged since the capture."""
-    prof = os.path.join(ROOT, "profiles", "gemv_mma_kernel.decode_layer.txt")
-    src = os.path.join(ROOT, "ternary_weight_only_b200", "csrc", "tern_gemv.cu")
+    prof = os.path.join(ROOT, "profiles", "gemv_tma_kernel.decode_layer.txt")
+    src = os.path.join(ROOT, "ternary_weight_only_b200", "csrc", "tern_gemv_tma.cu")
     try:
         text = open(prof).read()
         sha = hashlib.sha256(open(src, "rb").read()).hexdigest()
@@ -370,6 +373,20 @@ def traffic_from_profile():
     except OSError:
         pass
     return None
+
+
+def run_profile(args):
+    """Small case for ncu captures: a few layers' grouped launches, eager."""
+    torch.cuda.set_device(0)
+    from ternary_weight_only_b200 import tern as T
+    model = DecodeModel(T, n_layers=args.profile_layers)
+    for _ in range(3):
+        for grp in model.groups:
+            T.tern_gemv_grouped(grp, 1)
+    torch.cuda.synchronize()
+    print(json.dumps({"profile_layers": args.profile_layers,
+                      "bytes_per_launch": sum(wbytes(K, N) + 2 * K + 2 * N for _, K, N in synth.LAYER_PROJ)}))
+    return 0
 
 
 def run_tern(args):
@@ -460,7 +477,7 @@ def run_tern(args):
             "e2e": {"value": round(e2e_value, 1), "unit": "GB/s", "ms_per_step": round(e2e_ms, 4),
                     "h2d_bytes_per_step": int(model.x_all.numel() * 2),
                     "d2h_bytes_per_step": int(model.y_all.numel() * 2)},
-            "roofline": {"bound": "hbm", "kernel": "gemv_mma_kernel",
+            "roofline": {"bound": "hbm", "kernel": "gemv_tma_kernel",
                          "achieved": round(achieved, 1), "peak": peak_gbs, "unit": "GB/s",
                          "frac": round(achieved / peak_gbs, 4), "traffic": traffic,
                          "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)" if peak_src == "measured" else "fallback 6650 GB/s",
@@ -486,7 +503,11 @@ def main():
     ap.add_argument("--impl", choices=["tern", "reference"], default="tern")
     ap.add_argument("--no-rows", action="store_true", help="skip the per-shape breakdown")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
+    ap.add_argument("--profile-layers", type=int, default=0,
+                    help="profiling case: build this many layers, run their grouped launches 3x, exit")
     args = ap.parse_args()
+    if args.profile_layers > 0:
+        return run_profile(args)
     if args.warmup < 3:
         args.warmup = 3
     if args.impl == "reference":

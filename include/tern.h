@@ -132,9 +132,10 @@ tern_status tern_gemv(const uint16_t *x, const uint8_t *slots, const uint16_t *s
  * tern_gemm -- y[M][N] = x[M][K] * W^T for any M >= 1.
  *   x  fp16 [M][K] row-major (device, read);  y  fp16 [M][N] row-major (device, written).
  * M <= 8 (speculative-verify batches) runs the same bandwidth-bound kernel as
- * tern_gemv, reading the weights once for all rows.  Larger M runs the
- * tensor-core prefill kernel, which unpacks weight tiles on chip to s*t
- * (exact in fp16) and accumulates in fp32.
+ * tern_gemv, reading the weights once for all rows.  M >= 32 runs the
+ * tensor-core prefill kernel (tcgen05), which unpacks weight tiles on chip to
+ * s*t (exact in fp16) straight into tensor memory and accumulates in fp32;
+ * 8 < M < 32 runs the bandwidth kernel once per eight rows.
  */
 tern_status tern_gemm(const uint16_t *x, const uint8_t *slots, const uint16_t *scales, uint16_t *y,
                       int64_t M, int64_t N, int64_t K, void *workspace, size_t ws_bytes,
@@ -165,20 +166,43 @@ tern_status tern_gemv_grouped(const tern_gemv_desc *descs, int32_t count, int64_
                               size_t ws_bytes, void *stream);
 
 /*
+ * tern_sync_status -- wait for `stream`, then report whether any kernel of
+ * this library on the current device gave up a bounded on-device wait since
+ * the previous call (TERN_ERR_TIMEOUT), clearing that record.  No kernel of
+ * this library spins without a limit: a wait that exceeds it (1 s by default)
+ * makes the kernel stop, release its resources and return, leaving its output
+ * undefined and the CUDA context usable.
+ */
+tern_status tern_sync_status(void *stream);
+
+/*
  * Process-wide tuning knobs, for tests and benchmarks.  Value 0 restores the
- * built-in heuristic.  Not thread-safe.
- *   TERN_OPT_GEMV_KSPLIT   warps sharing one 16-row tile along K (1,2,4,8)
+ * built-in default.  Not thread-safe.
+ *   TERN_OPT_GEMV_KSPLIT   warps sharing one 16-row tile along K (1,2,4,8;
+ *                          the TMA kernel may lower it for short K)
  *   TERN_OPT_GEMV_CLUSTER  CTAs sharing one tile along K through a thread
  *                          block cluster and distributed shared memory (1,2,4,8)
  *   TERN_OPT_GEMV_CTAS     cap on resident CTAs per SM used for the grid
  *   TERN_OPT_GEMM_PATH     1 = force the bandwidth kernel (M<=8 chunks),
  *                          2 = force the tensor-core kernel
+ *   TERN_OPT_GEMM_MIN_M    smallest M (> 8) sent to the tensor-core kernel
+ *                          (default 32)
+ *   TERN_OPT_GEMV_VARIANT  bandwidth kernel: 0 = TMA-staged (default),
+ *                          1 = register-ring loads (kept for comparison)
+ *   TERN_OPT_TEST_STALL_US TESTS ONLY: the TMA loaders of the tensor-core and
+ *                          the TMA-staged bandwidth kernels issue no loads, so
+ *                          their waits can never complete, and every bounded
+ *                          wait gives up after this many microseconds.
+ *                          Exercises the timeout path; 0 = normal operation.
  */
 enum {
     TERN_OPT_GEMV_KSPLIT = 1,
     TERN_OPT_GEMV_CLUSTER = 2,
     TERN_OPT_GEMV_CTAS = 3,
-    TERN_OPT_GEMM_PATH = 4
+    TERN_OPT_GEMM_PATH = 4,
+    TERN_OPT_GEMM_MIN_M = 5,
+    TERN_OPT_TEST_STALL_US = 6,
+    TERN_OPT_GEMV_VARIANT = 7
 };
 tern_status tern_set_option(int option, int64_t value);
 

@@ -1,5 +1,7 @@
 // C entry points of libtern: argument checks on the host, then dispatch to
 // the kernels.  Nothing here allocates device memory.
+#include <cudaTypedefs.h>
+
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
@@ -59,11 +61,45 @@ tern_status current_device(DeviceInfo *out) {
     return TERN_OK;
 }
 
+namespace {
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::once_flag g_encode_once;
+cudaError_t g_encode_err = cudaSuccess;
+}  // namespace
+
+tern_status encode_tiled_2d(CUtensorMap *map, CUtensorMapDataType dt, const void *base, uint64_t inner,
+                            uint64_t outer, uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer,
+                            CUtensorMapSwizzle swizzle) {
+    std::call_once(g_encode_once, [] {
+        void *fn = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        g_encode_err = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q);
+        if (g_encode_err == cudaSuccess && q == cudaDriverEntryPointSuccess)
+            g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    });
+    if (!g_encode)
+        return fail(TERN_ERR_CUDA, "cuTensorMapEncodeTiled unavailable (%s)", cudaGetErrorString(g_encode_err));
+    std::memset(map, 0, sizeof(*map));
+    const cuuint64_t dims[2] = {inner, outer};
+    const cuuint64_t strides[1] = {row_bytes};
+    const cuuint32_t box[2] = {box_inner, box_outer};
+    const cuuint32_t estr[2] = {1, 1};
+    CUresult r = g_encode(map, dt, 2, const_cast<void *>(base), dims, strides, box, estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(TERN_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
+    return TERN_OK;
+}
+
 }  // namespace tern
 
 using namespace tern;
 
 namespace {
+
+// Smallest M sent to the tensor-core kernel by default; below it the
+// bandwidth kernel runs in chunks of eight token rows.
+constexpr int64_t kTensorCoreMinM = 32;
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -182,11 +218,14 @@ tern_status tern_gemm(const uint16_t *x, const uint8_t *slots, const uint16_t *s
     st = check_mat(x, slots, scales, y);
     if (st != TERN_OK) return st;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const int64_t min_m = g_opt.gemm_min_m > 0 ? g_opt.gemm_min_m : kTensorCoreMinM;
+    const bool tensor = (g_opt.gemm_path == 2) || (g_opt.gemm_path != 1 && M > 8 && M >= min_m);
+    if (tensor) return launch_gemm_tc(mat(x, slots, scales, y, N, K), static_cast<int>(M), s);
     // Bandwidth kernel, eight token rows per launch (weights re-read per chunk).
     for (int64_t m0 = 0; m0 < M; m0 += 8) {
         const int mc = static_cast<int>(M - m0 < 8 ? M - m0 : 8);
         MatDesc d = mat(x + m0 * K, slots, scales, y + m0 * N, N, K);
-        st = launch_gemv_mma(&d, 1, mc, s);
+        st = (g_opt.gemv_variant == 1) ? launch_gemv_mma(&d, 1, mc, s) : launch_gemv_tma(&d, 1, mc, s);
         if (st != TERN_OK) return st;
     }
     return TERN_OK;
@@ -215,17 +254,44 @@ tern_status tern_gemv_grouped(const tern_gemv_desc *descs, int32_t count, int64_
         if (st != TERN_OK) return st;
         d[i] = mat(descs[i].x, descs[i].slots, descs[i].scales, descs[i].y, descs[i].N, descs[i].K);
     }
-    return launch_gemv_mma(d, count, static_cast<int>(M), static_cast<cudaStream_t>(stream));
+    if (g_opt.gemv_variant == 1) return launch_gemv_mma(d, count, static_cast<int>(M), static_cast<cudaStream_t>(stream));
+    return launch_gemv_tma(d, count, static_cast<int>(M), static_cast<cudaStream_t>(stream));
+}
+
+tern_status tern_sync_status(void *stream) {
+    clear_error();
+    cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+    unsigned int v = 0, w = 0;
+    tern_status st = read_gemm_status(true, &v);
+    if (st != TERN_OK) return st;
+    st = read_gemv_status(true, &w);
+    if (st != TERN_OK) return st;
+    if (v == 0) v = w;
+    if (v != 0) return fail(static_cast<tern_status>(v), "a kernel gave up a bounded wait on the device");
+    return TERN_OK;
 }
 
 tern_status tern_set_option(int option, int64_t value) {
     clear_error();
-    if (value < 0 || value > 1024) return fail(TERN_ERR_INVALID_ARG, "option value %lld", static_cast<long long>(value));
+    if (value < 0 || value > 100000000) return fail(TERN_ERR_INVALID_ARG, "option value %lld", static_cast<long long>(value));
     switch (option) {
         case TERN_OPT_GEMV_KSPLIT: g_opt.gemv_ksplit = static_cast<int>(value); return TERN_OK;
         case TERN_OPT_GEMV_CLUSTER: g_opt.gemv_cluster = static_cast<int>(value); return TERN_OK;
         case TERN_OPT_GEMV_CTAS: g_opt.gemv_ctas = static_cast<int>(value); return TERN_OK;
-        case TERN_OPT_GEMM_PATH: g_opt.gemm_path = static_cast<int>(value); return TERN_OK;
+        case TERN_OPT_GEMM_PATH:
+            if (value > 2) return fail(TERN_ERR_INVALID_ARG, "gemm path %lld", static_cast<long long>(value));
+            g_opt.gemm_path = static_cast<int>(value);
+            return TERN_OK;
+        case TERN_OPT_GEMM_MIN_M: g_opt.gemm_min_m = static_cast<int>(value); return TERN_OK;
+        case TERN_OPT_GEMV_VARIANT:
+            if (value > 1) return fail(TERN_ERR_INVALID_ARG, "gemv variant %lld", static_cast<long long>(value));
+            g_opt.gemv_variant = static_cast<int>(value);
+            return TERN_OK;
+        case TERN_OPT_TEST_STALL_US:
+            g_gemm_skip_loads = value > 0 ? 1 : 0;
+            g_gemm_timeout_ns = value > 0 ? static_cast<unsigned long long>(value) * 1000ull : 1000000000ull;
+            return TERN_OK;
         default: return fail(TERN_ERR_INVALID_ARG, "unknown option %d", option);
     }
 }

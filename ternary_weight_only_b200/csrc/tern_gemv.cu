@@ -68,35 +68,6 @@ struct GParams {
     int xs_halves;  // size of the x staging area
 };
 
-// Two fp16 codes -> exact fp16 ternary pair, see the header comment.
-// Pair j of a 32-bit slot word holds weights j (low half) and j+8 (high half).
-__device__ __forceinline__ void unpack_word(uint32_t w, uint32_t (&t)[8]) {
-    constexpr uint32_t kExp = 0x64006400u;  // fp16 1024.0 in both halves
-    const uint32_t w10 = w >> 10;
-    t[0] = hfma2_u32(lop3_and_or(w, 0x00030003u, kExp), 0x3C003C00u, 0xE401E401u);    // *1    -1025
-    t[1] = hfma2_u32(lop3_and_or(w, 0x000C000Cu, kExp), 0x34003400u, 0xDC04DC04u);    // *1/4  -257
-    t[2] = hfma2_u32(lop3_and_or(w, 0x00300030u, kExp), 0x2C002C00u, 0xD410D410u);    // *1/16 -65
-    t[3] = hfma2_u32(lop3_and_or(w, 0x00C000C0u, kExp), 0x24002400u, 0xCC40CC40u);    // *1/64 -17
-    t[4] = hfma2_u32(lop3_and_or(w, 0x03000300u, kExp), 0x1C001C00u, 0xC500C500u);    // *1/256 -5
-    t[5] = hfma2_u32(lop3_and_or(w10, 0x00030003u, kExp), 0x3C003C00u, 0xE401E401u);
-    t[6] = hfma2_u32(lop3_and_or(w10, 0x000C000Cu, kExp), 0x34003400u, 0xDC04DC04u);
-    t[7] = hfma2_u32(lop3_and_or(w10, 0x00300030u, kExp), 0x2C002C00u, 0xD410D410u);
-}
-
-// Index (in halves) of x[m][kl] in the fragment-order staging area.
-// Unit = 4 halves {x[b+2r], x[b+2r+8], x[b+2r+1], x[b+2r+9]} with b the start
-// of a 16-weight word; units are laid out [group][word][m][lane q][r].
-__device__ __forceinline__ int xs_index(int m, int kl, int M) {
-    const int grp = kl >> 7;
-    const int kk = kl & 127;
-    const int q = kk >> 5;
-    const int wi = (kk >> 4) & 1;
-    const int hi = (kk >> 3) & 1;
-    const int j = kk & 7;
-    const int unit = (((grp * 2 + wi) * M + m) * 4 + q) * 4 + (j >> 1);
-    return unit * 4 + (j & 1) * 2 + hi;
-}
-
 struct Item {
     uint2 a, b;          // slot bytes of rows g and g+8 for one scale group
     uint32_t sa, sb;     // their fp16 scales (low 16 bits)

@@ -1,6 +1,7 @@
 // Internal declarations shared by the CUDA sources of libtern (not installed).
 #pragma once
 
+#include <cuda.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -31,6 +32,8 @@ struct Options {
     int gemv_cluster = 0;
     int gemv_ctas = 0;
     int gemm_path = 0;
+    int gemm_min_m = 0;
+    int gemv_variant = 0;
 };
 extern Options g_opt;
 
@@ -48,10 +51,69 @@ struct MatDesc {
     __half *y;
     int N, K;
 };
-// Bandwidth-bound product for M in [1,8] over `count` matrices in one launch.
+// Bandwidth-bound product for M in [1,8] over `count` matrices in one launch:
+// TMA-staged kernel (default) and the register-ring kernel (variant 1).
+tern_status launch_gemv_tma(const MatDesc *d, int count, int M, cudaStream_t stream);
 tern_status launch_gemv_mma(const MatDesc *d, int count, int M, cudaStream_t stream);
+// 2-D tiled tensor map (row-major: `inner` contiguous elements per row, `outer`
+// rows `row_bytes` apart) for TMA loads of `box_inner` x `box_outer` boxes.
+tern_status encode_tiled_2d(CUtensorMap *map, CUtensorMapDataType dt, const void *base, uint64_t inner,
+                            uint64_t outer, uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer,
+                            CUtensorMapSwizzle swizzle);
+// Tensor-core prefill product (any M; meant for large M).
+tern_status launch_gemm_tc(const MatDesc &d, int M, cudaStream_t stream);
+// Device-side status words written by bounded waits that gave up (one per
+// kernel source file; read and optionally cleared).
+tern_status read_gemm_status(bool reset, unsigned int *out);
+tern_status read_gemv_status(bool reset, unsigned int *out);
+extern unsigned long long g_gemm_timeout_ns;
+extern int g_gemm_skip_loads;
 
 // ---- device helpers -------------------------------------------------------
+__device__ __forceinline__ uint32_t smem_u32(const void *p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ unsigned long long globaltimer() {
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint64_t *bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+                 : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+
+__device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, int c0, int c1, uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
+        ::"r"(smem_u32(dst)), "l"(map), "r"(c0), "r"(c1), "r"(smem_u32(bar))
+        : "memory");
+}
+
+__device__ __forceinline__ void named_bar_sync(int id, int count) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
 __device__ __forceinline__ uint32_t lop3_and_or(uint32_t a, uint32_t b, uint32_t c) {
     // (a & b) | c
     uint32_t d;
@@ -102,8 +164,42 @@ __device__ __forceinline__ float4 ld_shared_cluster_f4(uint32_t addr) {
     return v;
 }
 
-__device__ __forceinline__ uint32_t smem_u32(const void *p) {
-    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+
+// Two fp16 codes -> exact fp16 ternary pair.  One LOP3 places the 2-bit code c
+// of two weights into the mantissas of an fp16 pair whose exponent field makes
+// each half 1024 + c*4^j (j = bit pair inside the half); one HFMA2 with the
+// constants (4^-j, -(1024*4^-j + 1)) gives c - 1 = t exactly, because every
+// intermediate is an exactly representable fp16 value.  Pair j of a 32-bit
+// slot word holds weights j (low half) and j+8 (high half).  Code 3 (invalid)
+// gives 2, a finite value.
+__device__ __forceinline__ void unpack_word(uint32_t w, uint32_t (&t)[8]) {
+    constexpr uint32_t kExp = 0x64006400u;  // fp16 1024.0 in both halves
+    const uint32_t w10 = w >> 10;
+    t[0] = hfma2_u32(lop3_and_or(w, 0x00030003u, kExp), 0x3C003C00u, 0xE401E401u);  // *1     -1025
+    t[1] = hfma2_u32(lop3_and_or(w, 0x000C000Cu, kExp), 0x34003400u, 0xDC04DC04u);  // *1/4   -257
+    t[2] = hfma2_u32(lop3_and_or(w, 0x00300030u, kExp), 0x2C002C00u, 0xD410D410u);  // *1/16  -65
+    t[3] = hfma2_u32(lop3_and_or(w, 0x00C000C0u, kExp), 0x24002400u, 0xCC40CC40u);  // *1/64  -17
+    t[4] = hfma2_u32(lop3_and_or(w, 0x03000300u, kExp), 0x1C001C00u, 0xC500C500u);  // *1/256 -5
+    t[5] = hfma2_u32(lop3_and_or(w10, 0x00030003u, kExp), 0x3C003C00u, 0xE401E401u);
+    t[6] = hfma2_u32(lop3_and_or(w10, 0x000C000Cu, kExp), 0x34003400u, 0xDC04DC04u);
+    t[7] = hfma2_u32(lop3_and_or(w10, 0x00300030u, kExp), 0x2C002C00u, 0xD410D410u);
+}
+
+// Index (in halves) of x[m][kl] in the "fragment order" staging area of the
+// bandwidth kernels.  Unit = 4 halves {x[b+2r], x[b+2r+8], x[b+2r+1], x[b+2r+9]}
+// with b the start of a 16-weight slot word, so that unit r is exactly the B
+// fragment of the mma that consumes pairs 2r and 2r+1 of that word; units are
+// laid out [group][word][m][lane q][r] so that a warp's fragment loads are
+// contiguous (no bank conflicts).
+__device__ __forceinline__ int xs_index(int m, int kl, int M) {
+    const int grp = kl >> 7;
+    const int kk = kl & 127;
+    const int q = kk >> 5;
+    const int wi = (kk >> 4) & 1;
+    const int hi = (kk >> 3) & 1;
+    const int j = kk & 7;
+    const int unit = (((grp * 2 + wi) * M + m) * 4 + q) * 4 + (j >> 1);
+    return unit * 4 + (j & 1) * 2 + hi;
 }
 
 __device__ __forceinline__ uint2 ldg_nc_u2(const void *p) {

@@ -33,6 +33,9 @@ TERN_OPT_GEMV_KSPLIT = 1
 TERN_OPT_GEMV_CLUSTER = 2
 TERN_OPT_GEMV_CTAS = 3
 TERN_OPT_GEMM_PATH = 4
+TERN_OPT_GEMM_MIN_M = 5
+TERN_OPT_TEST_STALL_US = 6
+TERN_OPT_GEMV_VARIANT = 7
 TERN_MAX_GROUP = 16
 
 _i64, _vp, _sz, _i32, _int = ctypes.c_int64, ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int32, ctypes.c_int
@@ -55,6 +58,7 @@ _SIGS = {
     "tern_gemm": ([_vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp, _sz, _vp], _int),
     "tern_gemv_grouped": ([ctypes.POINTER(tern_gemv_desc), _i32, _i64, _vp, _sz, _vp], _int),
     "tern_set_option": ([_int, _i64], _int),
+    "tern_sync_status": ([_vp], _int),
 }
 for _name, (_args, _res) in _SIGS.items():
     _f = getattr(_L, _name)
@@ -112,6 +116,11 @@ def tern_workspace_bytes(M: int, N: int, K: int) -> int:
 
 def tern_set_option(option: int, value: int):
     _check(_L.tern_set_option(option, value), "tern_set_option")
+
+
+def tern_sync_status(stream=None):
+    """Wait for the stream; raise TernError if a kernel gave up a bounded wait."""
+    _check(_L.tern_sync_status(_stream(stream)), "tern_sync_status")
 
 
 def tern_pack_g128(codes: torch.Tensor, scales: torch.Tensor, slots_out: Optional[torch.Tensor] = None,

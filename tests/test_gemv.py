@@ -20,7 +20,7 @@ def T():
     build.build()
     from ternary_weight_only_b200 import tern
     yield tern
-    for o in (1, 2, 3, 4):
+    for o in (1, 2, 3, 4, 5, 6, 7):
         tern.tern_set_option(o, 0)
 
 
@@ -72,20 +72,55 @@ def test_ragged(T, orc, M, K, N):
     run_case(T, orc, x, codes, scales, f"M={M} K={K} N={N}")
 
 
+@pytest.mark.parametrize("variant", [0, 1])
 @pytest.mark.parametrize("ks", [1, 2, 4, 8])
 @pytest.mark.parametrize("cl", [1, 2, 4])
-def test_split_options(T, orc, ks, cl):
+def test_split_options(T, orc, ks, cl, variant):
+    """Every forced k split inside the CTA and across a cluster, both kernels."""
     from ternary_weight_only_b200 import synth
-    x, codes, scales = synth.case(3, 2048, 200, seed=ks * 10 + cl, codes="sparse")
+    x, codes, scales = synth.case(3, 17408, 200, seed=ks * 10 + cl, codes="sparse")
+    T.tern_set_option(T.TERN_OPT_GEMV_VARIANT, variant)
     T.tern_set_option(T.TERN_OPT_GEMV_KSPLIT, ks)
     T.tern_set_option(T.TERN_OPT_GEMV_CLUSTER, cl)
     try:
-        run_case(T, orc, x, codes, scales, f"ks={ks} cl={cl}")
-        x1, c1, s1 = synth.case(1, 5120, 1024, seed=ks * 10 + cl + 1, codes="sparse")
-        run_case(T, orc, x1, c1, s1, f"M=1 ks={ks} cl={cl}")
+        run_case(T, orc, x, codes, scales, f"v{variant} ks={ks} cl={cl}")
+        x1, c1, s1 = synth.case(1, 17408, 1040, seed=ks * 10 + cl + 1, codes="sparse")
+        run_case(T, orc, x1, c1, s1, f"M=1 v{variant} ks={ks} cl={cl}")
     finally:
         T.tern_set_option(T.TERN_OPT_GEMV_KSPLIT, 0)
         T.tern_set_option(T.TERN_OPT_GEMV_CLUSTER, 0)
+        T.tern_set_option(T.TERN_OPT_GEMV_VARIANT, 0)
+
+
+@pytest.mark.parametrize("M,K,N", [(1, 5120, 1024), (8, 384, 33), (5, 640, 100), (4, 25600, 64)])
+def test_register_ring_variant(T, orc, M, K, N):
+    from ternary_weight_only_b200 import synth
+    x, codes, scales = synth.case(M, K, N, seed=M + K + N + 5, codes="sparse", outlier_p=0.01)
+    T.tern_set_option(T.TERN_OPT_GEMV_VARIANT, 1)
+    try:
+        run_case(T, orc, x, codes, scales, f"ring M={M} K={K} N={N}")
+    finally:
+        T.tern_set_option(T.TERN_OPT_GEMV_VARIANT, 0)
+
+
+def test_timeout_path_reports_and_recovers(T, orc):
+    """A TMA wait that can never complete (nothing is loaded) gives up after its
+    limit; the status reaches the host and the context stays usable."""
+    from ternary_weight_only_b200 import synth
+    x, codes, scales = synth.case(2, 2048, 700, seed=78, codes="sparse")
+    xn, cn, sn = np_inputs(x, codes, scales)
+    slots, sc, _, _ = orc.pack(cn, sn)
+    xd, sd, scd = x.cuda(), torch.from_numpy(slots).cuda(), scales.cuda()
+    T.tern_set_option(T.TERN_OPT_TEST_STALL_US, 2000)
+    try:
+        T.tern_gemm(xd, sd, scd)
+        with pytest.raises(T.TernError) as ei:
+            T.tern_sync_status()
+        assert ei.value.status == T.TERN_ERR_TIMEOUT
+    finally:
+        T.tern_set_option(T.TERN_OPT_TEST_STALL_US, 0)
+    T.tern_sync_status()
+    run_case(T, orc, x, codes, scales, "after timeout")
 
 
 def test_grid_cap(T, orc):
