@@ -262,6 +262,30 @@ def proj_rows(T, model, peak_gbs, l2_bytes):
     return out
 
 
+def prefill_rows(T, peak_tf):
+    """Prefill GEMM (tensor cores) at M = 2048 and 8192 for both shapes:
+    TFLOP/s = 2*M*N*K / device time, against the measured dense fp16 peak."""
+    out = {}
+    s = torch.cuda.Stream()
+    for ci, (K, N) in enumerate(synth.PREFILL):
+        g = synth.gen(3000 + 10 * ci, "cuda")
+        codes = synth.codes_uniform(N, K, g, device="cuda")
+        scales = synth.scales_uniform(N, K, g, device="cuda")
+        slots, sc = T.tern_pack_g128(codes, scales)
+        del codes
+        for M in synth.PREFILL_M:
+            x = synth.activations(M, K, g, device="cuda")
+            y = torch.empty(M, N, dtype=torch.float16, device="cuda")
+            ms = graph_time([lambda: T.tern_gemm(x, slots, sc, y)], s, reps=5)
+            tf = 2.0 * M * N * K / (ms * 1e-3) / 1e12
+            out[f"prefill_K{K}_N{N}_M{M}"] = {"ms": round(ms, 4), "TFLOPs": round(tf, 1),
+                                              "frac": round(tf / peak_tf, 4)}
+            del x, y
+        del slots, sc
+    torch.cuda.empty_cache()
+    return out
+
+
 def graph_time(fns, stream, reps=3, flush=0):
     """Average device time per call of fns (captured once into a graph, the
     graph replayed `reps` times; with `flush` > 0 an L2-sized buffer is
@@ -293,13 +317,41 @@ def graph_time(fns, stream, reps=3, flush=0):
 
 
 # --------------------------------------------------------------- oracle ---
+_ORACLE_JOBS = None
+
+
 def oracle_sample(target_s: float = 12.0, max_s: float = 30.0):
-    """Time the fp64 oracle on a bounded sample of the decode step: every
-    projection of layer 0 and a slice of the head, inputs drawn on the host
-    and packed by the oracle itself.  Returns (GB/s, threads, description)."""
+    """Time the fp64 oracle on a bounded sample of the decode step: the
+    projections of one decode layer and a slice of the head, inputs drawn on the
+    host and packed by the oracle itself (packing untimed), run in passes until
+    `target_s` of oracle time (at least one matrix, at most `max_s`).
+    Returns (GB/s, threads, description)."""
+    global _ORACLE_JOBS
     import oracle
     orc = oracle.load()
     threads = os.cpu_count() or 1
+    if _ORACLE_JOBS is None:
+        _ORACLE_JOBS = _oracle_jobs(orc)
+    packed = _ORACLE_JOBS
+    done_bytes, t_total, mats = 0, 0.0, 0
+    while t_total < target_s:
+        for name, K, N, xb, sl, sc in packed:
+            t0 = time.perf_counter()
+            orc.matmul(xb, sl, sc, threads=threads)
+            t_total += time.perf_counter() - t0
+            done_bytes += wbytes(K, N) + 2 * K + 2 * N
+            mats += 1
+            if t_total >= target_s or t_total > max_s:
+                break
+        if t_total > max_s:
+            break
+    used = orc.threads_used
+    desc = (f"{mats} matrix products from one decode layer (q,k,v,o,gate,up,down, M=1) and 16384 rows "
+            f"of the 5120x151936 head, in that order, fp64 oracle, {used} OpenMP threads, {t_total:.1f} s")
+    return done_bytes / t_total / 1e9, used, desc
+
+
+def _oracle_jobs(orc):
     jobs = []
     for i, (name, K, N) in enumerate(synth.LAYER_PROJ):
         x, codes, scales = synth.case(1, K, N, seed=6000 + i, codes="sparse")
@@ -312,20 +364,7 @@ def oracle_sample(target_s: float = 12.0, max_s: float = 30.0):
         xb = x.view(torch.int16).numpy().view(np.uint16)
         sl, sc, _, _ = orc.pack(codes.numpy(), scales.view(torch.int16).numpy().view(np.uint16))
         packed.append((name, K, N, xb, sl, sc))
-    done_bytes, t_total, passes = 0, 0.0, 0
-    while t_total < target_s:
-        for name, K, N, xb, sl, sc in packed:
-            t0 = time.perf_counter()
-            orc.matmul(xb, sl, sc, threads=threads)
-            t_total += time.perf_counter() - t0
-            done_bytes += wbytes(K, N) + 2 * K + 2 * N
-        passes += 1
-        if t_total > max_s:
-            break
-    used = orc.threads_used
-    desc = (f"{passes} pass(es) over one decode layer (q,k,v,o,gate,up,down, M=1) plus 16384 "
-            f"rows of the 5120x151936 head, fp64 oracle, {used} OpenMP threads, {t_total:.1f} s")
-    return done_bytes / t_total / 1e9, used, desc
+    return packed
 
 
 def run_reference(args):
@@ -335,8 +374,9 @@ def run_reference(args):
     wb, xin, yout = step_bytes()
     total = wb + xin + yout
     vals = []
+    per_step = max(0.05, min(2.0, 150.0 / (args.warmup + args.steps)))  # whole run ~<= 3 min
     for i in range(args.warmup + args.steps):
-        gbs, used, desc = oracle_sample(target_s=2.0, max_s=6.0)
+        gbs, used, desc = oracle_sample(target_s=per_step, max_s=3 * per_step)
         if i >= args.warmup:
             vals.append(gbs)
     gbs = statistics.mean(vals)
@@ -379,6 +419,8 @@ def run_profile(args):
     """Small case for ncu captures: a few layers' grouped launches, eager."""
     torch.cuda.set_device(0)
     from ternary_weight_only_b200 import tern as T
+    if args.gemv_variant:
+        T.tern_set_option(T.TERN_OPT_GEMV_VARIANT, args.gemv_variant)
     model = DecodeModel(T, n_layers=args.profile_layers)
     for _ in range(3):
         for grp in model.groups:
@@ -449,6 +491,7 @@ def run_tern(args):
     rows = None
     if rank == 0 and not args.no_rows:
         rows = proj_rows(T, model, peak_gbs, l2)
+        rows.update(prefill_rows(T, peak_tf))
 
     cpu = None
     if rank == 0 and ws == 1 and not args.no_cpu:
@@ -505,6 +548,8 @@ def main():
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
     ap.add_argument("--profile-layers", type=int, default=0,
                     help="profiling case: build this many layers, run their grouped launches 3x, exit")
+    ap.add_argument("--gemv-variant", type=int, default=0,
+                    help="profiling case only: bandwidth kernel variant (0 TMA-staged, 1 register ring)")
     args = ap.parse_args()
     if args.profile_layers > 0:
         return run_profile(args)

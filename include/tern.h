@@ -182,7 +182,9 @@ tern_status tern_sync_status(void *stream);
  *                          the TMA kernel may lower it for short K)
  *   TERN_OPT_GEMV_CLUSTER  CTAs sharing one tile along K through a thread
  *                          block cluster and distributed shared memory (1,2,4,8)
- *   TERN_OPT_GEMV_CTAS     cap on resident CTAs per SM used for the grid
+ *   TERN_OPT_GEMV_CTAS     cap on resident CTAs per SM used for the grid; for
+ *                          the TMA-staged kernel 3 also selects the build with
+ *                          the smaller register budget (default: 2 per SM)
  *   TERN_OPT_GEMM_PATH     1 = force the bandwidth kernel (M<=8 chunks),
  *                          2 = force the tensor-core kernel
  *   TERN_OPT_GEMM_MIN_M    smallest M (> 8) sent to the tensor-core kernel

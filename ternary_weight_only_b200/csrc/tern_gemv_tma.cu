@@ -12,11 +12,11 @@
 //    slots, one TMA box from a 2-D tensor map over the slot matrix, written
 //    into shared memory with the 128-byte swizzle so that the lanes' 8-byte
 //    fragment loads hit distinct banks.
-//  * Every warp runs its own 4-stage ring of slices (lane 0 issues the TMA
-//    loads and refills a stage as soon as the warp has read it), so a 2-CTA
-//    SM keeps 128 KB of weight loads in flight without spending registers on
-//    them; the per-row fp16 scales ride along in a 2-register-per-lane ring of
-//    plain loads issued four slices ahead.
+//  * Every warp runs its own 3-stage ring of slices (lane 0 issues the TMA
+//    loads and refills a stage as soon as the warp has read it), so an SM
+//    with 2-3 CTAs keeps 96-144 KB of weight loads in flight without spending
+//    registers on them; the per-row fp16 scales ride along in a
+//    2-register-per-lane ring of plain loads issued three slices ahead.
 //  * Unpack: one LOP3 + one HFMA2 per pair of weights gives exact fp16 t; the
 //    multiply-accumulate runs on the tensor cores (mma.sync m16n8k16, fp32
 //    accumulate) with the 16 weight rows as the A operand straight from
@@ -47,7 +47,7 @@ namespace {
 
 constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
-constexpr int kNS = 4;             // stages per warp
+constexpr int kNS = 3;             // stages per warp
 constexpr int kSliceRows = 16;
 constexpr int kSliceBytes = 128;   // per row: 512 weights
 constexpr int kSliceGroups = 4;    // scale groups per slice
@@ -86,7 +86,15 @@ __device__ __forceinline__ bool wait_bounded(uint64_t *bar, uint32_t parity, uns
     return true;
 }
 
-__global__ void __launch_bounds__(kThreads, 2) gemv_tma_kernel(const __grid_constant__ TParams p) {
+// Tile row handled as mma row g (and g + 8): even rows for g < 4, odd rows for
+// g >= 4.  With the 128-byte swizzle this makes the 16 lanes of each half-warp
+// read 16 distinct 8-byte bank pairs (four rows 2 apart cover all eight swizzle
+// phases of the two 16-byte chunks of a scale group).
+__device__ __forceinline__ int tile_row(int g) { return g < 4 ? 2 * g : 2 * g - 7; }
+
+// MINB = resident CTAs per SM the register budget is sized for (2 or 3).
+template <int MT, int MINB>
+__global__ void __launch_bounds__(kThreads, MINB) gemv_tma_kernel(const __grid_constant__ TParams p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *stages = smem;                                                   // [warp][stage] 2 KB each
@@ -98,6 +106,7 @@ __global__ void __launch_bounds__(kThreads, 2) gemv_tma_kernel(const __grid_cons
     const int S = p.S, M = p.M;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int g = lane >> 2, q = lane & 3;
+    const int row = tile_row(g);
     const int cl = blockIdx.x / S;
     const int rank = (S > 1) ? static_cast<int>(cluster_ctarank()) : 0;
 
@@ -131,32 +140,29 @@ __global__ void __launch_bounds__(kThreads, 2) gemv_tma_kernel(const __grid_cons
     }
     __syncwarp();
 
-    // Issue stream (lane 0 only issues TMA; every lane tracks it for scales).
-    int is_it = 0, is_b = 0;  // slice (iteration, k block) of the next issue
-    uint32_t n_issued = 0;    // 8 bits per stage: loads issued into it (lane 0)
-    auto issue_next = [&](int stage) {
+    // Issue stream: slice (is_it, is_b) goes next.  Lane 0 issues the TMA;
+    // every lane loads its two scales of that slice (rows row and row + 8,
+    // group q of the slice; 0 beyond K so that padded groups contribute 0).
+    int is_it = 0, is_b = 0;
+    uint32_t n_issued = 0;  // 8 bits per stage: loads issued into it (lane 0)
+    const unsigned short *sc = reinterpret_cast<const unsigned short *>(d.scales);
+    auto issue_next = [&](int stage, uint32_t &sa, uint32_t &sb) {
         const int tile = tile0 + is_it * stride;
-        if (is_it < nit && tile < d.ntile && lane == 0 && !p.skip_loads) {
+        const bool ok = is_it < nit && tile < d.ntile;
+        if (ok && lane == 0 && !p.skip_loads) {
             mbar_expect_tx(&wfull[stage], kStageBytes);
             tma_load_2d(wst + stage * kStageBytes, &d.map, (b0 + is_b) * kSliceBytes, tile * kSliceRows,
                         &wfull[stage]);
             n_issued += 1u << (8 * stage);
         }
-    };
-    // Scale ring: lane (g,q) holds the scales of rows g and g+8 for group q of a slice.
-    const unsigned short *sc = reinterpret_cast<const unsigned short *>(d.scales);
-    auto load_scales = [&](uint32_t &sa, uint32_t &sb) {
-        const int tile = tile0 + is_it * stride;
         const int grp = (b0 + is_b) * kSliceGroups + q;
         sa = sb = 0;
-        if (is_it < nit && tile < d.ntile && grp < G) {
-            const int r0 = min(tile * kSliceRows + g, N - 1);
-            const int r1 = min(tile * kSliceRows + g + 8, N - 1);
+        if (ok && grp < G) {
+            const int r0 = min(tile * kSliceRows + row, N - 1);
+            const int r1 = min(tile * kSliceRows + row + 8, N - 1);
             sa = __ldg(sc + static_cast<size_t>(r0) * G + grp);
             sb = __ldg(sc + static_cast<size_t>(r1) * G + grp);
         }
-    };
-    auto advance_issue = [&]() {
         if (++is_b == nb) {
             is_b = 0;
             is_it++;
@@ -165,39 +171,40 @@ __global__ void __launch_bounds__(kThreads, 2) gemv_tma_kernel(const __grid_cons
 
     uint32_t sra[kNS], srb[kNS];
 #pragma unroll
-    for (int s = 0; s < kNS; s++) {
-        issue_next(s);
-        load_scales(sra[s], srb[s]);
-        advance_issue();
-    }
+    for (int s = 0; s < kNS; s++) issue_next(s, sra[s], srb[s]);
 
-    // Stage this CTA's K range of x in fragment order (overlaps the first loads).
+    // Stage this CTA's K range of x in fragment order (overlaps the first
+    // loads); groups past K are zero so that padded slices contribute 0.
+    const int gA = bA * kSliceGroups;
     {
-        const int gA = bA * kSliceGroups;
-        const int gB = min(bB * kSliceGroups, G);
-        const int KC = (gB - gA) * kGroup;
-        const int per_m = KC / 8;
+        const int gB = bB * kSliceGroups;
+        const int per_m = (gB - gA) * (kGroup / 8);
         for (int idx = threadIdx.x; idx < M * per_m; idx += kThreads) {
             const int m = idx / per_m, c8 = idx - m * per_m;
-            const uint4 v = *reinterpret_cast<const uint4 *>(d.x + static_cast<size_t>(m) * K +
-                                                             static_cast<size_t>(gA) * kGroup + c8 * 8);
+            const int k = gA * kGroup + c8 * 8;
+            uint4 v = make_uint4(0, 0, 0, 0);
+            if (k < K) v = *reinterpret_cast<const uint4 *>(d.x + static_cast<size_t>(m) * K + k);
             const __half *hv = reinterpret_cast<const __half *>(&v);
 #pragma unroll
-            for (int e = 0; e < 8; e++) xs[xs_index(m, c8 * 8 + e, M)] = hv[e];
+            for (int e = 0; e < 8; e++) xs[xs_index(m, c8 * 8 + e, MT)] = hv[e];
         }
     }
     __syncthreads();
 
-    // Per-lane swizzled offsets of its 8-byte fragment for group j of a slice
-    // (row g; row g+8 is 1024 bytes further and has the same swizzle phase).
+    // Per-lane swizzled byte offsets of its 8-byte fragment of group j (row
+    // `row`; row + 8 is 1024 bytes further with the same swizzle phase).
     uint32_t off[kSliceGroups];
 #pragma unroll
     for (int j = 0; j < kSliceGroups; j++)
-        off[j] = g * kSliceBytes + (((2 * j + (q >> 1)) ^ g) << 4) + (q & 1) * 8;
+        off[j] = row * kSliceBytes + (((2 * j + (q >> 1)) ^ (row & 7)) << 4) + (q & 1) * 8;
 
-    const bool has_x = g < M;
-    const int xw_stride = M * 64;  // halves between word 0 and word 1 of a group
-    const int gA_x = bA * kSliceGroups;
+    // B column g holds token min(g, M-1): columns past M repeat the last token
+    // (never stored), so every lane loads unconditionally.
+    const int gx = g < M ? g : M - 1;
+    const __half *xlane = xs + (gx * 4 + q) * 16;  // fragment of word 0, group 0
+    constexpr int kGroupHalves = 2 * MT * 64;    // x halves per scale group
+    constexpr int kWordHalves = MT * 64;         // word 1 of a group is this far
+    const int shfl_base = lane & ~3;
     float acc[4] = {0.f, 0.f, 0.f, 0.f};
     int c_it = 0, c_b = 0, buf = 0;
     bool dead = false;  // this warp gave up a wait: no more loads, computes or stores
@@ -216,56 +223,48 @@ __global__ void __launch_bounds__(kThreads, 2) gemv_tma_kernel(const __grid_cons
                 }
                 if (live && !dead) {
                     const uint8_t *st = wst + u * kStageBytes;
-                    const int gbase = (b0 + c_b) * kSliceGroups;
+                    const __half *xg = xlane + ((b0 + c_b) * kSliceGroups - gA) * kGroupHalves;
+                    const float fa = __half2float(__ushort_as_half(static_cast<unsigned short>(sra[u])));
+                    const float fb2 = __half2float(__ushort_as_half(static_cast<unsigned short>(srb[u])));
 #pragma unroll
                     for (int j = 0; j < kSliceGroups; j++) {
-                        if (gbase + j < G) {
-                            const uint2 a = *reinterpret_cast<const uint2 *>(st + off[j]);
-                            const uint2 b = *reinterpret_cast<const uint2 *>(st + off[j] + 1024);
-                            const __half *xb = xs + (((gbase + j - gA_x) * 2 * M + g) * 4 + q) * 16;
-                            uint4 x0 = make_uint4(0, 0, 0, 0), x1 = x0, x2 = x0, x3 = x0;
-                            if (has_x) {
-                                x0 = *reinterpret_cast<const uint4 *>(xb);
-                                x1 = *reinterpret_cast<const uint4 *>(xb + 8);
-                                x2 = *reinterpret_cast<const uint4 *>(xb + xw_stride);
-                                x3 = *reinterpret_cast<const uint4 *>(xb + xw_stride + 8);
-                            }
-                            float c0[4] = {0.f, 0.f, 0.f, 0.f}, c1[4] = {0.f, 0.f, 0.f, 0.f};
-                            {
-                                uint32_t ta[8], tb[8];
-                                unpack_word(a.x, ta);
-                                unpack_word(b.x, tb);
-                                mma_16816(c0, ta[0], tb[0], ta[1], tb[1], x0.x, x0.y);
-                                mma_16816(c0, ta[2], tb[2], ta[3], tb[3], x0.z, x0.w);
-                                mma_16816(c0, ta[4], tb[4], ta[5], tb[5], x1.x, x1.y);
-                                mma_16816(c0, ta[6], tb[6], ta[7], tb[7], x1.z, x1.w);
-                            }
-                            {
-                                uint32_t ta[8], tb[8];
-                                unpack_word(a.y, ta);
-                                unpack_word(b.y, tb);
-                                mma_16816(c1, ta[0], tb[0], ta[1], tb[1], x2.x, x2.y);
-                                mma_16816(c1, ta[2], tb[2], ta[3], tb[3], x2.z, x2.w);
-                                mma_16816(c1, ta[4], tb[4], ta[5], tb[5], x3.x, x3.y);
-                                mma_16816(c1, ta[6], tb[6], ta[7], tb[7], x3.z, x3.w);
-                            }
-                            const int src = (lane & ~3) | j;
-                            const uint32_t ha = __shfl_sync(0xffffffffu, sra[u], src);
-                            const uint32_t hb = __shfl_sync(0xffffffffu, srb[u], src);
-                            const float sa = __half2float(__ushort_as_half(static_cast<unsigned short>(ha)));
-                            const float sb = __half2float(__ushort_as_half(static_cast<unsigned short>(hb)));
-                            acc[0] = fmaf(sa, c0[0] + c1[0], acc[0]);
-                            acc[1] = fmaf(sa, c0[1] + c1[1], acc[1]);
-                            acc[2] = fmaf(sb, c0[2] + c1[2], acc[2]);
-                            acc[3] = fmaf(sb, c0[3] + c1[3], acc[3]);
+                        const uint2 a = *reinterpret_cast<const uint2 *>(st + off[j]);
+                        const uint2 b = *reinterpret_cast<const uint2 *>(st + off[j] + 1024);
+                        const __half *xb = xg + j * kGroupHalves;
+                        const uint4 x0 = *reinterpret_cast<const uint4 *>(xb);
+                        const uint4 x1 = *reinterpret_cast<const uint4 *>(xb + 8);
+                        const uint4 x2 = *reinterpret_cast<const uint4 *>(xb + kWordHalves);
+                        const uint4 x3 = *reinterpret_cast<const uint4 *>(xb + kWordHalves + 8);
+                        float c[4];
+                        {
+                            uint32_t ta[8], tb[8];
+                            unpack_word(a.x, ta);
+                            unpack_word(b.x, tb);
+                            mma_16816_zc(c, ta[0], tb[0], ta[1], tb[1], x0.x, x0.y);
+                            mma_16816(c, ta[2], tb[2], ta[3], tb[3], x0.z, x0.w);
+                            mma_16816(c, ta[4], tb[4], ta[5], tb[5], x1.x, x1.y);
+                            mma_16816(c, ta[6], tb[6], ta[7], tb[7], x1.z, x1.w);
                         }
+                        {
+                            uint32_t ta[8], tb[8];
+                            unpack_word(a.y, ta);
+                            unpack_word(b.y, tb);
+                            mma_16816(c, ta[0], tb[0], ta[1], tb[1], x2.x, x2.y);
+                            mma_16816(c, ta[2], tb[2], ta[3], tb[3], x2.z, x2.w);
+                            mma_16816(c, ta[4], tb[4], ta[5], tb[5], x3.x, x3.y);
+                            mma_16816(c, ta[6], tb[6], ta[7], tb[7], x3.z, x3.w);
+                        }
+                        const float sa = __shfl_sync(0xffffffffu, fa, shfl_base | j);
+                        const float sb = __shfl_sync(0xffffffffu, fb2, shfl_base | j);
+                        acc[0] = fmaf(sa, c[0], acc[0]);
+                        acc[1] = fmaf(sa, c[1], acc[1]);
+                        acc[2] = fmaf(sb, c[2], acc[2]);
+                        acc[3] = fmaf(sb, c[3], acc[3]);
                     }
                 }
                 // Stage u is free again: refill it with the slice kNS ahead.
                 __syncwarp();
-                if (!dead) issue_next(u);
-                load_scales(sra[u], srb[u]);
-                advance_issue();
+                if (!dead) issue_next(u, sra[u], srb[u]);
                 if (++c_b == nb) {
                     // ---- end of this warp's share of a tile: reduce and store ----
                     float v[4] = {acc[0], acc[1], acc[2], acc[3]};
@@ -303,7 +302,7 @@ __global__ void __launch_bounds__(kThreads, 2) gemv_tma_kernel(const __grid_cons
                         buf ^= 1;
                     }
                     if (writer && live && !dead) {
-                        const int n0 = tile * kSliceRows + g, n1 = n0 + 8;
+                        const int n0 = tile * kSliceRows + row, n1 = n0 + 8;
                         const int m0 = 2 * q, m1 = 2 * q + 1;
                         if (m0 < M) {
                             if (n0 < N) d.y[static_cast<size_t>(m0) * N + n0] = __float2half_rn(v[0]);
@@ -333,8 +332,8 @@ __global__ void __launch_bounds__(kThreads, 2) gemv_tma_kernel(const __grid_cons
     if (S > 1) cluster_sync_all();
 }
 
-bool g_attr_done[64];
-int g_occ[64][256];
+bool g_attr_done[64][8];
+int g_occ[64][8][256];
 
 // Per-CTA work (slices per warp) of matrix i with P warps per tile and c clusters.
 long long cta_work(int ntile, int nb_cta, int P, long long c) {
@@ -360,8 +359,15 @@ tern_status launch_gemv_tma(const MatDesc *md, int count, int M, cudaStream_t st
     }
     // Cluster split along K only when x would not fit next to the stages.
     int S = 1;
+    const int MT = M == 1 ? 1 : (M == 2 ? 2 : (M <= 4 ? 4 : 8));
+    // Register budget: 2 CTAs per SM (128 registers) unless the knob asks for 3.
+    const bool two = g_opt.gemv_ctas != 3;
+    using KernFn = void (*)(TParams);
+    KernFn kern;
+    if (two) kern = MT == 1 ? gemv_tma_kernel<1, 2> : (MT == 2 ? gemv_tma_kernel<2, 2> : (MT == 4 ? gemv_tma_kernel<4, 2> : gemv_tma_kernel<8, 2>));
+    else kern = MT == 1 ? gemv_tma_kernel<1, 3> : (MT == 2 ? gemv_tma_kernel<2, 3> : (MT == 4 ? gemv_tma_kernel<4, 3> : gemv_tma_kernel<8, 3>));
     auto xs_bytes = [&](int s) {
-        return static_cast<long long>(M) * ((bmax + s - 1) / s) * kSliceGroups * kGroup * 2;
+        return static_cast<long long>(MT) * ((bmax + s - 1) / s) * kSliceGroups * kGroup * 2;
     };
     while (S < 8 && S * 2 <= bmin && xs_bytes(S) > 96 * 1024) S *= 2;
     if (g_opt.gemv_cluster > 0) S = g_opt.gemv_cluster;
@@ -373,18 +379,19 @@ tern_status launch_gemv_tma(const MatDesc *md, int count, int M, cudaStream_t st
                         static_cast<size_t>(xs_halves) * 2 + 2 * kWarps * 32 * 4 * sizeof(float) +
                         (S > 1 ? 2 * kWarps * 32 * 4 * sizeof(float) : 0);
     if (smem > dev.max_smem_optin) return fail(TERN_ERR_SHAPE, "needs %zu B of shared memory", smem);
-    if (!g_attr_done[dev.device]) {
-        cudaError_t e = cudaFuncSetAttribute(gemv_tma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    const int mi = (MT == 1 ? 0 : (MT == 2 ? 1 : (MT == 4 ? 2 : 3))) + (two ? 4 : 0);
+    if (!g_attr_done[dev.device][mi]) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              static_cast<int>(dev.max_smem_optin));
         if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
-        g_attr_done[dev.device] = true;
+        g_attr_done[dev.device][mi] = true;
     }
     const int skb = static_cast<int>((smem + 1023) / 1024);
-    int occ = (skb < 256) ? g_occ[dev.device][skb] : 0;
+    int occ = (skb < 256) ? g_occ[dev.device][mi][skb] : 0;
     if (occ == 0) {
-        cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, gemv_tma_kernel, kThreads, skb * 1024);
+        cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, kThreads, skb * 1024);
         if (e != cudaSuccess) return cuda_fail(e, "occupancy query");
-        if (skb < 256) g_occ[dev.device][skb] = occ;
+        if (skb < 256) g_occ[dev.device][mi][skb] = occ;
     }
     if (occ < 1) return fail(TERN_ERR_SHAPE, "kernel does not fit on an SM (smem %zu)", smem);
     if (g_opt.gemv_ctas > 0) occ = std::min(occ, g_opt.gemv_ctas);
@@ -508,7 +515,7 @@ tern_status launch_gemv_tma(const MatDesc *md, int count, int M, cudaStream_t st
         cfg.attrs = attr;
         cfg.numAttrs = 1;
     }
-    cudaError_t e = cudaLaunchKernelEx(&cfg, gemv_tma_kernel, p);
+    cudaError_t e = cudaLaunchKernelEx(&cfg, kern, p);
     if (e != cudaSuccess) return cuda_fail(e, "gemv kernel launch");
     return TERN_OK;
 }
