@@ -83,9 +83,25 @@ const char *tern_last_error(void);
 size_t tern_slots_bytes(int64_t N, int64_t K);
 size_t tern_scales_bytes(int64_t N, int64_t K);
 
-/* Workspace needed by tern_gemv / tern_gemm / tern_gemv_grouped for this
- * shape.  The current kernels need none and return 0; a caller that passes a
- * workspace anyway is fine.  A non-zero value would be stated here. */
+/*
+ * Workspace.  With TERN_OPT_GEMV_VARIANT = 3 and M <= 4 the bandwidth kernel
+ * splits long rows along K over several warpgroups when the caller passes a
+ * workspace of at least
+ * tern_workspace_bytes(M, N, K) bytes (tern_gemv_grouped_workspace_bytes() for
+ * a grouped call): partial sums go there and the last part of each 16x128-row
+ * tile to finish adds them up in a fixed order, so results do not depend on
+ * scheduling.  Without it (NULL or too small) tiles are not split: the result
+ * is the same, the balance across SMs may be worse.
+ *   - The workspace is device memory owned by the caller, 256-byte aligned,
+ *     and its first 128 KiB (per-tile arrival counters) must be ZERO before
+ *     its first use; every call that completes leaves them zero again, so one
+ *     workspace can serve calls of any shape in turn.  The rest holds partial
+ *     sums and needs no initialisation.  After a call that reported
+ *     TERN_ERR_TIMEOUT, zero the first 128 KiB again.
+ *   - Calls that may run concurrently must not share a workspace.
+ *   - The size depends on the current device's SM count (148 is assumed when
+ *     no device is visible) and is 0 when no split is planned.
+ */
 size_t tern_workspace_bytes(int64_t M, int64_t N, int64_t K);
 
 /*
@@ -121,9 +137,9 @@ tern_status tern_unpack_g128(const uint8_t *slots, int64_t N, int64_t K, int8_t 
  *   slots   uint8 [N][K/4]  (device, read)
  *   scales  fp16 [N][K/128] (device, read)
  *   y       fp16 [N]        (device, written)
- *   workspace / ws_bytes: may be NULL / 0 (see tern_workspace_bytes).
- * Bandwidth-bound: the weights are streamed from HBM once, unpacked in
- * registers and never written back in any other precision.
+ *   workspace / ws_bytes: optional, see tern_workspace_bytes.
+ * Bandwidth-bound: the weights are streamed from HBM once, unpacked on chip
+ * and never written back in any other precision.
  */
 tern_status tern_gemv(const uint16_t *x, const uint8_t *slots, const uint16_t *scales, uint16_t *y,
                       int64_t N, int64_t K, void *workspace, size_t ws_bytes, void *stream);
@@ -131,7 +147,7 @@ tern_status tern_gemv(const uint16_t *x, const uint8_t *slots, const uint16_t *s
 /*
  * tern_gemm -- y[M][N] = x[M][K] * W^T for any M >= 1.
  *   x  fp16 [M][K] row-major (device, read);  y  fp16 [M][N] row-major (device, written).
- * M <= 8 (speculative-verify batches) runs the same bandwidth-bound kernel as
+ * M <= 8 (speculative-verify batches) runs the same bandwidth-bound kernels as
  * tern_gemv, reading the weights once for all rows.  M >= 32 runs the
  * tensor-core prefill kernel (tcgen05), which unpacks weight tiles on chip to
  * s*t (exact in fp16) straight into tensor memory and accumulates in fp32;
@@ -165,6 +181,10 @@ typedef struct tern_gemv_desc {
 tern_status tern_gemv_grouped(const tern_gemv_desc *descs, int32_t count, int64_t M, void *workspace,
                               size_t ws_bytes, void *stream);
 
+/* Workspace for one tern_gemv_grouped call with these descriptors (only N and
+ * K are read); 0 if none is needed or the arguments are invalid. */
+size_t tern_gemv_grouped_workspace_bytes(const tern_gemv_desc *descs, int32_t count, int64_t M);
+
 /*
  * tern_sync_status -- wait for `stream`, then report whether any kernel of
  * this library on the current device gave up a bounded on-device wait since
@@ -189,8 +209,10 @@ tern_status tern_sync_status(void *stream);
  *                          2 = force the tensor-core kernel
  *   TERN_OPT_GEMM_MIN_M    smallest M (> 8) sent to the tensor-core kernel
  *                          (default 32)
- *   TERN_OPT_GEMV_VARIANT  bandwidth kernel: 0 = TMA-staged (default),
- *                          1 = register-ring loads (kept for comparison)
+ *   TERN_OPT_GEMV_VARIANT  bandwidth kernel: 0 = default (TMA-staged mma.sync),
+ *                          1 = register-ring mma.sync, 2 = TMA-staged mma.sync,
+ *                          3 = tcgen05 kernel for M <= 4 (splits K through the
+ *                          workspace); all kept for comparison
  *   TERN_OPT_TEST_STALL_US TESTS ONLY: the TMA loaders of the tensor-core and
  *                          the TMA-staged bandwidth kernels issue no loads, so
  *                          their waits can never complete, and every bounded

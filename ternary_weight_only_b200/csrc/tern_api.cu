@@ -4,6 +4,7 @@
 
 #include <cstdarg>
 #include <cstdio>
+#include <algorithm>
 #include <cstring>
 #include <mutex>
 
@@ -125,6 +126,33 @@ tern_status check_mat(const void *x, const void *slots, const void *scales, cons
     return TERN_OK;
 }
 
+// Streaming-multiprocessor count of the current device (148 on B200 when no
+// device is visible, so that sizes can be planned on a machine without one).
+int planning_sms() {
+    DeviceInfo dev;
+    if (current_device(&dev) == TERN_OK) return dev.sms;
+    clear_error();
+    return 148;
+}
+
+// Bandwidth kernels (M <= 8).  Default: the TMA-staged mma.sync kernel,
+// the fastest measured so far; the knob selects the others for comparison.
+enum { kVarDefault = 0, kVarRing = 1, kVarTma = 2, kVarTc = 3 };
+
+bool use_tc(int M) { return g_opt.gemv_variant == kVarTc && M <= 4; }
+
+tern_status launch_bandwidth(const MatDesc *d, int count, int M, void *workspace, size_t ws_bytes,
+                             cudaStream_t s) {
+    if (g_opt.gemv_variant == kVarRing) return launch_gemv_mma(d, count, M, s);
+    if (use_tc(M)) return launch_gemv_tc(d, count, M, workspace, ws_bytes, s);
+    return launch_gemv_tma(d, count, M, s);
+}
+
+size_t bandwidth_workspace(const MatDesc *d, int count, int M) {
+    if (!use_tc(M)) return 0;
+    return gemv_tc_workspace_bytes(d, count, M, planning_sms());
+}
+
 MatDesc mat(const uint16_t *x, const uint8_t *slots, const uint16_t *scales, uint16_t *y, int64_t N,
             int64_t K) {
     MatDesc d;
@@ -170,10 +198,30 @@ size_t tern_scales_bytes(int64_t N, int64_t K) {
 }
 
 size_t tern_workspace_bytes(int64_t M, int64_t N, int64_t K) {
-    (void)M;
-    (void)N;
-    (void)K;
-    return 0;
+    if (M < 1 || check_nk(N, K) != TERN_OK) {
+        clear_error();
+        return 0;
+    }
+    MatDesc d = mat(nullptr, nullptr, nullptr, nullptr, N, K);
+    size_t best = 0;
+    for (int64_t m0 = 0; m0 < M && M <= 8; m0 += 8) {
+        const int mc = static_cast<int>(M - m0 < 8 ? M - m0 : 8);
+        best = std::max(best, bandwidth_workspace(&d, 1, mc));
+    }
+    return best;
+}
+
+size_t tern_gemv_grouped_workspace_bytes(const tern_gemv_desc *descs, int32_t count, int64_t M) {
+    if (!descs || count < 1 || count > TERN_MAX_GROUP || M < 1 || M > 8) return 0;
+    MatDesc d[TERN_MAX_GROUP];
+    for (int i = 0; i < count; i++) {
+        if (check_nk(descs[i].N, descs[i].K) != TERN_OK) {
+            clear_error();
+            return 0;
+        }
+        d[i] = mat(nullptr, nullptr, nullptr, nullptr, descs[i].N, descs[i].K);
+    }
+    return bandwidth_workspace(d, count, static_cast<int>(M));
 }
 
 tern_status tern_pack_g128(const int8_t *codes, const uint16_t *scales_in, int64_t N, int64_t K,
@@ -209,8 +257,6 @@ tern_status tern_gemm(const uint16_t *x, const uint8_t *slots, const uint16_t *s
                       int64_t M, int64_t N, int64_t K, void *workspace, size_t ws_bytes,
                       void *stream) {
     clear_error();
-    (void)workspace;
-    (void)ws_bytes;
     if (M < 1) return fail(TERN_ERR_SHAPE, "M must be >= 1 (got %lld)", static_cast<long long>(M));
     if (M > (int64_t(1) << 24)) return fail(TERN_ERR_SHAPE, "M too large");
     tern_status st = check_nk(N, K);
@@ -225,7 +271,7 @@ tern_status tern_gemm(const uint16_t *x, const uint8_t *slots, const uint16_t *s
     for (int64_t m0 = 0; m0 < M; m0 += 8) {
         const int mc = static_cast<int>(M - m0 < 8 ? M - m0 : 8);
         MatDesc d = mat(x + m0 * K, slots, scales, y + m0 * N, N, K);
-        st = (g_opt.gemv_variant == 1) ? launch_gemv_mma(&d, 1, mc, s) : launch_gemv_tma(&d, 1, mc, s);
+        st = launch_bandwidth(&d, 1, mc, workspace, ws_bytes, s);
         if (st != TERN_OK) return st;
     }
     return TERN_OK;
@@ -239,8 +285,6 @@ tern_status tern_gemv(const uint16_t *x, const uint8_t *slots, const uint16_t *s
 tern_status tern_gemv_grouped(const tern_gemv_desc *descs, int32_t count, int64_t M,
                               void *workspace, size_t ws_bytes, void *stream) {
     clear_error();
-    (void)workspace;
-    (void)ws_bytes;
     if (!descs) return fail(TERN_ERR_INVALID_ARG, "descs is NULL");
     if (count < 1 || count > TERN_MAX_GROUP)
         return fail(TERN_ERR_INVALID_ARG, "count must be 1..%d (got %d)", TERN_MAX_GROUP, count);
@@ -254,20 +298,22 @@ tern_status tern_gemv_grouped(const tern_gemv_desc *descs, int32_t count, int64_
         if (st != TERN_OK) return st;
         d[i] = mat(descs[i].x, descs[i].slots, descs[i].scales, descs[i].y, descs[i].N, descs[i].K);
     }
-    if (g_opt.gemv_variant == 1) return launch_gemv_mma(d, count, static_cast<int>(M), static_cast<cudaStream_t>(stream));
-    return launch_gemv_tma(d, count, static_cast<int>(M), static_cast<cudaStream_t>(stream));
+    return launch_bandwidth(d, count, static_cast<int>(M), workspace, ws_bytes, static_cast<cudaStream_t>(stream));
 }
 
 tern_status tern_sync_status(void *stream) {
     clear_error();
     cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
-    unsigned int v = 0, w = 0;
+    unsigned int v = 0, w = 0, u = 0;
     tern_status st = read_gemm_status(true, &v);
     if (st != TERN_OK) return st;
     st = read_gemv_status(true, &w);
     if (st != TERN_OK) return st;
+    st = read_gemvtc_status(true, &u);
+    if (st != TERN_OK) return st;
     if (v == 0) v = w;
+    if (v == 0) v = u;
     if (v != 0) return fail(static_cast<tern_status>(v), "a kernel gave up a bounded wait on the device");
     return TERN_OK;
 }
@@ -285,7 +331,7 @@ tern_status tern_set_option(int option, int64_t value) {
             return TERN_OK;
         case TERN_OPT_GEMM_MIN_M: g_opt.gemm_min_m = static_cast<int>(value); return TERN_OK;
         case TERN_OPT_GEMV_VARIANT:
-            if (value > 1) return fail(TERN_ERR_INVALID_ARG, "gemv variant %lld", static_cast<long long>(value));
+            if (value > 3) return fail(TERN_ERR_INVALID_ARG, "gemv variant %lld", static_cast<long long>(value));
             g_opt.gemv_variant = static_cast<int>(value);
             return TERN_OK;
         case TERN_OPT_TEST_STALL_US:

@@ -54,6 +54,11 @@ struct MatDesc {
 // Bandwidth-bound product for M in [1,8] over `count` matrices in one launch:
 // TMA-staged kernel (default) and the register-ring kernel (variant 1).
 tern_status launch_gemv_tma(const MatDesc *d, int count, int M, cudaStream_t stream);
+// Tensor-core (tcgen05) bandwidth kernel for M in [1,4]; splits tiles along K
+// when a large enough zero-initialised workspace is given.
+tern_status launch_gemv_tc(const MatDesc *d, int count, int M, void *workspace, size_t ws_bytes,
+                           cudaStream_t stream);
+size_t gemv_tc_workspace_bytes(const MatDesc *d, int count, int M, int sms);
 tern_status launch_gemv_mma(const MatDesc *d, int count, int M, cudaStream_t stream);
 // 2-D tiled tensor map (row-major: `inner` contiguous elements per row, `outer`
 // rows `row_bytes` apart) for TMA loads of `box_inner` x `box_outer` boxes.
@@ -66,6 +71,7 @@ tern_status launch_gemm_tc(const MatDesc &d, int M, cudaStream_t stream);
 // kernel source file; read and optionally cleared).
 tern_status read_gemm_status(bool reset, unsigned int *out);
 tern_status read_gemv_status(bool reset, unsigned int *out);
+tern_status read_gemvtc_status(bool reset, unsigned int *out);
 extern unsigned long long g_gemm_timeout_ns;
 extern int g_gemm_skip_loads;
 

@@ -36,6 +36,7 @@ TERN_OPT_GEMM_PATH = 4
 TERN_OPT_GEMM_MIN_M = 5
 TERN_OPT_TEST_STALL_US = 6
 TERN_OPT_GEMV_VARIANT = 7
+GEMV_VARIANT_DEFAULT, GEMV_VARIANT_RING, GEMV_VARIANT_TMA, GEMV_VARIANT_TC = 0, 1, 2, 3
 TERN_MAX_GROUP = 16
 
 _i64, _vp, _sz, _i32, _int = ctypes.c_int64, ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int32, ctypes.c_int
@@ -59,6 +60,7 @@ _SIGS = {
     "tern_gemv_grouped": ([ctypes.POINTER(tern_gemv_desc), _i32, _i64, _vp, _sz, _vp], _int),
     "tern_set_option": ([_int, _i64], _int),
     "tern_sync_status": ([_vp], _int),
+    "tern_gemv_grouped_workspace_bytes": ([ctypes.POINTER(tern_gemv_desc), _i32, _i64], _sz),
 }
 for _name, (_args, _res) in _SIGS.items():
     _f = getattr(_L, _name)
@@ -114,6 +116,40 @@ def tern_workspace_bytes(M: int, N: int, K: int) -> int:
     return _L.tern_workspace_bytes(M, N, K)
 
 
+# Zero-initialised workspaces owned by this binding, one per (device, stream):
+# the library leaves a workspace zeroed after every call that completes, so a
+# cached buffer can be reused by later calls on the same stream.
+_WS: dict = {}
+_WS_RETIRED: list = []  # outgrown buffers stay alive: a captured graph may still use them
+
+
+def _workspace(nbytes: int, device: torch.device, stream: int):
+    if nbytes <= 0:
+        return None, 0
+    key = (device.index, stream)
+    buf = _WS.get(key)
+    if buf is None or buf.numel() < nbytes:
+        if buf is not None:
+            _WS_RETIRED.append(buf)
+        buf = torch.zeros(((nbytes + 255) // 256) * 256, dtype=torch.uint8, device=device)
+        _WS[key] = buf
+    return buf.data_ptr(), buf.numel()
+
+
+def tern_reset_workspaces():
+    """Zero every cached workspace (needed after a call reported TERN_ERR_TIMEOUT)."""
+    for buf in list(_WS.values()) + _WS_RETIRED:
+        buf.zero_()
+
+
+def _ws_args(workspace, nbytes, device, stream):
+    if workspace is False:
+        return None, 0
+    if isinstance(workspace, torch.Tensor):
+        return _dev(workspace, "workspace"), workspace.numel() * workspace.element_size()
+    return _workspace(nbytes, device, stream)
+
+
 def tern_set_option(option: int, value: int):
     _check(_L.tern_set_option(option, value), "tern_set_option")
 
@@ -151,33 +187,39 @@ def tern_unpack_g128(slots: torch.Tensor, K: int, codes_out: Optional[torch.Tens
 
 
 def tern_gemv(x: torch.Tensor, slots: torch.Tensor, scales: torch.Tensor,
-              y: Optional[torch.Tensor] = None, stream=None):
-    """x fp16 [K] -> y fp16 [N]."""
+              y: Optional[torch.Tensor] = None, stream=None, workspace=None):
+    """x fp16 [K] -> y fp16 [N].  workspace: None = a cached zeroed buffer of
+    tern_workspace_bytes(1, N, K) bytes, False = none, or a uint8 CUDA tensor."""
     N = slots.shape[0]
     K = x.shape[-1]
     if y is None:
         y = torch.empty((N,), dtype=torch.float16, device=x.device)
+    st = _stream(stream)
+    wp, wn = _ws_args(workspace, _L.tern_workspace_bytes(1, N, K) if workspace is None else 0, x.device, st)
     _check(_L.tern_gemv(_dev(x, "x", torch.float16), _dev(slots, "slots", torch.uint8),
                         _dev(scales, "scales", torch.float16), _dev(y, "y", torch.float16), N, K,
-                        None, 0, _stream(stream)), "tern_gemv")
+                        wp, wn, st), "tern_gemv")
     return y
 
 
 def tern_gemm(x: torch.Tensor, slots: torch.Tensor, scales: torch.Tensor,
-              y: Optional[torch.Tensor] = None, stream=None):
-    """x fp16 [M,K] -> y fp16 [M,N]."""
+              y: Optional[torch.Tensor] = None, stream=None, workspace=None):
+    """x fp16 [M,K] -> y fp16 [M,N].  workspace as for tern_gemv."""
     M, K = x.shape
     N = slots.shape[0]
     if y is None:
         y = torch.empty((M, N), dtype=torch.float16, device=x.device)
+    st = _stream(stream)
+    wp, wn = _ws_args(workspace, _L.tern_workspace_bytes(M, N, K) if workspace is None else 0, x.device, st)
     _check(_L.tern_gemm(_dev(x, "x", torch.float16), _dev(slots, "slots", torch.uint8),
                         _dev(scales, "scales", torch.float16), _dev(y, "y", torch.float16), M, N, K,
-                        None, 0, _stream(stream)), "tern_gemm")
+                        wp, wn, st), "tern_gemm")
     return y
 
 
-def tern_gemv_grouped(mats: Sequence, M: int, stream=None):
-    """mats: sequence of (x [M,K], slots [N,K/4], scales [N,K/128], y [M,N]) CUDA tensors."""
+def tern_gemv_grouped(mats: Sequence, M: int, stream=None, workspace=None):
+    """mats: sequence of (x [M,K], slots [N,K/4], scales [N,K/128], y [M,N]) CUDA tensors.
+    workspace as for tern_gemv (sized by tern_gemv_grouped_workspace_bytes)."""
     arr = (tern_gemv_desc * len(mats))()
     for i, (x, s, sc, y) in enumerate(mats):
         arr[i].x = _dev(x, "x", torch.float16)
@@ -186,4 +228,15 @@ def tern_gemv_grouped(mats: Sequence, M: int, stream=None):
         arr[i].y = _dev(y, "y", torch.float16)
         arr[i].N = s.shape[0]
         arr[i].K = x.shape[-1]
-    _check(_L.tern_gemv_grouped(arr, len(mats), M, None, 0, _stream(stream)), "tern_gemv_grouped")
+    st = _stream(stream)
+    need = _L.tern_gemv_grouped_workspace_bytes(arr, len(mats), M) if workspace is None else 0
+    wp, wn = _ws_args(workspace, need, mats[0][0].device, st)
+    _check(_L.tern_gemv_grouped(arr, len(mats), M, wp, wn, st), "tern_gemv_grouped")
+
+
+def tern_gemv_grouped_workspace_bytes(mats: Sequence, M: int) -> int:
+    arr = (tern_gemv_desc * len(mats))()
+    for i, (x, s, sc, y) in enumerate(mats):
+        arr[i].N = s.shape[0]
+        arr[i].K = x.shape[-1]
+    return _L.tern_gemv_grouped_workspace_bytes(arr, len(mats), M)

@@ -52,8 +52,30 @@ def test_sizes(lib):
         151936 * 5120 * 17 // 64
     for bad in [(0, 128), (4, 0), (4, 100), (-1, 128), (4, -128)]:
         assert lib.tern_slots_bytes(*bad) == 0 and lib.tern_scales_bytes(*bad) == 0
-    assert lib.tern_workspace_bytes(1, 1024, 5120) == 0
     assert lib.tern_version() >= 100
+
+
+def test_workspace_sizes(lib):
+    """With the tcgen05 bandwidth kernel selected, workspace is planned for
+    M <= 4 (it splits K), none for M = 5..8 and for the prefill kernel; invalid
+    shapes give 0; a grouped query for one matrix equals the single-matrix
+    query.  The default kernel needs none."""
+    from ternary_weight_only_b200 import tern
+    assert lib.tern_workspace_bytes(1, 5120, 17408) == 0
+    assert lib.tern_set_option(7, 3) == 0
+    for M in (1, 2, 4):
+        n = lib.tern_workspace_bytes(M, 5120, 17408)
+        assert n > 0 and n % 4 == 0
+    for M in (5, 8, 64, 2048):
+        assert lib.tern_workspace_bytes(M, 1024, 5120) == 0
+    for bad in [(0, 1024, 5120), (1, 0, 5120), (1, 1024, 100)]:
+        assert lib.tern_workspace_bytes(*bad) == 0
+    arr = (tern.tern_gemv_desc * 1)()
+    arr[0].N, arr[0].K = 17408, 5120
+    assert lib.tern_gemv_grouped_workspace_bytes(arr, 1, 1) == lib.tern_workspace_bytes(1, 17408, 5120)
+    assert lib.tern_gemv_grouped_workspace_bytes(arr, 0, 1) == 0
+    assert lib.tern_gemv_grouped_workspace_bytes(None, 1, 1) == 0
+    assert lib.tern_set_option(7, 0) == 0
 
 
 def test_status_strings(lib):

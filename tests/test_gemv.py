@@ -24,12 +24,12 @@ def T():
         tern.tern_set_option(o, 0)
 
 
-def run_case(T, orc, x, codes, scales, what="", threads=None):
+def run_case(T, orc, x, codes, scales, what="", threads=None, workspace=None):
     """Pack with the oracle (host), run the GPU product on those slots, compare."""
     xn, cn, sn = np_inputs(x, codes, scales)
     slots, sc, bad, _ = orc.pack(cn, sn)
     assert bad == 0
-    yd = T.tern_gemm(x.cuda(), torch.from_numpy(slots).cuda(), scales.cuda())
+    yd = T.tern_gemm(x.cuda(), torch.from_numpy(slots).cuda(), scales.cuda(), workspace=workspace)
     torch.cuda.synchronize()
     y_ref, bound = orc.matmul(xn, slots, sc, threads=threads or NCPU)
     return check_close(yd, y_ref, bound, what)
@@ -72,11 +72,11 @@ def test_ragged(T, orc, M, K, N):
     run_case(T, orc, x, codes, scales, f"M={M} K={K} N={N}")
 
 
-@pytest.mark.parametrize("variant", [0, 1])
+@pytest.mark.parametrize("variant", [2, 1])
 @pytest.mark.parametrize("ks", [1, 2, 4, 8])
 @pytest.mark.parametrize("cl", [1, 2, 4])
 def test_split_options(T, orc, ks, cl, variant):
-    """Every forced k split inside the CTA and across a cluster, both kernels."""
+    """Every forced k split inside the CTA and across a cluster, both mma.sync kernels."""
     from ternary_weight_only_b200 import synth
     x, codes, scales = synth.case(3, 17408, 200, seed=ks * 10 + cl, codes="sparse")
     T.tern_set_option(T.TERN_OPT_GEMV_VARIANT, variant)
@@ -89,6 +89,88 @@ def test_split_options(T, orc, ks, cl, variant):
     finally:
         T.tern_set_option(T.TERN_OPT_GEMV_KSPLIT, 0)
         T.tern_set_option(T.TERN_OPT_GEMV_CLUSTER, 0)
+        T.tern_set_option(T.TERN_OPT_GEMV_VARIANT, 0)
+
+
+@pytest.fixture
+def tc(T):
+    """Select the tcgen05 bandwidth kernel for the duration of a test."""
+    T.tern_set_option(T.TERN_OPT_GEMV_VARIANT, 3)
+    yield T
+    T.tern_set_option(T.TERN_OPT_GEMV_VARIANT, 0)
+
+
+@pytest.mark.parametrize("M", [1, 2, 3, 4])
+@pytest.mark.parametrize("K,N", [(128, 1), (384, 130), (5120, 1024), (6144, 5120), (17408, 640), (1152, 4000)])
+def test_tensor_core_split_and_whole(tc, orc, M, K, N):
+    """The tcgen05 kernel with its K split (cached workspace) and without (no workspace)."""
+    from ternary_weight_only_b200 import synth
+    x, codes, scales = synth.case(M, K, N, seed=M * 7 + K + N, codes="sparse", outlier_p=0.01)
+    run_case(tc, orc, x, codes, scales, f"tc split M={M} K={K} N={N}")
+    run_case(tc, orc, x, codes, scales, f"tc whole M={M} K={K} N={N}", workspace=False)
+
+
+@pytest.mark.parametrize("M", [1, 2, 4])
+@pytest.mark.parametrize("i", range(7))
+def test_tensor_core_decode_layer(tc, orc, i, M):
+    from ternary_weight_only_b200 import synth
+    x, codes, scales = synth.decode_proj(i, M=M)
+    run_case(tc, orc, x, codes, scales, f"tc {synth.LAYER_PROJ[i][0]} M={M}")
+
+
+def test_workspace_shared_by_shapes(tc, orc):
+    """One workspace serves calls of different shapes in turn (the counters of a
+    larger call never land on a smaller call's leftover partial sums)."""
+    from ternary_weight_only_b200 import synth
+    shapes = [(2, 6144, 5120), (2, 5120, 17408), (1, 17408, 5120), (4, 5120, 1024), (2, 5120, 17408)]
+    need = max(tc.tern_workspace_bytes(M, N, K) for M, K, N in shapes)
+    ws = torch.zeros(need, dtype=torch.uint8, device="cuda")
+    for i, (M, K, N) in enumerate(shapes):
+        x, codes, scales = synth.case(M, K, N, seed=500 + i, codes="sparse")
+        run_case(tc, orc, x, codes, scales, f"shared ws M={M} K={K} N={N}", workspace=ws)
+
+
+def test_split_is_deterministic_and_workspace_reusable(tc, orc):
+    T = tc
+    """Repeated calls sharing one workspace give bit-identical results (fixed
+    reduction order, counters reset by every call)."""
+    from ternary_weight_only_b200 import synth
+    x, codes, scales = synth.case(1, 17408, 5120, seed=99, codes="sparse")
+    xd, cd, sd = x.cuda(), codes.cuda(), scales.cuda()
+    slots, sc = T.tern_pack_g128(cd, sd)
+    need = T.tern_workspace_bytes(1, 5120, 17408)
+    assert need > 0
+    ws = torch.zeros(need, dtype=torch.uint8, device="cuda")
+    ys = [T.tern_gemv(xd[0], slots, sc, workspace=ws).clone() for _ in range(4)]
+    torch.cuda.synchronize()
+    for y in ys[1:]:
+        assert torch.equal(y.view(torch.int16), ys[0].view(torch.int16))
+    assert int(ws[: 128 * 1024].view(torch.int32).abs().sum().item()) == 0  # counters back to zero
+    xn, cn, sn = np_inputs(x, codes, scales)
+    ref_slots, ref_sc, _, _ = orc.pack(cn, sn)
+    y_ref, bound = orc.matmul(xn, ref_slots, ref_sc, threads=NCPU)
+    check_close(ys[0].view(1, -1), y_ref, bound, "deterministic split")
+
+
+@pytest.mark.parametrize("variant", [3, 2])
+def test_variant_grouped_layer(T, orc, variant):
+    from ternary_weight_only_b200 import synth
+    T.tern_set_option(T.TERN_OPT_GEMV_VARIANT, variant)
+    try:
+        mats, refs = [], []
+        for i in range(7):
+            x, codes, scales = synth.decode_proj(i, M=2)
+            xn, cn, sn = np_inputs(x, codes, scales)
+            slots, sc, _, _ = orc.pack(cn, sn)
+            y = torch.full((2, codes.shape[0]), float("nan"), dtype=torch.float16, device="cuda")
+            mats.append((x.cuda(), torch.from_numpy(slots).cuda(), scales.cuda(), y))
+            refs.append((xn, slots, sc))
+        T.tern_gemv_grouped(mats, 2)
+        torch.cuda.synchronize()
+        for i, ((xn, slots, sc), m) in enumerate(zip(refs, mats)):
+            y_ref, bound = orc.matmul(xn, slots, sc, threads=NCPU)
+            check_close(m[3], y_ref, bound, f"v{variant} grouped {synth.LAYER_PROJ[i][0]}")
+    finally:
         T.tern_set_option(T.TERN_OPT_GEMV_VARIANT, 0)
 
 
@@ -111,16 +193,20 @@ def test_timeout_path_reports_and_recovers(T, orc):
     xn, cn, sn = np_inputs(x, codes, scales)
     slots, sc, _, _ = orc.pack(cn, sn)
     xd, sd, scd = x.cuda(), torch.from_numpy(slots).cuda(), scales.cuda()
-    T.tern_set_option(T.TERN_OPT_TEST_STALL_US, 2000)
-    try:
-        T.tern_gemm(xd, sd, scd)
-        with pytest.raises(T.TernError) as ei:
-            T.tern_sync_status()
-        assert ei.value.status == T.TERN_ERR_TIMEOUT
-    finally:
-        T.tern_set_option(T.TERN_OPT_TEST_STALL_US, 0)
-    T.tern_sync_status()
-    run_case(T, orc, x, codes, scales, "after timeout")
+    for variant in (3, 2):
+        T.tern_set_option(T.TERN_OPT_GEMV_VARIANT, variant)
+        T.tern_set_option(T.TERN_OPT_TEST_STALL_US, 2000)
+        try:
+            T.tern_gemm(xd, sd, scd)
+            with pytest.raises(T.TernError) as ei:
+                T.tern_sync_status()
+            assert ei.value.status == T.TERN_ERR_TIMEOUT
+        finally:
+            T.tern_set_option(T.TERN_OPT_TEST_STALL_US, 0)
+            T.tern_set_option(T.TERN_OPT_GEMV_VARIANT, 0)
+        T.tern_reset_workspaces()
+        T.tern_sync_status()
+        run_case(T, orc, x, codes, scales, f"after timeout v{variant}")
 
 
 def test_grid_cap(T, orc):
