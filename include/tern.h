@@ -157,6 +157,29 @@ tern_status tern_gemm(const uint16_t *x, const uint8_t *slots, const uint16_t *s
                       int64_t M, int64_t N, int64_t K, void *workspace, size_t ws_bytes,
                       void *stream);
 
+/*
+ * tern_gemv_noalloc -- the same product as tern_gemv (M = 1), for callers that
+ * may not allocate device memory themselves: code running while a CUDA graph
+ * is captured into a memory pool it does not own, runtimes that forbid
+ * allocation after start-up, plug-ins whose host framework owns all device
+ * memory.  It runs the tensor-core (tcgen05) bandwidth kernel and takes the
+ * kernel's split-K scratch from a 4 MiB area compiled into the library
+ * instead of a workspace, and allocates nothing (no cudaMalloc, no cudaFree).
+ * The method described by the pages has no counterpart to this entry point;
+ * it exists only for such callers.
+ *   x, slots, scales, y, N, K, stream: as for tern_gemv.
+ *   - Every GPU that loads the library holds the 4 MiB area until exit.
+ *   - The first call on a device looks the area up (once per device, with
+ *     that device current); make that first call before any stream capture.
+ *   - Shapes whose scratch would exceed 4 MiB return TERN_ERR_WORKSPACE and
+ *     launch nothing.  (The 5120 x 151936 output head at M = 1 fits.)
+ *   - All calls on a device share the area: calls that may overlap on the GPU
+ *     race on it and must be serialised by the caller.  Each call clears the
+ *     area's arrival counters on `stream` before its kernel.
+ */
+tern_status tern_gemv_noalloc(const uint16_t *x, const uint8_t *slots, const uint16_t *scales, uint16_t *y,
+                              int64_t N, int64_t K, void *stream);
+
 /* One matrix of a grouped product (all fields describe device buffers as in
  * tern_gemm; every descriptor of one call has the same M). */
 typedef struct tern_gemv_desc {

@@ -282,6 +282,16 @@ tern_status tern_gemv(const uint16_t *x, const uint8_t *slots, const uint16_t *s
     return tern_gemm(x, slots, scales, y, 1, N, K, workspace, ws_bytes, stream);
 }
 
+tern_status tern_gemv_noalloc(const uint16_t *x, const uint8_t *slots, const uint16_t *scales, uint16_t *y,
+                              int64_t N, int64_t K, void *stream) {
+    clear_error();
+    tern_status st = check_nk(N, K);
+    if (st != TERN_OK) return st;
+    st = check_mat(x, slots, scales, y);
+    if (st != TERN_OK) return st;
+    return gemv_noalloc(mat(x, slots, scales, y, N, K), static_cast<cudaStream_t>(stream));
+}
+
 tern_status tern_gemv_grouped(const tern_gemv_desc *descs, int32_t count, int64_t M,
                               void *workspace, size_t ws_bytes, void *stream) {
     clear_error();

@@ -36,6 +36,7 @@
 // result does not depend on scheduling.  Every wait is bounded.
 #include <algorithm>
 #include <cstring>
+#include <mutex>
 
 #include "tern_internal.cuh"
 
@@ -730,6 +731,61 @@ tern_status read_gemvtc_status(bool reset, unsigned int *out) {
     }
     *out = v;
     return TERN_OK;
+}
+
+}  // namespace tern
+
+// ---------------------------------------------------------------------------
+// Entry-point variant that allocates nothing: the M = 1 product of this
+// kernel with its split-K scratch (arrival counters + partial sums) taken from
+// a fixed area compiled into the library instead of a caller workspace.  It
+// serves callers that may not allocate device memory on their own: code that
+// runs while a CUDA graph is being captured into a pool the caller does not
+// control, runtimes that forbid allocation after start-up (real-time or
+// certified deployments), and plug-ins hosted by a framework that owns all
+// device memory.  The area is shared by every call on a device, so calls that
+// may overlap on the GPU (different streams, or graphs launched concurrently)
+// race on it; callers must serialise them.
+namespace tern {
+
+// Largest scratch the no-allocation entry point can use, per device.  Every
+// GPU that loads this library reserves it until the process exits.
+constexpr size_t kNoAllocScratchBytes = size_t(4) << 20;  // 4 MiB
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+namespace {
+std::mutex g_noalloc_mu;
+void *g_noalloc_ptr[64];
+}  // namespace
+
+tern_status gemv_noalloc(const MatDesc &d, cudaStream_t stream) {
+    DeviceInfo dev;
+    tern_status st = current_device(&dev);
+    if (st != TERN_OK) return st;
+    void *scratch = nullptr;
+    {
+        // One-time set-up per device, with that device current: the host can
+        // only use the symbol's device address, never the symbol itself.
+        std::lock_guard<std::mutex> lock(g_noalloc_mu);
+        if (g_noalloc_ptr[dev.device] == nullptr) {
+            void *ptr = nullptr;
+            cudaError_t e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
+            if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(no-allocation scratch)");
+            g_noalloc_ptr[dev.device] = ptr;
+        }
+        scratch = g_noalloc_ptr[dev.device];
+    }
+    const size_t need = gemv_tc_workspace_bytes(&d, 1, 1, dev.sms);
+    if (need > kNoAllocScratchBytes)
+        return fail(TERN_ERR_WORKSPACE,
+                    "N=%d K=%d needs %zu bytes of scratch; the no-allocation entry point has %zu", d.N, d.K, need,
+                    kNoAllocScratchBytes);
+    if (need == 0) return launch_gemv_tc(&d, 1, 1, nullptr, 0, stream);
+    // The area keeps the previous call's contents: clear the arrival counters,
+    // the only part that must start at zero (the partial sums are overwritten).
+    cudaError_t e = cudaMemsetAsync(scratch, 0, kCounterBytes, stream);
+    if (e != cudaSuccess) return cuda_fail(e, "clearing no-allocation scratch");
+    return launch_gemv_tc(&d, 1, 1, scratch, kNoAllocScratchBytes, stream);
 }
 
 }  // namespace tern

@@ -59,6 +59,8 @@ tern_status launch_gemv_tma(const MatDesc *d, int count, int M, cudaStream_t str
 tern_status launch_gemv_tc(const MatDesc *d, int count, int M, void *workspace, size_t ws_bytes,
                            cudaStream_t stream);
 size_t gemv_tc_workspace_bytes(const MatDesc *d, int count, int M, int sms);
+// M = 1 product of the tcgen05 kernel with its scratch in a static device area.
+tern_status gemv_noalloc(const MatDesc &d, cudaStream_t stream);
 tern_status launch_gemv_mma(const MatDesc *d, int count, int M, cudaStream_t stream);
 // 2-D tiled tensor map (row-major: `inner` contiguous elements per row, `outer`
 // rows `row_bytes` apart) for TMA loads of `box_inner` x `box_outer` boxes.

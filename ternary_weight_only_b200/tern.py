@@ -61,6 +61,7 @@ _SIGS = {
     "tern_set_option": ([_int, _i64], _int),
     "tern_sync_status": ([_vp], _int),
     "tern_gemv_grouped_workspace_bytes": ([ctypes.POINTER(tern_gemv_desc), _i32, _i64], _sz),
+    "tern_gemv_noalloc": ([_vp, _vp, _vp, _vp, _i64, _i64, _vp], _int),
 }
 for _name, (_args, _res) in _SIGS.items():
     _f = getattr(_L, _name)
@@ -199,6 +200,18 @@ def tern_gemv(x: torch.Tensor, slots: torch.Tensor, scales: torch.Tensor,
     _check(_L.tern_gemv(_dev(x, "x", torch.float16), _dev(slots, "slots", torch.uint8),
                         _dev(scales, "scales", torch.float16), _dev(y, "y", torch.float16), N, K,
                         wp, wn, st), "tern_gemv")
+    return y
+
+
+def tern_gemv_noalloc(x: torch.Tensor, slots: torch.Tensor, scales: torch.Tensor,
+                      y: torch.Tensor, stream=None):
+    """x fp16 [K] -> y fp16 [N] (preallocated); the library uses its static
+    scratch area and allocates nothing.  Calls must not overlap on the GPU."""
+    N = slots.shape[0]
+    K = x.shape[-1]
+    _check(_L.tern_gemv_noalloc(_dev(x, "x", torch.float16), _dev(slots, "slots", torch.uint8),
+                                _dev(scales, "scales", torch.float16), _dev(y, "y", torch.float16), N, K,
+                                _stream(stream)), "tern_gemv_noalloc")
     return y
 
 
