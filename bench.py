@@ -398,18 +398,25 @@ def run_reference(args):
 
 
 # ----------------------------------------------------------------- main ---
-def traffic_from_profile():
+# The kernel that carries the decode step (every grouped layer and the head).
+DOMINANT_KERNEL, DOMINANT_SOURCE = "gemv_pc_kernel", "tern_gemv_pc.cu"
+
+
+def traffic_from_profile(avg_launch_bytes):
     """Per-launch DRAM bytes of the dominant kernel from the committed ncu
     summary, only if the kernel source is unchanged since the capture."""
-    prof = os.path.join(ROOT, "profiles", "gemv_tma_kernel.decode_layer.txt")
-    src = os.path.join(ROOT, "ternary_weight_only_b200", "csrc", "tern_gemv_tma.cu")
+    prof = os.path.join(ROOT, "profiles", f"{DOMINANT_KERNEL}.decode_layer.txt")
+    src = os.path.join(ROOT, "ternary_weight_only_b200", "csrc", DOMINANT_SOURCE)
     try:
         text = open(prof).read()
         sha = hashlib.sha256(open(src, "rb").read()).hexdigest()
         m_sha = re.search(r"source_sha256:\s*([0-9a-f]{64})", text)
         m_b = re.search(r"dram_bytes_per_launch:\s*([0-9.eE+]+)", text)
-        if m_sha and m_b and m_sha.group(1) == sha:
-            return float(m_b.group(1))
+        m_a = re.search(r"algorithmic_bytes_per_launch:\s*([0-9.eE+]+)", text)
+        if m_sha and m_b and m_a and m_sha.group(1) == sha:
+            # DRAM bytes per algorithmic byte of the captured launch, applied
+            # to the average launch of the step.
+            return float(m_b.group(1)) / float(m_a.group(1)) * avg_launch_bytes
     except OSError:
         pass
     return None
@@ -501,7 +508,7 @@ def run_tern(args):
     launches = model.launches_per_step * args.steps
     per_launch_ms = ms_local / model.launches_per_step
     achieved = total_bytes / model.launches_per_step / (per_launch_ms * 1e-3) / 1e9
-    traffic = traffic_from_profile()
+    traffic = traffic_from_profile(total_bytes / model.launches_per_step)
     if rank == 0:
         line = {
             "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": ws,
@@ -520,9 +527,9 @@ def run_tern(args):
             "e2e": {"value": round(e2e_value, 1), "unit": "GB/s", "ms_per_step": round(e2e_ms, 4),
                     "h2d_bytes_per_step": int(model.x_all.numel() * 2),
                     "d2h_bytes_per_step": int(model.y_all.numel() * 2)},
-            "roofline": {"bound": "hbm", "kernel": "gemv_tma_kernel",
+            "roofline": {"bound": "hbm", "kernel": DOMINANT_KERNEL,
                          "achieved": round(achieved, 1), "peak": peak_gbs, "unit": "GB/s",
-                         "frac": round(achieved / peak_gbs, 4), "traffic": traffic,
+                         "frac": round(achieved / peak_gbs, 4), "traffic": round(traffic) if traffic else None,
                          "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)" if peak_src == "measured" else "fallback 6650 GB/s",
                          "per_launch": "device time of the timed region / launches (gaps included)"},
             "cpu_baseline": cpu,

@@ -232,10 +232,17 @@ tern_status tern_sync_status(void *stream);
  *                          2 = force the tensor-core kernel
  *   TERN_OPT_GEMM_MIN_M    smallest M (> 8) sent to the tensor-core kernel
  *                          (default 32)
- *   TERN_OPT_GEMV_VARIANT  bandwidth kernel: 0 = default (TMA-staged mma.sync),
+ *   TERN_OPT_GEMV_VARIANT  bandwidth kernel: 0 = default (variant 4 where its
+ *                          shape rules hold, else variant 2),
  *                          1 = register-ring mma.sync, 2 = TMA-staged mma.sync,
  *                          3 = tcgen05 kernel for M <= 4 (splits K through the
- *                          workspace); all kept for comparison
+ *                          workspace), 4 = producer/consumer mma.sync kernel
+ *                          for K a multiple of 1024 (one CTA per SM, one
+ *                          logic operation per weight pair; other shapes take
+ *                          the default kernel); all kept for comparison
+ *   TERN_OPT_GEMV_GRID     cap on the CTAs of the producer/consumer kernel
+ *                          (0 = one per SM); smaller grids give every CTA
+ *                          more tiles to split among its warps
  *   TERN_OPT_TEST_STALL_US TESTS ONLY: the TMA loaders of the tensor-core and
  *                          the TMA-staged bandwidth kernels issue no loads, so
  *                          their waits can never complete, and every bounded
@@ -249,7 +256,8 @@ enum {
     TERN_OPT_GEMM_PATH = 4,
     TERN_OPT_GEMM_MIN_M = 5,
     TERN_OPT_TEST_STALL_US = 6,
-    TERN_OPT_GEMV_VARIANT = 7
+    TERN_OPT_GEMV_VARIANT = 7,
+    TERN_OPT_GEMV_GRID = 8
 };
 tern_status tern_set_option(int option, int64_t value);
 

@@ -137,7 +137,7 @@ int planning_sms() {
 
 // Bandwidth kernels (M <= 8).  Default: the TMA-staged mma.sync kernel,
 // the fastest measured so far; the knob selects the others for comparison.
-enum { kVarDefault = 0, kVarRing = 1, kVarTma = 2, kVarTc = 3 };
+enum { kVarDefault = 0, kVarRing = 1, kVarTma = 2, kVarTc = 3, kVarPc = 4 };
 
 bool use_tc(int M) { return g_opt.gemv_variant == kVarTc && M <= 4; }
 
@@ -145,6 +145,10 @@ tern_status launch_bandwidth(const MatDesc *d, int count, int M, void *workspace
                              cudaStream_t s) {
     if (g_opt.gemv_variant == kVarRing) return launch_gemv_mma(d, count, M, s);
     if (use_tc(M)) return launch_gemv_tc(d, count, M, workspace, ws_bytes, s);
+    // Default: the producer/consumer kernel where its shape rules hold (K a
+    // multiple of 1024, x fits its shared memory), else the TMA-staged one.
+    if ((g_opt.gemv_variant == kVarPc || g_opt.gemv_variant == kVarDefault) && gemv_pc_supports(d, count, M))
+        return launch_gemv_pc(d, count, M, s);
     return launch_gemv_tma(d, count, M, s);
 }
 
@@ -322,8 +326,12 @@ tern_status tern_sync_status(void *stream) {
     if (st != TERN_OK) return st;
     st = read_gemvtc_status(true, &u);
     if (st != TERN_OK) return st;
+    unsigned int z = 0;
+    st = read_gemvpc_status(true, &z);
+    if (st != TERN_OK) return st;
     if (v == 0) v = w;
     if (v == 0) v = u;
+    if (v == 0) v = z;
     if (v != 0) return fail(static_cast<tern_status>(v), "a kernel gave up a bounded wait on the device");
     return TERN_OK;
 }
@@ -341,9 +349,10 @@ tern_status tern_set_option(int option, int64_t value) {
             return TERN_OK;
         case TERN_OPT_GEMM_MIN_M: g_opt.gemm_min_m = static_cast<int>(value); return TERN_OK;
         case TERN_OPT_GEMV_VARIANT:
-            if (value > 3) return fail(TERN_ERR_INVALID_ARG, "gemv variant %lld", static_cast<long long>(value));
+            if (value > 4) return fail(TERN_ERR_INVALID_ARG, "gemv variant %lld", static_cast<long long>(value));
             g_opt.gemv_variant = static_cast<int>(value);
             return TERN_OK;
+        case TERN_OPT_GEMV_GRID: g_opt.gemv_grid = static_cast<int>(value); return TERN_OK;
         case TERN_OPT_TEST_STALL_US:
             g_gemm_skip_loads = value > 0 ? 1 : 0;
             g_gemm_timeout_ns = value > 0 ? static_cast<unsigned long long>(value) * 1000ull : 1000000000ull;

@@ -1,0 +1,587 @@
+// Bandwidth-bound ternary-g128 product for M = 1..8 token rows: producer /
+// consumer form of the TMA-staged mma.sync kernel, for K a multiple of 1024.
+//
+// What it computes: y[m][n] = sum_k x[m][k] * s[n][k/128] * t[n][k] with t
+// read straight from the 2-bit slots and the group scale applied inside the
+// product ("Ternary-Bonsai-27B" model summary, aitrends.kr, section
+// "Technical features"); decode is bound by memory bandwidth ("Bonsai 27B
+// ternary / 1-bit quantization", ThakiCloud blog, section "Throughput and
+// speculative decoding").
+//
+// Arithmetic (mma.sync m16n8k16, weight rows as A, token rows as B, fp32
+// accumulate, group scale applied in fp32) with a one-instruction unpack:
+//  * A slot word holds 16 codes; its "pair j" is field j of both 16-bit halves
+//    (weights j and j+8).  One AND with 0x00030003 << 2j' (j' = j for j < 5,
+//    j - 5 on the word shifted right by 10 for j >= 5) leaves an fp16 pair
+//    whose halves are the subnormals c * 4^j' * 2^-24: exact, no offset.
+//  * Every mma takes pair j of the lane's four words, so one mma sees one
+//    factor 4^j'.  The staged x carries the inverse: the B operand of pair j
+//    is x * 2^(E - 2j'), an exact power-of-two scaling for E = min(8, 15 - e),
+//    e the binary exponent of max|x| (no overflow; for max|x| < 256 nothing
+//    is rounded).  Each product is then c * x * 2^(E-24), exact in fp32.
+//  * t = c - 1, so a group's sum is D(codes) - D(all ones); D(all ones) is
+//    computed per group and token once per CTA with the very same mma chain,
+//    so an all-zero row of weights gives exactly 0.  The fp32 accumulator is
+//    multiplied by 2^(24-E) at the end of a tile.
+// One CTA per SM: twelve consumer warps and one producer warp (13 warps, at
+// most four on a scheduler, so 128 registers a thread).  Each consumer owns a
+// private ring of `ns` stages; a stage is one "slice" of 16 weight rows x
+// 1024 k: two 128-byte-swizzled TMA boxes of slots (2 x 2 KB) and one TMA box
+// of the matching 16 x 8 fp16 scales (256 B, which needs the scale rows to be
+// a multiple of 16 bytes, i.e. K a multiple of 1024).  Lane c of the producer
+// warp refills consumer c's ring as soon as a stage is free, polling with
+// non-blocking waits, so no consumer waits for another.
+#include <algorithm>
+#include <cstring>
+
+#include "tern_internal.cuh"
+
+namespace tern {
+
+// Device-side record of a bounded wait in this kernel that gave up.
+__device__ unsigned int g_tern_gemvpc_status;
+
+namespace {
+
+constexpr int kCons = 12;                       // consumer warps
+constexpr int kThreads = (kCons + 1) * 32;      // + one producer warp
+constexpr int kRows = 16;                       // tile rows (mma M)
+constexpr int kSG = 8;                          // scale groups per slice (1024 k)
+constexpr int kBox = 128;                       // bytes per row of one slot box (4 groups)
+constexpr int kSlotBytes = kRows * kBox * 2;    // 4 KB
+constexpr int kScaleBytes = kRows * kSG * 2;    // 256 B
+constexpr int kMaxNS = 4;                       // ring stages per consumer, at most
+constexpr int kGroupK = 128;
+constexpr int kBarBytes = 2 * kCons * kMaxNS * 8;
+constexpr int kRecBytes = kCons * 2 * 32 * 4 * 4;  // partial tiles, two per consumer
+constexpr size_t kSmemBudget = 232448;          // opt-in shared memory per block on sm_100
+constexpr int kMaxDesc = TERN_MAX_GROUP;
+
+struct alignas(64) PDesc {
+    CUtensorMap smap;   // slots uint8 [N][K/4], box 128 B x 16 rows, 128-byte swizzle
+    CUtensorMap cmap;   // scales fp16 [N][K/128], box 8 x 16, no swizzle
+    const __half *x;    // [M][K]
+    __half *y;          // [M][N]
+    int N, K, B;        // B = K / 1024 slices per row
+    int ntile;          // ceil(N / 16)
+    int c_begin, c_count;  // CTAs of this matrix
+};
+
+struct PParams {
+    PDesc d[kMaxDesc];
+    int count, M;
+    int ns;             // ring stages per consumer
+    int kmax;           // largest K of the launch (sizes the all-ones table)
+    int xs_halves;
+    int skip_loads;
+    unsigned long long timeout_ns;
+};
+
+size_t smem_bytes(int ns, int xs_halves, int kmax) {
+    return 1024 + static_cast<size_t>(kCons) * ns * (kSlotBytes + kScaleBytes) + kBarBytes + kRecBytes + 160 +
+           static_cast<size_t>(kmax / kGroupK) * 8 * 4 + static_cast<size_t>(xs_halves) * 2;
+}
+
+constexpr uint32_t kOnes = 0x55555555u;  // every 2-bit field = code 1 (t = 0)
+
+// D = A * B + C and D = A * B, m16n8k16, fp16 in, fp32 accumulate (no side
+// effects, so the compiler may interleave the chains of neighbouring groups).
+__device__ __forceinline__ void mma_acc(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                        uint32_t b0, uint32_t b1) {
+    asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 "
+        "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ void mma_zero(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                         uint32_t b0, uint32_t b1) {
+    asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 "
+        "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%10,%10,%10,%10};"
+        : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "f"(0.0f));
+}
+
+// Index (in halves) of x[m][kl] in this kernel's staging area.  Per group
+// of 128 k the B fragments of its eight mmas: chunk i (pairs j = 2i, 2i+1)
+// holds, per token m and lane q (words 2q, 2q+1 of the group), 8 halves
+// [j & 1][word 2q + wi][half] = x at word position j (lo) and j+8 (hi).
+// Layout [group][chunk][m][q][8]: a lane's four 16-byte loads hit distinct
+// banks within every quarter warp.
+template <int MT>
+__device__ __forceinline__ int xs_pair_index(int m, int kl) {
+    const int grp = kl >> 7;
+    const int word = (kl >> 4) & 7;
+    const int hi = (kl >> 3) & 1;
+    const int j = kl & 7;
+    return (((grp * 4 + (j >> 1)) * MT + m) * 4 + (word >> 1)) * 8 + (j & 1) * 4 + (word & 1) * 2 + hi;
+}
+
+// The eight mmas of one 16-row x 128-k group: pair j of the lane's words
+// (a = row g, b = row g+8; .x = word 2q, .y = word 2q+1) against the staged x
+// of pair j, as two independent chains (pairs 0-3 and 4-7) added at the end.
+// Shared by the weight path and the all-ones pass, so the two round
+// identically.
+template <int MT>
+__device__ __forceinline__ void group_mma(float (&c)[4], uint32_t ax, uint32_t ay, uint32_t bx, uint32_t by,
+                                          const __half *xb) {
+    constexpr int kChunk = MT * 32;
+    const uint4 x0 = *reinterpret_cast<const uint4 *>(xb);
+    const uint4 x1 = *reinterpret_cast<const uint4 *>(xb + kChunk);
+    const uint4 x2 = *reinterpret_cast<const uint4 *>(xb + 2 * kChunk);
+    const uint4 x3 = *reinterpret_cast<const uint4 *>(xb + 3 * kChunk);
+    const uint32_t ax5 = ax >> 10, ay5 = ay >> 10, bx5 = bx >> 10, by5 = by >> 10;
+    float e[4];
+    mma_zero(c, ax & 0x00030003u, bx & 0x00030003u, ay & 0x00030003u, by & 0x00030003u, x0.x, x0.y);
+    mma_zero(e, ax & 0x03000300u, bx & 0x03000300u, ay & 0x03000300u, by & 0x03000300u, x2.x, x2.y);
+    mma_acc(c, ax & 0x000C000Cu, bx & 0x000C000Cu, ay & 0x000C000Cu, by & 0x000C000Cu, x0.z, x0.w);
+    mma_acc(e, ax5 & 0x00030003u, bx5 & 0x00030003u, ay5 & 0x00030003u, by5 & 0x00030003u, x2.z, x2.w);
+    mma_acc(c, ax & 0x00300030u, bx & 0x00300030u, ay & 0x00300030u, by & 0x00300030u, x1.x, x1.y);
+    mma_acc(e, ax5 & 0x000C000Cu, bx5 & 0x000C000Cu, ay5 & 0x000C000Cu, by5 & 0x000C000Cu, x3.x, x3.y);
+    mma_acc(c, ax & 0x00C000C0u, bx & 0x00C000C0u, ay & 0x00C000C0u, by & 0x00C000C0u, x1.z, x1.w);
+    mma_acc(e, ax5 & 0x00300030u, bx5 & 0x00300030u, ay5 & 0x00300030u, by5 & 0x00300030u, x3.z, x3.w);
+    c[0] += e[0];
+    c[1] += e[1];
+    c[2] += e[2];
+    c[3] += e[3];
+}
+
+__device__ __forceinline__ bool mbar_test_wait(uint64_t *bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+__device__ __forceinline__ bool pc_wait(uint64_t *bar, uint32_t parity, unsigned long long deadline) {
+    while (!mbar_try_wait(bar, parity)) {
+        if (globaltimer() > deadline) {
+            atomicExch(&g_tern_gemvpc_status, static_cast<unsigned int>(TERN_ERR_TIMEOUT));
+            return false;
+        }
+    }
+    return true;
+}
+
+__device__ __forceinline__ int tile_row(int g) { return g < 4 ? 2 * g : 2 * g - 7; }
+
+// Work of warp w (consumer w, or producer lane w) of CTA lc of a matrix: the
+// CTA owns tiles [t0, t1) (balanced to one tile), whose (tile, slice) units
+// in tile-major order are split evenly over the consumer warps: units
+// [u0, u1), unit u = slice u % B of tile t0 + u / B.
+struct Range {
+    int t0, u0, u1;
+    __device__ void init(const PDesc &d, int lc, int w) {
+        t0 = static_cast<int>((static_cast<long long>(lc) * d.ntile) / d.c_count);
+        const int t1 = static_cast<int>((static_cast<long long>(lc + 1) * d.ntile) / d.c_count);
+        const int U = (t1 - t0) * d.B;
+        u0 = (U * w) / kCons;
+        u1 = (U * (w + 1)) / kCons;
+    }
+};
+
+template <int MT>
+__global__ void __launch_bounds__(kThreads, 1) gemv_pc_kernel(const __grid_constant__ PParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const int ns = p.ns;
+    uint8_t *slot_ring = base;                                   // [kCons][ns][4096], 1024-aligned boxes
+    uint8_t *scale_ring = slot_ring + kCons * ns * kSlotBytes;   // [kCons][ns][256]
+    uint64_t *full = reinterpret_cast<uint64_t *>(scale_ring + kCons * ns * kScaleBytes);  // [kCons][kMaxNS]
+    uint64_t *empty = full + kCons * kMaxNS;
+    float *rec = reinterpret_cast<float *>(empty + kCons * kMaxNS);  // [kCons][2][32][4] partial tiles
+    int *rec_tile = reinterpret_cast<int *>(rec + kCons * 2 * 32 * 4);  // [kCons][2]
+    unsigned int *wmax = reinterpret_cast<unsigned int *>(rec_tile + 2 * kCons);  // [kCons]
+    float *d1 = reinterpret_cast<float *>(wmax + 16);            // [K/128][8]
+    __half *xs = reinterpret_cast<__half *>(d1 + (p.kmax / kGroupK) * 8);
+
+    const int M = p.M;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    int di = 0;
+#pragma unroll 1
+    while (di + 1 < p.count && static_cast<int>(blockIdx.x) >= p.d[di + 1].c_begin) di++;
+    const PDesc &d = p.d[di];
+    const int lc = blockIdx.x - d.c_begin;
+    const int B = d.B;
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < kCons * kMaxNS; i++) {
+            mbar_init(&full[i], 1);
+            mbar_init(&empty[i], 1);
+        }
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    __syncthreads();
+    const unsigned long long deadline = globaltimer() + p.timeout_ns;
+
+    if (warp == kCons) {
+        // ======================= producer warp =======================
+        // Lane c (< kCons) feeds consumer warp c its units in order, one ring
+        // stage each.
+        Range r;
+        int u = 0, s = 0, issued = 0;
+        uint32_t ph = 0;
+        bool done = true;
+        if (lane < kCons && !p.skip_loads) {
+            r.init(d, lc, lane);
+            u = r.u0;
+            done = u >= r.u1;
+        }
+        uint8_t *my_slots = slot_ring + lane * ns * kSlotBytes;
+        uint8_t *my_scales = scale_ring + lane * ns * kScaleBytes;
+        uint64_t *my_full = full + lane * kMaxNS;
+        uint64_t *my_empty = empty + lane * kMaxNS;
+        while (__any_sync(0xffffffffu, !done)) {
+            bool progressed = false;
+            if (!done) {
+                if (mbar_test_wait(&my_empty[s], ph ^ 1)) {
+                    const int tile = r.t0 + u / B;
+                    const int kbx = u - (u / B) * B;
+                    mbar_expect_tx(&my_full[s], kSlotBytes + kScaleBytes);
+                    tma_load_2d(my_slots + s * kSlotBytes, &d.smap, kbx * 2 * kBox, tile * kRows, &my_full[s]);
+                    tma_load_2d(my_slots + s * kSlotBytes + kRows * kBox, &d.smap, kbx * 2 * kBox + kBox,
+                                tile * kRows, &my_full[s]);
+                    tma_load_2d(my_scales + s * kScaleBytes, &d.cmap, kbx * kSG, tile * kRows, &my_full[s]);
+                    issued++;
+                    if (++s == ns) {
+                        s = 0;
+                        ph ^= 1;
+                    }
+                    progressed = true;
+                    done = ++u >= r.u1;
+                } else if (globaltimer() > deadline) {
+                    atomicExch(&g_tern_gemvpc_status, static_cast<unsigned int>(TERN_ERR_TIMEOUT));
+                    done = true;
+                }
+            }
+            if (!__any_sync(0xffffffffu, progressed)) __nanosleep(128);
+        }
+        // The last min(ns, issued) stages are the only ones that can still be
+        // in flight: they must land before the CTA exits, also when the
+        // consumer gave up on them (bounded; normally already complete).
+        const unsigned long long dl2 = globaltimer() + p.timeout_ns;
+        for (int i = 0; i < ns && i < issued; i++) {
+            const int uu = issued - 1 - i;
+            pc_wait(&my_full[uu % ns], (uu / ns) & 1, dl2);
+        }
+    } else {
+        // ======================= consumer warps =======================
+        const int K = d.K, N = d.N;
+        const int nthr = kCons * 32;
+        // (1) E from the largest finite |x| of all token rows.
+        {
+            unsigned int mx = 0;
+            for (int idx = threadIdx.x; idx < M * K / 8; idx += nthr) {
+                const uint4 v = *reinterpret_cast<const uint4 *>(d.x + static_cast<size_t>(idx) * 8);
+                const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                for (int e = 0; e < 4; e++) {
+                    mx = max(mx, min(wv[e] & 0x7FFFu, 0x7BFFu));
+                    mx = max(mx, min((wv[e] >> 16) & 0x7FFFu, 0x7BFFu));
+                }
+            }
+            mx = __reduce_max_sync(0xffffffffu, mx);
+            if (lane == 0) wmax[warp] = mx;
+            if (lane < 2) rec_tile[warp * 2 + lane] = -1;
+        }
+        named_bar_sync(1, nthr);
+        unsigned int mx = 0;
+#pragma unroll
+        for (int i = 0; i < kCons; i++) mx = max(mx, wmax[i]);
+        // binary exponent of max|x| (subnormal and zero count as -14)
+        const int ex = max(static_cast<int>(mx >> 10), 1) - 15;
+        const int E = min(8, 15 - ex);
+        // (2) stage x in pair order, pair j scaled by 2^(E - 2j').
+        {
+            float fac[8];
+#pragma unroll
+            for (int j = 0; j < 8; j++) fac[j] = ldexpf(1.0f, E - 2 * (j < 5 ? j : j - 5));
+            const int per_m = K / 8;
+            for (int idx = threadIdx.x; idx < M * per_m; idx += nthr) {
+                const int m = idx / per_m, c8 = idx - m * per_m;
+                const uint4 v = *reinterpret_cast<const uint4 *>(d.x + static_cast<size_t>(m) * K + c8 * 8);
+                const __half *hv = reinterpret_cast<const __half *>(&v);
+                __half *dst = xs + xs_pair_index<MT>(m, c8 * 8);  // element e: chunk e/2, slot (e&1)*4
+#pragma unroll
+                for (int e = 0; e < 8; e++)
+                    dst[(e >> 1) * MT * 32 + (e & 1) * 4] = __float2half_rn(__half2float(hv[e]) * fac[e]);
+            }
+        }
+        named_bar_sync(1, nthr);
+        const int g = lane >> 2, q = lane & 3;
+        const int gx = g < M ? g : M - 1;
+        const int G = K / kGroupK;
+        constexpr int kGroupHalves = MT * 4 * 32;
+        const __half *xlane = xs + (gx * 4 + q) * 8;
+        // (3) the all-ones pass: D(ones) per group and B column (token).
+        for (int grp = warp; grp < G; grp += kCons) {
+            float c[4];
+            group_mma<MT>(c, kOnes, kOnes, kOnes, kOnes, xlane + grp * kGroupHalves);
+            if (g == 0) *reinterpret_cast<float2 *>(d1 + grp * 8 + 2 * q) = make_float2(c[0], c[1]);
+        }
+        named_bar_sync(1, nthr);
+
+        const int row = tile_row(g);
+        Range r;
+        r.init(d, lc, warp);
+        uint32_t off[4];
+#pragma unroll
+        for (int j = 0; j < 4; j++) off[j] = row * kBox + (((2 * j + (q >> 1)) ^ (row & 7)) << 4) + (q & 1) * 8;
+        const float *d1lane = d1 + 2 * q;
+        const uint8_t *my_slots = slot_ring + warp * ns * kSlotBytes;
+        const uint8_t *my_scales = scale_ring + warp * ns * kScaleBytes;
+        uint64_t *my_full = full + warp * kMaxNS;
+        uint64_t *my_empty = empty + warp * kMaxNS;
+        const float post = ldexpf(1.0f, 24 - E);
+        float acc[4] = {0.f, 0.f, 0.f, 0.f};
+        int s = 0;
+        uint32_t ph = 0;
+        bool dead = false;
+        int tl = r.u0 / B;                 // tile (relative to t0) being accumulated
+        int kb = r.u0 - tl * B;            // its next slice
+        const int kb_first = kb;           // first slice of the first tile
+        for (int u = r.u0; u < r.u1; u++) {
+            bool ok = !dead;
+            if (ok) ok = __all_sync(0xffffffffu, pc_wait(&my_full[s], ph, deadline));
+            dead = dead || !ok;
+            if (ok) {
+                const uint8_t *sl = my_slots + s * kSlotBytes;
+                const unsigned short *sc = reinterpret_cast<const unsigned short *>(my_scales + s * kScaleBytes);
+                const int grp0 = kb * kSG;
+#pragma unroll 4
+                for (int j = 0; j < kSG; j++) {
+                    const uint8_t *bx = sl + (j >> 2) * (kRows * kBox);
+                    const uint2 a = *reinterpret_cast<const uint2 *>(bx + off[j & 3]);
+                    const uint2 b = *reinterpret_cast<const uint2 *>(bx + off[j & 3] + 8 * kBox);
+                    float c[4];
+                    group_mma<MT>(c, a.x, a.y, b.x, b.y, xlane + (grp0 + j) * kGroupHalves);
+                    const float2 o = *reinterpret_cast<const float2 *>(d1lane + (grp0 + j) * 8);
+                    const float sa = __half2float(__ushort_as_half(sc[row * kSG + j]));
+                    const float sb = __half2float(__ushort_as_half(sc[(row + 8) * kSG + j]));
+                    acc[0] = fmaf(sa, c[0] - o.x, acc[0]);
+                    acc[1] = fmaf(sa, c[1] - o.y, acc[1]);
+                    acc[2] = fmaf(sb, c[2] - o.x, acc[2]);
+                    acc[3] = fmaf(sb, c[3] - o.y, acc[3]);
+                }
+            }
+            // Release the stage.  A warp that gave up a wait stops arriving,
+            // so its producer lane gives up too.
+            __syncwarp();
+            if (lane == 0 && !dead) mbar_arrive(&my_empty[s]);
+            if (++s == ns) {
+                s = 0;
+                ph ^= 1;
+            }
+            ++kb;
+            if (kb == B || u + 1 == r.u1) {
+                // ---- this warp's part of a tile is complete ----
+                const int tile = r.t0 + tl;
+                const bool whole = kb == B && (tl != r.u0 / B || kb_first == 0);
+                const float v0 = acc[0] * post, v1 = acc[1] * post, v2 = acc[2] * post, v3 = acc[3] * post;
+                if (whole) {
+                    if (!dead) {
+                        const int n0 = tile * kRows + row, n1 = n0 + 8;
+                        const int m0 = 2 * q, m1 = 2 * q + 1;
+                        if (m0 < M) {
+                            if (n0 < N) d.y[static_cast<size_t>(m0) * N + n0] = __float2half_rn(v0);
+                            if (n1 < N) d.y[static_cast<size_t>(m0) * N + n1] = __float2half_rn(v2);
+                        }
+                        if (m1 < M) {
+                            if (n0 < N) d.y[static_cast<size_t>(m1) * N + n0] = __float2half_rn(v1);
+                            if (n1 < N) d.y[static_cast<size_t>(m1) * N + n1] = __float2half_rn(v3);
+                        }
+                    }
+                } else {
+                    // A tile shared with neighbouring warps: keep the partial
+                    // (slot 0 = the range's first tile, slot 1 = its last).
+                    const int slot = (tl == r.u0 / B) ? 0 : 1;
+                    *reinterpret_cast<float4 *>(rec + ((warp * 2 + slot) * 32 + lane) * 4) =
+                        make_float4(v0, v1, v2, v3);
+                    if (lane == 0) rec_tile[warp * 2 + slot] = dead ? -2 : tile;
+                }
+                acc[0] = acc[1] = acc[2] = acc[3] = 0.f;
+                kb = 0;
+                tl++;
+            }
+        }
+        // ---- tiles split over several warps: summed in warp order by the
+        // first warp that holds a part ----
+        named_bar_sync(1, nthr);
+#pragma unroll 1
+        for (int slot = 0; slot < 2; slot++) {
+            const int tile = rec_tile[warp * 2 + slot];
+            if (tile < 0) continue;
+            bool owner = true;
+            for (int w2 = 0; w2 < warp; w2++)
+                if (rec_tile[w2 * 2] == tile || rec_tile[w2 * 2 + 1] == tile) owner = false;
+            if (!owner) continue;
+            float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
+            bool bad = false;
+            for (int w2 = warp; w2 < kCons; w2++) {
+                for (int s2 = 0; s2 < 2; s2++) {
+                    if (rec_tile[w2 * 2 + s2] != tile) continue;
+                    const float4 o = *reinterpret_cast<const float4 *>(rec + ((w2 * 2 + s2) * 32 + lane) * 4);
+                    sum.x += o.x; sum.y += o.y; sum.z += o.z; sum.w += o.w;
+                }
+            }
+            // a part that gave up is marked -2; then the tile is not stored
+            for (int w2 = 0; w2 < kCons; w2++)
+                if (rec_tile[w2 * 2] == -2 || rec_tile[w2 * 2 + 1] == -2) bad = true;
+            if (bad) continue;
+            const int n0 = tile * kRows + row, n1 = n0 + 8;
+            const int m0 = 2 * q, m1 = 2 * q + 1;
+            if (m0 < M) {
+                if (n0 < N) d.y[static_cast<size_t>(m0) * N + n0] = __float2half_rn(sum.x);
+                if (n1 < N) d.y[static_cast<size_t>(m0) * N + n1] = __float2half_rn(sum.z);
+            }
+            if (m1 < M) {
+                if (n0 < N) d.y[static_cast<size_t>(m1) * N + n0] = __float2half_rn(sum.y);
+                if (n1 < N) d.y[static_cast<size_t>(m1) * N + n1] = __float2half_rn(sum.w);
+            }
+        }
+    }
+}
+
+bool g_attr_pc[64][4];
+int g_occ_pc[64][4];
+
+int pc_mt(int M) { return M == 1 ? 1 : (M == 2 ? 2 : (M <= 4 ? 4 : 8)); }
+
+}  // namespace
+
+bool gemv_pc_supports(const MatDesc *md, int count, int M) {
+    if (M < 1 || M > 8) return false;
+    int kmax = 0;
+    for (int i = 0; i < count; i++) {
+        if (md[i].K % 1024 != 0) return false;
+        kmax = std::max(kmax, md[i].K);
+    }
+    // x is staged whole per CTA; at least two ring stages must fit beside it.
+    return smem_bytes(2, pc_mt(M) * kmax, kmax) <= kSmemBudget;
+}
+
+tern_status launch_gemv_pc(const MatDesc *md, int count, int M, cudaStream_t stream) {
+    DeviceInfo dev;
+    tern_status st = current_device(&dev);
+    if (st != TERN_OK) return st;
+    if (count < 1 || count > kMaxDesc) return fail(TERN_ERR_INVALID_ARG, "descriptor count %d", count);
+    if (!gemv_pc_supports(md, count, M)) return fail(TERN_ERR_SHAPE, "producer/consumer kernel: unsupported shape");
+    const int MT = pc_mt(M);
+    auto kern = MT == 1 ? gemv_pc_kernel<1> : (MT == 2 ? gemv_pc_kernel<2> : (MT == 4 ? gemv_pc_kernel<4> : gemv_pc_kernel<8>));
+    const int mi = MT == 1 ? 0 : (MT == 2 ? 1 : (MT == 4 ? 2 : 3));
+    int kmax = 0;
+    for (int i = 0; i < count; i++) kmax = std::max(kmax, md[i].K);
+    const int xs_halves = MT * kmax;
+    const size_t budget = std::min<size_t>(kSmemBudget, dev.max_smem_optin);
+    int ns = kMaxNS;
+    while (ns > 2 && smem_bytes(ns, xs_halves, kmax) > budget) ns--;
+    const size_t smem = smem_bytes(ns, xs_halves, kmax);
+    if (smem > budget) return fail(TERN_ERR_SHAPE, "needs %zu B of shared memory", smem);
+    if (!g_attr_pc[dev.device][mi]) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             static_cast<int>(dev.max_smem_optin));
+        if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(gemv pc)");
+        int occ = 0;
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, kThreads, static_cast<size_t>(kSmemBudget));
+        if (e != cudaSuccess) return cuda_fail(e, "occupancy query");
+        if (occ < 1) return fail(TERN_ERR_SHAPE, "producer/consumer kernel does not fit on an SM");
+        g_occ_pc[dev.device][mi] = occ;
+        g_attr_pc[dev.device][mi] = true;
+    }
+    // One CTA per SM (a CTA holds most of the SM's shared memory).  Each
+    // matrix gets CTAs in proportion to its slices: start from one each and
+    // hand the rest, one at a time, to the matrix whose CTAs carry the most
+    // (tiles per CTA, rounded up, x slices per tile); never more CTAs than tiles.
+    long long cap = static_cast<long long>(dev.sms);
+    if (g_opt.gemv_grid > 0) cap = std::min<long long>(cap, g_opt.gemv_grid);
+    cap = std::max<long long>(cap, count);
+    int ntile[kMaxDesc];
+    long long cl[kMaxDesc];
+    long long used = 0;
+    for (int i = 0; i < count; i++) {
+        ntile[i] = (md[i].N + kRows - 1) / kRows;
+        cl[i] = 1;
+        used++;
+    }
+    auto load = [&](int i, long long c) {
+        return ((ntile[i] + c - 1) / c) * static_cast<long long>(md[i].K / 1024);
+    };
+    while (used < cap) {
+        int worst = -1;
+        long long wv = -1;
+        for (int i = 0; i < count; i++) {
+            if (cl[i] >= ntile[i]) continue;
+            const long long l = load(i, cl[i]);
+            if (l > wv) {
+                wv = l;
+                worst = i;
+            }
+        }
+        if (worst < 0) break;
+        cl[worst]++;
+        used++;
+    }
+    // Then trim CTAs that do not lower their matrix's largest load.
+    for (int i = 0; i < count; i++)
+        while (cl[i] > 1 && load(i, cl[i] - 1) == load(i, cl[i])) cl[i]--;
+
+    PParams p;
+    std::memset(&p, 0, sizeof(p));
+    p.count = count;
+    p.M = M;
+    p.ns = ns;
+    p.kmax = kmax;
+    p.xs_halves = xs_halves;
+    p.skip_loads = g_gemm_skip_loads;
+    p.timeout_ns = g_gemm_timeout_ns;
+    int next = 0;
+    for (int i = 0; i < count; i++) {
+        PDesc &g = p.d[i];
+        st = encode_tiled_2d(&g.smap, CU_TENSOR_MAP_DATA_TYPE_UINT8, md[i].slots, static_cast<uint64_t>(md[i].K / 4),
+                             static_cast<uint64_t>(md[i].N), static_cast<uint64_t>(md[i].K / 4), kBox, kRows,
+                             CU_TENSOR_MAP_SWIZZLE_128B);
+        if (st != TERN_OK) return st;
+        const int G = md[i].K / kGroup;
+        st = encode_tiled_2d(&g.cmap, CU_TENSOR_MAP_DATA_TYPE_UINT16, md[i].scales, static_cast<uint64_t>(G),
+                             static_cast<uint64_t>(md[i].N), static_cast<uint64_t>(G) * 2, kSG, kRows,
+                             CU_TENSOR_MAP_SWIZZLE_NONE);
+        if (st != TERN_OK) return st;
+        g.x = md[i].x;
+        g.y = md[i].y;
+        g.N = md[i].N;
+        g.K = md[i].K;
+        g.B = md[i].K / 1024;
+        g.ntile = ntile[i];
+        g.c_begin = next;
+        g.c_count = static_cast<int>(cl[i]);
+        next += g.c_count;
+    }
+    cudaLaunchConfig_t cfg;
+    std::memset(&cfg, 0, sizeof(cfg));
+    cfg.gridDim = dim3(static_cast<unsigned>(next));
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, kern, p);
+    if (e != cudaSuccess) return cuda_fail(e, "gemv pc kernel launch");
+    return TERN_OK;
+}
+
+tern_status read_gemvpc_status(bool reset, unsigned int *out) {
+    unsigned int v = 0;
+    cudaError_t e = cudaMemcpyFromSymbol(&v, g_tern_gemvpc_status, sizeof(v));
+    if (e != cudaSuccess) return cuda_fail(e, "reading device status");
+    if (reset && v != 0) {
+        const unsigned int zero = 0;
+        e = cudaMemcpyToSymbol(g_tern_gemvpc_status, &zero, sizeof(zero));
+        if (e != cudaSuccess) return cuda_fail(e, "clearing device status");
+    }
+    *out = v;
+    return TERN_OK;
+}
+
+}  // namespace tern

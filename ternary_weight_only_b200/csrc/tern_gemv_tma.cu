@@ -335,14 +335,86 @@ __global__ void __launch_bounds__(kThreads, MINB) gemv_tma_kernel(const __grid_c
 bool g_attr_done[64][8];
 int g_occ[64][8][256];
 
-// Per-CTA work (slices per warp) of matrix i with P warps per tile and c clusters.
-long long cta_work(int ntile, int nb_cta, int P, long long c) {
-    const long long spc = kWarps / P;
+}  // namespace
+
+namespace {
+// Per-CTA work (slices per warp) with P warps per tile and c CTAs (clusters).
+long long cta_work(int ntile, int nb_cta, int P, long long c, int warps) {
+    const long long spc = warps / P;
     const long long rounds = (ntile + c * spc - 1) / (c * spc);
     return rounds * ((nb_cta + P - 1) / P);
 }
-
 }  // namespace
+
+tern_status plan_partition(const int *ntile, const int *nbc, const int *nbmin, int count, int warps,
+                           long long cap, int forced_P, int *Pout, long long *cl_out) {
+    // For every matrix choose P (warps per 16-row tile, a divisor of `warps`) and its
+    // CTA count so that the largest per-CTA work is as small as possible with
+    // at most `cap` CTAs (clusters) in total: binary search on that bound, then
+    // hand leftover CTAs to the matrices whose CTAs work longest.
+    auto best_for = [&](int i, long long tau, int *Pc) -> long long {
+        long long best = -1;
+        for (int P = 1; P <= warps; P++) {
+            if (warps % P != 0) continue;  // every slot of P warps is whole
+            if (forced_P > 0 && P != forced_P) continue;
+            if (P > nbmin[i]) continue;  // every warp's part keeps at least one slice
+            const long long per_tile = (nbc[i] + P - 1) / P;
+            if (per_tile > tau) continue;
+            const long long rounds = tau / per_tile;
+            const long long spc = warps / P;
+            const long long c = (ntile[i] + rounds * spc - 1) / (rounds * spc);
+            if (best < 0 || c < best || (c == best && P > *Pc)) {
+                best = c;
+                *Pc = P;
+            }
+        }
+        return best;
+    };
+    long long lo = 1, hi = 1;
+    for (int i = 0; i < count; i++) hi = std::max<long long>(hi, static_cast<long long>(ntile[i]) * nbc[i]);
+    while (lo < hi) {
+        const long long mid = (lo + hi) / 2;
+        long long need = 0;
+        bool ok = true;
+        for (int i = 0; i < count && ok; i++) {
+            int P = 1;
+            const long long c = best_for(i, mid, &P);
+            if (c < 0) ok = false;
+            else need += c;
+        }
+        if (ok && need <= cap) hi = mid;
+        else lo = mid + 1;
+    }
+    long long used = 0;
+    for (int i = 0; i < count; i++) {
+        int P = 1;
+        const long long c = best_for(i, lo, &P);
+        if (c < 0) return fail(TERN_ERR_SHAPE, "no valid k split for matrix %d", i);
+        Pout[i] = P;
+        cl_out[i] = c;
+        used += c;
+    }
+    while (used < cap) {
+        int worst = -1;
+        long long wv = -1;
+        for (int i = 0; i < count; i++) {
+            const long long w = cta_work(ntile[i], nbc[i], Pout[i], cl_out[i], warps);
+            const long long spc = warps / Pout[i];
+            if (cl_out[i] * spc >= ntile[i]) continue;  // already one tile per slot
+            if (w > wv) {
+                wv = w;
+                worst = i;
+            }
+        }
+        if (worst < 0) break;
+        const long long before = cta_work(ntile[worst], nbc[worst], Pout[worst], cl_out[worst], warps);
+        const long long after = cta_work(ntile[worst], nbc[worst], Pout[worst], cl_out[worst] + 1, warps);
+        if (after >= before) break;
+        cl_out[worst]++;
+        used++;
+    }
+    return TERN_OK;
+}
 
 tern_status launch_gemv_tma(const MatDesc *md, int count, int M, cudaStream_t stream) {
     DeviceInfo dev;
@@ -397,77 +469,16 @@ tern_status launch_gemv_tma(const MatDesc *md, int count, int M, cudaStream_t st
     if (g_opt.gemv_ctas > 0) occ = std::min(occ, g_opt.gemv_ctas);
     const long long cap = std::max<long long>(count, static_cast<long long>(dev.sms) * occ / S);
 
-    // For every matrix choose P (warps per tile) and its cluster count so that
-    // the largest per-CTA work is as small as possible with at most `cap`
-    // clusters in total: binary search on that work bound.
-    int ntile[kMaxDesc], nbc[kMaxDesc];
+    int ntile[kMaxDesc], nbc[kMaxDesc], nbmin[kMaxDesc], Pch[kMaxDesc];
+    long long cl_count[kMaxDesc];
     for (int i = 0; i < count; i++) {
         ntile[i] = (md[i].N + kSliceRows - 1) / kSliceRows;
         const int B = (md[i].K / kGroup + kSliceGroups - 1) / kSliceGroups;
         nbc[i] = (B + S - 1) / S;  // slices of the widest CTA range
+        nbmin[i] = B / S;          // ... and of the narrowest
     }
-    auto best_for = [&](int i, long long tau, int *Pout) -> long long {
-        long long best = -1;
-        for (int P = 1; P <= kWarps; P *= 2) {
-            if (g_opt.gemv_ksplit > 0 && P != g_opt.gemv_ksplit) continue;
-            if (P * S > (md[i].K / kGroup + kSliceGroups - 1) / kSliceGroups) continue;
-            const long long per_tile = (nbc[i] + P - 1) / P;
-            if (per_tile > tau) continue;
-            const long long rounds = tau / per_tile;
-            const long long spc = kWarps / P;
-            const long long c = (ntile[i] + rounds * spc - 1) / (rounds * spc);
-            if (best < 0 || c < best || (c == best && P > *Pout)) {
-                best = c;
-                *Pout = P;
-            }
-        }
-        return best;
-    };
-    long long lo = 1, hi = 1;
-    for (int i = 0; i < count; i++) hi = std::max<long long>(hi, static_cast<long long>(ntile[i]) * nbc[i]);
-    int Pch[kMaxDesc];
-    while (lo < hi) {
-        const long long mid = (lo + hi) / 2;
-        long long need = 0;
-        bool ok = true;
-        for (int i = 0; i < count && ok; i++) {
-            int P = 1;
-            const long long c = best_for(i, mid, &P);
-            if (c < 0) ok = false;
-            else need += c;
-        }
-        if (ok && need <= cap) hi = mid;
-        else lo = mid + 1;
-    }
-    long long used = 0, cl_count[kMaxDesc];
-    for (int i = 0; i < count; i++) {
-        int P = 1;
-        long long c = best_for(i, lo, &P);
-        if (c < 0) return fail(TERN_ERR_SHAPE, "no valid k split for matrix %d (K=%d)", i, md[i].K);
-        Pch[i] = P;
-        cl_count[i] = c;
-        used += c;
-    }
-    // Spread leftover clusters over the matrices whose CTAs work longest.
-    while (used < cap) {
-        int worst = -1;
-        long long wv = -1;
-        for (int i = 0; i < count; i++) {
-            const long long w = cta_work(ntile[i], nbc[i], Pch[i], cl_count[i]);
-            const long long spc = kWarps / Pch[i];
-            if (cl_count[i] * spc >= ntile[i]) continue;  // already one tile per slot
-            if (w > wv) {
-                wv = w;
-                worst = i;
-            }
-        }
-        if (worst < 0) break;
-        const long long before = cta_work(ntile[worst], nbc[worst], Pch[worst], cl_count[worst]);
-        const long long after = cta_work(ntile[worst], nbc[worst], Pch[worst], cl_count[worst] + 1);
-        if (after >= before) break;
-        cl_count[worst]++;
-        used++;
-    }
+    st = plan_partition(ntile, nbc, nbmin, count, kWarps, cap, g_opt.gemv_ksplit, Pch, cl_count);
+    if (st != TERN_OK) return st;
 
     TParams p;  // copied into the launch by cudaLaunchKernelEx
     std::memset(&p, 0, sizeof(p));

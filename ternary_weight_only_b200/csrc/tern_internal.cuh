@@ -34,6 +34,7 @@ struct Options {
     int gemm_path = 0;
     int gemm_min_m = 0;
     int gemv_variant = 0;
+    int gemv_grid = 0;
 };
 extern Options g_opt;
 
@@ -54,6 +55,9 @@ struct MatDesc {
 // Bandwidth-bound product for M in [1,8] over `count` matrices in one launch:
 // TMA-staged kernel (default) and the register-ring kernel (variant 1).
 tern_status launch_gemv_tma(const MatDesc *d, int count, int M, cudaStream_t stream);
+// Producer/consumer form of the same kernel (K a multiple of 1024, x small).
+bool gemv_pc_supports(const MatDesc *d, int count, int M);
+tern_status launch_gemv_pc(const MatDesc *d, int count, int M, cudaStream_t stream);
 // Tensor-core (tcgen05) bandwidth kernel for M in [1,4]; splits tiles along K
 // when a large enough zero-initialised workspace is given.
 tern_status launch_gemv_tc(const MatDesc *d, int count, int M, void *workspace, size_t ws_bytes,
@@ -62,6 +66,12 @@ size_t gemv_tc_workspace_bytes(const MatDesc *d, int count, int M, int sms);
 // M = 1 product of the tcgen05 kernel with its scratch in a static device area.
 tern_status gemv_noalloc(const MatDesc &d, cudaStream_t stream);
 tern_status launch_gemv_mma(const MatDesc *d, int count, int M, cudaStream_t stream);
+// Partition of a grouped bandwidth launch: for each matrix i with ntile[i]
+// 16-row tiles and between nbmin[i] and nbc[i] k-slices per CTA, choose
+// Pout[i] warps per tile (power of two, <= nbmin[i]) and cl_out[i] CTAs (or
+// clusters) within `cap` in total (see tern_gemv_tma.cu).
+tern_status plan_partition(const int *ntile, const int *nbc, const int *nbmin, int count, int warps,
+                           long long cap, int forced_P, int *Pout, long long *cl_out);
 // 2-D tiled tensor map (row-major: `inner` contiguous elements per row, `outer`
 // rows `row_bytes` apart) for TMA loads of `box_inner` x `box_outer` boxes.
 tern_status encode_tiled_2d(CUtensorMap *map, CUtensorMapDataType dt, const void *base, uint64_t inner,
@@ -74,6 +84,7 @@ tern_status launch_gemm_tc(const MatDesc &d, int M, cudaStream_t stream);
 tern_status read_gemm_status(bool reset, unsigned int *out);
 tern_status read_gemv_status(bool reset, unsigned int *out);
 tern_status read_gemvtc_status(bool reset, unsigned int *out);
+tern_status read_gemvpc_status(bool reset, unsigned int *out);
 extern unsigned long long g_gemm_timeout_ns;
 extern int g_gemm_skip_loads;
 

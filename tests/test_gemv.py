@@ -210,14 +210,16 @@ def test_timeout_path_reports_and_recovers(T, orc):
 
 
 def test_grid_cap(T, orc):
-    """Few resident CTAs: every CTA walks many tiles."""
+    """TMA-staged kernel with few resident CTAs: every CTA walks many tiles."""
     from ternary_weight_only_b200 import synth
     x, codes, scales = synth.case(1, 1024, 4000, seed=3, codes="sparse")
+    T.tern_set_option(T.TERN_OPT_GEMV_VARIANT, 2)
     T.tern_set_option(T.TERN_OPT_GEMV_CTAS, 1)
     try:
         run_case(T, orc, x, codes, scales, "one CTA per SM")
     finally:
         T.tern_set_option(T.TERN_OPT_GEMV_CTAS, 0)
+        T.tern_set_option(T.TERN_OPT_GEMV_VARIANT, 0)
 
 
 def test_exact_special_cases(T, orc):
@@ -321,3 +323,122 @@ def test_stream_argument(T, orc):
     s.synchronize()
     y_ref, bound = orc.matmul(xn, slots, sc)
     check_close(y, y_ref, bound, "side stream")
+
+
+@pytest.fixture
+def pc(T):
+    """Select the producer/consumer bandwidth kernel (K a multiple of 1024)."""
+    T.tern_set_option(T.TERN_OPT_GEMV_VARIANT, 4)
+    yield T
+    T.tern_set_option(T.TERN_OPT_GEMV_VARIANT, 0)
+
+
+@pytest.mark.parametrize("M", [1, 2, 4, 8])
+@pytest.mark.parametrize("i", range(7))
+def test_producer_consumer_layer(pc, orc, i, M):
+    from ternary_weight_only_b200 import synth
+    x, codes, scales = synth.decode_proj(i, M=M)
+    run_case(pc, orc, x, codes, scales, f"pc {synth.LAYER_PROJ[i][0]} M={M}")
+
+
+@pytest.mark.parametrize("grid", [0, 1, 5, 37])
+@pytest.mark.parametrize("M,K,N", [(1, 1024, 17), (1, 17408, 1000), (2, 5120, 4000), (3, 2048, 250),
+                                   (1, 20480, 33), (8, 2048, 129), (1, 12288, 5000), (4, 3072, 7)])
+def test_producer_consumer_grids(pc, orc, grid, M, K, N):
+    """Capped grids give each CTA many tiles, whose (tile, slice) units its
+    twelve warps split evenly: tiles shared by neighbouring warps are summed
+    at the end of the CTA."""
+    from ternary_weight_only_b200 import synth
+    x, codes, scales = synth.case(M, K, N, seed=grid * 31 + M + K + N, codes="sparse", outlier_p=0.01)
+    pc.tern_set_option(pc.TERN_OPT_GEMV_GRID, grid)
+    try:
+        run_case(pc, orc, x, codes, scales, f"pc grid={grid} M={M} K={K} N={N}")
+    finally:
+        pc.tern_set_option(pc.TERN_OPT_GEMV_GRID, 0)
+
+
+@pytest.mark.parametrize("grid", [0, 7, 30])
+def test_producer_consumer_layer_grids(pc, orc, grid):
+    """A grouped decode layer (K = 5120, 6144 and 17408: 5, 6 and 17 slices
+    of 1024 per row) on full and capped grids, twice in a row."""
+    from ternary_weight_only_b200 import synth
+    mats, refs = [], []
+    for i in range(7):
+        x, codes, scales = synth.decode_proj(i, M=2)
+        xn, cn, sn = np_inputs(x, codes, scales)
+        slots, sc, _, _ = orc.pack(cn, sn)
+        y = torch.full((2, codes.shape[0]), float("nan"), dtype=torch.float16, device="cuda")
+        mats.append((x.cuda(), torch.from_numpy(slots).cuda(), scales.cuda(), y))
+        refs.append((xn, slots, sc))
+    pc.tern_set_option(pc.TERN_OPT_GEMV_GRID, grid)
+    try:
+        for _ in range(2):
+            pc.tern_gemv_grouped(mats, 2)
+        pc.tern_sync_status()
+    finally:
+        pc.tern_set_option(pc.TERN_OPT_GEMV_GRID, 0)
+    for i, ((xn, slots, sc), m) in enumerate(zip(refs, mats)):
+        y_ref, bound = orc.matmul(xn, slots, sc, threads=NCPU)
+        check_close(m[3], y_ref, bound, f"pc grid={grid} {synth.LAYER_PROJ[i][0]}")
+
+
+def test_producer_consumer_exact_cases(pc, orc):
+    """All-zero weights give exactly zero; one-hot x gives s * t exactly; large
+    activations (|x| > 256, where the staged x is scaled down) stay in bound."""
+    from ternary_weight_only_b200 import synth
+    N, K = 64, 2048
+    g = synth.gen(99, "cuda")
+    scales = synth.scales_uniform(N, K, g, device="cuda")
+    x = synth.activations(1, K, g, device="cuda")
+    codes = torch.zeros((N, K), dtype=torch.int8, device="cuda")  # t = 0 everywhere
+    slots, sc = pc.tern_pack_g128(codes, scales)
+    y = pc.tern_gemv(x[0], slots, sc)
+    pc.tern_sync_status()
+    assert bool(torch.all(y == 0)), y.abs().max()
+    codes = synth.codes_uniform(N, K, g, device="cuda")
+    slots, sc = pc.tern_pack_g128(codes, scales)
+    for k in (0, 1, 7, 8, 15, 127, 128, 1000, 2047):
+        xe = torch.zeros(K, dtype=torch.float16, device="cuda")
+        xe[k] = 3.0
+        y = pc.tern_gemv(xe, slots, sc)
+        want = (3.0 * scales[:, k // 128].float() * codes[:, k].float()).half()
+        assert torch.equal(y, want), (k, (y.float() - want.float()).abs().max())
+    for amp in (300.0, 20000.0):
+        xb = (x.float() * amp / x.float().abs().max()).half()
+        y = pc.tern_gemv(xb[0], slots, sc)
+        xn, cn, sn = np_inputs(xb.cpu(), codes.cpu(), scales.cpu())
+        ref_slots, ref_sc, _, _ = orc.pack(cn, sn)
+        y_ref, bound = orc.matmul(xn, ref_slots, ref_sc, threads=NCPU)
+        check_close(y.view(1, -1), y_ref, bound, f"pc |x| up to {amp}")
+    pc.tern_sync_status()
+
+
+def test_producer_consumer_grouped_and_timeout(pc, orc):
+    from ternary_weight_only_b200 import synth
+    mats, refs = [], []
+    for i in range(7):
+        x, codes, scales = synth.decode_proj(i, M=1)
+        xn, cn, sn = np_inputs(x, codes, scales)
+        slots, sc, _, _ = orc.pack(cn, sn)
+        y = torch.full((1, codes.shape[0]), float("nan"), dtype=torch.float16, device="cuda")
+        mats.append((x.cuda(), torch.from_numpy(slots).cuda(), scales.cuda(), y))
+        refs.append((xn, slots, sc))
+    pc.tern_gemv_grouped(mats, 1)
+    pc.tern_sync_status()
+    for i, ((xn, slots, sc), m) in enumerate(zip(refs, mats)):
+        y_ref, bound = orc.matmul(xn, slots, sc, threads=NCPU)
+        check_close(m[3], y_ref, bound, f"pc grouped {synth.LAYER_PROJ[i][0]}")
+    # a wait that can never complete gives up, is reported, and the context survives
+    pc.tern_set_option(pc.TERN_OPT_TEST_STALL_US, 2000)
+    try:
+        pc.tern_gemv_grouped(mats, 1)
+        with pytest.raises(pc.TernError) as ei:
+            pc.tern_sync_status()
+        assert ei.value.status == pc.TERN_ERR_TIMEOUT
+    finally:
+        pc.tern_set_option(pc.TERN_OPT_TEST_STALL_US, 0)
+    pc.tern_gemv_grouped(mats, 1)
+    pc.tern_sync_status()
+    xn, slots, sc = refs[4]
+    y_ref, bound = orc.matmul(xn, slots, sc, threads=NCPU)
+    check_close(mats[4][3], y_ref, bound, "pc after timeout")
