@@ -227,7 +227,9 @@ tern_status tern_sync_status(void *stream);
  *                          block cluster and distributed shared memory (1,2,4,8)
  *   TERN_OPT_GEMV_CTAS     cap on resident CTAs per SM used for the grid; for
  *                          the TMA-staged kernel 3 also selects the build with
- *                          the smaller register budget (default: 2 per SM)
+ *                          the smaller register budget (default: 2 per SM);
+ *                          for the tensor-memory kernel 1 selects one
+ *                          warpgroup per CTA instead of two
  *   TERN_OPT_GEMM_PATH     1 = force the bandwidth kernel (M<=8 chunks),
  *                          2 = force the tensor-core kernel
  *   TERN_OPT_GEMM_MIN_M    smallest M (> 8) sent to the tensor-core kernel
@@ -239,8 +241,12 @@ tern_status tern_sync_status(void *stream);
  *                          workspace), 4 = producer/consumer mma.sync kernel
  *                          for K a multiple of 1024 (one CTA per SM, one
  *                          logic operation per weight pair; other shapes take
- *                          the default kernel); all kept for comparison
- *   TERN_OPT_GEMV_GRID     cap on the CTAs of the producer/consumer kernel
+ *                          the default kernel), 5 = tensor-memory kernel for K
+ *                          a multiple of 1024 (tcgen05, weights unpacked
+ *                          into tensor memory by one thread per row); all
+ *                          kept for comparison
+ *   TERN_OPT_GEMV_GRID     cap on the CTAs of the producer/consumer and
+ *                          tensor-memory kernels
  *                          (0 = one per SM); smaller grids give every CTA
  *                          more tiles to split among its warps
  *   TERN_OPT_TEST_STALL_US TESTS ONLY: the TMA loaders of the tensor-core and

@@ -68,9 +68,8 @@ std::once_flag g_encode_once;
 cudaError_t g_encode_err = cudaSuccess;
 }  // namespace
 
-tern_status encode_tiled_2d(CUtensorMap *map, CUtensorMapDataType dt, const void *base, uint64_t inner,
-                            uint64_t outer, uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer,
-                            CUtensorMapSwizzle swizzle) {
+// Resolves cuTensorMapEncodeTiled from the driver once per process.
+static bool resolve_encode() {
     std::call_once(g_encode_once, [] {
         void *fn = nullptr;
         cudaDriverEntryPointQueryResult q;
@@ -78,7 +77,13 @@ tern_status encode_tiled_2d(CUtensorMap *map, CUtensorMapDataType dt, const void
         if (g_encode_err == cudaSuccess && q == cudaDriverEntryPointSuccess)
             g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
     });
-    if (!g_encode)
+    return g_encode != nullptr;
+}
+
+tern_status encode_tiled_2d(CUtensorMap *map, CUtensorMapDataType dt, const void *base, uint64_t inner,
+                            uint64_t outer, uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer,
+                            CUtensorMapSwizzle swizzle) {
+    if (!resolve_encode())
         return fail(TERN_ERR_CUDA, "cuTensorMapEncodeTiled unavailable (%s)", cudaGetErrorString(g_encode_err));
     std::memset(map, 0, sizeof(*map));
     const cuuint64_t dims[2] = {inner, outer};
@@ -89,6 +94,21 @@ tern_status encode_tiled_2d(CUtensorMap *map, CUtensorMapDataType dt, const void
                           CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return fail(TERN_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
+    return TERN_OK;
+}
+
+tern_status encode_tiled_3d(CUtensorMap *map, CUtensorMapDataType dt, const void *base, const uint64_t dims[3],
+                            const uint64_t strides[2], const uint32_t box[3], CUtensorMapSwizzle swizzle) {
+    if (!resolve_encode())
+        return fail(TERN_ERR_CUDA, "cuTensorMapEncodeTiled unavailable (%s)", cudaGetErrorString(g_encode_err));
+    std::memset(map, 0, sizeof(*map));
+    const cuuint64_t d[3] = {dims[0], dims[1], dims[2]};
+    const cuuint64_t str[2] = {strides[0], strides[1]};
+    const cuuint32_t bx[3] = {box[0], box[1], box[2]};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = g_encode(map, dt, 3, const_cast<void *>(base), d, str, bx, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                          swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(TERN_ERR_CUDA, "cuTensorMapEncodeTiled (3-D) failed (%d)", static_cast<int>(r));
     return TERN_OK;
 }
 
@@ -137,7 +157,7 @@ int planning_sms() {
 
 // Bandwidth kernels (M <= 8).  Default: the TMA-staged mma.sync kernel,
 // the fastest measured so far; the knob selects the others for comparison.
-enum { kVarDefault = 0, kVarRing = 1, kVarTma = 2, kVarTc = 3, kVarPc = 4 };
+enum { kVarDefault = 0, kVarRing = 1, kVarTma = 2, kVarTc = 3, kVarPc = 4, kVarTmem = 5 };
 
 bool use_tc(int M) { return g_opt.gemv_variant == kVarTc && M <= 4; }
 
@@ -145,6 +165,7 @@ tern_status launch_bandwidth(const MatDesc *d, int count, int M, void *workspace
                              cudaStream_t s) {
     if (g_opt.gemv_variant == kVarRing) return launch_gemv_mma(d, count, M, s);
     if (use_tc(M)) return launch_gemv_tc(d, count, M, workspace, ws_bytes, s);
+    if (g_opt.gemv_variant == kVarTmem && gemv_tmem_supports(d, count, M)) return launch_gemv_tmem(d, count, M, s);
     // Default: the producer/consumer kernel where its shape rules hold (K a
     // multiple of 1024, x fits its shared memory), else the TMA-staged one.
     if ((g_opt.gemv_variant == kVarPc || g_opt.gemv_variant == kVarDefault) && gemv_pc_supports(d, count, M))
@@ -329,9 +350,13 @@ tern_status tern_sync_status(void *stream) {
     unsigned int z = 0;
     st = read_gemvpc_status(true, &z);
     if (st != TERN_OK) return st;
+    unsigned int t5 = 0;
+    st = read_gemvtm_status(true, &t5);
+    if (st != TERN_OK) return st;
     if (v == 0) v = w;
     if (v == 0) v = u;
     if (v == 0) v = z;
+    if (v == 0) v = t5;
     if (v != 0) return fail(static_cast<tern_status>(v), "a kernel gave up a bounded wait on the device");
     return TERN_OK;
 }
@@ -349,7 +374,7 @@ tern_status tern_set_option(int option, int64_t value) {
             return TERN_OK;
         case TERN_OPT_GEMM_MIN_M: g_opt.gemm_min_m = static_cast<int>(value); return TERN_OK;
         case TERN_OPT_GEMV_VARIANT:
-            if (value > 4) return fail(TERN_ERR_INVALID_ARG, "gemv variant %lld", static_cast<long long>(value));
+            if (value > 5) return fail(TERN_ERR_INVALID_ARG, "gemv variant %lld", static_cast<long long>(value));
             g_opt.gemv_variant = static_cast<int>(value);
             return TERN_OK;
         case TERN_OPT_GEMV_GRID: g_opt.gemv_grid = static_cast<int>(value); return TERN_OK;

@@ -58,7 +58,7 @@ constexpr size_t kSmemBudget = 232448;          // opt-in shared memory per bloc
 constexpr int kMaxDesc = TERN_MAX_GROUP;
 
 struct alignas(64) PDesc {
-    CUtensorMap smap;   // slots uint8 [N][K/4], box 128 B x 16 rows, 128-byte swizzle
+    CUtensorMap smap;   // slots as uint8 [K/512][N][128], box 128 B x 16 rows x 2, 128-byte swizzle
     CUtensorMap cmap;   // scales fp16 [N][K/128], box 8 x 16, no swizzle
     const __half *x;    // [M][K]
     __half *y;          // [M][N]
@@ -79,7 +79,7 @@ struct PParams {
 
 size_t smem_bytes(int ns, int xs_halves, int kmax) {
     return 1024 + static_cast<size_t>(kCons) * ns * (kSlotBytes + kScaleBytes) + kBarBytes + kRecBytes + 160 +
-           static_cast<size_t>(kmax / kGroupK) * 8 * 4 + static_cast<size_t>(xs_halves) * 2;
+           (static_cast<size_t>(kmax / kGroupK) * 8 + 16) * 4 + static_cast<size_t>(xs_halves) * 2;
 }
 
 constexpr uint32_t kOnes = 0x55555555u;  // every 2-bit field = code 1 (t = 0)
@@ -118,9 +118,9 @@ __device__ __forceinline__ int xs_pair_index(int m, int kl) {
 
 // The eight mmas of one 16-row x 128-k group: pair j of the lane's words
 // (a = row g, b = row g+8; .x = word 2q, .y = word 2q+1) against the staged x
-// of pair j, as two independent chains (pairs 0-3 and 4-7) added at the end.
-// Shared by the weight path and the all-ones pass, so the two round
-// identically.
+// of pair j, one accumulation chain (the unrolled groups of a slice give the
+// scheduler independent chains).  Shared by the weight path and the all-ones
+// pass, so the two round identically.
 template <int MT>
 __device__ __forceinline__ void group_mma(float (&c)[4], uint32_t ax, uint32_t ay, uint32_t bx, uint32_t by,
                                           const __half *xb) {
@@ -130,19 +130,14 @@ __device__ __forceinline__ void group_mma(float (&c)[4], uint32_t ax, uint32_t a
     const uint4 x2 = *reinterpret_cast<const uint4 *>(xb + 2 * kChunk);
     const uint4 x3 = *reinterpret_cast<const uint4 *>(xb + 3 * kChunk);
     const uint32_t ax5 = ax >> 10, ay5 = ay >> 10, bx5 = bx >> 10, by5 = by >> 10;
-    float e[4];
     mma_zero(c, ax & 0x00030003u, bx & 0x00030003u, ay & 0x00030003u, by & 0x00030003u, x0.x, x0.y);
-    mma_zero(e, ax & 0x03000300u, bx & 0x03000300u, ay & 0x03000300u, by & 0x03000300u, x2.x, x2.y);
     mma_acc(c, ax & 0x000C000Cu, bx & 0x000C000Cu, ay & 0x000C000Cu, by & 0x000C000Cu, x0.z, x0.w);
-    mma_acc(e, ax5 & 0x00030003u, bx5 & 0x00030003u, ay5 & 0x00030003u, by5 & 0x00030003u, x2.z, x2.w);
     mma_acc(c, ax & 0x00300030u, bx & 0x00300030u, ay & 0x00300030u, by & 0x00300030u, x1.x, x1.y);
-    mma_acc(e, ax5 & 0x000C000Cu, bx5 & 0x000C000Cu, ay5 & 0x000C000Cu, by5 & 0x000C000Cu, x3.x, x3.y);
     mma_acc(c, ax & 0x00C000C0u, bx & 0x00C000C0u, ay & 0x00C000C0u, by & 0x00C000C0u, x1.z, x1.w);
-    mma_acc(e, ax5 & 0x00300030u, bx5 & 0x00300030u, ay5 & 0x00300030u, by5 & 0x00300030u, x3.z, x3.w);
-    c[0] += e[0];
-    c[1] += e[1];
-    c[2] += e[2];
-    c[3] += e[3];
+    mma_acc(c, ax & 0x03000300u, bx & 0x03000300u, ay & 0x03000300u, by & 0x03000300u, x2.x, x2.y);
+    mma_acc(c, ax5 & 0x00030003u, bx5 & 0x00030003u, ay5 & 0x00030003u, by5 & 0x00030003u, x2.z, x2.w);
+    mma_acc(c, ax5 & 0x000C000Cu, bx5 & 0x000C000Cu, ay5 & 0x000C000Cu, by5 & 0x000C000Cu, x3.x, x3.y);
+    mma_acc(c, ax5 & 0x00300030u, bx5 & 0x00300030u, ay5 & 0x00300030u, by5 & 0x00300030u, x3.z, x3.w);
 }
 
 __device__ __forceinline__ bool mbar_test_wait(uint64_t *bar, uint32_t parity) {
@@ -196,8 +191,10 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_pc_kernel(const __grid_const
     float *rec = reinterpret_cast<float *>(empty + kCons * kMaxNS);  // [kCons][2][32][4] partial tiles
     int *rec_tile = reinterpret_cast<int *>(rec + kCons * 2 * 32 * 4);  // [kCons][2]
     unsigned int *wmax = reinterpret_cast<unsigned int *>(rec_tile + 2 * kCons);  // [kCons]
-    float *d1 = reinterpret_cast<float *>(wmax + 16);            // [K/128][8]
-    __half *xs = reinterpret_cast<__half *>(d1 + (p.kmax / kGroupK) * 8);
+    // [lane q][2 G + 4]: two floats per group, rows padded so that the four
+    // lanes q of a quarter warp read distinct banks
+    float *d1 = reinterpret_cast<float *>(wmax + 16);
+    __half *xs = reinterpret_cast<__half *>(d1 + (p.kmax / kGroupK) * 8 + 16);
 
     const int M = p.M;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -217,6 +214,10 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_pc_kernel(const __grid_const
     }
     __syncthreads();
     const unsigned long long deadline = globaltimer() + p.timeout_ns;
+    // Programmatic dependent launch: the next launch in the stream may start
+    // its CTAs as SMs free up.  It prefetches only weights (which no GEMV
+    // writes) before its grid-dependency wait, and reads x and writes y after.
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
     if (warp == kCons) {
         // ======================= producer warp =======================
@@ -242,9 +243,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_pc_kernel(const __grid_const
                     const int tile = r.t0 + u / B;
                     const int kbx = u - (u / B) * B;
                     mbar_expect_tx(&my_full[s], kSlotBytes + kScaleBytes);
-                    tma_load_2d(my_slots + s * kSlotBytes, &d.smap, kbx * 2 * kBox, tile * kRows, &my_full[s]);
-                    tma_load_2d(my_slots + s * kSlotBytes + kRows * kBox, &d.smap, kbx * 2 * kBox + kBox,
-                                tile * kRows, &my_full[s]);
+                    tma_load_3d(my_slots + s * kSlotBytes, &d.smap, 0, tile * kRows, kbx * 2, &my_full[s]);
                     tma_load_2d(my_scales + s * kScaleBytes, &d.cmap, kbx * kSG, tile * kRows, &my_full[s]);
                     issued++;
                     if (++s == ns) {
@@ -272,6 +271,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_pc_kernel(const __grid_const
         // ======================= consumer warps =======================
         const int K = d.K, N = d.N;
         const int nthr = kCons * 32;
+        // x may be the output of the preceding launch: wait for it to finish.
+        asm volatile("griddepcontrol.wait;" ::: "memory");
         // (1) E from the largest finite |x| of all token rows.
         {
             unsigned int mx = 0;
@@ -279,11 +280,9 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_pc_kernel(const __grid_const
                 const uint4 v = *reinterpret_cast<const uint4 *>(d.x + static_cast<size_t>(idx) * 8);
                 const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-                for (int e = 0; e < 4; e++) {
-                    mx = max(mx, min(wv[e] & 0x7FFFu, 0x7BFFu));
-                    mx = max(mx, min((wv[e] >> 16) & 0x7FFFu, 0x7BFFu));
-                }
+                for (int e = 0; e < 4; e++) mx = __vmaxu2(mx, __vminu2(wv[e] & 0x7FFF7FFFu, 0x7BFF7BFFu));
             }
+            mx = max(mx & 0xFFFFu, mx >> 16);
             mx = __reduce_max_sync(0xffffffffu, mx);
             if (lane == 0) wmax[warp] = mx;
             if (lane < 2) rec_tile[warp * 2 + lane] = -1;
@@ -297,18 +296,29 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_pc_kernel(const __grid_const
         const int E = min(8, 15 - ex);
         // (2) stage x in pair order, pair j scaled by 2^(E - 2j').
         {
-            float fac[8];
+            // factor pairs for elements (2i, 2i+1) of an 8-element run: 2^(E - 2j'),
+            // as fp16x2 (exact powers of two); the multiply rounds only subnormal results
+            uint32_t fac2[4];
 #pragma unroll
-            for (int j = 0; j < 8; j++) fac[j] = ldexpf(1.0f, E - 2 * (j < 5 ? j : j - 5));
+            for (int i = 0; i < 4; i++) {
+                const int e0 = E - 2 * (2 * i < 5 ? 2 * i : 2 * i - 5);
+                const int e1 = E - 2 * (2 * i + 1 < 5 ? 2 * i + 1 : 2 * i + 1 - 5);
+                fac2[i] = (static_cast<uint32_t>(15 + e0) << 10) | (static_cast<uint32_t>(15 + e1) << 26);
+            }
             const int per_m = K / 8;
             for (int idx = threadIdx.x; idx < M * per_m; idx += nthr) {
                 const int m = idx / per_m, c8 = idx - m * per_m;
                 const uint4 v = *reinterpret_cast<const uint4 *>(d.x + static_cast<size_t>(m) * K + c8 * 8);
-                const __half *hv = reinterpret_cast<const __half *>(&v);
-                __half *dst = xs + xs_pair_index<MT>(m, c8 * 8);  // element e: chunk e/2, slot (e&1)*4
+                const uint32_t pr[4] = {v.x, v.y, v.z, v.w};
+                unsigned short *dst = reinterpret_cast<unsigned short *>(xs + xs_pair_index<MT>(m, c8 * 8));
 #pragma unroll
-                for (int e = 0; e < 8; e++)
-                    dst[(e >> 1) * MT * 32 + (e & 1) * 4] = __float2half_rn(__half2float(hv[e]) * fac[e]);
+                for (int i = 0; i < 4; i++) {
+                    uint32_t h2;
+                    asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(h2) : "r"(pr[i]), "r"(fac2[i]));
+                    // element e = 2i + t lands at chunk e / 2 = i, slot t * 4
+                    dst[i * MT * 32] = static_cast<unsigned short>(h2);
+                    dst[i * MT * 32 + 4] = static_cast<unsigned short>(h2 >> 16);
+                }
             }
         }
         named_bar_sync(1, nthr);
@@ -321,7 +331,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_pc_kernel(const __grid_const
         for (int grp = warp; grp < G; grp += kCons) {
             float c[4];
             group_mma<MT>(c, kOnes, kOnes, kOnes, kOnes, xlane + grp * kGroupHalves);
-            if (g == 0) *reinterpret_cast<float2 *>(d1 + grp * 8 + 2 * q) = make_float2(c[0], c[1]);
+            if (g == 0) *reinterpret_cast<float2 *>(d1 + q * (2 * G + 4) + grp * 2) = make_float2(c[0], c[1]);
         }
         named_bar_sync(1, nthr);
 
@@ -331,7 +341,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_pc_kernel(const __grid_const
         uint32_t off[4];
 #pragma unroll
         for (int j = 0; j < 4; j++) off[j] = row * kBox + (((2 * j + (q >> 1)) ^ (row & 7)) << 4) + (q & 1) * 8;
-        const float *d1lane = d1 + 2 * q;
+        const float *d1lane = d1 + q * (2 * G + 4);
         const uint8_t *my_slots = slot_ring + warp * ns * kSlotBytes;
         const uint8_t *my_scales = scale_ring + warp * ns * kScaleBytes;
         uint64_t *my_full = full + warp * kMaxNS;
@@ -350,22 +360,37 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_pc_kernel(const __grid_const
             dead = dead || !ok;
             if (ok) {
                 const uint8_t *sl = my_slots + s * kSlotBytes;
-                const unsigned short *sc = reinterpret_cast<const unsigned short *>(my_scales + s * kScaleBytes);
+                const uint8_t *scb = my_scales + s * kScaleBytes;
                 const int grp0 = kb * kSG;
-#pragma unroll 4
-                for (int j = 0; j < kSG; j++) {
-                    const uint8_t *bx = sl + (j >> 2) * (kRows * kBox);
-                    const uint2 a = *reinterpret_cast<const uint2 *>(bx + off[j & 3]);
-                    const uint2 b = *reinterpret_cast<const uint2 *>(bx + off[j & 3] + 8 * kBox);
-                    float c[4];
-                    group_mma<MT>(c, a.x, a.y, b.x, b.y, xlane + (grp0 + j) * kGroupHalves);
-                    const float2 o = *reinterpret_cast<const float2 *>(d1lane + (grp0 + j) * 8);
-                    const float sa = __half2float(__ushort_as_half(sc[row * kSG + j]));
-                    const float sb = __half2float(__ushort_as_half(sc[(row + 8) * kSG + j]));
-                    acc[0] = fmaf(sa, c[0] - o.x, acc[0]);
-                    acc[1] = fmaf(sa, c[1] - o.y, acc[1]);
-                    acc[2] = fmaf(sb, c[2] - o.x, acc[2]);
-                    acc[3] = fmaf(sb, c[3] - o.y, acc[3]);
+                const __half *xg = xlane + grp0 * kGroupHalves;
+                const float *dg = d1lane + grp0 * 2;
+#pragma unroll
+                for (int h = 0; h < 2; h++) {
+                    // four groups of one 512-k box: their scales (rows row, row+8)
+                    // and all-ones sums come in with four vector loads
+                    const uint2 sa4 = *reinterpret_cast<const uint2 *>(scb + row * 16 + h * 8);
+                    const uint2 sb4 = *reinterpret_cast<const uint2 *>(scb + (row + 8) * 16 + h * 8);
+                    const float4 o01 = *reinterpret_cast<const float4 *>(dg + h * 8);
+                    const float4 o23 = *reinterpret_cast<const float4 *>(dg + h * 8 + 4);
+                    const uint8_t *bx = sl + h * (kRows * kBox);
+                    const __half *xh = xg + h * 4 * kGroupHalves;
+                    const float ox[4] = {o01.x, o01.z, o23.x, o23.z};
+                    const float oy[4] = {o01.y, o01.w, o23.y, o23.w};
+                    const uint32_t sav[2] = {sa4.x, sa4.y}, sbv[2] = {sb4.x, sb4.y};
+#pragma unroll
+                    for (int jj = 0; jj < 4; jj++) {
+                        const uint2 a = *reinterpret_cast<const uint2 *>(bx + off[jj]);
+                        const uint2 b = *reinterpret_cast<const uint2 *>(bx + off[jj] + 8 * kBox);
+                        float c[4];
+                        group_mma<MT>(c, a.x, a.y, b.x, b.y, xh + jj * kGroupHalves);
+                        const uint32_t wa = sav[jj >> 1], wb = sbv[jj >> 1];
+                        const float sa = __half2float(__ushort_as_half(static_cast<unsigned short>((jj & 1) ? (wa >> 16) : wa)));
+                        const float sb = __half2float(__ushort_as_half(static_cast<unsigned short>((jj & 1) ? (wb >> 16) : wb)));
+                        acc[0] = fmaf(sa, c[0] - ox[jj], acc[0]);
+                        acc[1] = fmaf(sa, c[1] - oy[jj], acc[1]);
+                        acc[2] = fmaf(sb, c[2] - ox[jj], acc[2]);
+                        acc[3] = fmaf(sb, c[3] - oy[jj], acc[3]);
+                    }
                 }
             }
             // Release the stage.  A warp that gave up a wait stops arriving,
@@ -541,8 +566,13 @@ tern_status launch_gemv_pc(const MatDesc *md, int count, int M, cudaStream_t str
     int next = 0;
     for (int i = 0; i < count; i++) {
         PDesc &g = p.d[i];
-        st = encode_tiled_2d(&g.smap, CU_TENSOR_MAP_DATA_TYPE_UINT8, md[i].slots, static_cast<uint64_t>(md[i].K / 4),
-                             static_cast<uint64_t>(md[i].N), static_cast<uint64_t>(md[i].K / 4), kBox, kRows,
+        // The slot matrix seen as [K/512 chunks][N rows][128 bytes]: one copy
+        // brings both 512-k boxes of a slice (chunk stride 128 B, row stride K/4 B).
+        const uint64_t sdims[3] = {static_cast<uint64_t>(kBox), static_cast<uint64_t>(md[i].N),
+                                   static_cast<uint64_t>(md[i].K / 512)};
+        const uint64_t sstr[2] = {static_cast<uint64_t>(md[i].K / 4), static_cast<uint64_t>(kBox)};
+        const uint32_t sbox[3] = {static_cast<uint32_t>(kBox), static_cast<uint32_t>(kRows), 2};
+        st = encode_tiled_3d(&g.smap, CU_TENSOR_MAP_DATA_TYPE_UINT8, md[i].slots, sdims, sstr, sbox,
                              CU_TENSOR_MAP_SWIZZLE_128B);
         if (st != TERN_OK) return st;
         const int G = md[i].K / kGroup;
@@ -566,6 +596,11 @@ tern_status launch_gemv_pc(const MatDesc *md, int count, int M, cudaStream_t str
     cfg.blockDim = dim3(kThreads);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
     cudaError_t e = cudaLaunchKernelEx(&cfg, kern, p);
     if (e != cudaSuccess) return cuda_fail(e, "gemv pc kernel launch");
     return TERN_OK;

@@ -57,6 +57,9 @@ struct MatDesc {
 tern_status launch_gemv_tma(const MatDesc *d, int count, int M, cudaStream_t stream);
 // Producer/consumer form of the same kernel (K a multiple of 1024, x small).
 bool gemv_pc_supports(const MatDesc *d, int count, int M);
+bool gemv_tmem_supports(const MatDesc *md, int count, int M);
+tern_status launch_gemv_tmem(const MatDesc *md, int count, int M, cudaStream_t stream);
+tern_status read_gemvtm_status(bool reset, unsigned int *out);
 tern_status launch_gemv_pc(const MatDesc *d, int count, int M, cudaStream_t stream);
 // Tensor-core (tcgen05) bandwidth kernel for M in [1,4]; splits tiles along K
 // when a large enough zero-initialised workspace is given.
@@ -77,6 +80,10 @@ tern_status plan_partition(const int *ntile, const int *nbc, const int *nbmin, i
 tern_status encode_tiled_2d(CUtensorMap *map, CUtensorMapDataType dt, const void *base, uint64_t inner,
                             uint64_t outer, uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer,
                             CUtensorMapSwizzle swizzle);
+// Rank-3 tiled map: dims[0] innermost (elements), strides[] in bytes for
+// dims 1 and 2 (multiples of 16), box[] in elements.
+tern_status encode_tiled_3d(CUtensorMap *map, CUtensorMapDataType dt, const void *base, const uint64_t dims[3],
+                            const uint64_t strides[2], const uint32_t box[3], CUtensorMapSwizzle swizzle);
 // Tensor-core prefill product (any M; meant for large M).
 tern_status launch_gemm_tc(const MatDesc &d, int M, cudaStream_t stream);
 // Device-side status words written by bounded waits that gave up (one per
@@ -126,6 +133,13 @@ __device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, i
     asm volatile(
         "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
         ::"r"(smem_u32(dst)), "l"(map), "r"(c0), "r"(c1), "r"(smem_u32(bar))
+        : "memory");
+}
+
+__device__ __forceinline__ void tma_load_3d(void *dst, const CUtensorMap *map, int c0, int c1, int c2, uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], [%5];"
+        ::"r"(smem_u32(dst)), "l"(map), "r"(c0), "r"(c1), "r"(c2), "r"(smem_u32(bar))
         : "memory");
 }
 

@@ -38,6 +38,7 @@ TERN_OPT_TEST_STALL_US = 6
 TERN_OPT_GEMV_VARIANT = 7
 TERN_OPT_GEMV_GRID = 8
 GEMV_VARIANT_DEFAULT, GEMV_VARIANT_RING, GEMV_VARIANT_TMA, GEMV_VARIANT_TC, GEMV_VARIANT_PC = 0, 1, 2, 3, 4
+GEMV_VARIANT_TMEM = 5
 TERN_MAX_GROUP = 16
 
 _i64, _vp, _sz, _i32, _int = ctypes.c_int64, ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int32, ctypes.c_int

@@ -325,12 +325,17 @@ def test_stream_argument(T, orc):
     check_close(y, y_ref, bound, "side stream")
 
 
-@pytest.fixture
-def pc(T):
-    """Select the producer/consumer bandwidth kernel (K a multiple of 1024)."""
-    T.tern_set_option(T.TERN_OPT_GEMV_VARIANT, 4)
+@pytest.fixture(params=[(4, 0), (5, 0), (5, 1)], ids=["pc", "tmem", "tmem1wg"])
+def pc(T, request):
+    """Select one of the bandwidth kernels for K a multiple of 1024: the
+    producer/consumer mma.sync kernel (4) or the tensor-memory kernel (5) with
+    two warpgroups per CTA or one."""
+    variant, ctas = request.param
+    T.tern_set_option(T.TERN_OPT_GEMV_VARIANT, variant)
+    T.tern_set_option(T.TERN_OPT_GEMV_CTAS, ctas)
     yield T
     T.tern_set_option(T.TERN_OPT_GEMV_VARIANT, 0)
+    T.tern_set_option(T.TERN_OPT_GEMV_CTAS, 0)
 
 
 @pytest.mark.parametrize("M", [1, 2, 4, 8])
