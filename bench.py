@@ -429,12 +429,18 @@ def run_profile(args):
     if args.gemv_variant:
         T.tern_set_option(T.TERN_OPT_GEMV_VARIANT, args.gemv_variant)
     model = DecodeModel(T, n_layers=args.profile_layers)
+    _, hK, hN, hslots, hsc = model.head
     for _ in range(3):
-        for grp in model.groups:
-            T.tern_gemv_grouped(grp, 1)
+        if args.profile_head:
+            T.tern_gemv(model.head_io[0], hslots, hsc, model.head_io[1])
+        else:
+            for grp in model.groups:
+                T.tern_gemv_grouped(grp, 1)
     torch.cuda.synchronize()
-    print(json.dumps({"profile_layers": args.profile_layers,
-                      "bytes_per_launch": sum(wbytes(K, N) + 2 * K + 2 * N for _, K, N in synth.LAYER_PROJ)}))
+    per_launch = (wbytes(hK, hN) + 2 * hK + 2 * hN if args.profile_head
+                  else sum(wbytes(K, N) + 2 * K + 2 * N for _, K, N in synth.LAYER_PROJ))
+    print(json.dumps({"profile_layers": args.profile_layers, "profile_head": bool(args.profile_head),
+                      "bytes_per_launch": per_launch}))
     return 0
 
 
@@ -555,6 +561,8 @@ def main():
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
     ap.add_argument("--profile-layers", type=int, default=0,
                     help="profiling case: build this many layers, run their grouped launches 3x, exit")
+    ap.add_argument("--profile-head", action="store_true",
+                    help="profiling case: run the 5120x151936 head launch 3x instead of the layers")
     ap.add_argument("--gemv-variant", type=int, default=0,
                     help="profiling case only: bandwidth kernel variant (0 TMA-staged, 1 register ring)")
     args = ap.parse_args()

@@ -243,12 +243,19 @@ tern_status tern_sync_status(void *stream);
  *                          logic operation per weight pair; other shapes take
  *                          the default kernel), 5 = tensor-memory kernel for K
  *                          a multiple of 1024 (tcgen05, weights unpacked
- *                          into tensor memory by one thread per row); all
+ *                          into tensor memory by one thread per row),
+ *                          6 = variant 4 with token rows in the mma columns
+ *                          also at M = 1 (variant 4 puts the eight scale
+ *                          groups of a 1024-k slice there when M = 1); all
  *                          kept for comparison
  *   TERN_OPT_GEMV_GRID     cap on the CTAs of the producer/consumer and
  *                          tensor-memory kernels
  *                          (0 = one per SM); smaller grids give every CTA
  *                          more tiles to split among its warps
+ *   TERN_OPT_GEMV_PREFETCH L2 prefetch distance of the producer/consumer
+ *                          kernel, in 16-row x 1024-k units per consumer warp;
+ *                          0 or n <= ring depth = none (the default: measured
+ *                          slower)
  *   TERN_OPT_TEST_STALL_US TESTS ONLY: the TMA loaders of the tensor-core and
  *                          the TMA-staged bandwidth kernels issue no loads, so
  *                          their waits can never complete, and every bounded
@@ -263,7 +270,8 @@ enum {
     TERN_OPT_GEMM_MIN_M = 5,
     TERN_OPT_TEST_STALL_US = 6,
     TERN_OPT_GEMV_VARIANT = 7,
-    TERN_OPT_GEMV_GRID = 8
+    TERN_OPT_GEMV_GRID = 8,
+    TERN_OPT_GEMV_PREFETCH = 9
 };
 tern_status tern_set_option(int option, int64_t value);
 

@@ -157,7 +157,7 @@ int planning_sms() {
 
 // Bandwidth kernels (M <= 8).  Default: the TMA-staged mma.sync kernel,
 // the fastest measured so far; the knob selects the others for comparison.
-enum { kVarDefault = 0, kVarRing = 1, kVarTma = 2, kVarTc = 3, kVarPc = 4, kVarTmem = 5 };
+enum { kVarDefault = 0, kVarRing = 1, kVarTma = 2, kVarTc = 3, kVarPc = 4, kVarTmem = 5, kVarPcTok = 6 };
 
 bool use_tc(int M) { return g_opt.gemv_variant == kVarTc && M <= 4; }
 
@@ -168,8 +168,9 @@ tern_status launch_bandwidth(const MatDesc *d, int count, int M, void *workspace
     if (g_opt.gemv_variant == kVarTmem && gemv_tmem_supports(d, count, M)) return launch_gemv_tmem(d, count, M, s);
     // Default: the producer/consumer kernel where its shape rules hold (K a
     // multiple of 1024, x fits its shared memory), else the TMA-staged one.
-    if ((g_opt.gemv_variant == kVarPc || g_opt.gemv_variant == kVarDefault) && gemv_pc_supports(d, count, M))
-        return launch_gemv_pc(d, count, M, s);
+    if ((g_opt.gemv_variant == kVarPc || g_opt.gemv_variant == kVarDefault || g_opt.gemv_variant == kVarPcTok) &&
+        gemv_pc_supports(d, count, M))
+        return launch_gemv_pc(d, count, M, g_opt.gemv_variant == kVarPcTok, s);
     return launch_gemv_tma(d, count, M, s);
 }
 
@@ -374,10 +375,11 @@ tern_status tern_set_option(int option, int64_t value) {
             return TERN_OK;
         case TERN_OPT_GEMM_MIN_M: g_opt.gemm_min_m = static_cast<int>(value); return TERN_OK;
         case TERN_OPT_GEMV_VARIANT:
-            if (value > 5) return fail(TERN_ERR_INVALID_ARG, "gemv variant %lld", static_cast<long long>(value));
+            if (value > 6) return fail(TERN_ERR_INVALID_ARG, "gemv variant %lld", static_cast<long long>(value));
             g_opt.gemv_variant = static_cast<int>(value);
             return TERN_OK;
         case TERN_OPT_GEMV_GRID: g_opt.gemv_grid = static_cast<int>(value); return TERN_OK;
+        case TERN_OPT_GEMV_PREFETCH: g_opt.gemv_prefetch = static_cast<int>(value); return TERN_OK;
         case TERN_OPT_TEST_STALL_US:
             g_gemm_skip_loads = value > 0 ? 1 : 0;
             g_gemm_timeout_ns = value > 0 ? static_cast<unsigned long long>(value) * 1000ull : 1000000000ull;

@@ -43,8 +43,11 @@ __device__ unsigned int g_tern_gemvpc_status;
 
 namespace {
 
-constexpr int kCons = 12;                       // consumer warps
-constexpr int kThreads = (kCons + 1) * 32;      // + one producer warp
+// Consumer warps: twelve fed by one producer warp (token-per-column form), or
+// sixteen that load their own rings (group-per-column form).
+constexpr int kConsTok = 12, kConsGC = 16;
+__host__ __device__ constexpr int ncons(bool gc) { return gc ? kConsGC : kConsTok; }
+__host__ __device__ constexpr int nthreads(bool gc) { return gc ? kConsGC * 32 : (kConsTok + 1) * 32; }
 constexpr int kRows = 16;                       // tile rows (mma M)
 constexpr int kSG = 8;                          // scale groups per slice (1024 k)
 constexpr int kBox = 128;                       // bytes per row of one slot box (4 groups)
@@ -52,8 +55,10 @@ constexpr int kSlotBytes = kRows * kBox * 2;    // 4 KB
 constexpr int kScaleBytes = kRows * kSG * 2;    // 256 B
 constexpr int kMaxNS = 4;                       // ring stages per consumer, at most
 constexpr int kGroupK = 128;
-constexpr int kBarBytes = 2 * kCons * kMaxNS * 8;
-constexpr int kRecBytes = kCons * 2 * 32 * 4 * 4;  // partial tiles, two per consumer
+__host__ __device__ constexpr int barbytes(bool gc) { return 2 * ncons(gc) * kMaxNS * 8; }
+// partial tiles, two per consumer: float4 per lane, or (group-per-column form,
+// after the sum over the four lanes of a row) float2 per mma row g
+__host__ __device__ constexpr int recbytes(bool gc) { return gc ? ncons(gc) * 2 * 8 * 8 : ncons(gc) * 2 * 32 * 4 * 4; }
 constexpr size_t kSmemBudget = 232448;          // opt-in shared memory per block on sm_100
 constexpr int kMaxDesc = TERN_MAX_GROUP;
 
@@ -70,16 +75,23 @@ struct alignas(64) PDesc {
 struct PParams {
     PDesc d[kMaxDesc];
     int count, M;
-    int ns;             // ring stages per consumer
+    unsigned int smem_usable;  // dynamic shared memory past the 1024-byte alignment
     int kmax;           // largest K of the launch (sizes the all-ones table)
     int xs_halves;
     int skip_loads;
+    int pf;             // L2 prefetch distance in units (0: none)
     unsigned long long timeout_ns;
 };
 
-size_t smem_bytes(int ns, int xs_halves, int kmax) {
-    return 1024 + static_cast<size_t>(kCons) * ns * (kSlotBytes + kScaleBytes) + kBarBytes + kRecBytes + 160 +
-           (static_cast<size_t>(kmax / kGroupK) * 8 + 16) * 4 + static_cast<size_t>(xs_halves) * 2;
+// Bytes before the staged x: barriers, partial tiles, tile ids, maxima, d1.
+__host__ __device__ constexpr uint32_t fixed_bytes(int kmax, bool gc) {
+    return barbytes(gc) + recbytes(gc) + 2 * ncons(gc) * 4 + 16 * 4 + (static_cast<uint32_t>(kmax / kGroupK) * 8 + 16) * 4;
+}
+// Dynamic shared memory for rings of ns stages beside xs_halves of staged x
+// (+1024 for the alignment of the start).
+size_t smem_bytes(int ns, int xs_halves, int kmax, bool gc) {
+    const size_t ring_off = (fixed_bytes(kmax, gc) + static_cast<size_t>(xs_halves) * 2 + 1023) & ~size_t(1023);
+    return 1024 + ring_off + static_cast<size_t>(ncons(gc)) * ns * (kSlotBytes + kScaleBytes);
 }
 
 constexpr uint32_t kOnes = 0x55555555u;  // every 2-bit field = code 1 (t = 0)
@@ -121,14 +133,8 @@ __device__ __forceinline__ int xs_pair_index(int m, int kl) {
 // of pair j, one accumulation chain (the unrolled groups of a slice give the
 // scheduler independent chains).  Shared by the weight path and the all-ones
 // pass, so the two round identically.
-template <int MT>
-__device__ __forceinline__ void group_mma(float (&c)[4], uint32_t ax, uint32_t ay, uint32_t bx, uint32_t by,
-                                          const __half *xb) {
-    constexpr int kChunk = MT * 32;
-    const uint4 x0 = *reinterpret_cast<const uint4 *>(xb);
-    const uint4 x1 = *reinterpret_cast<const uint4 *>(xb + kChunk);
-    const uint4 x2 = *reinterpret_cast<const uint4 *>(xb + 2 * kChunk);
-    const uint4 x3 = *reinterpret_cast<const uint4 *>(xb + 3 * kChunk);
+__device__ __forceinline__ void group_mma_b(float (&c)[4], uint32_t ax, uint32_t ay, uint32_t bx, uint32_t by,
+                                            const uint4 &x0, const uint4 &x1, const uint4 &x2, const uint4 &x3) {
     const uint32_t ax5 = ax >> 10, ay5 = ay >> 10, bx5 = bx >> 10, by5 = by >> 10;
     mma_zero(c, ax & 0x00030003u, bx & 0x00030003u, ay & 0x00030003u, by & 0x00030003u, x0.x, x0.y);
     mma_acc(c, ax & 0x000C000Cu, bx & 0x000C000Cu, ay & 0x000C000Cu, by & 0x000C000Cu, x0.z, x0.w);
@@ -138,6 +144,29 @@ __device__ __forceinline__ void group_mma(float (&c)[4], uint32_t ax, uint32_t a
     mma_acc(c, ax5 & 0x00030003u, bx5 & 0x00030003u, ay5 & 0x00030003u, by5 & 0x00030003u, x2.z, x2.w);
     mma_acc(c, ax5 & 0x000C000Cu, bx5 & 0x000C000Cu, ay5 & 0x000C000Cu, by5 & 0x000C000Cu, x3.x, x3.y);
     mma_acc(c, ax5 & 0x00300030u, bx5 & 0x00300030u, ay5 & 0x00300030u, by5 & 0x00300030u, x3.z, x3.w);
+}
+
+// The four B-fragment loads of one group (chunks of MT x 32 x 8 halves).
+template <int MT>
+__device__ __forceinline__ void load_xfrag(const __half *xb, uint4 (&xf)[4]) {
+    constexpr int kChunk = MT * 32;
+#pragma unroll
+    for (int i = 0; i < 4; i++) xf[i] = *reinterpret_cast<const uint4 *>(xb + i * kChunk);
+}
+
+template <int MT>
+__device__ __forceinline__ void group_mma(float (&c)[4], uint32_t ax, uint32_t ay, uint32_t bx, uint32_t by,
+                                          const __half *xb) {
+    uint4 xf[4];
+    load_xfrag<MT>(xb, xf);
+    group_mma_b(c, ax, ay, bx, by, xf[0], xf[1], xf[2], xf[3]);
+}
+
+// Lane q's pick among four values (q = 0..3).
+__device__ __forceinline__ float sel4(int q, float a, float b, float c, float d) {
+    const float lo = (q & 1) ? b : a;
+    const float hi = (q & 1) ? d : c;
+    return (q & 2) ? hi : lo;
 }
 
 __device__ __forceinline__ bool mbar_test_wait(uint64_t *bar, uint32_t parity) {
@@ -170,7 +199,7 @@ __device__ __forceinline__ int tile_row(int g) { return g < 4 ? 2 * g : 2 * g - 
 // [u0, u1), unit u = slice u % B of tile t0 + u / B.
 struct Range {
     int t0, u0, u1;
-    __device__ void init(const PDesc &d, int lc, int w) {
+    __device__ void init(const PDesc &d, int lc, int w, int kCons) {
         t0 = static_cast<int>((static_cast<long long>(lc) * d.ntile) / d.c_count);
         const int t1 = static_cast<int>((static_cast<long long>(lc + 1) * d.ntile) / d.c_count);
         const int U = (t1 - t0) * d.B;
@@ -179,23 +208,18 @@ struct Range {
     }
 };
 
-template <int MT>
-__global__ void __launch_bounds__(kThreads, 1) gemv_pc_kernel(const __grid_constant__ PParams p) {
+// GC (M = 1 only): the eight B columns carry the eight scale groups of a
+// slice instead of eight token rows, so one set of B fragments serves all
+// eight groups (see gc_note below).
+template <int MT, bool GC>
+__global__ void __launch_bounds__(nthreads(GC), 1) gemv_pc_kernel(const __grid_constant__ PParams p) {
+    constexpr int kCons = ncons(GC);
+    // Layout width of the staged x: token rows, or the eight groups of a slice.
+    constexpr int XT = GC ? 8 : MT;
     extern __shared__ uint8_t smem_raw[];
-    uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    const int ns = p.ns;
-    uint8_t *slot_ring = base;                                   // [kCons][ns][4096], 1024-aligned boxes
-    uint8_t *scale_ring = slot_ring + kCons * ns * kSlotBytes;   // [kCons][ns][256]
-    uint64_t *full = reinterpret_cast<uint64_t *>(scale_ring + kCons * ns * kScaleBytes);  // [kCons][kMaxNS]
-    uint64_t *empty = full + kCons * kMaxNS;
-    float *rec = reinterpret_cast<float *>(empty + kCons * kMaxNS);  // [kCons][2][32][4] partial tiles
-    int *rec_tile = reinterpret_cast<int *>(rec + kCons * 2 * 32 * 4);  // [kCons][2]
-    unsigned int *wmax = reinterpret_cast<unsigned int *>(rec_tile + 2 * kCons);  // [kCons]
-    // [lane q][2 G + 4]: two floats per group, rows padded so that the four
-    // lanes q of a quarter warp read distinct banks
-    float *d1 = reinterpret_cast<float *>(wmax + 16);
-    __half *xs = reinterpret_cast<__half *>(d1 + (p.kmax / kGroupK) * 8 + 16);
-
+    // 1024-byte aligned start (offset arithmetic on the shared array keeps the
+    // compiler's knowledge that every derived pointer is shared memory)
+    uint8_t *base = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     const int M = p.M;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     int di = 0;
@@ -204,6 +228,23 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_pc_kernel(const __grid_const
     const PDesc &d = p.d[di];
     const int lc = blockIdx.x - d.c_begin;
     const int B = d.B;
+
+    uint64_t *full = reinterpret_cast<uint64_t *>(base);  // [kCons][kMaxNS]
+    uint64_t *empty = full + kCons * kMaxNS;
+    float *rec = reinterpret_cast<float *>(empty + kCons * kMaxNS);  // partial tiles (recbytes)
+    int *rec_tile = reinterpret_cast<int *>(reinterpret_cast<uint8_t *>(rec) + recbytes(GC));  // [kCons][2]
+    unsigned int *wmax = reinterpret_cast<unsigned int *>(rec_tile + 2 * kCons);  // [kCons]
+    // [lane q][2 G + 4]: two floats per group, rows padded so that the four
+    // lanes q of a quarter warp read distinct banks (group-per-column form:
+    // one float per group)
+    float *d1 = reinterpret_cast<float *>(wmax + 16);
+    __half *xs = reinterpret_cast<__half *>(d1 + (p.kmax / kGroupK) * 8 + 16);
+    // The rings take what is left after this CTA's own staged x (a grouped
+    // launch is sized for its largest K; CTAs of smaller K get deeper rings).
+    const uint32_t ring_off = (fixed_bytes(p.kmax, GC) + static_cast<uint32_t>(GC ? 1 : MT) * d.K * 2 + 1023u) & ~1023u;
+    const int ns = min(kMaxNS, static_cast<int>((p.smem_usable - ring_off) / (kCons * (kSlotBytes + kScaleBytes))));
+    uint8_t *slot_ring = base + ring_off;                        // [kCons][ns][4096], 1024-aligned boxes
+    uint8_t *scale_ring = slot_ring + kCons * ns * kSlotBytes;   // [kCons][ns][256]
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < kCons * kMaxNS; i++) {
@@ -227,8 +268,9 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_pc_kernel(const __grid_const
         int u = 0, s = 0, issued = 0;
         uint32_t ph = 0;
         bool done = true;
-        if (lane < kCons && !p.skip_loads) {
-            r.init(d, lc, lane);
+        // (the group-per-column form loads its own rings: nothing to do here)
+        if (lane < kCons && !p.skip_loads && !GC) {
+            r.init(d, lc, lane, kCons);
             u = r.u0;
             done = u >= r.u1;
         }
@@ -236,6 +278,16 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_pc_kernel(const __grid_const
         uint8_t *my_scales = scale_ring + lane * ns * kScaleBytes;
         uint64_t *my_full = full + lane * kMaxNS;
         uint64_t *my_empty = empty + lane * kMaxNS;
+        // L2 prefetch `pf` units ahead of the ring (the ring itself covers the
+        // next ns units): the later TMA loads then hit L2.
+        auto prefetch = [&](int v) {
+            const int tile = r.t0 + v / B;
+            const int kbx = v - (v / B) * B;
+            tma_prefetch_3d(&d.smap, 0, tile * kRows, kbx * 2);
+            tma_prefetch_2d(&d.cmap, kbx * kSG, tile * kRows);
+        };
+        if (!done && p.pf > ns)
+            for (int v = u + ns; v < r.u1 && v < u + p.pf; v++) prefetch(v);
         while (__any_sync(0xffffffffu, !done)) {
             bool progressed = false;
             if (!done) {
@@ -245,6 +297,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_pc_kernel(const __grid_const
                     mbar_expect_tx(&my_full[s], kSlotBytes + kScaleBytes);
                     tma_load_3d(my_slots + s * kSlotBytes, &d.smap, 0, tile * kRows, kbx * 2, &my_full[s]);
                     tma_load_2d(my_scales + s * kScaleBytes, &d.cmap, kbx * kSG, tile * kRows, &my_full[s]);
+                    if (p.pf > ns && u + p.pf < r.u1) prefetch(u + p.pf);
                     issued++;
                     if (++s == ns) {
                         s = 0;
@@ -271,6 +324,28 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_pc_kernel(const __grid_const
         // ======================= consumer warps =======================
         const int K = d.K, N = d.N;
         const int nthr = kCons * 32;
+        Range r;
+        r.init(d, lc, warp, kCons);
+        uint8_t *my_slots = slot_ring + warp * ns * kSlotBytes;
+        uint8_t *my_scales = scale_ring + warp * ns * kScaleBytes;
+        uint64_t *my_full = full + warp * kMaxNS;
+        uint64_t *my_empty = empty + warp * kMaxNS;
+        // Group-per-column form: lane 0 loads the warp's own ring (unit v into
+        // stage `st`); the first ns units go out before the grid-dependency
+        // wait (weights are never written by a preceding launch).
+        auto issue = [&](int v, int st) {
+            const int tile = r.t0 + v / B;
+            const int kbx = v - (v / B) * B;
+            mbar_expect_tx(&my_full[st], kSlotBytes + kScaleBytes);
+            tma_load_3d(my_slots + st * kSlotBytes, &d.smap, 0, tile * kRows, kbx * 2, &my_full[st]);
+            tma_load_2d(my_scales + st * kScaleBytes, &d.cmap, kbx * kSG, tile * kRows, &my_full[st]);
+        };
+        int issued_end = r.u0;  // units [r.u0, issued_end) have been issued
+        if (GC && !p.skip_loads) {
+            issued_end = min(r.u0 + ns, r.u1);
+            if (lane == 0)
+                for (int v = r.u0; v < issued_end; v++) issue(v, v - r.u0);
+        }
         // x may be the output of the preceding launch: wait for it to finish.
         asm volatile("griddepcontrol.wait;" ::: "memory");
         // (1) E from the largest finite |x| of all token rows.
@@ -310,14 +385,18 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_pc_kernel(const __grid_const
                 const int m = idx / per_m, c8 = idx - m * per_m;
                 const uint4 v = *reinterpret_cast<const uint4 *>(d.x + static_cast<size_t>(m) * K + c8 * 8);
                 const uint32_t pr[4] = {v.x, v.y, v.z, v.w};
-                unsigned short *dst = reinterpret_cast<unsigned short *>(xs + xs_pair_index<MT>(m, c8 * 8));
+                // GC: group n of slice b is staged as "token" n of a 1024-k group b
+                const int kl = c8 * 8;
+                const int di = GC ? xs_pair_index<8>((kl >> 7) & 7, ((kl >> 10) << 7) | (kl & 127))
+                                  : xs_pair_index<MT>(m, kl);
+                unsigned short *dst = reinterpret_cast<unsigned short *>(xs + di);
 #pragma unroll
                 for (int i = 0; i < 4; i++) {
                     uint32_t h2;
                     asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(h2) : "r"(pr[i]), "r"(fac2[i]));
                     // element e = 2i + t lands at chunk e / 2 = i, slot t * 4
-                    dst[i * MT * 32] = static_cast<unsigned short>(h2);
-                    dst[i * MT * 32 + 4] = static_cast<unsigned short>(h2 >> 16);
+                    dst[i * XT * 32] = static_cast<unsigned short>(h2);
+                    dst[i * XT * 32 + 4] = static_cast<unsigned short>(h2 >> 16);
                 }
             }
         }
@@ -325,40 +404,119 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_pc_kernel(const __grid_const
         const int g = lane >> 2, q = lane & 3;
         const int gx = g < M ? g : M - 1;
         const int G = K / kGroupK;
-        constexpr int kGroupHalves = MT * 4 * 32;
-        const __half *xlane = xs + (gx * 4 + q) * 8;
-        // (3) the all-ones pass: D(ones) per group and B column (token).
-        for (int grp = warp; grp < G; grp += kCons) {
-            float c[4];
-            group_mma<MT>(c, kOnes, kOnes, kOnes, kOnes, xlane + grp * kGroupHalves);
-            if (g == 0) *reinterpret_cast<float2 *>(d1 + q * (2 * G + 4) + grp * 2) = make_float2(c[0], c[1]);
+        constexpr int kGroupHalves = XT * 4 * 32;
+        const __half *xlane = xs + ((GC ? g : gx) * 4 + q) * 8;
+        // (3) the all-ones pass: D(ones) per group and B column (token).  GC:
+        // one chain per slice gives all eight groups, column n = group n;
+        // stored as d1[group].
+        if (GC) {
+            for (int sl = warp; sl < G / kSG; sl += kCons) {
+                float c[4];
+                group_mma<8>(c, kOnes, kOnes, kOnes, kOnes, xlane + sl * kGroupHalves);
+                if (g == 0) *reinterpret_cast<float2 *>(d1 + sl * kSG + 2 * q) = make_float2(c[0], c[1]);
+            }
+        } else {
+            for (int grp = warp; grp < G; grp += kCons) {
+                float c[4];
+                group_mma<MT>(c, kOnes, kOnes, kOnes, kOnes, xlane + grp * kGroupHalves);
+                if (g == 0) *reinterpret_cast<float2 *>(d1 + q * (2 * G + 4) + grp * 2) = make_float2(c[0], c[1]);
+            }
         }
         named_bar_sync(1, nthr);
 
         const int row = tile_row(g);
-        Range r;
-        r.init(d, lc, warp);
         uint32_t off[4];
 #pragma unroll
         for (int j = 0; j < 4; j++) off[j] = row * kBox + (((2 * j + (q >> 1)) ^ (row & 7)) << 4) + (q & 1) * 8;
         const float *d1lane = d1 + q * (2 * G + 4);
-        const uint8_t *my_slots = slot_ring + warp * ns * kSlotBytes;
-        const uint8_t *my_scales = scale_ring + warp * ns * kScaleBytes;
-        uint64_t *my_full = full + warp * kMaxNS;
-        uint64_t *my_empty = empty + warp * kMaxNS;
         const float post = ldexpf(1.0f, 24 - E);
         float acc[4] = {0.f, 0.f, 0.f, 0.f};
         int s = 0;
         uint32_t ph = 0;
         bool dead = false;
+        int dead_u = r.u1, dead_s = 0;
+        uint32_t dead_ph = 0;
         int tl = r.u0 / B;                 // tile (relative to t0) being accumulated
         int kb = r.u0 - tl * B;            // its next slice
         const int kb_first = kb;           // first slice of the first tile
         for (int u = r.u0; u < r.u1; u++) {
             bool ok = !dead;
             if (ok) ok = __all_sync(0xffffffffu, pc_wait(&my_full[s], ph, deadline));
+            if (!ok && !dead) {
+                dead_u = u;
+                dead_s = s;
+                dead_ph = ph;
+            }
             dead = dead || !ok;
-            if (ok) {
+            if (ok && GC) {
+                // gc_note: the slice's B fragments (x of all eight groups, group
+                // n in column n) are loaded once; weight group G runs its
+                // eight-mma chain into its own accumulator dd[G], of which only
+                // column G is meaningful.  Lane (g, q) holds columns 2q, 2q+1,
+                // i.e. groups 2q and 2q+1 of rows `row` and `row` + 8.
+                const uint8_t *sl = my_slots + s * kSlotBytes;
+                const uint8_t *scb = my_scales + s * kScaleBytes;
+                uint4 xf[4];
+                load_xfrag<8>(xlane + kb * kGroupHalves, xf);
+                const float2 on = *reinterpret_cast<const float2 *>(d1 + kb * kSG + 2 * q);
+                const __half2 sa2 = *reinterpret_cast<const __half2 *>(scb + row * 16 + 4 * q);
+                const __half2 sb2 = *reinterpret_cast<const __half2 *>(scb + (row + 8) * 16 + 4 * q);
+                // All eight groups' words first, then the mmas field by field
+                // (j outer, group inner): eight independent accumulation chains
+                // between two dependent mmas.
+                uint32_t wd[kSG][4];
+#pragma unroll
+                for (int G8 = 0; G8 < kSG; G8++) {
+                    const uint8_t *bx = sl + (G8 >> 2) * (kRows * kBox);
+                    const uint2 a = *reinterpret_cast<const uint2 *>(bx + off[G8 & 3]);
+                    const uint2 b = *reinterpret_cast<const uint2 *>(bx + off[G8 & 3] + 8 * kBox);
+                    wd[G8][0] = a.x;  // row g,   word 2q
+                    wd[G8][1] = b.x;  // row g+8, word 2q
+                    wd[G8][2] = a.y;  // row g,   word 2q+1
+                    wd[G8][3] = b.y;  // row g+8, word 2q+1
+                }
+                // Everything this unit needs from the stage is in registers:
+                // refill it now, so that the next load is in flight during the
+                // mmas below (the warp barrier orders the reads before the
+                // proxy fence and the copy that overwrites the stage).
+                __syncwarp();
+                if (issued_end < r.u1) {
+                    if (lane == 0) {
+                        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                        issue(issued_end, s);
+                    }
+                    issued_end++;
+                }
+                float dd[kSG][4];
+#pragma unroll
+                for (int j = 0; j < 8; j++) {
+                    if (j == 5) {
+#pragma unroll
+                        for (int G8 = 0; G8 < kSG; G8++)
+#pragma unroll
+                            for (int i = 0; i < 4; i++) wd[G8][i] >>= 10;
+                    }
+                    const uint32_t m = 0x00030003u << (2 * (j < 5 ? j : j - 5));
+                    const uint4 &xv = xf[j >> 1];
+                    const uint32_t b0 = (j & 1) ? xv.z : xv.x, b1 = (j & 1) ? xv.w : xv.y;
+#pragma unroll
+                    for (int G8 = 0; G8 < kSG; G8++) {
+                        if (j == 0)
+                            mma_zero(dd[G8], wd[G8][0] & m, wd[G8][1] & m, wd[G8][2] & m, wd[G8][3] & m, b0, b1);
+                        else
+                            mma_acc(dd[G8], wd[G8][0] & m, wd[G8][1] & m, wd[G8][2] & m, wd[G8][3] & m, b0, b1);
+                    }
+                }
+                const float v0 = sel4(q, dd[0][0], dd[2][0], dd[4][0], dd[6][0]);
+                const float v1 = sel4(q, dd[1][1], dd[3][1], dd[5][1], dd[7][1]);
+                const float v2 = sel4(q, dd[0][2], dd[2][2], dd[4][2], dd[6][2]);
+                const float v3 = sel4(q, dd[1][3], dd[3][3], dd[5][3], dd[7][3]);
+                const float2 fa = __half22float2(sa2), fb = __half22float2(sb2);
+                acc[0] = fmaf(fa.x, v0 - on.x, acc[0]);
+                acc[0] = fmaf(fa.y, v1 - on.y, acc[0]);
+                acc[2] = fmaf(fb.x, v2 - on.x, acc[2]);
+                acc[2] = fmaf(fb.y, v3 - on.y, acc[2]);
+            } else if (ok) {
                 const uint8_t *sl = my_slots + s * kSlotBytes;
                 const uint8_t *scb = my_scales + s * kScaleBytes;
                 const int grp0 = kb * kSG;
@@ -393,10 +551,13 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_pc_kernel(const __grid_const
                     }
                 }
             }
-            // Release the stage.  A warp that gave up a wait stops arriving,
-            // so its producer lane gives up too.
-            __syncwarp();
-            if (lane == 0 && !dead) mbar_arrive(&my_empty[s]);
+            // Release the stage (the group-per-column form released it above).
+            // A warp that gave up a wait stops arriving, so its producer lane
+            // gives up too.
+            if (!(GC && ok)) {
+                __syncwarp();
+                if (lane == 0 && !dead) mbar_arrive(&my_empty[s]);
+            }
             if (++s == ns) {
                 s = 0;
                 ph ^= 1;
@@ -406,6 +567,13 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_pc_kernel(const __grid_const
                 // ---- this warp's part of a tile is complete ----
                 const int tile = r.t0 + tl;
                 const bool whole = kb == B && (tl != r.u0 / B || kb_first == 0);
+                if (GC) {
+                    // sum the four lanes q of a row (their groups differ)
+                    acc[0] += __shfl_xor_sync(0xffffffffu, acc[0], 1);
+                    acc[0] += __shfl_xor_sync(0xffffffffu, acc[0], 2);
+                    acc[2] += __shfl_xor_sync(0xffffffffu, acc[2], 1);
+                    acc[2] += __shfl_xor_sync(0xffffffffu, acc[2], 2);
+                }
                 const float v0 = acc[0] * post, v1 = acc[1] * post, v2 = acc[2] * post, v3 = acc[3] * post;
                 if (whole) {
                     if (!dead) {
@@ -424,13 +592,31 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_pc_kernel(const __grid_const
                     // A tile shared with neighbouring warps: keep the partial
                     // (slot 0 = the range's first tile, slot 1 = its last).
                     const int slot = (tl == r.u0 / B) ? 0 : 1;
-                    *reinterpret_cast<float4 *>(rec + ((warp * 2 + slot) * 32 + lane) * 4) =
-                        make_float4(v0, v1, v2, v3);
+                    if (GC) {
+                        if (q == 0) *reinterpret_cast<float2 *>(rec + ((warp * 2 + slot) * 8 + g) * 2) = make_float2(v0, v2);
+                    } else {
+                        *reinterpret_cast<float4 *>(rec + ((warp * 2 + slot) * 32 + lane) * 4) =
+                            make_float4(v0, v1, v2, v3);
+                    }
                     if (lane == 0) rec_tile[warp * 2 + slot] = dead ? -2 : tile;
                 }
                 acc[0] = acc[1] = acc[2] = acc[3] = 0.f;
                 kb = 0;
                 tl++;
+            }
+        }
+        // A warp that gave up may still have copies of its own in flight
+        // (group-per-column form): they must land before the CTA exits.
+        if (GC && dead) {
+            const unsigned long long dl2 = globaltimer() + p.timeout_ns;
+            int st = dead_s;
+            uint32_t phs = dead_ph;
+            for (int v = dead_u; v < issued_end; v++) {
+                pc_wait(&my_full[st], phs, dl2);
+                if (++st == ns) {
+                    st = 0;
+                    phs ^= 1;
+                }
             }
         }
         // ---- tiles split over several warps: summed in warp order by the
@@ -449,8 +635,13 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_pc_kernel(const __grid_const
             for (int w2 = warp; w2 < kCons; w2++) {
                 for (int s2 = 0; s2 < 2; s2++) {
                     if (rec_tile[w2 * 2 + s2] != tile) continue;
-                    const float4 o = *reinterpret_cast<const float4 *>(rec + ((w2 * 2 + s2) * 32 + lane) * 4);
-                    sum.x += o.x; sum.y += o.y; sum.z += o.z; sum.w += o.w;
+                    if (GC) {
+                        const float2 o = *reinterpret_cast<const float2 *>(rec + ((w2 * 2 + s2) * 8 + g) * 2);
+                        sum.x += o.x; sum.z += o.y;
+                    } else {
+                        const float4 o = *reinterpret_cast<const float4 *>(rec + ((w2 * 2 + s2) * 32 + lane) * 4);
+                        sum.x += o.x; sum.y += o.y; sum.z += o.z; sum.w += o.w;
+                    }
                 }
             }
             // a part that gave up is marked -2; then the tile is not stored
@@ -471,10 +662,24 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_pc_kernel(const __grid_const
     }
 }
 
-bool g_attr_pc[64][4];
-int g_occ_pc[64][4];
+bool g_attr_pc[64][5];
+int g_occ_pc[64][5];
 
 int pc_mt(int M) { return M == 1 ? 1 : (M == 2 ? 2 : (M <= 4 ? 4 : 8)); }
+
+// Kernel instance for M token rows; M = 1 takes the group-per-column form
+// unless `token_columns` asks for the token-per-column form.
+using PcKernel = void (*)(PParams);
+PcKernel pc_kernel(int M, bool token_columns, int *index) {
+    const int MT = pc_mt(M);
+    if (MT == 1 && !token_columns) {
+        *index = 4;
+        return gemv_pc_kernel<1, true>;
+    }
+    *index = MT == 1 ? 0 : (MT == 2 ? 1 : (MT == 4 ? 2 : 3));
+    return MT == 1 ? gemv_pc_kernel<1, false>
+                   : (MT == 2 ? gemv_pc_kernel<2, false> : (MT == 4 ? gemv_pc_kernel<4, false> : gemv_pc_kernel<8, false>));
+}
 
 }  // namespace
 
@@ -486,32 +691,33 @@ bool gemv_pc_supports(const MatDesc *md, int count, int M) {
         kmax = std::max(kmax, md[i].K);
     }
     // x is staged whole per CTA; at least two ring stages must fit beside it.
-    return smem_bytes(2, pc_mt(M) * kmax, kmax) <= kSmemBudget;
+    return smem_bytes(2, pc_mt(M) * kmax, kmax, false) <= kSmemBudget;
 }
 
-tern_status launch_gemv_pc(const MatDesc *md, int count, int M, cudaStream_t stream) {
+tern_status launch_gemv_pc(const MatDesc *md, int count, int M, bool token_columns, cudaStream_t stream) {
     DeviceInfo dev;
     tern_status st = current_device(&dev);
     if (st != TERN_OK) return st;
     if (count < 1 || count > kMaxDesc) return fail(TERN_ERR_INVALID_ARG, "descriptor count %d", count);
     if (!gemv_pc_supports(md, count, M)) return fail(TERN_ERR_SHAPE, "producer/consumer kernel: unsupported shape");
     const int MT = pc_mt(M);
-    auto kern = MT == 1 ? gemv_pc_kernel<1> : (MT == 2 ? gemv_pc_kernel<2> : (MT == 4 ? gemv_pc_kernel<4> : gemv_pc_kernel<8>));
-    const int mi = MT == 1 ? 0 : (MT == 2 ? 1 : (MT == 4 ? 2 : 3));
+    int mi = 0;
+    const PcKernel kern = pc_kernel(M, token_columns, &mi);
     int kmax = 0;
     for (int i = 0; i < count; i++) kmax = std::max(kmax, md[i].K);
     const int xs_halves = MT * kmax;
     const size_t budget = std::min<size_t>(kSmemBudget, dev.max_smem_optin);
-    int ns = kMaxNS;
-    while (ns > 2 && smem_bytes(ns, xs_halves, kmax) > budget) ns--;
-    const size_t smem = smem_bytes(ns, xs_halves, kmax);
-    if (smem > budget) return fail(TERN_ERR_SHAPE, "needs %zu B of shared memory", smem);
+    // The whole budget: every CTA sizes its rings (2..4 stages) from what its
+    // own staged x leaves.
+    const bool gc = mi == 4;
+    const size_t smem = std::min(budget, smem_bytes(kMaxNS, MT * 1024, kmax, gc));
+    if (smem_bytes(2, xs_halves, kmax, gc) > smem) return fail(TERN_ERR_SHAPE, "needs %zu B of shared memory", smem_bytes(2, xs_halves, kmax, gc));
     if (!g_attr_pc[dev.device][mi]) {
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              static_cast<int>(dev.max_smem_optin));
         if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(gemv pc)");
         int occ = 0;
-        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, kThreads, static_cast<size_t>(kSmemBudget));
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, nthreads(mi == 4), static_cast<size_t>(kSmemBudget));
         if (e != cudaSuccess) return cuda_fail(e, "occupancy query");
         if (occ < 1) return fail(TERN_ERR_SHAPE, "producer/consumer kernel does not fit on an SM");
         g_occ_pc[dev.device][mi] = occ;
@@ -558,10 +764,11 @@ tern_status launch_gemv_pc(const MatDesc *md, int count, int M, cudaStream_t str
     std::memset(&p, 0, sizeof(p));
     p.count = count;
     p.M = M;
-    p.ns = ns;
+    p.smem_usable = static_cast<unsigned int>(smem - 1024);
     p.kmax = kmax;
     p.xs_halves = xs_halves;
     p.skip_loads = g_gemm_skip_loads;
+    p.pf = g_opt.gemv_prefetch;
     p.timeout_ns = g_gemm_timeout_ns;
     int next = 0;
     for (int i = 0; i < count; i++) {
@@ -593,7 +800,7 @@ tern_status launch_gemv_pc(const MatDesc *md, int count, int M, cudaStream_t str
     cudaLaunchConfig_t cfg;
     std::memset(&cfg, 0, sizeof(cfg));
     cfg.gridDim = dim3(static_cast<unsigned>(next));
-    cfg.blockDim = dim3(kThreads);
+    cfg.blockDim = dim3(nthreads(gc));
     cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];

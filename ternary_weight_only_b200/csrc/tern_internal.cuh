@@ -35,6 +35,7 @@ struct Options {
     int gemm_min_m = 0;
     int gemv_variant = 0;
     int gemv_grid = 0;
+    int gemv_prefetch = 0;
 };
 extern Options g_opt;
 
@@ -60,7 +61,8 @@ bool gemv_pc_supports(const MatDesc *d, int count, int M);
 bool gemv_tmem_supports(const MatDesc *md, int count, int M);
 tern_status launch_gemv_tmem(const MatDesc *md, int count, int M, cudaStream_t stream);
 tern_status read_gemvtm_status(bool reset, unsigned int *out);
-tern_status launch_gemv_pc(const MatDesc *d, int count, int M, cudaStream_t stream);
+// M = 1 uses the group-per-column form unless token_columns is set.
+tern_status launch_gemv_pc(const MatDesc *d, int count, int M, bool token_columns, cudaStream_t stream);
 // Tensor-core (tcgen05) bandwidth kernel for M in [1,4]; splits tiles along K
 // when a large enough zero-initialised workspace is given.
 tern_status launch_gemv_tc(const MatDesc *d, int count, int M, void *workspace, size_t ws_bytes,
@@ -141,6 +143,17 @@ __device__ __forceinline__ void tma_load_3d(void *dst, const CUtensorMap *map, i
         "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], [%5];"
         ::"r"(smem_u32(dst)), "l"(map), "r"(c0), "r"(c1), "r"(c2), "r"(smem_u32(bar))
         : "memory");
+}
+
+// Bring a tile of a tensor into L2 only (no shared memory, no completion).
+__device__ __forceinline__ void tma_prefetch_2d(const CUtensorMap *map, int c0, int c1) {
+    asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(map), "r"(c0), "r"(c1)
+                 : "memory");
+}
+__device__ __forceinline__ void tma_prefetch_3d(const CUtensorMap *map, int c0, int c1, int c2) {
+    asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];" ::"l"(map), "r"(c0), "r"(c1),
+                 "r"(c2)
+                 : "memory");
 }
 
 __device__ __forceinline__ void named_bar_sync(int id, int count) {
