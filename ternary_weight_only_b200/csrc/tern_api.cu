@@ -318,6 +318,26 @@ tern_status tern_gemv_noalloc(const uint16_t *x, const uint8_t *slots, const uin
     return gemv_noalloc(mat(x, slots, scales, y, N, K), static_cast<cudaStream_t>(stream));
 }
 
+tern_status tern_gemv_step(const tern_gemv_desc *descs, int32_t count, void *stream) {
+    clear_error();
+    if (!descs) return fail(TERN_ERR_INVALID_ARG, "descs is NULL");
+    if (count < 1 || count > TERN_MAX_STEP)
+        return fail(TERN_ERR_INVALID_ARG, "count must be 1..%d (got %d)", TERN_MAX_STEP, count);
+    static MatDesc d[TERN_MAX_STEP];
+    for (int i = 0; i < count; i++) {
+        tern_status st = check_nk(descs[i].N, descs[i].K);
+        if (st != TERN_OK) return st;
+        if (descs[i].K % 1024 != 0)
+            return fail(TERN_ERR_SHAPE, "tern_gemv_step needs K a multiple of 1024 (descriptor %d has K=%lld)", i,
+                        static_cast<long long>(descs[i].K));
+        st = check_mat(descs[i].x, descs[i].slots, descs[i].scales, descs[i].y);
+        if (st != TERN_OK) return st;
+        d[i] = mat(descs[i].x, descs[i].slots, descs[i].scales, descs[i].y, descs[i].N, descs[i].K);
+    }
+    if (!gemv_step_supports(d, count)) return fail(TERN_ERR_SHAPE, "tern_gemv_step: K too large for shared memory");
+    return launch_gemv_step(d, count, static_cast<cudaStream_t>(stream));
+}
+
 tern_status tern_gemv_grouped(const tern_gemv_desc *descs, int32_t count, int64_t M,
                               void *workspace, size_t ws_bytes, void *stream) {
     clear_error();
@@ -354,10 +374,14 @@ tern_status tern_sync_status(void *stream) {
     unsigned int t5 = 0;
     st = read_gemvtm_status(true, &t5);
     if (st != TERN_OK) return st;
+    unsigned int t6 = 0;
+    st = read_gemvstep_status(true, &t6);
+    if (st != TERN_OK) return st;
     if (v == 0) v = w;
     if (v == 0) v = u;
     if (v == 0) v = z;
     if (v == 0) v = t5;
+    if (v == 0) v = t6;
     if (v != 0) return fail(static_cast<tern_status>(v), "a kernel gave up a bounded wait on the device");
     return TERN_OK;
 }

@@ -35,6 +35,7 @@
 #include <cstring>
 
 #include "tern_internal.cuh"
+#include "tern_unpack_mma.cuh"
 
 namespace tern {
 
@@ -94,81 +95,6 @@ size_t smem_bytes(int ns, int xs_halves, int kmax, bool gc) {
     return 1024 + ring_off + static_cast<size_t>(ncons(gc)) * ns * (kSlotBytes + kScaleBytes);
 }
 
-constexpr uint32_t kOnes = 0x55555555u;  // every 2-bit field = code 1 (t = 0)
-
-// D = A * B + C and D = A * B, m16n8k16, fp16 in, fp32 accumulate (no side
-// effects, so the compiler may interleave the chains of neighbouring groups).
-__device__ __forceinline__ void mma_acc(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
-                                        uint32_t b0, uint32_t b1) {
-    asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 "
-        "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
-        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
-}
-__device__ __forceinline__ void mma_zero(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
-                                         uint32_t b0, uint32_t b1) {
-    asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 "
-        "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%10,%10,%10,%10};"
-        : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
-        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "f"(0.0f));
-}
-
-// Index (in halves) of x[m][kl] in this kernel's staging area.  Per group
-// of 128 k the B fragments of its eight mmas: chunk i (pairs j = 2i, 2i+1)
-// holds, per token m and lane q (words 2q, 2q+1 of the group), 8 halves
-// [j & 1][word 2q + wi][half] = x at word position j (lo) and j+8 (hi).
-// Layout [group][chunk][m][q][8]: a lane's four 16-byte loads hit distinct
-// banks within every quarter warp.
-template <int MT>
-__device__ __forceinline__ int xs_pair_index(int m, int kl) {
-    const int grp = kl >> 7;
-    const int word = (kl >> 4) & 7;
-    const int hi = (kl >> 3) & 1;
-    const int j = kl & 7;
-    return (((grp * 4 + (j >> 1)) * MT + m) * 4 + (word >> 1)) * 8 + (j & 1) * 4 + (word & 1) * 2 + hi;
-}
-
-// The eight mmas of one 16-row x 128-k group: pair j of the lane's words
-// (a = row g, b = row g+8; .x = word 2q, .y = word 2q+1) against the staged x
-// of pair j, one accumulation chain (the unrolled groups of a slice give the
-// scheduler independent chains).  Shared by the weight path and the all-ones
-// pass, so the two round identically.
-__device__ __forceinline__ void group_mma_b(float (&c)[4], uint32_t ax, uint32_t ay, uint32_t bx, uint32_t by,
-                                            const uint4 &x0, const uint4 &x1, const uint4 &x2, const uint4 &x3) {
-    const uint32_t ax5 = ax >> 10, ay5 = ay >> 10, bx5 = bx >> 10, by5 = by >> 10;
-    mma_zero(c, ax & 0x00030003u, bx & 0x00030003u, ay & 0x00030003u, by & 0x00030003u, x0.x, x0.y);
-    mma_acc(c, ax & 0x000C000Cu, bx & 0x000C000Cu, ay & 0x000C000Cu, by & 0x000C000Cu, x0.z, x0.w);
-    mma_acc(c, ax & 0x00300030u, bx & 0x00300030u, ay & 0x00300030u, by & 0x00300030u, x1.x, x1.y);
-    mma_acc(c, ax & 0x00C000C0u, bx & 0x00C000C0u, ay & 0x00C000C0u, by & 0x00C000C0u, x1.z, x1.w);
-    mma_acc(c, ax & 0x03000300u, bx & 0x03000300u, ay & 0x03000300u, by & 0x03000300u, x2.x, x2.y);
-    mma_acc(c, ax5 & 0x00030003u, bx5 & 0x00030003u, ay5 & 0x00030003u, by5 & 0x00030003u, x2.z, x2.w);
-    mma_acc(c, ax5 & 0x000C000Cu, bx5 & 0x000C000Cu, ay5 & 0x000C000Cu, by5 & 0x000C000Cu, x3.x, x3.y);
-    mma_acc(c, ax5 & 0x00300030u, bx5 & 0x00300030u, ay5 & 0x00300030u, by5 & 0x00300030u, x3.z, x3.w);
-}
-
-// The four B-fragment loads of one group (chunks of MT x 32 x 8 halves).
-template <int MT>
-__device__ __forceinline__ void load_xfrag(const __half *xb, uint4 (&xf)[4]) {
-    constexpr int kChunk = MT * 32;
-#pragma unroll
-    for (int i = 0; i < 4; i++) xf[i] = *reinterpret_cast<const uint4 *>(xb + i * kChunk);
-}
-
-template <int MT>
-__device__ __forceinline__ void group_mma(float (&c)[4], uint32_t ax, uint32_t ay, uint32_t bx, uint32_t by,
-                                          const __half *xb) {
-    uint4 xf[4];
-    load_xfrag<MT>(xb, xf);
-    group_mma_b(c, ax, ay, bx, by, xf[0], xf[1], xf[2], xf[3]);
-}
-
-// Lane q's pick among four values (q = 0..3).
-__device__ __forceinline__ float sel4(int q, float a, float b, float c, float d) {
-    const float lo = (q & 1) ? b : a;
-    const float hi = (q & 1) ? d : c;
-    return (q & 2) ? hi : lo;
-}
-
 __device__ __forceinline__ bool mbar_test_wait(uint64_t *bar, uint32_t parity) {
     uint32_t ok;
     asm volatile(
@@ -191,7 +117,6 @@ __device__ __forceinline__ bool pc_wait(uint64_t *bar, uint32_t parity, unsigned
     return true;
 }
 
-__device__ __forceinline__ int tile_row(int g) { return g < 4 ? 2 * g : 2 * g - 7; }
 
 // Work of warp w (consumer w, or producer lane w) of CTA lc of a matrix: the
 // CTA owns tiles [t0, t1) (balanced to one tile), whose (tile, slice) units
@@ -487,30 +412,8 @@ __global__ void __launch_bounds__(nthreads(GC), 1) gemv_pc_kernel(const __grid_c
                     }
                     issued_end++;
                 }
-                float dd[kSG][4];
-#pragma unroll
-                for (int j = 0; j < 8; j++) {
-                    if (j == 5) {
-#pragma unroll
-                        for (int G8 = 0; G8 < kSG; G8++)
-#pragma unroll
-                            for (int i = 0; i < 4; i++) wd[G8][i] >>= 10;
-                    }
-                    const uint32_t m = 0x00030003u << (2 * (j < 5 ? j : j - 5));
-                    const uint4 &xv = xf[j >> 1];
-                    const uint32_t b0 = (j & 1) ? xv.z : xv.x, b1 = (j & 1) ? xv.w : xv.y;
-#pragma unroll
-                    for (int G8 = 0; G8 < kSG; G8++) {
-                        if (j == 0)
-                            mma_zero(dd[G8], wd[G8][0] & m, wd[G8][1] & m, wd[G8][2] & m, wd[G8][3] & m, b0, b1);
-                        else
-                            mma_acc(dd[G8], wd[G8][0] & m, wd[G8][1] & m, wd[G8][2] & m, wd[G8][3] & m, b0, b1);
-                    }
-                }
-                const float v0 = sel4(q, dd[0][0], dd[2][0], dd[4][0], dd[6][0]);
-                const float v1 = sel4(q, dd[1][1], dd[3][1], dd[5][1], dd[7][1]);
-                const float v2 = sel4(q, dd[0][2], dd[2][2], dd[4][2], dd[6][2]);
-                const float v3 = sel4(q, dd[1][3], dd[3][3], dd[5][3], dd[7][3]);
+                float v0, v1, v2, v3;
+                gc_slice(wd, xf, q, v0, v1, v2, v3);
                 const float2 fa = __half22float2(sa2), fb = __half22float2(sb2);
                 acc[0] = fmaf(fa.x, v0 - on.x, acc[0]);
                 acc[0] = fmaf(fa.y, v1 - on.y, acc[0]);

@@ -1,0 +1,521 @@
+// One persistent launch for a whole decode step of M = 1 ternary-g128
+// products: many independent matrices (every projection of every layer and
+// the output head) streamed by all SMs as one flat list of weight tiles.
+//
+// What it computes: y_i[n] = sum_k x_i[k] * s_i[n][k/128] * t_i[n][k] for
+// every matrix i, with t read straight from the 2-bit slots and the group
+// scale applied inside the product ("Ternary-Bonsai-27B" model summary,
+// aitrends.kr, section "Technical features").  Generation speed is set by the
+// bytes read per token ("Bonsai 27B ternary / 1-bit quantization",
+// ThakiCloud blog, section "Throughput and speculative decoding"): one launch
+// for the step removes the per-launch start-up and drain of every SM, which
+// per-matrix launches pay once per matrix.
+//
+// Work split: the tiles (16 weight rows) of all matrices, in order, form one
+// list; the host cuts it into one contiguous range per CTA with equal
+// numbers of 1024-k units (slices).  Inside a CTA each matrix's part is a
+// "piece": its x is staged once (all warps), its units are split evenly over
+// the sixteen warps, and tiles shared by two warps are summed in warp order
+// after the piece (deterministic, no atomics, no scratch).
+//
+// Loads: every warp keeps its own ring of ns stages; a stage is one unit, two
+// 128-byte-swizzled boxes of 16 slot rows x 128 bytes (one 3-D tensor copy)
+// plus the 16 x 8 fp16 scales (one 2-D tensor copy), completing on the
+// stage's mbarrier.  The tensor maps travel in the kernel parameters, which
+// bounds one launch to kMaxPer matrices; the host splits longer lists into
+// several launches.  The ring runs ahead across piece boundaries: weights
+// never depend on the preceding launch or piece.
+//
+// Arithmetic: the group-per-column mma.sync form (tern_unpack_mma.cuh).
+#include <algorithm>
+#include <cstring>
+
+#include "tern_internal.cuh"
+#include "tern_unpack_mma.cuh"
+
+namespace tern {
+
+// Device-side record of a bounded wait in this kernel that gave up.
+__device__ unsigned int g_tern_gemvstep_status;
+
+namespace {
+
+constexpr int kW = 16;                    // warps per CTA, all consumers
+constexpr int kThreads = kW * 32;
+constexpr int kRows = 16;                 // tile rows (mma M)
+constexpr int kSG = 8;                    // scale groups per unit (1024 k)
+constexpr int kBox = 128;                 // bytes per row of one slot box (512 k)
+constexpr int kSlotStage = kRows * kBox * 2;           // two boxes: 4096
+constexpr int kScaleStage = kRows * kSG * 2;           // 256
+constexpr int kStageBytes = kSlotStage + kScaleStage;  // 4352
+constexpr int kMaxNS = 4;
+constexpr int kMaxCtas = 160;
+constexpr int kMaxPer = 96;               // matrices per launch (parameter space)
+constexpr size_t kSmemBudget = 232448;
+
+struct SDesc {
+    const __half *x;
+    __half *y;
+    int N, K;
+    int tile0;   // first tile of this matrix in the flat tile list
+    int ntile;   // ceil(N / 16)
+};
+
+struct alignas(64) SMaps {
+    CUtensorMap smap;   // slots as uint8 [K/512][N][128], box 128 B x 16 rows x 2, 128-byte swizzle
+    CUtensorMap cmap;   // scales fp16 [N][K/128], box 8 x 16, no swizzle
+};
+
+struct SParams {
+    SMaps m[kMaxPer];
+    SDesc d[kMaxPer];
+    int cta_tile[kMaxCtas + 1];   // flat tile range [cta_tile[c], cta_tile[c + 1]) of CTA c
+    int count;
+    unsigned int smem_usable;     // dynamic shared memory past the 1024-byte alignment
+    int kmax;
+    int skip_loads;               // test only: issue no copies (exercises the timeout path)
+    unsigned long long timeout_ns;
+};
+
+// Shared memory layout (bytes from the 128-aligned base).
+__host__ __device__ constexpr int bar_off() { return 0; }
+__host__ __device__ constexpr int rec_off() { return kW * kMaxNS * 8; }               // [kW][2][8] float2
+__host__ __device__ constexpr int rtile_off() { return rec_off() + kW * 2 * 8 * 8; }  // [kW][2] int
+__host__ __device__ constexpr int wmax_off() { return rtile_off() + kW * 2 * 4; }     // [kW] uint
+__host__ __device__ constexpr int d1_off() { return wmax_off() + kW * 4; }            // [kmax / 128] float
+__host__ __device__ constexpr int xs_off(int kmax) { return d1_off() + (kmax / 128) * 4 + 64; }
+__host__ __device__ constexpr int ring_off(int kmax) { return (xs_off(kmax) + kmax * 2 + 1023) & ~1023; }
+size_t smem_bytes(int kmax, int ns) { return 1024 + static_cast<size_t>(ring_off(kmax)) + static_cast<size_t>(kW) * ns * kStageBytes; }
+
+__device__ __forceinline__ bool step_wait(uint64_t *bar, uint32_t parity, unsigned long long deadline) {
+    while (!mbar_try_wait(bar, parity)) {
+        if (globaltimer() > deadline) {
+            atomicExch(&g_tern_gemvstep_status, static_cast<unsigned int>(TERN_ERR_TIMEOUT));
+            return false;
+        }
+    }
+    return true;
+}
+
+// A warp's position in its own sequence of units: piece = matrix i inside
+// this CTA's tile range, units [v, vend) of it (tile-major, slice inner).
+struct Cursor {
+    int i;          // matrix, or -1 when the sequence is exhausted
+    int tbeg;       // first tile of the piece (matrix-relative)
+    int B;          // units per tile (K / 1024)
+    int v, vend;    // this warp's next unit and end within the piece
+};
+
+__device__ __forceinline__ void piece_range(const SDesc &d, int T0, int T1, int warp, int &tbeg, int &U, int &v0,
+                                            int &v1) {
+    tbeg = max(T0, d.tile0) - d.tile0;
+    const int tend = min(T1, d.tile0 + d.ntile) - d.tile0;
+    U = (tend - tbeg) * (d.K >> 10);
+    v0 = static_cast<int>((static_cast<long long>(U) * warp) / kW);
+    v1 = static_cast<int>((static_cast<long long>(U) * (warp + 1)) / kW);
+}
+
+__device__ __forceinline__ void cursor_settle(Cursor &c, const SParams &p, int T1, int warp, int T0) {
+    while (c.i >= 0 && c.v >= c.vend) {
+        c.i++;
+        if (c.i >= p.count || p.d[c.i].tile0 >= T1) {
+            c.i = -1;
+            return;
+        }
+        int U;
+        piece_range(p.d[c.i], T0, T1, warp, c.tbeg, U, c.v, c.vend);
+        c.B = p.d[c.i].K >> 10;
+    }
+}
+
+__global__ void __launch_bounds__(kThreads, 1) gemv_step_kernel(const __grid_constant__ SParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *base = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    uint64_t *full = reinterpret_cast<uint64_t *>(base + bar_off());  // [kW][kMaxNS]
+    float *rec = reinterpret_cast<float *>(base + rec_off());
+    int *rec_tile = reinterpret_cast<int *>(base + rtile_off());
+    unsigned int *wmax = reinterpret_cast<unsigned int *>(base + wmax_off());
+    float *d1 = reinterpret_cast<float *>(base + d1_off());
+    __half *xs = reinterpret_cast<__half *>(base + xs_off(p.kmax));
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int g = lane >> 2, q = lane & 3;
+    const int row = tile_row(g);
+    uint32_t off[4];  // 128-byte-swizzled position of words 2q, 2q+1 of group j (0..3 in a box) of `row`
+#pragma unroll
+    for (int j = 0; j < 4; j++) off[j] = row * kBox + (((2 * j + (q >> 1)) ^ (row & 7)) << 4) + (q & 1) * 8;
+    const int T0 = p.cta_tile[blockIdx.x], T1 = p.cta_tile[blockIdx.x + 1];
+    // first matrix with a tile at or after T0
+    int i0 = 0;
+    {
+        int lo = 0, hi = p.count - 1;
+        while (lo < hi) {
+            const int mid = (lo + hi) >> 1;
+            if (p.d[mid].tile0 + p.d[mid].ntile <= T0) lo = mid + 1; else hi = mid;
+        }
+        i0 = lo;
+    }
+    // The ring takes what this CTA's largest staged x leaves (2..4 stages).
+    int kcta = 1024;
+    for (int i = i0; T0 < T1 && i < p.count && p.d[i].tile0 < T1; i++) kcta = max(kcta, p.d[i].K);
+    const uint32_t roff = (static_cast<uint32_t>(xs_off(p.kmax)) + 2u * kcta + 1023u) & ~1023u;
+    const int ns = min(kMaxNS, static_cast<int>((p.smem_usable - roff) / (kW * kStageBytes)));
+    uint8_t *ring = base + roff;
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < kW * kMaxNS; i++) mbar_init(&full[i], 1);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    __syncthreads();
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    const unsigned long long deadline = globaltimer() + p.timeout_ns;
+    uint64_t *my_full = full + warp * kMaxNS;
+    // slot stages (4096 bytes, 1024-aligned: the 128-byte swizzle pattern is
+    // tied to the address) for all warps first, then the 256-byte scale stages
+    uint8_t *my_ring = ring + warp * ns * kSlotStage;
+    uint8_t *my_scl = ring + kW * ns * kSlotStage + warp * ns * kScaleStage;
+
+    // ---- issue side: this warp's units, in order, into its ring ----
+    Cursor ic;
+    ic.i = T0 < T1 ? i0 : -1;
+    if (ic.i >= 0) {
+        int U;
+        piece_range(p.d[ic.i], T0, T1, warp, ic.tbeg, U, ic.v, ic.vend);
+        ic.B = p.d[ic.i].K >> 10;
+        cursor_settle(ic, p, T1, warp, T0);
+    }
+    if (p.skip_loads) ic.i = -1;
+    long long issued = 0;
+    // Lane 0 issues; all lanes keep the cursor (uniform).  Rows past N are
+    // filled with zeros by the copy and never stored.
+    auto issue = [&](int st) {
+        const int tile = ic.tbeg + ic.v / ic.B;
+        const int kb = ic.v - (ic.v / ic.B) * ic.B;
+        if (lane == 0) {
+            uint8_t *stage = my_ring + st * kSlotStage;
+            mbar_expect_tx(&my_full[st], kStageBytes);
+            tma_load_3d(stage, &p.m[ic.i].smap, 0, tile * kRows, kb * 2, &my_full[st]);
+            tma_load_2d(my_scl + st * kScaleStage, &p.m[ic.i].cmap, kb * kSG, tile * kRows, &my_full[st]);
+        }
+        ic.v++;
+        cursor_settle(ic, p, T1, warp, T0);
+        issued++;
+    };
+    for (int st = 0; st < ns && ic.i >= 0; st++) issue(st);
+
+    // x may be the output of the preceding launch: wait for it to finish.
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+
+    int s = 0;
+    uint32_t ph = 0;
+    long long consumed = 0;
+    bool dead = false;
+    const int nthr = kThreads;
+    for (int i = i0; T0 < T1 && i < p.count && p.d[i].tile0 < T1; i++) {
+        const SDesc &d = p.d[i];
+        const int K = d.K, N = d.N, B = K >> 10;
+        // ---- stage x of matrix i: E from max |x|, pair order, all-ones sums ----
+        __syncthreads();  // the previous piece is finished with xs, d1, rec
+        {
+            unsigned int mx = 0;
+            for (int idx = threadIdx.x; idx < K / 8; idx += nthr) {
+                const uint4 v = *reinterpret_cast<const uint4 *>(d.x + static_cast<size_t>(idx) * 8);
+                const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                for (int e = 0; e < 4; e++) mx = __vmaxu2(mx, __vminu2(wv[e] & 0x7FFF7FFFu, 0x7BFF7BFFu));
+            }
+            mx = max(mx & 0xFFFFu, mx >> 16);
+            mx = __reduce_max_sync(0xffffffffu, mx);
+            if (lane == 0) wmax[warp] = mx;
+            if (lane < 2) rec_tile[warp * 2 + lane] = -1;
+        }
+        __syncthreads();
+        unsigned int mx = 0;
+#pragma unroll
+        for (int w = 0; w < kW; w++) mx = max(mx, wmax[w]);
+        const int ex = max(static_cast<int>(mx >> 10), 1) - 15;
+        const int E = min(8, 15 - ex);
+        {
+            uint32_t fac2[4];
+#pragma unroll
+            for (int c = 0; c < 4; c++) {
+                const int e0 = E - 2 * (2 * c < 5 ? 2 * c : 2 * c - 5);
+                const int e1 = E - 2 * (2 * c + 1 < 5 ? 2 * c + 1 : 2 * c + 1 - 5);
+                fac2[c] = (static_cast<uint32_t>(15 + e0) << 10) | (static_cast<uint32_t>(15 + e1) << 26);
+            }
+            for (int idx = threadIdx.x; idx < K / 8; idx += nthr) {
+                const uint4 v = *reinterpret_cast<const uint4 *>(d.x + static_cast<size_t>(idx) * 8);
+                const uint32_t pr[4] = {v.x, v.y, v.z, v.w};
+                const int kl = idx * 8;
+                unsigned short *dst =
+                    reinterpret_cast<unsigned short *>(xs + xs_pair_index<8>((kl >> 7) & 7, ((kl >> 10) << 7) | (kl & 127)));
+#pragma unroll
+                for (int c = 0; c < 4; c++) {
+                    uint32_t h2;
+                    asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(h2) : "r"(pr[c]), "r"(fac2[c]));
+                    dst[c * 256] = static_cast<unsigned short>(h2);
+                    dst[c * 256 + 4] = static_cast<unsigned short>(h2 >> 16);
+                }
+            }
+        }
+        __syncthreads();
+        const __half *xlane = xs + lane * 8;
+        for (int sl = warp; sl < B; sl += kW) {
+            float c[4];
+            group_mma<8>(c, kOnes, kOnes, kOnes, kOnes, xlane + sl * 1024);
+            if (g == 0) *reinterpret_cast<float2 *>(d1 + sl * kSG + 2 * q) = make_float2(c[0], c[1]);
+        }
+        __syncthreads();
+
+        // ---- this warp's units of the piece ----
+        int tbeg, U, v0, v1;
+        piece_range(d, T0, T1, warp, tbeg, U, v0, v1);
+        const float post = ldexpf(1.0f, 24 - E);
+        float acc0 = 0.f, acc2 = 0.f;
+        for (int v = v0; v < v1; v++) {
+            bool ok = !dead;
+            if (ok) ok = __all_sync(0xffffffffu, step_wait(&my_full[s], ph, deadline));
+            dead = dead || !ok;
+            const int kb = v % B;
+            if (ok) {
+                const uint8_t *stage = my_ring + s * kSlotStage;
+                const uint8_t *scs = my_scl + s * kScaleStage;
+                uint32_t wd[kSG][4];
+#pragma unroll
+                for (int G8 = 0; G8 < kSG; G8++) {
+                    const uint8_t *bx = stage + (G8 >> 2) * (kRows * kBox);
+                    const uint2 a = *reinterpret_cast<const uint2 *>(bx + off[G8 & 3]);
+                    const uint2 b = *reinterpret_cast<const uint2 *>(bx + off[G8 & 3] + 8 * kBox);
+                    wd[G8][0] = a.x;
+                    wd[G8][1] = b.x;
+                    wd[G8][2] = a.y;
+                    wd[G8][3] = b.y;
+                }
+                const __half2 sa2 = *reinterpret_cast<const __half2 *>(scs + row * 16 + 4 * q);
+                const __half2 sb2 = *reinterpret_cast<const __half2 *>(scs + (row + 8) * 16 + 4 * q);
+                // The stage is in registers: refill it with this warp's next
+                // unit (the warp barrier and the proxy fence order the reads
+                // before the copy that overwrites it).
+                __syncwarp();
+                consumed++;
+                if (ic.i >= 0) {
+                    if (lane == 0) asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                    issue(s);
+                }
+                uint4 xf[4];
+                load_xfrag<8>(xlane + kb * 1024, xf);
+                const float2 on = *reinterpret_cast<const float2 *>(d1 + kb * kSG + 2 * q);
+                float w0, w1, w2, w3;
+                gc_slice(wd, xf, q, w0, w1, w2, w3);
+                const float2 fa = __half22float2(sa2), fb = __half22float2(sb2);
+                acc0 = fmaf(fa.x, w0 - on.x, acc0);
+                acc0 = fmaf(fa.y, w1 - on.y, acc0);
+                acc2 = fmaf(fb.x, w2 - on.x, acc2);
+                acc2 = fmaf(fb.y, w3 - on.y, acc2);
+            }
+            if (++s == ns) {
+                s = 0;
+                ph ^= 1;
+            }
+            if (kb == B - 1 || v + 1 == v1) {
+                // ---- this warp's part of a tile is complete ----
+                acc0 += __shfl_xor_sync(0xffffffffu, acc0, 1);
+                acc0 += __shfl_xor_sync(0xffffffffu, acc0, 2);
+                acc2 += __shfl_xor_sync(0xffffffffu, acc2, 1);
+                acc2 += __shfl_xor_sync(0xffffffffu, acc2, 2);
+                const int tile = tbeg + v / B;
+                const bool whole = kb == B - 1 && (v / B != v0 / B || v0 % B == 0);
+                if (whole) {
+                    if (!dead && q == 0) {
+                        const int n0 = tile * kRows + row, n1 = n0 + 8;
+                        if (n0 < N) d.y[n0] = __float2half_rn(acc0 * post);
+                        if (n1 < N) d.y[n1] = __float2half_rn(acc2 * post);
+                    }
+                } else {
+                    const int slot = (v / B == v0 / B) ? 0 : 1;
+                    if (q == 0)
+                        *reinterpret_cast<float2 *>(rec + ((warp * 2 + slot) * 8 + g) * 2) =
+                            make_float2(acc0 * post, acc2 * post);
+                    if (lane == 0) rec_tile[warp * 2 + slot] = dead ? -2 : tile;
+                }
+                acc0 = acc2 = 0.f;
+            }
+        }
+        // ---- tiles of this piece split over several warps: summed in warp
+        // order by the first warp that holds a part ----
+        __syncthreads();
+#pragma unroll 1
+        for (int slot = 0; slot < 2; slot++) {
+            const int tile = rec_tile[warp * 2 + slot];
+            if (tile < 0) continue;
+            bool owner = true;
+            for (int w2 = 0; w2 < warp; w2++)
+                if (rec_tile[w2 * 2] == tile || rec_tile[w2 * 2 + 1] == tile) owner = false;
+            if (!owner) continue;
+            bool bad = false;
+            for (int w2 = 0; w2 < kW; w2++)
+                if (rec_tile[w2 * 2] == -2 || rec_tile[w2 * 2 + 1] == -2) bad = true;
+            if (bad) continue;
+            float s0 = 0.f, s2 = 0.f;
+            for (int w2 = warp; w2 < kW; w2++)
+                for (int s2i = 0; s2i < 2; s2i++) {
+                    if (rec_tile[w2 * 2 + s2i] != tile) continue;
+                    const float2 o = *reinterpret_cast<const float2 *>(rec + ((w2 * 2 + s2i) * 8 + g) * 2);
+                    s0 += o.x;
+                    s2 += o.y;
+                }
+            if (q == 0) {
+                const int n0 = tile * kRows + row, n1 = n0 + 8;
+                if (n0 < N) d.y[n0] = __float2half_rn(s0);
+                if (n1 < N) d.y[n1] = __float2half_rn(s2);
+            }
+        }
+    }
+    // A warp that gave up may still have copies of its own in flight: they
+    // must land before the CTA exits (bounded).
+    if (dead) {
+        const unsigned long long dl2 = globaltimer() + p.timeout_ns;
+        for (long long u = consumed; u < issued; u++) {
+            const int st = static_cast<int>(u % ns);
+            const uint32_t phs = static_cast<uint32_t>((u / ns) & 1);
+            step_wait(&my_full[st], phs, dl2);
+        }
+    }
+}
+
+bool g_attr_step[64];
+
+}  // namespace
+
+bool gemv_step_supports(const MatDesc *md, int count) {
+    if (count < 1 || count > TERN_MAX_STEP) return false;
+    int kmax = 0;
+    for (int i = 0; i < count; i++) {
+        if (md[i].K % 1024 != 0) return false;
+        kmax = std::max(kmax, md[i].K);
+    }
+    return smem_bytes(kmax, 2) <= kSmemBudget;
+}
+
+namespace {
+
+// One launch over md[0..count) (count <= kMaxPer).
+tern_status launch_chunk(const DeviceInfo &dev, const MatDesc *md, int count, cudaStream_t stream) {
+    static SParams p;  // large (parameter space); filled on the host for each launch
+    std::memset(&p, 0, sizeof(p));
+    int kmax = 0;
+    long long total_units = 0;
+    int tiles = 0;
+    for (int i = 0; i < count; i++) {
+        SDesc &d = p.d[i];
+        d.x = md[i].x;
+        d.y = md[i].y;
+        d.N = md[i].N;
+        d.K = md[i].K;
+        d.tile0 = tiles;
+        d.ntile = (md[i].N + kRows - 1) / kRows;
+        tiles += d.ntile;
+        total_units += static_cast<long long>(d.ntile) * (md[i].K / 1024);
+        kmax = std::max(kmax, md[i].K);
+        // the slot matrix seen as [K/512 chunks][N rows][128 bytes]: one copy
+        // brings both 512-k boxes of a unit
+        const uint64_t sdims[3] = {static_cast<uint64_t>(kBox), static_cast<uint64_t>(md[i].N),
+                                   static_cast<uint64_t>(md[i].K / 512)};
+        const uint64_t sstr[2] = {static_cast<uint64_t>(md[i].K / 4), static_cast<uint64_t>(kBox)};
+        const uint32_t sbox[3] = {static_cast<uint32_t>(kBox), static_cast<uint32_t>(kRows), 2};
+        tern_status st = encode_tiled_3d(&p.m[i].smap, CU_TENSOR_MAP_DATA_TYPE_UINT8, md[i].slots, sdims, sstr, sbox,
+                                         CU_TENSOR_MAP_SWIZZLE_128B);
+        if (st != TERN_OK) return st;
+        const int G = md[i].K / kGroup;
+        st = encode_tiled_2d(&p.m[i].cmap, CU_TENSOR_MAP_DATA_TYPE_UINT16, md[i].scales, static_cast<uint64_t>(G),
+                             static_cast<uint64_t>(md[i].N), static_cast<uint64_t>(G) * 2, kSG, kRows,
+                             CU_TENSOR_MAP_SWIZZLE_NONE);
+        if (st != TERN_OK) return st;
+    }
+    const size_t budget = std::min<size_t>(kSmemBudget, dev.max_smem_optin);
+    // The whole budget: every CTA sizes its ring from what its own staged x leaves.
+    const size_t smem = std::min(budget, smem_bytes(kmax, kMaxNS));
+    if (smem_bytes(kmax, 2) > smem) return fail(TERN_ERR_SHAPE, "step kernel needs %zu B of shared memory", smem_bytes(kmax, 2));
+    int grid = std::min<int>(std::min(dev.sms, kMaxCtas), tiles);
+    if (g_opt.gemv_grid > 0) grid = std::min(grid, g_opt.gemv_grid);
+    // Cut the flat tile list into `grid` ranges of about equal units: CTA c
+    // starts at the first tile boundary at or after c * total / grid units.
+    p.cta_tile[0] = 0;
+    {
+        int i = 0;
+        long long ubase = 0;  // units before matrix i
+        for (int c = 1; c < grid; c++) {
+            const long long target = (total_units * c) / grid;
+            while (i < count && ubase + static_cast<long long>(p.d[i].ntile) * (p.d[i].K / 1024) <= target) {
+                ubase += static_cast<long long>(p.d[i].ntile) * (p.d[i].K / 1024);
+                i++;
+            }
+            int t = tiles;
+            if (i < count) {
+                const long long B = p.d[i].K / 1024;
+                t = p.d[i].tile0 + static_cast<int>((target - ubase + B - 1) / B);
+            }
+            p.cta_tile[c] = std::max(p.cta_tile[c - 1], std::min(t, tiles));
+        }
+        p.cta_tile[grid] = tiles;
+    }
+    p.count = count;
+    p.smem_usable = static_cast<unsigned int>(smem - 1024);
+    p.kmax = kmax;
+    p.skip_loads = g_gemm_skip_loads;
+    p.timeout_ns = g_gemm_timeout_ns;
+    cudaLaunchConfig_t cfg;
+    std::memset(&cfg, 0, sizeof(cfg));
+    cfg.gridDim = dim3(static_cast<unsigned>(grid));
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, gemv_step_kernel, p);
+    if (e != cudaSuccess) return cuda_fail(e, "gemv step kernel launch");
+    return TERN_OK;
+}
+
+}  // namespace
+
+tern_status launch_gemv_step(const MatDesc *md, int count, cudaStream_t stream) {
+    DeviceInfo dev;
+    tern_status st = current_device(&dev);
+    if (st != TERN_OK) return st;
+    if (!gemv_step_supports(md, count)) return fail(TERN_ERR_SHAPE, "step kernel: unsupported shapes");
+    if (!g_attr_step[dev.device]) {
+        cudaError_t e = cudaFuncSetAttribute(gemv_step_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             static_cast<int>(dev.max_smem_optin));
+        if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(gemv step)");
+        g_attr_step[dev.device] = true;
+    }
+    // Equal-sized launches of at most kMaxPer matrices each.
+    const int launches = (count + kMaxPer - 1) / kMaxPer;
+    int done = 0;
+    for (int l = 0; l < launches; l++) {
+        const int n = (count - done) / (launches - l);
+        st = launch_chunk(dev, md + done, n, stream);
+        if (st != TERN_OK) return st;
+        done += n;
+    }
+    return TERN_OK;
+}
+
+tern_status read_gemvstep_status(bool reset, unsigned int *out) {
+    unsigned int v = 0;
+    cudaError_t e = cudaMemcpyFromSymbol(&v, g_tern_gemvstep_status, sizeof(v));
+    if (e != cudaSuccess) return cuda_fail(e, "reading device status");
+    if (reset && v != 0) {
+        const unsigned int zero = 0;
+        e = cudaMemcpyToSymbol(g_tern_gemvstep_status, &zero, sizeof(zero));
+        if (e != cudaSuccess) return cuda_fail(e, "clearing device status");
+    }
+    *out = v;
+    return TERN_OK;
+}
+
+}  // namespace tern

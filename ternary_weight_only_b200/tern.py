@@ -41,6 +41,8 @@ TERN_OPT_GEMV_PREFETCH = 9
 GEMV_VARIANT_DEFAULT, GEMV_VARIANT_RING, GEMV_VARIANT_TMA, GEMV_VARIANT_TC, GEMV_VARIANT_PC = 0, 1, 2, 3, 4
 GEMV_VARIANT_TMEM = 5
 TERN_MAX_GROUP = 16
+TERN_MAX_STEP = 512
+GEMV_VARIANT_PC_TOKEN_COLUMNS = 6
 
 _i64, _vp, _sz, _i32, _int = ctypes.c_int64, ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int32, ctypes.c_int
 
@@ -65,6 +67,7 @@ _SIGS = {
     "tern_sync_status": ([_vp], _int),
     "tern_gemv_grouped_workspace_bytes": ([ctypes.POINTER(tern_gemv_desc), _i32, _i64], _sz),
     "tern_gemv_noalloc": ([_vp, _vp, _vp, _vp, _i64, _i64, _vp], _int),
+    "tern_gemv_step": ([ctypes.POINTER(tern_gemv_desc), _i32, _vp], _int),
 }
 for _name, (_args, _res) in _SIGS.items():
     _f = getattr(_L, _name)
@@ -248,6 +251,20 @@ def tern_gemv_grouped(mats: Sequence, M: int, stream=None, workspace=None):
     need = _L.tern_gemv_grouped_workspace_bytes(arr, len(mats), M) if workspace is None else 0
     wp, wn = _ws_args(workspace, need, mats[0][0].device, st)
     _check(_L.tern_gemv_grouped(arr, len(mats), M, wp, wn, st), "tern_gemv_grouped")
+
+
+def tern_gemv_step(mats: Sequence, stream=None):
+    """mats: sequence of (x [K], slots [N,K/4], scales [N,K/128], y [N]) CUDA
+    tensors, M = 1, every K a multiple of 1024: one persistent launch."""
+    arr = (tern_gemv_desc * len(mats))()
+    for i, (x, s, sc, y) in enumerate(mats):
+        arr[i].x = _dev(x, "x", torch.float16)
+        arr[i].slots = _dev(s, "slots", torch.uint8)
+        arr[i].scales = _dev(sc, "scales", torch.float16)
+        arr[i].y = _dev(y, "y", torch.float16)
+        arr[i].N = s.shape[0]
+        arr[i].K = x.shape[-1]
+    _check(_L.tern_gemv_step(arr, len(mats), _stream(stream)), "tern_gemv_step")
 
 
 def tern_gemv_grouped_workspace_bytes(mats: Sequence, M: int) -> int:

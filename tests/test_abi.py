@@ -29,7 +29,7 @@ def lib():
 def test_header_declares_the_boundary():
     names = _declared()
     for n in ["tern_pack_g128", "tern_unpack_g128", "tern_gemv", "tern_gemm",
-              "tern_gemv_grouped", "tern_workspace_bytes", "tern_slots_bytes",
+              "tern_gemv_grouped", "tern_gemv_step", "tern_workspace_bytes", "tern_slots_bytes",
               "tern_scales_bytes", "tern_status_string", "tern_last_error", "tern_set_option",
               "tern_version"]:
         assert n in names
@@ -131,6 +131,30 @@ def test_grouped_rejects(lib):
     arr[1].K = 256
     arr[1].y = A + 2
     assert lib.tern_gemv_grouped(arr, 2, 1, None, 0, None) == 2
+
+
+def test_step_rejects(lib):
+    """tern_gemv_step: argument errors return before any launch."""
+    from ternary_weight_only_b200 import tern
+    arr = (tern.tern_gemv_desc * 3)()
+    for d in arr:
+        d.x, d.slots, d.scales, d.y, d.N, d.K = A, A, A, A, 16, 2048
+    assert lib.tern_gemv_step(None, 1, None) == 1
+    assert lib.tern_gemv_step(arr, 0, None) == 1
+    assert lib.tern_gemv_step(arr, tern.TERN_MAX_STEP + 1, None) == 1
+    arr[1].K = 1536                      # a multiple of 128 but not of 1024
+    assert lib.tern_gemv_step(arr, 3, None) == 3
+    arr[1].K = 1000                      # not a multiple of 128
+    assert lib.tern_gemv_step(arr, 3, None) == 3
+    arr[1].K = 2048
+    arr[2].N = 0
+    assert lib.tern_gemv_step(arr, 3, None) == 3
+    arr[2].N = 16
+    arr[2].slots = A + 8
+    assert lib.tern_gemv_step(arr, 3, None) == 2
+    arr[2].slots = A
+    arr[0].x = None
+    assert lib.tern_gemv_step(arr, 3, None) == 1
 
 
 def test_options(lib):

@@ -1,0 +1,143 @@
+"""The persistent decode-step launch (tern_gemv_step) against the fp64 oracle.
+
+Every output of every matrix of a call is compared, element by element, with
+the tolerance of helpers.check_close.  The cases cover: ragged N (partial last
+tiles), mixed K, many small matrices (several pieces per CTA), capped grids
+(pieces and split tiles in every CTA), a whole synthetic decode layer plus
+the output head at full size, exact cases, and the timeout path.
+"""
+import os
+
+import numpy as np
+import pytest
+import torch
+
+from helpers import check_close, np_inputs
+
+pytestmark = pytest.mark.gpu
+NCPU = os.cpu_count() or 1
+
+
+@pytest.fixture(scope="module")
+def T():
+    from ternary_weight_only_b200 import build
+    build.build()
+    from ternary_weight_only_b200 import tern
+    yield tern
+    tern.tern_set_option(tern.TERN_OPT_GEMV_GRID, 0)
+    tern.tern_set_option(tern.TERN_OPT_TEST_STALL_US, 0)
+
+
+def make_mats(orc, shapes, seed):
+    """Host inputs packed by the oracle; device copies; outputs pre-filled with NaN."""
+    from ternary_weight_only_b200 import synth
+    mats, refs = [], []
+    for j, (K, N) in enumerate(shapes):
+        x, codes, scales = synth.case(1, K, N, seed=seed + 17 * j, codes="sparse", outlier_p=0.01)
+        xn, cn, sn = np_inputs(x, codes, scales)
+        slots, sc, bad, _ = orc.pack(cn, sn)
+        assert bad == 0
+        y = torch.full((N,), float("nan"), dtype=torch.float16, device="cuda")
+        mats.append((x[0].cuda(), torch.from_numpy(slots).cuda(), scales.cuda(), y))
+        refs.append((xn, slots, sc))
+    return mats, refs
+
+
+def check_all(orc, mats, refs, what):
+    for j, ((xn, slots, sc), m) in enumerate(zip(refs, mats)):
+        y_ref, bound = orc.matmul(xn, slots, sc, threads=NCPU)
+        check_close(m[3].view(1, -1), y_ref, bound, f"{what} matrix {j} (K={m[0].shape[0]}, N={m[1].shape[0]})")
+
+
+@pytest.mark.parametrize("grid", [0, 1, 3, 7, 40])
+def test_mixed_shapes(T, orc, grid):
+    shapes = [(1024, 1), (2048, 17), (5120, 100), (1024, 16), (3072, 333), (6144, 64), (1024, 250),
+              (17408, 40), (4096, 129), (2048, 7)]
+    mats, refs = make_mats(orc, shapes, seed=7000 + grid)
+    T.tern_set_option(T.TERN_OPT_GEMV_GRID, grid)
+    try:
+        T.tern_gemv_step(mats)
+        T.tern_sync_status()
+    finally:
+        T.tern_set_option(T.TERN_OPT_GEMV_GRID, 0)
+    check_all(orc, mats, refs, f"step grid={grid}")
+
+
+def test_many_small_matrices(T, orc):
+    """More matrices than CTAs; every CTA crosses several pieces."""
+    rng = np.random.default_rng(5)
+    shapes = [(int(1024 * rng.integers(1, 5)), int(rng.integers(1, 90))) for _ in range(300)]
+    mats, refs = make_mats(orc, shapes, seed=7100)
+    T.tern_gemv_step(mats)
+    T.tern_sync_status()
+    check_all(orc, mats, refs, "step x300")
+
+
+def test_decode_layer_and_head(T, orc):
+    """The seven projections of a synthetic decode layer plus the 5120x151936
+    head, one launch, every output."""
+    from ternary_weight_only_b200 import synth
+    shapes = [(K, N) for _, K, N in synth.LAYER_PROJ] + [(synth.HEAD[1], synth.HEAD[2])]
+    mats, refs = make_mats(orc, shapes, seed=7200)
+    T.tern_gemv_step(mats)
+    T.tern_sync_status()
+    check_all(orc, mats, refs, "step layer+head")
+
+
+def test_matches_single_launches(T, orc):
+    """Each matrix of a step call meets the tolerance and agrees with tern_gemv
+    on the same inputs within it (the two differ only in summation order)."""
+    shapes = [(5120, 6144), (6144, 5120), (17408, 512)]
+    mats, refs = make_mats(orc, shapes, seed=7300)
+    T.tern_gemv_step(mats)
+    T.tern_sync_status()
+    for j, (x, slots, sc, y) in enumerate(mats):
+        y1 = T.tern_gemv(x, slots, sc)
+        T.tern_sync_status()
+        xn, sl, scn = refs[j]
+        y_ref, bound = orc.matmul(xn, sl, scn, threads=NCPU)
+        check_close(y.view(1, -1), y_ref, bound, f"step {j}")
+        check_close(y1.view(1, -1), y_ref, bound, f"single {j}")
+
+
+def test_exact_cases(T):
+    """All-zero codes give exactly zero; one-hot x gives s * t exactly."""
+    from ternary_weight_only_b200 import synth
+    N, K = 80, 3072
+    g = synth.gen(98, "cuda")
+    scales = synth.scales_uniform(N, K, g, device="cuda")
+    zero = torch.zeros((N, K), dtype=torch.int8, device="cuda")
+    zslots, zsc = T.tern_pack_g128(zero, scales)
+    codes = synth.codes_uniform(N, K, g, device="cuda")
+    slots, sc = T.tern_pack_g128(codes, scales)
+    x = synth.activations(1, K, g, device="cuda")[0]
+    ks = (0, 1, 7, 8, 15, 127, 128, 1000, 3071)
+    xes = []
+    for k in ks:
+        xe = torch.zeros(K, dtype=torch.float16, device="cuda")
+        xe[k] = 3.0
+        xes.append(xe)
+    y0 = torch.empty(N, dtype=torch.float16, device="cuda")
+    ys = [torch.empty(N, dtype=torch.float16, device="cuda") for _ in ks]
+    T.tern_gemv_step([(x, zslots, zsc, y0)] + [(xe, slots, sc, y) for xe, y in zip(xes, ys)])
+    T.tern_sync_status()
+    assert bool(torch.all(y0 == 0)), y0.abs().max()
+    for k, y in zip(ks, ys):
+        want = (3.0 * scales[:, k // 128].float() * codes[:, k].float()).half()
+        assert torch.equal(y, want), (k, (y.float() - want.float()).abs().max())
+
+
+def test_timeout_reported_and_context_survives(T, orc):
+    shapes = [(2048, 300), (1024, 64)]
+    mats, refs = make_mats(orc, shapes, seed=7400)
+    T.tern_set_option(T.TERN_OPT_TEST_STALL_US, 2000)
+    try:
+        T.tern_gemv_step(mats)
+        with pytest.raises(T.TernError) as ei:
+            T.tern_sync_status()
+        assert ei.value.status == T.TERN_ERR_TIMEOUT
+    finally:
+        T.tern_set_option(T.TERN_OPT_TEST_STALL_US, 0)
+    T.tern_gemv_step(mats)
+    T.tern_sync_status()
+    check_all(orc, mats, refs, "step after timeout")
