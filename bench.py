@@ -36,6 +36,7 @@ from ternary_weight_only_b200 import synth  # noqa: E402
 GROUP = 128
 METRIC = "ternary-g128 GEMV HBM GB/s (% of B200 peak); decode-step weight-stream ms"
 BYTES_PER_WEIGHT = 0.25 + 2.0 / GROUP  # 2-bit slot + fp16 scale per 128
+STEP_PER_LAUNCH = 96  # matrices one launch of the step kernel takes (tern_gemv_step splits longer lists)
 
 
 def wbytes(K, N):
@@ -70,7 +71,7 @@ class ClockSampler:
         0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting",
     }
 
-    def __init__(self, index: int, period_s: float = 0.005):
+    def __init__(self, index: int, period_s: float = 0.002):
         self.samples, self.reasons = [], 0
         self.period = period_s
         self.ok = False
@@ -195,7 +196,17 @@ class DecodeModel:
             self.groups.append(grp)
         self.head_io = (self.x_all[xo:xo + 5120], self.y_all[yo:yo + synth.HEAD[2]])
 
+    def all_mats(self):
+        _, K, N, slots, sc = self.head
+        return [m for grp in self.groups for m in grp] + [(self.head_io[0], slots, sc, self.head_io[1])]
+
     def step(self):
+        """One decode step: every projection of every layer and the head in
+        one tern_gemv_step call (the inputs are independent)."""
+        self.T.tern_gemv_step(self.all_mats())
+
+    def step_per_layer(self):
+        """The same step as one grouped launch per layer plus the head."""
         T = self.T
         for grp in self.groups:
             T.tern_gemv_grouped(grp, 1)
@@ -204,7 +215,8 @@ class DecodeModel:
 
     @property
     def launches_per_step(self):
-        return self.n_layers + 1
+        n = len(self.all_mats())
+        return (n + STEP_PER_LAUNCH - 1) // STEP_PER_LAUNCH
 
 
 def cuda_time(fn, iters, stream=None):
@@ -253,6 +265,18 @@ def proj_rows(T, model, peak_gbs, l2_bytes):
                 2 * synth.LAYER_PROJ[i][1] + 2 * synth.LAYER_PROJ[i][2] for i in idx)
         out[f"{label}_M1"] = {"us": round(ms * 1e3, 3), "GBps": round(b / ms / 1e6, 1),
                               "frac": round(b / ms / 1e6 / peak_gbs, 4)}
+    # one layer (seven projections) through the step kernel, rotating layers
+    fns = [lambda grp=grp: T.tern_gemv_step(grp) for grp in model.groups]
+    ms = graph_time(fns, s)
+    b = sum(wbytes(K, N) + 2 * K + 2 * N for _, K, N in synth.LAYER_PROJ)
+    out["layer_step_kernel_M1"] = {"us": round(ms * 1e3, 3), "GBps": round(b / ms / 1e6, 1),
+                                   "frac": round(b / ms / 1e6 / peak_gbs, 4)}
+    # the whole decode step as one grouped launch per layer plus the head
+    wb, xin, yout = step_bytes()
+    ms = graph_time([model.step_per_layer], s, reps=5)
+    out["decode_step_per_layer_launches"] = {"ms": round(ms, 4), "GBps": round((wb + xin + yout) / ms / 1e6, 1),
+                                             "frac": round((wb + xin + yout) / ms / 1e6 / peak_gbs, 4),
+                                             "launches": model.n_layers + 1}
     _, K, N, slots, sc = model.head
     # 206 MB of head weights per call: larger than L2, streamed cold each replay
     ms = graph_time([lambda: T.tern_gemv(model.head_io[0], slots, sc, model.head_io[1])], s, reps=20)
@@ -399,13 +423,13 @@ def run_reference(args):
 
 # ----------------------------------------------------------------- main ---
 # The kernel that carries the decode step (every grouped layer and the head).
-DOMINANT_KERNEL, DOMINANT_SOURCE = "gemv_pc_kernel", "tern_gemv_pc.cu"
+DOMINANT_KERNEL, DOMINANT_SOURCE = "gemv_step_kernel", "tern_gemv_step.cu"
 
 
 def traffic_from_profile(avg_launch_bytes):
     """Per-launch DRAM bytes of the dominant kernel from the committed ncu
     summary, only if the kernel source is unchanged since the capture."""
-    prof = os.path.join(ROOT, "profiles", f"{DOMINANT_KERNEL}.decode_layer.txt")
+    prof = os.path.join(ROOT, "profiles", f"{DOMINANT_KERNEL}.decode_step.txt")
     src = os.path.join(ROOT, "ternary_weight_only_b200", "csrc", DOMINANT_SOURCE)
     try:
         text = open(prof).read()
@@ -431,15 +455,22 @@ def run_profile(args):
     model = DecodeModel(T, n_layers=args.profile_layers)
     _, hK, hN, hslots, hsc = model.head
     for _ in range(3):
-        if args.profile_head:
+        if args.profile_step:
+            model.step()
+        elif args.profile_head:
             T.tern_gemv(model.head_io[0], hslots, hsc, model.head_io[1])
         else:
             for grp in model.groups:
                 T.tern_gemv_grouped(grp, 1)
     torch.cuda.synchronize()
-    per_launch = (wbytes(hK, hN) + 2 * hK + 2 * hN if args.profile_head
-                  else sum(wbytes(K, N) + 2 * K + 2 * N for _, K, N in synth.LAYER_PROJ))
+    layer = sum(wbytes(K, N) + 2 * K + 2 * N for _, K, N in synth.LAYER_PROJ)
+    head = wbytes(hK, hN) + 2 * hK + 2 * hN
+    if args.profile_step:
+        per_launch = (args.profile_layers * layer + head) / model.launches_per_step
+    else:
+        per_launch = head if args.profile_head else layer
     print(json.dumps({"profile_layers": args.profile_layers, "profile_head": bool(args.profile_head),
+                      "profile_step": bool(args.profile_step), "launches": model.launches_per_step,
                       "bytes_per_launch": per_launch}))
     return 0
 
@@ -527,7 +558,8 @@ def run_tern(args):
                                    "x N(0,1)",
                        "weights_bytes": wb, "bytes_per_step": total_bytes,
                        "l2": f"inputs {wb/1e9:.2f} GB >> L2 {l2/1e6:.0f} MB, no flush needed",
-                       "launch": "CUDA graph of 65 launches/step (one grouped launch per layer + head)",
+                       "launch": f"CUDA graph of {model.launches_per_step} launches/step (tern_gemv_step over all "
+                                 f"{len(model.all_mats())} products, at most {STEP_PER_LAUNCH} per launch)",
                        "parallelism": f"replicas x{ws}" if ws > 1 else "1 GPU"},
             "pct_of_peak_hbm": round(100 * value / ws / peak_gbs, 2),
             "e2e": {"value": round(e2e_value, 1), "unit": "GB/s", "ms_per_step": round(e2e_ms, 4),
@@ -561,6 +593,8 @@ def main():
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
     ap.add_argument("--profile-layers", type=int, default=0,
                     help="profiling case: build this many layers, run their grouped launches 3x, exit")
+    ap.add_argument("--profile-step", action="store_true",
+                    help="profiling case: run the layers and the head as tern_gemv_step calls 3x")
     ap.add_argument("--profile-head", action="store_true",
                     help="profiling case: run the 5120x151936 head launch 3x instead of the layers")
     ap.add_argument("--gemv-variant", type=int, default=0,
