@@ -258,18 +258,23 @@ __global__ void __launch_bounds__(nthreads(GC), 1) gemv_pc_kernel(const __grid_c
         // Group-per-column form: lane 0 loads the warp's own ring (unit v into
         // stage `st`); the first ns units go out before the grid-dependency
         // wait (weights are never written by a preceding launch).
-        auto issue = [&](int v, int st) {
-            const int tile = r.t0 + v / B;
-            const int kbx = v - (v / B) * B;
-            mbar_expect_tx(&my_full[st], kSlotBytes + kScaleBytes);
-            tma_load_3d(my_slots + st * kSlotBytes, &d.smap, 0, tile * kRows, kbx * 2, &my_full[st]);
-            tma_load_2d(my_scales + st * kScaleBytes, &d.cmap, kbx * kSG, tile * kRows, &my_full[st]);
+        // (tile, slice) of the next unit to issue, advanced by increments
+        int is_tile = r.t0 + r.u0 / B, is_kb = r.u0 - (r.u0 / B) * B;
+        auto issue = [&](int st) {
+            if (lane == 0) {
+                mbar_expect_tx(&my_full[st], kSlotBytes + kScaleBytes);
+                tma_load_3d(my_slots + st * kSlotBytes, &d.smap, 0, is_tile * kRows, is_kb * 2, &my_full[st]);
+                tma_load_2d(my_scales + st * kScaleBytes, &d.cmap, is_kb * kSG, is_tile * kRows, &my_full[st]);
+            }
+            if (++is_kb == B) {
+                is_kb = 0;
+                is_tile++;
+            }
         };
         int issued_end = r.u0;  // units [r.u0, issued_end) have been issued
         if (GC && !p.skip_loads) {
             issued_end = min(r.u0 + ns, r.u1);
-            if (lane == 0)
-                for (int v = r.u0; v < issued_end; v++) issue(v, v - r.u0);
+            for (int v = r.u0; v < issued_end; v++) issue(v - r.u0);
         }
         // x may be the output of the preceding launch: wait for it to finish.
         asm volatile("griddepcontrol.wait;" ::: "memory");
@@ -406,10 +411,8 @@ __global__ void __launch_bounds__(nthreads(GC), 1) gemv_pc_kernel(const __grid_c
                 // proxy fence and the copy that overwrites the stage).
                 __syncwarp();
                 if (issued_end < r.u1) {
-                    if (lane == 0) {
-                        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-                        issue(issued_end, s);
-                    }
+                    if (lane == 0) asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                    issue(s);
                     issued_end++;
                 }
                 float v0, v1, v2, v3;

@@ -98,12 +98,14 @@ __device__ __forceinline__ bool step_wait(uint64_t *bar, uint32_t parity, unsign
 }
 
 // A warp's position in its own sequence of units: piece = matrix i inside
-// this CTA's tile range, units [v, vend) of it (tile-major, slice inner).
+// this CTA's tile range; the next unit is slice kb of tile `tile`
+// (matrix-relative), `left` units of this warp's share remain.  Advanced by
+// increments: no division per unit.
 struct Cursor {
     int i;          // matrix, or -1 when the sequence is exhausted
-    int tbeg;       // first tile of the piece (matrix-relative)
+    int tile, kb;   // next unit
     int B;          // units per tile (K / 1024)
-    int v, vend;    // this warp's next unit and end within the piece
+    int left;       // units left in this piece
 };
 
 __device__ __forceinline__ void piece_range(const SDesc &d, int T0, int T1, int warp, int &tbeg, int &U, int &v0,
@@ -115,16 +117,33 @@ __device__ __forceinline__ void piece_range(const SDesc &d, int T0, int T1, int 
     v1 = static_cast<int>((static_cast<long long>(U) * (warp + 1)) / kW);
 }
 
-__device__ __forceinline__ void cursor_settle(Cursor &c, const SParams &p, int T1, int warp, int T0) {
-    while (c.i >= 0 && c.v >= c.vend) {
-        c.i++;
+// Enter matrix i's piece (and skip pieces where this warp has no unit).
+__device__ __forceinline__ void cursor_enter(Cursor &c, const SParams &p, int i, int T0, int T1, int warp) {
+    for (c.i = i;; c.i++) {
         if (c.i >= p.count || p.d[c.i].tile0 >= T1) {
             c.i = -1;
             return;
         }
-        int U;
-        piece_range(p.d[c.i], T0, T1, warp, c.tbeg, U, c.v, c.vend);
-        c.B = p.d[c.i].K >> 10;
+        int tbeg, U, v0, v1;
+        piece_range(p.d[c.i], T0, T1, warp, tbeg, U, v0, v1);
+        if (v1 > v0) {
+            c.B = p.d[c.i].K >> 10;
+            c.tile = tbeg + v0 / c.B;
+            c.kb = v0 - (v0 / c.B) * c.B;
+            c.left = v1 - v0;
+            return;
+        }
+    }
+}
+
+__device__ __forceinline__ void cursor_next(Cursor &c, const SParams &p, int T0, int T1, int warp) {
+    if (--c.left == 0) {
+        cursor_enter(c, p, c.i + 1, T0, T1, warp);
+        return;
+    }
+    if (++c.kb == c.B) {
+        c.kb = 0;
+        c.tile++;
     }
 }
 
@@ -177,28 +196,19 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_step_kernel(const __grid_con
 
     // ---- issue side: this warp's units, in order, into its ring ----
     Cursor ic;
-    ic.i = T0 < T1 ? i0 : -1;
-    if (ic.i >= 0) {
-        int U;
-        piece_range(p.d[ic.i], T0, T1, warp, ic.tbeg, U, ic.v, ic.vend);
-        ic.B = p.d[ic.i].K >> 10;
-        cursor_settle(ic, p, T1, warp, T0);
-    }
-    if (p.skip_loads) ic.i = -1;
+    ic.i = -1;
+    if (T0 < T1 && !p.skip_loads) cursor_enter(ic, p, i0, T0, T1, warp);
     long long issued = 0;
     // Lane 0 issues; all lanes keep the cursor (uniform).  Rows past N are
     // filled with zeros by the copy and never stored.
     auto issue = [&](int st) {
-        const int tile = ic.tbeg + ic.v / ic.B;
-        const int kb = ic.v - (ic.v / ic.B) * ic.B;
         if (lane == 0) {
             uint8_t *stage = my_ring + st * kSlotStage;
             mbar_expect_tx(&my_full[st], kStageBytes);
-            tma_load_3d(stage, &p.m[ic.i].smap, 0, tile * kRows, kb * 2, &my_full[st]);
-            tma_load_2d(my_scl + st * kScaleStage, &p.m[ic.i].cmap, kb * kSG, tile * kRows, &my_full[st]);
+            tma_load_3d(stage, &p.m[ic.i].smap, 0, ic.tile * kRows, ic.kb * 2, &my_full[st]);
+            tma_load_2d(my_scl + st * kScaleStage, &p.m[ic.i].cmap, ic.kb * kSG, ic.tile * kRows, &my_full[st]);
         }
-        ic.v++;
-        cursor_settle(ic, p, T1, warp, T0);
+        cursor_next(ic, p, T0, T1, warp);
         issued++;
     };
     for (int st = 0; st < ns && ic.i >= 0; st++) issue(st);
@@ -272,11 +282,14 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_step_kernel(const __grid_con
         piece_range(d, T0, T1, warp, tbeg, U, v0, v1);
         const float post = ldexpf(1.0f, 24 - E);
         float acc0 = 0.f, acc2 = 0.f;
+        // (tile, slice) of unit v, by increments
+        const int tl_first = v0 / B;
+        const bool first_partial = v0 - tl_first * B != 0;
+        int tl = tl_first, kb = v0 - tl_first * B;
         for (int v = v0; v < v1; v++) {
             bool ok = !dead;
             if (ok) ok = __all_sync(0xffffffffu, step_wait(&my_full[s], ph, deadline));
             dead = dead || !ok;
-            const int kb = v % B;
             if (ok) {
                 const uint8_t *stage = my_ring + s * kSlotStage;
                 const uint8_t *scs = my_scl + s * kScaleStage;
@@ -323,8 +336,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_step_kernel(const __grid_con
                 acc0 += __shfl_xor_sync(0xffffffffu, acc0, 2);
                 acc2 += __shfl_xor_sync(0xffffffffu, acc2, 1);
                 acc2 += __shfl_xor_sync(0xffffffffu, acc2, 2);
-                const int tile = tbeg + v / B;
-                const bool whole = kb == B - 1 && (v / B != v0 / B || v0 % B == 0);
+                const int tile = tbeg + tl;
+                const bool whole = kb == B - 1 && (tl != tl_first || !first_partial);
                 if (whole) {
                     if (!dead && q == 0) {
                         const int n0 = tile * kRows + row, n1 = n0 + 8;
@@ -332,13 +345,17 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_step_kernel(const __grid_con
                         if (n1 < N) d.y[n1] = __float2half_rn(acc2 * post);
                     }
                 } else {
-                    const int slot = (v / B == v0 / B) ? 0 : 1;
+                    const int slot = (tl == tl_first) ? 0 : 1;
                     if (q == 0)
                         *reinterpret_cast<float2 *>(rec + ((warp * 2 + slot) * 8 + g) * 2) =
                             make_float2(acc0 * post, acc2 * post);
                     if (lane == 0) rec_tile[warp * 2 + slot] = dead ? -2 : tile;
                 }
                 acc0 = acc2 = 0.f;
+            }
+            if (++kb == B) {
+                kb = 0;
+                tl++;
             }
         }
         // ---- tiles of this piece split over several warps: summed in warp
