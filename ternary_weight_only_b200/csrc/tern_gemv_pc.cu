@@ -108,7 +108,7 @@ __device__ __forceinline__ bool mbar_test_wait(uint64_t *bar, uint32_t parity) {
 }
 
 __device__ __forceinline__ bool pc_wait(uint64_t *bar, uint32_t parity, unsigned long long deadline) {
-    while (!mbar_try_wait(bar, parity)) {
+    while (!mbar_try_wait_sleep(bar, parity, 20000u)) {
         if (globaltimer() > deadline) {
             atomicExch(&g_tern_gemvpc_status, static_cast<unsigned int>(TERN_ERR_TIMEOUT));
             return false;
@@ -355,6 +355,7 @@ __global__ void __launch_bounds__(nthreads(GC), 1) gemv_pc_kernel(const __grid_c
         named_bar_sync(1, nthr);
 
         const int row = tile_row(g);
+        const float4 qm = make_float4(q == 0 ? 1.f : 0.f, q == 1 ? 1.f : 0.f, q == 2 ? 1.f : 0.f, q == 3 ? 1.f : 0.f);
         uint32_t off[4];
 #pragma unroll
         for (int j = 0; j < 4; j++) off[j] = row * kBox + (((2 * j + (q >> 1)) ^ (row & 7)) << 4) + (q & 1) * 8;
@@ -416,7 +417,7 @@ __global__ void __launch_bounds__(nthreads(GC), 1) gemv_pc_kernel(const __grid_c
                     issued_end++;
                 }
                 float v0, v1, v2, v3;
-                gc_slice(wd, xf, q, v0, v1, v2, v3);
+                gc_slice(wd, xf, qm, v0, v1, v2, v3);
                 const float2 fa = __half22float2(sa2), fb = __half22float2(sb2);
                 acc[0] = fmaf(fa.x, v0 - on.x, acc[0]);
                 acc[0] = fmaf(fa.y, v1 - on.y, acc[0]);

@@ -88,7 +88,7 @@ __host__ __device__ constexpr int ring_off(int kmax) { return (xs_off(kmax) + km
 size_t smem_bytes(int kmax, int ns) { return 1024 + static_cast<size_t>(ring_off(kmax)) + static_cast<size_t>(kW) * ns * kStageBytes; }
 
 __device__ __forceinline__ bool step_wait(uint64_t *bar, uint32_t parity, unsigned long long deadline) {
-    while (!mbar_try_wait(bar, parity)) {
+    while (!mbar_try_wait_sleep(bar, parity, 20000u)) {
         if (globaltimer() > deadline) {
             atomicExch(&g_tern_gemvstep_status, static_cast<unsigned int>(TERN_ERR_TIMEOUT));
             return false;
@@ -160,6 +160,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_step_kernel(const __grid_con
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int g = lane >> 2, q = lane & 3;
     const int row = tile_row(g);
+    const float4 qm = make_float4(q == 0 ? 1.f : 0.f, q == 1 ? 1.f : 0.f, q == 2 ? 1.f : 0.f, q == 3 ? 1.f : 0.f);
     uint32_t off[4];  // 128-byte-swizzled position of words 2q, 2q+1 of group j (0..3 in a box) of `row`
 #pragma unroll
     for (int j = 0; j < 4; j++) off[j] = row * kBox + (((2 * j + (q >> 1)) ^ (row & 7)) << 4) + (q & 1) * 8;
@@ -319,7 +320,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_step_kernel(const __grid_con
                 load_xfrag<8>(xlane + kb * 1024, xf);
                 const float2 on = *reinterpret_cast<const float2 *>(d1 + kb * kSG + 2 * q);
                 float w0, w1, w2, w3;
-                gc_slice(wd, xf, q, w0, w1, w2, w3);
+                gc_slice(wd, xf, qm, w0, w1, w2, w3);
                 const float2 fa = __half22float2(sa2), fb = __half22float2(sb2);
                 acc0 = fmaf(fa.x, w0 - on.x, acc0);
                 acc0 = fmaf(fa.y, w1 - on.y, acc0);

@@ -88,6 +88,13 @@ __device__ __forceinline__ float sel4(int q, float a, float b, float c, float d)
     return (q & 2) ? hi : lo;
 }
 
+// The same pick as a dot product with the one-hot weights m = (q == 0..3),
+// on the floating-point pipe instead of the integer one (exact for finite
+// values: the other terms are +-0 and adding them changes nothing).
+__device__ __forceinline__ float pick4(const float4 &m, float a, float b, float c, float d) {
+    return fmaf(m.w, d, fmaf(m.z, c, fmaf(m.y, b, m.x * a)));
+}
+
 // Tile row read by mma row g (row g + 8 reads tile row tile_row(g) + 8): the
 // rows of one half warp fall on distinct shared-memory banks for 128-byte
 // and 272-byte row strides alike.
@@ -101,10 +108,10 @@ __device__ __forceinline__ int tile_row(int g) { return g < 4 ? 2 * g : 2 * g - 
 // word 2q+1} of group G (overwritten).  The mmas go field by field (j outer,
 // group inner), so eight independent chains separate two dependent mmas.
 // Returns, for lane (g, q): v0 / v2 = group 2q of rows g / g+8, v1 / v3 =
-// group 2q+1 of rows g / g+8.  The chain per group is the one group_mma_b
+// group 2q+1 of rows g / g+8 (qm = one-hot (q == 0..3) as floats).  The chain per group is the one group_mma_b
 // runs, so the all-ones pass through group_mma_b rounds identically.
-__device__ __forceinline__ void gc_slice(uint32_t (&wd)[8][4], const uint4 (&xf)[4], int q, float &v0, float &v1,
-                                         float &v2, float &v3) {
+__device__ __forceinline__ void gc_slice(uint32_t (&wd)[8][4], const uint4 (&xf)[4], const float4 &qm, float &v0,
+                                         float &v1, float &v2, float &v3) {
     float dd[8][4];
 #pragma unroll
     for (int j = 0; j < 8; j++) {
@@ -125,10 +132,10 @@ __device__ __forceinline__ void gc_slice(uint32_t (&wd)[8][4], const uint4 (&xf)
                 mma_acc(dd[G8], wd[G8][0] & m, wd[G8][1] & m, wd[G8][2] & m, wd[G8][3] & m, b0, b1);
         }
     }
-    v0 = sel4(q, dd[0][0], dd[2][0], dd[4][0], dd[6][0]);
-    v1 = sel4(q, dd[1][1], dd[3][1], dd[5][1], dd[7][1]);
-    v2 = sel4(q, dd[0][2], dd[2][2], dd[4][2], dd[6][2]);
-    v3 = sel4(q, dd[1][3], dd[3][3], dd[5][3], dd[7][3]);
+    v0 = pick4(qm, dd[0][0], dd[2][0], dd[4][0], dd[6][0]);
+    v1 = pick4(qm, dd[1][1], dd[3][1], dd[5][1], dd[7][1]);
+    v2 = pick4(qm, dd[0][2], dd[2][2], dd[4][2], dd[6][2]);
+    v3 = pick4(qm, dd[1][3], dd[3][3], dd[5][3], dd[7][3]);
 }
 
 }  // namespace tern
