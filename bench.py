@@ -239,6 +239,7 @@ def proj_rows(T, model, peak_gbs, l2_bytes):
     names = [p[0] for p in synth.LAYER_PROJ]
     xbuf = torch.randn(8 * 17408, device="cuda").half()
     ybuf = torch.empty(8 * 17408, dtype=torch.float16, device="cuda")
+    ybuf_l = [torch.empty(8 * N, dtype=torch.float16, device="cuda") for _, _, N in synth.LAYER_PROJ]
     for M in (1, 2, 4, 8):
         for i, name in enumerate(names):
             _, K, N = synth.LAYER_PROJ[i]
@@ -264,6 +265,20 @@ def proj_rows(T, model, peak_gbs, l2_bytes):
         b = sum(wbytes(synth.LAYER_PROJ[i][1], synth.LAYER_PROJ[i][2]) +
                 2 * synth.LAYER_PROJ[i][1] + 2 * synth.LAYER_PROJ[i][2] for i in idx)
         out[f"{label}_M1"] = {"us": round(ms * 1e3, 3), "GBps": round(b / ms / 1e6, 1),
+                              "frac": round(b / ms / 1e6 / peak_gbs, 4)}
+    # grouped layers at M = 2, 4, 8 (verify batch): one launch per layer
+    for M in (2, 4, 8):
+        fns = []
+        for l in range(synth.N_LAYERS):
+            grp = []
+            for i, (x, slots, sc, y) in enumerate(model.groups[l]):
+                K = synth.LAYER_PROJ[i][1]
+                N = synth.LAYER_PROJ[i][2]
+                grp.append((xbuf[:M * K].view(M, K), slots, sc, ybuf_l[i][:M * N].view(M, N)))
+            fns.append(lambda grp=grp, M=M: T.tern_gemv_grouped(grp, M))
+        ms = graph_time(fns, s)
+        b = sum(wbytes(K, N) + 2 * M * K + 2 * M * N for _, K, N in synth.LAYER_PROJ)
+        out[f"layer_M{M}"] = {"us": round(ms * 1e3, 3), "GBps": round(b / ms / 1e6, 1),
                               "frac": round(b / ms / 1e6 / peak_gbs, 4)}
     # one layer (seven projections) through the step kernel, rotating layers
     fns = [lambda grp=grp: T.tern_gemv_step(grp) for grp in model.groups]

@@ -169,7 +169,7 @@ tern_status launch_bandwidth(const MatDesc *d, int count, int M, void *workspace
     // Default: the producer/consumer kernel where its shape rules hold (K a
     // multiple of 1024, x fits its shared memory), else the TMA-staged one.
     if ((g_opt.gemv_variant == kVarPc || g_opt.gemv_variant == kVarDefault || g_opt.gemv_variant == kVarPcTok) &&
-        gemv_pc_supports(d, count, M))
+        gemv_pc_supports(d, count, M, g_opt.gemv_variant == kVarPcTok))
         return launch_gemv_pc(d, count, M, g_opt.gemv_variant == kVarPcTok, s);
     return launch_gemv_tma(d, count, M, s);
 }

@@ -59,7 +59,7 @@ constexpr int kGroupK = 128;
 __host__ __device__ constexpr int barbytes(bool gc) { return 2 * ncons(gc) * kMaxNS * 8; }
 // partial tiles, two per consumer: float4 per lane, or (group-per-column form,
 // after the sum over the four lanes of a row) float2 per mma row g
-__host__ __device__ constexpr int recbytes(bool gc) { return gc ? ncons(gc) * 2 * 8 * 8 : ncons(gc) * 2 * 32 * 4 * 4; }
+__host__ __device__ constexpr int recbytes(bool gc) { return gc ? ncons(gc) * 2 * 16 * 16 : ncons(gc) * 2 * 32 * 4 * 4; }
 constexpr size_t kSmemBudget = 232448;          // opt-in shared memory per block on sm_100
 constexpr int kMaxDesc = TERN_MAX_GROUP;
 
@@ -166,7 +166,7 @@ __global__ void __launch_bounds__(nthreads(GC), 1) gemv_pc_kernel(const __grid_c
     __half *xs = reinterpret_cast<__half *>(d1 + (p.kmax / kGroupK) * 8 + 16);
     // The rings take what is left after this CTA's own staged x (a grouped
     // launch is sized for its largest K; CTAs of smaller K get deeper rings).
-    const uint32_t ring_off = (fixed_bytes(p.kmax, GC) + static_cast<uint32_t>(GC ? 1 : MT) * d.K * 2 + 1023u) & ~1023u;
+    const uint32_t ring_off = (fixed_bytes(p.kmax, GC) + static_cast<uint32_t>(MT) * d.K * 2 + 1023u) & ~1023u;
     const int ns = min(kMaxNS, static_cast<int>((p.smem_usable - ring_off) / (kCons * (kSlotBytes + kScaleBytes))));
     uint8_t *slot_ring = base + ring_off;                        // [kCons][ns][4096], 1024-aligned boxes
     uint8_t *scale_ring = slot_ring + kCons * ns * kSlotBytes;   // [kCons][ns][256]
@@ -311,13 +311,17 @@ __global__ void __launch_bounds__(nthreads(GC), 1) gemv_pc_kernel(const __grid_c
                 fac2[i] = (static_cast<uint32_t>(15 + e0) << 10) | (static_cast<uint32_t>(15 + e1) << 26);
             }
             const int per_m = K / 8;
-            for (int idx = threadIdx.x; idx < M * per_m; idx += nthr) {
+            // GC: MT token rows (M real, the rest zero) and 8 / MT groups per
+            // set share the eight columns: column (G % GPB) * MT + m of set G / GPB
+            constexpr int GPB = GC ? 8 / MT : 1;
+            for (int idx = threadIdx.x; idx < (GC ? MT : M) * per_m; idx += nthr) {
                 const int m = idx / per_m, c8 = idx - m * per_m;
-                const uint4 v = *reinterpret_cast<const uint4 *>(d.x + static_cast<size_t>(m) * K + c8 * 8);
+                uint4 v = make_uint4(0u, 0u, 0u, 0u);
+                if (m < M) v = *reinterpret_cast<const uint4 *>(d.x + static_cast<size_t>(m) * K + c8 * 8);
                 const uint32_t pr[4] = {v.x, v.y, v.z, v.w};
-                // GC: group n of slice b is staged as "token" n of a 1024-k group b
                 const int kl = c8 * 8;
-                const int di = GC ? xs_pair_index<8>((kl >> 7) & 7, ((kl >> 10) << 7) | (kl & 127))
+                const int gk = kl >> 7;
+                const int di = GC ? xs_pair_index<8>((gk % GPB) * MT + m, ((gk / GPB) << 7) | (kl & 127))
                                   : xs_pair_index<MT>(m, kl);
                 unsigned short *dst = reinterpret_cast<unsigned short *>(xs + di);
 #pragma unroll
@@ -340,7 +344,8 @@ __global__ void __launch_bounds__(nthreads(GC), 1) gemv_pc_kernel(const __grid_c
         // one chain per slice gives all eight groups, column n = group n;
         // stored as d1[group].
         if (GC) {
-            for (int sl = warp; sl < G / kSG; sl += kCons) {
+            // one chain per set: d1[set * 8 + column]
+            for (int sl = warp; sl < G * MT / kSG; sl += kCons) {
                 float c[4];
                 group_mma<8>(c, kOnes, kOnes, kOnes, kOnes, xlane + sl * kGroupHalves);
                 if (g == 0) *reinterpret_cast<float2 *>(d1 + sl * kSG + 2 * q) = make_float2(c[0], c[1]);
@@ -356,6 +361,25 @@ __global__ void __launch_bounds__(nthreads(GC), 1) gemv_pc_kernel(const __grid_c
 
         const int row = tile_row(g);
         const float4 qm = make_float4(q == 0 ? 1.f : 0.f, q == 1 ? 1.f : 0.f, q == 2 ? 1.f : 0.f, q == 3 ? 1.f : 0.f);
+        const float2 qh = make_float2(q < 2 ? 1.f : 0.f, q < 2 ? 0.f : 1.f);
+        // Group-per-column form: lanes q < kGcLanes hold complete sums after
+        // the tile's lane reduction; lane (g, q) stores v = (row g: tokens t0,
+        // t1; row g+8: tokens t0, t1) with t0 = 2q, t1 = 2q + 1 (MT = 4),
+        // t0 = 0, t1 = 1 (MT = 2) or only token 0 from v.x, v.z (MT = 1).
+        constexpr int kGcLanes = MT == 4 ? 2 : 1;
+        auto gc_store = [&](int tile, float4 v) {
+            if (q >= kGcLanes) return;
+            const int n0 = tile * kRows + row, n1 = n0 + 8;
+            const int t0 = MT == 4 ? 2 * q : 0, t1 = t0 + 1;
+            if (n0 < N) {
+                if (t0 < M) d.y[static_cast<size_t>(t0) * N + n0] = __float2half_rn(v.x);
+                if (MT > 1 && t1 < M) d.y[static_cast<size_t>(t1) * N + n0] = __float2half_rn(v.y);
+            }
+            if (n1 < N) {
+                if (t0 < M) d.y[static_cast<size_t>(t0) * N + n1] = __float2half_rn(v.z);
+                if (MT > 1 && t1 < M) d.y[static_cast<size_t>(t1) * N + n1] = __float2half_rn(v.w);
+            }
+        };
         uint32_t off[4];
 #pragma unroll
         for (int j = 0; j < 4; j++) off[j] = row * kBox + (((2 * j + (q >> 1)) ^ (row & 7)) << 4) + (q & 1) * 8;
@@ -380,18 +404,26 @@ __global__ void __launch_bounds__(nthreads(GC), 1) gemv_pc_kernel(const __grid_c
             }
             dead = dead || !ok;
             if (ok && GC) {
-                // gc_note: the slice's B fragments (x of all eight groups, group
-                // n in column n) are loaded once; weight group G runs its
-                // eight-mma chain into its own accumulator dd[G], of which only
-                // column G is meaningful.  Lane (g, q) holds columns 2q, 2q+1,
-                // i.e. groups 2q and 2q+1 of rows `row` and `row` + 8.
+                // gc_note: the slice's B fragments carry (group, token) pairs
+                // (gcm_slice); weight group G runs its eight-mma chain into its
+                // own accumulator, of which only its own columns are kept.
                 const uint8_t *sl = my_slots + s * kSlotBytes;
                 const uint8_t *scb = my_scales + s * kScaleBytes;
-                uint4 xf[4];
-                load_xfrag<8>(xlane + kb * kGroupHalves, xf);
-                const float2 on = *reinterpret_cast<const float2 *>(d1 + kb * kSG + 2 * q);
-                const __half2 sa2 = *reinterpret_cast<const __half2 *>(scb + row * 16 + 4 * q);
-                const __half2 sb2 = *reinterpret_cast<const __half2 *>(scb + (row + 8) * 16 + 4 * q);
+                // scales of the lane's groups (rows `row`, `row` + 8), read before
+                // the stage is refilled: MT = 1 groups 2q, 2q+1; otherwise one
+                // group per set h (4h + q, or 2h + q/2)
+                __half2 sh[MT == 1 ? 2 : MT];
+                if (MT == 1) {
+                    sh[0] = *reinterpret_cast<const __half2 *>(scb + row * 16 + 4 * q);
+                    sh[MT == 1 ? 1 : 0] = *reinterpret_cast<const __half2 *>(scb + (row + 8) * 16 + 4 * q);
+                } else {
+#pragma unroll
+                    for (int h = 0; h < MT; h++) {
+                        const int grp = MT == 2 ? 4 * h + q : 2 * h + (q >> 1);
+                        sh[h] = __halves2half2(*reinterpret_cast<const __half *>(scb + row * 16 + 2 * grp),
+                                               *reinterpret_cast<const __half *>(scb + (row + 8) * 16 + 2 * grp));
+                    }
+                }
                 // All eight groups' words first, then the mmas field by field
                 // (j outer, group inner): eight independent accumulation chains
                 // between two dependent mmas.
@@ -416,13 +448,26 @@ __global__ void __launch_bounds__(nthreads(GC), 1) gemv_pc_kernel(const __grid_c
                     issue(s);
                     issued_end++;
                 }
-                float v0, v1, v2, v3;
-                gc_slice(wd, xf, qm, v0, v1, v2, v3);
-                const float2 fa = __half22float2(sa2), fb = __half22float2(sb2);
-                acc[0] = fmaf(fa.x, v0 - on.x, acc[0]);
-                acc[0] = fmaf(fa.y, v1 - on.y, acc[0]);
-                acc[2] = fmaf(fb.x, v2 - on.x, acc[2]);
-                acc[2] = fmaf(fb.y, v3 - on.y, acc[2]);
+                float out[MT][4];
+                gcm_slice<MT>(wd, xlane + kb * MT * kGroupHalves, qm, qh, out);
+                // acc[0..1] = row g, columns 2q, 2q+1; acc[2..3] = row g+8
+#pragma unroll
+                for (int h = 0; h < MT; h++) {
+                    const float2 on = *reinterpret_cast<const float2 *>(d1 + (kb * MT + h) * kSG + 2 * q);
+                    float sa0, sa1, sb0, sb1;
+                    if (MT == 1) {
+                        const float2 fa = __half22float2(sh[0]), fb = __half22float2(sh[MT == 1 ? 1 : 0]);
+                        sa0 = fa.x; sa1 = fa.y; sb0 = fb.x; sb1 = fb.y;
+                    } else {
+                        const float2 f = __half22float2(sh[h]);
+                        sa0 = sa1 = f.x;
+                        sb0 = sb1 = f.y;
+                    }
+                    acc[0] = fmaf(sa0, out[h][0] - on.x, acc[0]);
+                    acc[1] = fmaf(sa1, out[h][1] - on.y, acc[1]);
+                    acc[2] = fmaf(sb0, out[h][2] - on.x, acc[2]);
+                    acc[3] = fmaf(sb1, out[h][3] - on.y, acc[3]);
+                }
             } else if (ok) {
                 const uint8_t *sl = my_slots + s * kSlotBytes;
                 const uint8_t *scb = my_scales + s * kScaleBytes;
@@ -475,14 +520,31 @@ __global__ void __launch_bounds__(nthreads(GC), 1) gemv_pc_kernel(const __grid_c
                 const int tile = r.t0 + tl;
                 const bool whole = kb == B && (tl != r.u0 / B || kb_first == 0);
                 if (GC) {
-                    // sum the four lanes q of a row (their groups differ)
-                    acc[0] += __shfl_xor_sync(0xffffffffu, acc[0], 1);
-                    acc[0] += __shfl_xor_sync(0xffffffffu, acc[0], 2);
-                    acc[2] += __shfl_xor_sync(0xffffffffu, acc[2], 1);
-                    acc[2] += __shfl_xor_sync(0xffffffffu, acc[2], 2);
+                    // sum the lanes q that hold other groups of the same tokens
+                    // (all four for MT <= 2, the pair q, q ^ 2 for MT = 4)
+                    if (MT == 1) {
+                        acc[0] += acc[1];
+                        acc[2] += acc[3];
+                        acc[1] = acc[3] = 0.f;
+                    }
+#pragma unroll
+                    for (int i = 0; i < 4; i++) {
+                        if (MT <= 2) acc[i] += __shfl_xor_sync(0xffffffffu, acc[i], 1);
+                        acc[i] += __shfl_xor_sync(0xffffffffu, acc[i], 2);
+                    }
                 }
                 const float v0 = acc[0] * post, v1 = acc[1] * post, v2 = acc[2] * post, v3 = acc[3] * post;
-                if (whole) {
+                if (GC) {
+                    if (whole) {
+                        if (!dead) gc_store(tile, make_float4(v0, v1, v2, v3));
+                    } else {
+                        const int slot = (tl == r.u0 / B) ? 0 : 1;
+                        if (q < kGcLanes)
+                            *reinterpret_cast<float4 *>(rec + (((warp * 2 + slot) * 8 + g) * 2 + q) * 4) =
+                                make_float4(v0, v1, v2, v3);
+                        if (lane == 0) rec_tile[warp * 2 + slot] = dead ? -2 : tile;
+                    }
+                } else if (whole) {
                     if (!dead) {
                         const int n0 = tile * kRows + row, n1 = n0 + 8;
                         const int m0 = 2 * q, m1 = 2 * q + 1;
@@ -499,12 +561,7 @@ __global__ void __launch_bounds__(nthreads(GC), 1) gemv_pc_kernel(const __grid_c
                     // A tile shared with neighbouring warps: keep the partial
                     // (slot 0 = the range's first tile, slot 1 = its last).
                     const int slot = (tl == r.u0 / B) ? 0 : 1;
-                    if (GC) {
-                        if (q == 0) *reinterpret_cast<float2 *>(rec + ((warp * 2 + slot) * 8 + g) * 2) = make_float2(v0, v2);
-                    } else {
-                        *reinterpret_cast<float4 *>(rec + ((warp * 2 + slot) * 32 + lane) * 4) =
-                            make_float4(v0, v1, v2, v3);
-                    }
+                    *reinterpret_cast<float4 *>(rec + ((warp * 2 + slot) * 32 + lane) * 4) = make_float4(v0, v1, v2, v3);
                     if (lane == 0) rec_tile[warp * 2 + slot] = dead ? -2 : tile;
                 }
                 acc[0] = acc[1] = acc[2] = acc[3] = 0.f;
@@ -543,8 +600,10 @@ __global__ void __launch_bounds__(nthreads(GC), 1) gemv_pc_kernel(const __grid_c
                 for (int s2 = 0; s2 < 2; s2++) {
                     if (rec_tile[w2 * 2 + s2] != tile) continue;
                     if (GC) {
-                        const float2 o = *reinterpret_cast<const float2 *>(rec + ((w2 * 2 + s2) * 8 + g) * 2);
-                        sum.x += o.x; sum.z += o.y;
+                        if (q < kGcLanes) {
+                            const float4 o = *reinterpret_cast<const float4 *>(rec + (((w2 * 2 + s2) * 8 + g) * 2 + q) * 4);
+                            sum.x += o.x; sum.y += o.y; sum.z += o.z; sum.w += o.w;
+                        }
                     } else {
                         const float4 o = *reinterpret_cast<const float4 *>(rec + ((w2 * 2 + s2) * 32 + lane) * 4);
                         sum.x += o.x; sum.y += o.y; sum.z += o.z; sum.w += o.w;
@@ -555,6 +614,10 @@ __global__ void __launch_bounds__(nthreads(GC), 1) gemv_pc_kernel(const __grid_c
             for (int w2 = 0; w2 < kCons; w2++)
                 if (rec_tile[w2 * 2] == -2 || rec_tile[w2 * 2 + 1] == -2) bad = true;
             if (bad) continue;
+            if (GC) {
+                gc_store(tile, sum);
+                continue;
+            }
             const int n0 = tile * kRows + row, n1 = n0 + 8;
             const int m0 = 2 * q, m1 = 2 * q + 1;
             if (m0 < M) {
@@ -569,19 +632,21 @@ __global__ void __launch_bounds__(nthreads(GC), 1) gemv_pc_kernel(const __grid_c
     }
 }
 
-bool g_attr_pc[64][5];
-int g_occ_pc[64][5];
+bool g_attr_pc[64][7];
+int g_occ_pc[64][7];
 
 int pc_mt(int M) { return M == 1 ? 1 : (M == 2 ? 2 : (M <= 4 ? 4 : 8)); }
 
-// Kernel instance for M token rows; M = 1 takes the group-per-column form
-// unless `token_columns` asks for the token-per-column form.
+// Kernel instance for M token rows: M <= 4 takes the group-per-column form
+// (M = 3 padded to 4) unless `token_columns` asks for the token-per-column
+// form; M = 5..8 always take the latter.
 using PcKernel = void (*)(PParams);
-PcKernel pc_kernel(int M, bool token_columns, int *index) {
+PcKernel pc_kernel(int M, bool token_columns, int *index, bool *gc) {
     const int MT = pc_mt(M);
-    if (MT == 1 && !token_columns) {
-        *index = 4;
-        return gemv_pc_kernel<1, true>;
+    *gc = MT <= 4 && !token_columns;
+    if (*gc) {
+        *index = MT == 1 ? 4 : (MT == 2 ? 5 : 6);
+        return MT == 1 ? gemv_pc_kernel<1, true> : (MT == 2 ? gemv_pc_kernel<2, true> : gemv_pc_kernel<4, true>);
     }
     *index = MT == 1 ? 0 : (MT == 2 ? 1 : (MT == 4 ? 2 : 3));
     return MT == 1 ? gemv_pc_kernel<1, false>
@@ -590,7 +655,7 @@ PcKernel pc_kernel(int M, bool token_columns, int *index) {
 
 }  // namespace
 
-bool gemv_pc_supports(const MatDesc *md, int count, int M) {
+bool gemv_pc_supports(const MatDesc *md, int count, int M, bool token_columns) {
     if (M < 1 || M > 8) return false;
     int kmax = 0;
     for (int i = 0; i < count; i++) {
@@ -598,7 +663,8 @@ bool gemv_pc_supports(const MatDesc *md, int count, int M) {
         kmax = std::max(kmax, md[i].K);
     }
     // x is staged whole per CTA; at least two ring stages must fit beside it.
-    return smem_bytes(2, pc_mt(M) * kmax, kmax, false) <= kSmemBudget;
+    const bool gc = pc_mt(M) <= 4 && !token_columns;
+    return smem_bytes(2, pc_mt(M) * kmax, kmax, gc) <= kSmemBudget;
 }
 
 tern_status launch_gemv_pc(const MatDesc *md, int count, int M, bool token_columns, cudaStream_t stream) {
@@ -606,17 +672,18 @@ tern_status launch_gemv_pc(const MatDesc *md, int count, int M, bool token_colum
     tern_status st = current_device(&dev);
     if (st != TERN_OK) return st;
     if (count < 1 || count > kMaxDesc) return fail(TERN_ERR_INVALID_ARG, "descriptor count %d", count);
-    if (!gemv_pc_supports(md, count, M)) return fail(TERN_ERR_SHAPE, "producer/consumer kernel: unsupported shape");
+    if (!gemv_pc_supports(md, count, M, token_columns))
+        return fail(TERN_ERR_SHAPE, "producer/consumer kernel: unsupported shape");
     const int MT = pc_mt(M);
     int mi = 0;
-    const PcKernel kern = pc_kernel(M, token_columns, &mi);
+    bool gc = false;
+    const PcKernel kern = pc_kernel(M, token_columns, &mi, &gc);
     int kmax = 0;
     for (int i = 0; i < count; i++) kmax = std::max(kmax, md[i].K);
     const int xs_halves = MT * kmax;
     const size_t budget = std::min<size_t>(kSmemBudget, dev.max_smem_optin);
     // The whole budget: every CTA sizes its rings (2..4 stages) from what its
     // own staged x leaves.
-    const bool gc = mi == 4;
     const size_t smem = std::min(budget, smem_bytes(kMaxNS, MT * 1024, kmax, gc));
     if (smem_bytes(2, xs_halves, kmax, gc) > smem) return fail(TERN_ERR_SHAPE, "needs %zu B of shared memory", smem_bytes(2, xs_halves, kmax, gc));
     if (!g_attr_pc[dev.device][mi]) {
@@ -624,7 +691,7 @@ tern_status launch_gemv_pc(const MatDesc *md, int count, int M, bool token_colum
                                              static_cast<int>(dev.max_smem_optin));
         if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(gemv pc)");
         int occ = 0;
-        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, nthreads(mi == 4), static_cast<size_t>(kSmemBudget));
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, nthreads(gc), static_cast<size_t>(kSmemBudget));
         if (e != cudaSuccess) return cuda_fail(e, "occupancy query");
         if (occ < 1) return fail(TERN_ERR_SHAPE, "producer/consumer kernel does not fit on an SM");
         g_occ_pc[dev.device][mi] = occ;

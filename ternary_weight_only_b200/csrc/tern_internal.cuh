@@ -57,7 +57,7 @@ struct MatDesc {
 // TMA-staged kernel (default) and the register-ring kernel (variant 1).
 tern_status launch_gemv_tma(const MatDesc *d, int count, int M, cudaStream_t stream);
 // Producer/consumer form of the same kernel (K a multiple of 1024, x small).
-bool gemv_pc_supports(const MatDesc *d, int count, int M);
+bool gemv_pc_supports(const MatDesc *d, int count, int M, bool token_columns);
 bool gemv_tmem_supports(const MatDesc *md, int count, int M);
 tern_status launch_gemv_tmem(const MatDesc *md, int count, int M, cudaStream_t stream);
 tern_status read_gemvtm_status(bool reset, unsigned int *out);

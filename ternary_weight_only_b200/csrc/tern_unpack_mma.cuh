@@ -138,4 +138,67 @@ __device__ __forceinline__ void gc_slice(uint32_t (&wd)[8][4], const uint4 (&xf)
     v3 = pick4(qm, dd[1][3], dd[3][3], dd[5][3], dd[7][3]);
 }
 
+// Group-per-column slice for MG token rows (MG = 1, 2 or 4): the eight B
+// columns carry (group, token) pairs, column n = group n / MG of a "set",
+// token n % MG; a 1024-k slice has MG sets of 8 / MG groups, staged by
+// xs_pair_index<8>(column, set * 128 + k % 128), so `xs` (the lane's
+// fragments of the slice's first set) reaches set h at xs + 1024 h.  Weight
+// group G (set G / (8/MG)) runs its eight-mma chain into its own accumulator;
+// only the columns of its own group are kept.  Lane (g, q) holds columns 2q,
+// 2q+1 of every set: out[h][0..1] = row g, out[h][2..3] = row g+8, for
+//   MG = 1: groups 2q, 2q+1 (token 0);
+//   MG = 2: group 4h + q, tokens 0, 1;
+//   MG = 4: group 2h + q/2, tokens 2(q%2), 2(q%2)+1.
+// qm = one-hot (q == 0..3), qh = one-hot (q/2 == 0..1), as floats.  The chain
+// per group is the one group_mma_b runs (same fragments, same order), so the
+// all-ones pass through group_mma_b rounds identically.
+template <int MG>
+__device__ __forceinline__ void gcm_slice(uint32_t (&wd)[8][4], const __half *xs, const float4 &qm, const float2 &qh,
+                                          float (&out)[MG][4]) {
+    constexpr int GPB = 8 / MG;  // groups per set
+    float dd[8][4];
+    uint4 xq[MG];
+#pragma unroll
+    for (int j = 0; j < 8; j++) {
+        if ((j & 1) == 0) {
+#pragma unroll
+            for (int h = 0; h < MG; h++) xq[h] = *reinterpret_cast<const uint4 *>(xs + h * 1024 + (j >> 1) * 256);
+        }
+        if (j == 5) {
+#pragma unroll
+            for (int G8 = 0; G8 < 8; G8++)
+#pragma unroll
+                for (int i = 0; i < 4; i++) wd[G8][i] >>= 10;
+        }
+        const uint32_t m = 0x00030003u << (2 * (j < 5 ? j : j - 5));
+#pragma unroll
+        for (int G8 = 0; G8 < 8; G8++) {
+            const uint4 &xv = xq[G8 / GPB];
+            const uint32_t b0 = (j & 1) ? xv.z : xv.x, b1 = (j & 1) ? xv.w : xv.y;
+            if (j == 0)
+                mma_zero(dd[G8], wd[G8][0] & m, wd[G8][1] & m, wd[G8][2] & m, wd[G8][3] & m, b0, b1);
+            else
+                mma_acc(dd[G8], wd[G8][0] & m, wd[G8][1] & m, wd[G8][2] & m, wd[G8][3] & m, b0, b1);
+        }
+    }
+    if (MG == 1) {
+#pragma unroll
+        for (int c = 0; c < 4; c++) {
+            const int o = c & 1;  // column 2q + o: group 2q + o
+            out[0][c] = pick4(qm, dd[o][c], dd[2 + o][c], dd[4 + o][c], dd[6 + o][c]);
+        }
+    } else if (MG == 2) {
+#pragma unroll
+        for (int h = 0; h < MG; h++)
+#pragma unroll
+            for (int c = 0; c < 4; c++)
+                out[h][c] = pick4(qm, dd[4 * h][c], dd[4 * h + 1][c], dd[4 * h + 2][c], dd[4 * h + 3][c]);
+    } else {
+#pragma unroll
+        for (int h = 0; h < MG; h++)
+#pragma unroll
+            for (int c = 0; c < 4; c++) out[h][c] = fmaf(qh.y, dd[(2 * h + 1) % 8][c], qh.x * dd[(2 * h) % 8][c]);
+    }
+}
+
 }  // namespace tern
