@@ -280,6 +280,21 @@ def proj_rows(T, model, peak_gbs, l2_bytes):
         b = sum(wbytes(K, N) + 2 * M * K + 2 * M * N for _, K, N in synth.LAYER_PROJ)
         out[f"layer_M{M}"] = {"us": round(ms * 1e3, 3), "GBps": round(b / ms / 1e6, 1),
                               "frac": round(b / ms / 1e6 / peak_gbs, 4)}
+    # the verify step: every projection of all layers at M = 2, 4 token rows,
+    # one tern_gemv_step call (5 launches)
+    for M in (2, 4):
+        mats, b = [], 0
+        for l in range(synth.N_LAYERS):
+            for i, (x, slots, sc, y) in enumerate(model.groups[l]):
+                K, N = synth.LAYER_PROJ[i][1], synth.LAYER_PROJ[i][2]
+                mats.append((xbuf[:M * K].view(M, K), slots, sc,
+                             torch.empty(M, N, dtype=torch.float16, device="cuda")))
+                b += wbytes(K, N) + 2 * M * K + 2 * M * N
+        ms = graph_time([lambda mats=mats, M=M: T.tern_gemv_step(mats, M)], s, reps=5)
+        out[f"verify_step_M{M}"] = {"ms": round(ms, 4), "GBps": round(b / ms / 1e6, 1),
+                                    "frac": round(b / ms / 1e6 / peak_gbs, 4),
+                                    "products": len(mats)}
+        del mats
     # one layer (seven projections) through the step kernel, rotating layers
     fns = [lambda grp=grp: T.tern_gemv_step(grp) for grp in model.groups]
     ms = graph_time(fns, s)

@@ -212,25 +212,30 @@ size_t tern_gemv_grouped_workspace_bytes(const tern_gemv_desc *descs, int32_t co
 #define TERN_MAX_STEP 512
 
 /*
- * tern_gemv_step -- M = 1 products of up to TERN_MAX_STEP independent
- * matrices (e.g. every projection of every layer plus the output head of one
- * decode step whose inputs do not depend on each other) in ONE persistent
- * launch.  Generation speed is set by the bytes of weights read per token
- * ("Bonsai 27B ternary / 1-bit quantization", ThakiCloud blog, section
- * "Throughput and speculative decoding"); one launch streams all of them
- * without the start-up and drain every separate launch pays.
- *   descs   count descriptors as for tern_gemv_grouped with M = 1: x fp16
- *           [K], slots uint8 [N][K/4], scales fp16 [N][K/128], y fp16 [N];
- *           device buffers owned by the caller, 16-byte aligned; read on the
- *           host during the call (the array need not outlive it)
+ * tern_gemv_step -- products of up to TERN_MAX_STEP independent matrices with
+ * the same M (1..4 token rows: a decode step, M = 1, or a speculative-verify
+ * step) in ONE persistent launch, e.g. every projection of every layer plus
+ * the output head of one step whose inputs do not depend on each other.
+ * Generation speed is set by the bytes of weights read per token ("Bonsai
+ * 27B ternary / 1-bit quantization", ThakiCloud blog, section "Throughput
+ * and speculative decoding"); one launch streams all of them without the
+ * start-up and drain every separate launch pays.
+ *   descs   count descriptors as for tern_gemv_grouped: x fp16 [M][K], slots
+ *           uint8 [N][K/4], scales fp16 [N][K/128], y fp16 [M][N]; device
+ *           buffers owned by the caller, 16-byte aligned; read on the host
+ *           during the call (the array need not outlive it)
  *   count   1..TERN_MAX_STEP
- * Every K must be a multiple of 1024 (TERN_ERR_SHAPE otherwise; use
- * tern_gemv_grouped for other shapes).  Results are those of tern_gemv for
- * each matrix (same arithmetic, fixed summation order per tile); outputs must
- * not overlap inputs or each other.  Argument errors return before any
- * launch; a device wait that gives up is reported by tern_sync_status.
+ *   M       1..4 (TERN_ERR_SHAPE otherwise)
+ * Every K must be a multiple of 1024, and M x (largest K) x 2 bytes of x
+ * must fit in shared memory beside the weight rings (TERN_ERR_SHAPE
+ * otherwise; use tern_gemv_grouped then).  Results are those of tern_gemv /
+ * tern_gemm for each matrix (same arithmetic, fixed summation order per tile);
+ * outputs must not overlap inputs or each other.  Argument errors return
+ * before any launch; a device wait that gives up is reported by
+ * tern_sync_status.  Internally a list longer than 96 matrices becomes a few
+ * launches of equal size (the tensor maps travel in the kernel parameters).
  */
-tern_status tern_gemv_step(const tern_gemv_desc *descs, int32_t count, void *stream);
+tern_status tern_gemv_step(const tern_gemv_desc *descs, int32_t count, int64_t M, void *stream);
 
 /*
  * tern_sync_status -- wait for `stream`, then report whether any kernel of

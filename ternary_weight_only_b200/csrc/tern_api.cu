@@ -318,11 +318,12 @@ tern_status tern_gemv_noalloc(const uint16_t *x, const uint8_t *slots, const uin
     return gemv_noalloc(mat(x, slots, scales, y, N, K), static_cast<cudaStream_t>(stream));
 }
 
-tern_status tern_gemv_step(const tern_gemv_desc *descs, int32_t count, void *stream) {
+tern_status tern_gemv_step(const tern_gemv_desc *descs, int32_t count, int64_t M, void *stream) {
     clear_error();
     if (!descs) return fail(TERN_ERR_INVALID_ARG, "descs is NULL");
     if (count < 1 || count > TERN_MAX_STEP)
         return fail(TERN_ERR_INVALID_ARG, "count must be 1..%d (got %d)", TERN_MAX_STEP, count);
+    if (M < 1 || M > 4) return fail(TERN_ERR_SHAPE, "tern_gemv_step takes M in 1..4 (got %lld)", static_cast<long long>(M));
     static MatDesc d[TERN_MAX_STEP];
     for (int i = 0; i < count; i++) {
         tern_status st = check_nk(descs[i].N, descs[i].K);
@@ -334,8 +335,9 @@ tern_status tern_gemv_step(const tern_gemv_desc *descs, int32_t count, void *str
         if (st != TERN_OK) return st;
         d[i] = mat(descs[i].x, descs[i].slots, descs[i].scales, descs[i].y, descs[i].N, descs[i].K);
     }
-    if (!gemv_step_supports(d, count)) return fail(TERN_ERR_SHAPE, "tern_gemv_step: K too large for shared memory");
-    return launch_gemv_step(d, count, static_cast<cudaStream_t>(stream));
+    if (!gemv_step_supports(d, count, static_cast<int>(M)))
+        return fail(TERN_ERR_SHAPE, "tern_gemv_step: M x K too large for shared memory");
+    return launch_gemv_step(d, count, static_cast<int>(M), static_cast<cudaStream_t>(stream));
 }
 
 tern_status tern_gemv_grouped(const tern_gemv_desc *descs, int32_t count, int64_t M,

@@ -71,6 +71,7 @@ struct SParams {
     SDesc d[kMaxPer];
     int cta_tile[kMaxCtas + 1];   // flat tile range [cta_tile[c], cta_tile[c + 1]) of CTA c
     int count;
+    int M;                        // token rows of every product (x [M][K], y [M][N])
     unsigned int smem_usable;     // dynamic shared memory past the 1024-byte alignment
     int kmax;
     int skip_loads;               // test only: issue no copies (exercises the timeout path)
@@ -79,13 +80,17 @@ struct SParams {
 
 // Shared memory layout (bytes from the 128-aligned base).
 __host__ __device__ constexpr int bar_off() { return 0; }
-__host__ __device__ constexpr int rec_off() { return kW * kMaxNS * 8; }               // [kW][2][8] float2
-__host__ __device__ constexpr int rtile_off() { return rec_off() + kW * 2 * 8 * 8; }  // [kW][2] int
+__host__ __device__ constexpr int rec_off() { return kW * kMaxNS * 8; }               // [kW][2][8][2] float4
+__host__ __device__ constexpr int rtile_off() { return rec_off() + kW * 2 * 16 * 16; }  // [kW][2] int
 __host__ __device__ constexpr int wmax_off() { return rtile_off() + kW * 2 * 4; }     // [kW] uint
 __host__ __device__ constexpr int d1_off() { return wmax_off() + kW * 4; }            // [kmax / 128] float
-__host__ __device__ constexpr int xs_off(int kmax) { return d1_off() + (kmax / 128) * 4 + 64; }
-__host__ __device__ constexpr int ring_off(int kmax) { return (xs_off(kmax) + kmax * 2 + 1023) & ~1023; }
-size_t smem_bytes(int kmax, int ns) { return 1024 + static_cast<size_t>(ring_off(kmax)) + static_cast<size_t>(kW) * ns * kStageBytes; }
+// d1 holds one float per (set, column): kmax / 128 * MT floats, MT <= 4
+__host__ __device__ constexpr int xs_off(int kmax) { return d1_off() + (kmax / 128) * 16 + 64; }
+// staged x: MT token rows (M real, the rest zero)
+__host__ __device__ constexpr int ring_off(int kmax, int mt) { return (xs_off(kmax) + kmax * 2 * mt + 1023) & ~1023; }
+size_t smem_bytes(int kmax, int mt, int ns) {
+    return 1024 + static_cast<size_t>(ring_off(kmax, mt)) + static_cast<size_t>(kW) * ns * kStageBytes;
+}
 
 __device__ __forceinline__ bool step_wait(uint64_t *bar, uint32_t parity, unsigned long long deadline) {
     while (!mbar_try_wait_sleep(bar, parity, 20000u)) {
@@ -147,7 +152,11 @@ __device__ __forceinline__ void cursor_next(Cursor &c, const SParams &p, int T0,
     }
 }
 
+// MT = token rows padded to 1, 2 or 4: the group-per-column form with
+// (group, token) pairs in the mma columns (gcm_slice).
+template <int MT>
 __global__ void __launch_bounds__(kThreads, 1) gemv_step_kernel(const __grid_constant__ SParams p) {
+    constexpr int GPB = 8 / MT;  // groups per set
     extern __shared__ uint8_t smem_raw[];
     uint8_t *base = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     uint64_t *full = reinterpret_cast<uint64_t *>(base + bar_off());  // [kW][kMaxNS]
@@ -161,6 +170,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_step_kernel(const __grid_con
     const int g = lane >> 2, q = lane & 3;
     const int row = tile_row(g);
     const float4 qm = make_float4(q == 0 ? 1.f : 0.f, q == 1 ? 1.f : 0.f, q == 2 ? 1.f : 0.f, q == 3 ? 1.f : 0.f);
+    const float2 qh = make_float2(q < 2 ? 1.f : 0.f, q < 2 ? 0.f : 1.f);
     uint32_t off[4];  // 128-byte-swizzled position of words 2q, 2q+1 of group j (0..3 in a box) of `row`
 #pragma unroll
     for (int j = 0; j < 4; j++) off[j] = row * kBox + (((2 * j + (q >> 1)) ^ (row & 7)) << 4) + (q & 1) * 8;
@@ -178,8 +188,9 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_step_kernel(const __grid_con
     // The ring takes what this CTA's largest staged x leaves (2..4 stages).
     int kcta = 1024;
     for (int i = i0; T0 < T1 && i < p.count && p.d[i].tile0 < T1; i++) kcta = max(kcta, p.d[i].K);
-    const uint32_t roff = (static_cast<uint32_t>(xs_off(p.kmax)) + 2u * kcta + 1023u) & ~1023u;
+    const uint32_t roff = (static_cast<uint32_t>(xs_off(p.kmax)) + 2u * MT * kcta + 1023u) & ~1023u;
     const int ns = min(kMaxNS, static_cast<int>((p.smem_usable - roff) / (kW * kStageBytes)));
+    const int M = p.M;
     uint8_t *ring = base + roff;
 
     if (threadIdx.x == 0) {
@@ -229,7 +240,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_step_kernel(const __grid_con
         __syncthreads();  // the previous piece is finished with xs, d1, rec
         {
             unsigned int mx = 0;
-            for (int idx = threadIdx.x; idx < K / 8; idx += nthr) {
+            for (int idx = threadIdx.x; idx < M * K / 8; idx += nthr) {
                 const uint4 v = *reinterpret_cast<const uint4 *>(d.x + static_cast<size_t>(idx) * 8);
                 const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
@@ -254,12 +265,17 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_step_kernel(const __grid_con
                 const int e1 = E - 2 * (2 * c + 1 < 5 ? 2 * c + 1 : 2 * c + 1 - 5);
                 fac2[c] = (static_cast<uint32_t>(15 + e0) << 10) | (static_cast<uint32_t>(15 + e1) << 26);
             }
-            for (int idx = threadIdx.x; idx < K / 8; idx += nthr) {
-                const uint4 v = *reinterpret_cast<const uint4 *>(d.x + static_cast<size_t>(idx) * 8);
+            // token m of group G sits in column (G % GPB) * MT + m of set G / GPB
+            const int per_m = K / 8;
+            for (int idx = threadIdx.x; idx < MT * per_m; idx += nthr) {
+                const int m = idx / per_m, c8 = idx - m * per_m;
+                uint4 v = make_uint4(0u, 0u, 0u, 0u);
+                if (m < M) v = *reinterpret_cast<const uint4 *>(d.x + static_cast<size_t>(m) * K + c8 * 8);
                 const uint32_t pr[4] = {v.x, v.y, v.z, v.w};
-                const int kl = idx * 8;
-                unsigned short *dst =
-                    reinterpret_cast<unsigned short *>(xs + xs_pair_index<8>((kl >> 7) & 7, ((kl >> 10) << 7) | (kl & 127)));
+                const int kl = c8 * 8;
+                const int gk = kl >> 7;
+                unsigned short *dst = reinterpret_cast<unsigned short *>(
+                    xs + xs_pair_index<8>((gk % GPB) * MT + m, ((gk / GPB) << 7) | (kl & 127)));
 #pragma unroll
                 for (int c = 0; c < 4; c++) {
                     uint32_t h2;
@@ -271,18 +287,38 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_step_kernel(const __grid_con
         }
         __syncthreads();
         const __half *xlane = xs + lane * 8;
-        for (int sl = warp; sl < B; sl += kW) {
+        // one all-ones chain per set: d1[set * 8 + column]
+        for (int sl = warp; sl < B * MT; sl += kW) {
             float c[4];
             group_mma<8>(c, kOnes, kOnes, kOnes, kOnes, xlane + sl * 1024);
             if (g == 0) *reinterpret_cast<float2 *>(d1 + sl * kSG + 2 * q) = make_float2(c[0], c[1]);
         }
         __syncthreads();
 
+        // Lanes q < kGcLanes hold complete sums after a tile's lane
+        // reduction; lane (g, q) stores v = (row g: tokens t0, t1; row g+8:
+        // tokens t0, t1), t0 = 2q, t1 = 2q + 1 (MT = 4), 0, 1 (MT = 2), or
+        // token 0 only from v.x, v.z (MT = 1).
+        constexpr int kGcLanes = MT == 4 ? 2 : 1;
+        auto gc_store = [&](int tile, float4 v) {
+            if (q >= kGcLanes) return;
+            const int n0 = tile * kRows + row, n1 = n0 + 8;
+            const int t0 = MT == 4 ? 2 * q : 0, t1 = t0 + 1;
+            if (n0 < N) {
+                if (t0 < M) d.y[static_cast<size_t>(t0) * N + n0] = __float2half_rn(v.x);
+                if (MT > 1 && t1 < M) d.y[static_cast<size_t>(t1) * N + n0] = __float2half_rn(v.y);
+            }
+            if (n1 < N) {
+                if (t0 < M) d.y[static_cast<size_t>(t0) * N + n1] = __float2half_rn(v.z);
+                if (MT > 1 && t1 < M) d.y[static_cast<size_t>(t1) * N + n1] = __float2half_rn(v.w);
+            }
+        };
+
         // ---- this warp's units of the piece ----
         int tbeg, U, v0, v1;
         piece_range(d, T0, T1, warp, tbeg, U, v0, v1);
         const float post = ldexpf(1.0f, 24 - E);
-        float acc0 = 0.f, acc2 = 0.f;
+        float acc[4] = {0.f, 0.f, 0.f, 0.f};
         // (tile, slice) of unit v, by increments
         const int tl_first = v0 / B;
         const bool first_partial = v0 - tl_first * B != 0;
@@ -305,8 +341,21 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_step_kernel(const __grid_con
                     wd[G8][2] = a.y;
                     wd[G8][3] = b.y;
                 }
-                const __half2 sa2 = *reinterpret_cast<const __half2 *>(scs + row * 16 + 4 * q);
-                const __half2 sb2 = *reinterpret_cast<const __half2 *>(scs + (row + 8) * 16 + 4 * q);
+                // scales of the lane's groups (rows `row`, `row` + 8): MT = 1
+                // groups 2q, 2q+1; otherwise one group per set h (4h + q, or
+                // 2h + q/2)
+                __half2 sh[MT == 1 ? 2 : MT];
+                if (MT == 1) {
+                    sh[0] = *reinterpret_cast<const __half2 *>(scs + row * 16 + 4 * q);
+                    sh[MT == 1 ? 1 : 0] = *reinterpret_cast<const __half2 *>(scs + (row + 8) * 16 + 4 * q);
+                } else {
+#pragma unroll
+                    for (int h = 0; h < MT; h++) {
+                        const int grp = MT == 2 ? 4 * h + q : 2 * h + (q >> 1);
+                        sh[h] = __halves2half2(*reinterpret_cast<const __half *>(scs + row * 16 + 2 * grp),
+                                               *reinterpret_cast<const __half *>(scs + (row + 8) * 16 + 2 * grp));
+                    }
+                }
                 // The stage is in registers: refill it with this warp's next
                 // unit (the warp barrier and the proxy fence order the reads
                 // before the copy that overwrites it).
@@ -316,43 +365,55 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_step_kernel(const __grid_con
                     if (lane == 0) asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
                     issue(s);
                 }
-                uint4 xf[4];
-                load_xfrag<8>(xlane + kb * 1024, xf);
-                const float2 on = *reinterpret_cast<const float2 *>(d1 + kb * kSG + 2 * q);
-                float w0, w1, w2, w3;
-                gc_slice(wd, xf, qm, w0, w1, w2, w3);
-                const float2 fa = __half22float2(sa2), fb = __half22float2(sb2);
-                acc0 = fmaf(fa.x, w0 - on.x, acc0);
-                acc0 = fmaf(fa.y, w1 - on.y, acc0);
-                acc2 = fmaf(fb.x, w2 - on.x, acc2);
-                acc2 = fmaf(fb.y, w3 - on.y, acc2);
+                float out[MT][4];
+                gcm_slice<MT>(wd, xlane + kb * MT * 1024, qm, qh, out);
+                // acc[0..1] = row g, columns 2q, 2q+1; acc[2..3] = row g+8
+#pragma unroll
+                for (int h = 0; h < MT; h++) {
+                    const float2 on = *reinterpret_cast<const float2 *>(d1 + (kb * MT + h) * kSG + 2 * q);
+                    float sa0, sa1, sb0, sb1;
+                    if (MT == 1) {
+                        const float2 fa = __half22float2(sh[0]), fb = __half22float2(sh[MT == 1 ? 1 : 0]);
+                        sa0 = fa.x; sa1 = fa.y; sb0 = fb.x; sb1 = fb.y;
+                    } else {
+                        const float2 f = __half22float2(sh[h]);
+                        sa0 = sa1 = f.x;
+                        sb0 = sb1 = f.y;
+                    }
+                    acc[0] = fmaf(sa0, out[h][0] - on.x, acc[0]);
+                    acc[1] = fmaf(sa1, out[h][1] - on.y, acc[1]);
+                    acc[2] = fmaf(sb0, out[h][2] - on.x, acc[2]);
+                    acc[3] = fmaf(sb1, out[h][3] - on.y, acc[3]);
+                }
             }
             if (++s == ns) {
                 s = 0;
                 ph ^= 1;
             }
             if (kb == B - 1 || v + 1 == v1) {
-                // ---- this warp's part of a tile is complete ----
-                acc0 += __shfl_xor_sync(0xffffffffu, acc0, 1);
-                acc0 += __shfl_xor_sync(0xffffffffu, acc0, 2);
-                acc2 += __shfl_xor_sync(0xffffffffu, acc2, 1);
-                acc2 += __shfl_xor_sync(0xffffffffu, acc2, 2);
+                // ---- this warp's part of a tile is complete: sum the lanes q
+                // that hold other groups of the same tokens ----
+                if (MT == 1) {
+                    acc[0] += acc[1];
+                    acc[2] += acc[3];
+                    acc[1] = acc[3] = 0.f;
+                }
+#pragma unroll
+                for (int c = 0; c < 4; c++) {
+                    if (MT <= 2) acc[c] += __shfl_xor_sync(0xffffffffu, acc[c], 1);
+                    acc[c] += __shfl_xor_sync(0xffffffffu, acc[c], 2);
+                }
                 const int tile = tbeg + tl;
                 const bool whole = kb == B - 1 && (tl != tl_first || !first_partial);
+                const float4 vv = make_float4(acc[0] * post, acc[1] * post, acc[2] * post, acc[3] * post);
                 if (whole) {
-                    if (!dead && q == 0) {
-                        const int n0 = tile * kRows + row, n1 = n0 + 8;
-                        if (n0 < N) d.y[n0] = __float2half_rn(acc0 * post);
-                        if (n1 < N) d.y[n1] = __float2half_rn(acc2 * post);
-                    }
+                    if (!dead) gc_store(tile, vv);
                 } else {
                     const int slot = (tl == tl_first) ? 0 : 1;
-                    if (q == 0)
-                        *reinterpret_cast<float2 *>(rec + ((warp * 2 + slot) * 8 + g) * 2) =
-                            make_float2(acc0 * post, acc2 * post);
+                    if (q < kGcLanes) *reinterpret_cast<float4 *>(rec + (((warp * 2 + slot) * 8 + g) * 2 + q) * 4) = vv;
                     if (lane == 0) rec_tile[warp * 2 + slot] = dead ? -2 : tile;
                 }
-                acc0 = acc2 = 0.f;
+                acc[0] = acc[1] = acc[2] = acc[3] = 0.f;
             }
             if (++kb == B) {
                 kb = 0;
@@ -374,19 +435,19 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_step_kernel(const __grid_con
             for (int w2 = 0; w2 < kW; w2++)
                 if (rec_tile[w2 * 2] == -2 || rec_tile[w2 * 2 + 1] == -2) bad = true;
             if (bad) continue;
-            float s0 = 0.f, s2 = 0.f;
-            for (int w2 = warp; w2 < kW; w2++)
-                for (int s2i = 0; s2i < 2; s2i++) {
-                    if (rec_tile[w2 * 2 + s2i] != tile) continue;
-                    const float2 o = *reinterpret_cast<const float2 *>(rec + ((w2 * 2 + s2i) * 8 + g) * 2);
-                    s0 += o.x;
-                    s2 += o.y;
-                }
-            if (q == 0) {
-                const int n0 = tile * kRows + row, n1 = n0 + 8;
-                if (n0 < N) d.y[n0] = __float2half_rn(s0);
-                if (n1 < N) d.y[n1] = __float2half_rn(s2);
+            float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (q < kGcLanes) {
+                for (int w2 = warp; w2 < kW; w2++)
+                    for (int s2i = 0; s2i < 2; s2i++) {
+                        if (rec_tile[w2 * 2 + s2i] != tile) continue;
+                        const float4 o = *reinterpret_cast<const float4 *>(rec + (((w2 * 2 + s2i) * 8 + g) * 2 + q) * 4);
+                        sum.x += o.x;
+                        sum.y += o.y;
+                        sum.z += o.z;
+                        sum.w += o.w;
+                    }
             }
+            gc_store(tile, sum);
         }
     }
     // A warp that gave up may still have copies of its own in flight: they
@@ -401,26 +462,30 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_step_kernel(const __grid_con
     }
 }
 
-bool g_attr_step[64];
+bool g_attr_step[64][3];
+
+int step_mt(int M) { return M == 1 ? 1 : (M == 2 ? 2 : 4); }
 
 }  // namespace
 
-bool gemv_step_supports(const MatDesc *md, int count) {
-    if (count < 1 || count > TERN_MAX_STEP) return false;
+bool gemv_step_supports(const MatDesc *md, int count, int M) {
+    if (count < 1 || count > TERN_MAX_STEP || M < 1 || M > 4) return false;
     int kmax = 0;
     for (int i = 0; i < count; i++) {
         if (md[i].K % 1024 != 0) return false;
         kmax = std::max(kmax, md[i].K);
     }
-    return smem_bytes(kmax, 2) <= kSmemBudget;
+    // one ring stage per warp at least (refilled as soon as it is read)
+    return smem_bytes(kmax, step_mt(M), 1) <= kSmemBudget;
 }
 
 namespace {
 
 // One launch over md[0..count) (count <= kMaxPer).
-tern_status launch_chunk(const DeviceInfo &dev, const MatDesc *md, int count, cudaStream_t stream) {
+tern_status launch_chunk(const DeviceInfo &dev, const MatDesc *md, int count, int M, cudaStream_t stream) {
     static SParams p;  // large (parameter space); filled on the host for each launch
     std::memset(&p, 0, sizeof(p));
+    const int mt = step_mt(M);
     int kmax = 0;
     long long total_units = 0;
     int tiles = 0;
@@ -452,8 +517,9 @@ tern_status launch_chunk(const DeviceInfo &dev, const MatDesc *md, int count, cu
     }
     const size_t budget = std::min<size_t>(kSmemBudget, dev.max_smem_optin);
     // The whole budget: every CTA sizes its ring from what its own staged x leaves.
-    const size_t smem = std::min(budget, smem_bytes(kmax, kMaxNS));
-    if (smem_bytes(kmax, 2) > smem) return fail(TERN_ERR_SHAPE, "step kernel needs %zu B of shared memory", smem_bytes(kmax, 2));
+    const size_t smem = std::min(budget, smem_bytes(kmax, mt, kMaxNS));
+    if (smem_bytes(kmax, mt, 1) > smem)
+        return fail(TERN_ERR_SHAPE, "step kernel needs %zu B of shared memory", smem_bytes(kmax, mt, 1));
     int grid = std::min<int>(std::min(dev.sms, kMaxCtas), tiles);
     if (g_opt.gemv_grid > 0) grid = std::min(grid, g_opt.gemv_grid);
     // Cut the flat tile list into `grid` ranges of about equal units: CTA c
@@ -478,6 +544,7 @@ tern_status launch_chunk(const DeviceInfo &dev, const MatDesc *md, int count, cu
         p.cta_tile[grid] = tiles;
     }
     p.count = count;
+    p.M = M;
     p.smem_usable = static_cast<unsigned int>(smem - 1024);
     p.kmax = kmax;
     p.skip_loads = g_gemm_skip_loads;
@@ -493,30 +560,33 @@ tern_status launch_chunk(const DeviceInfo &dev, const MatDesc *md, int count, cu
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    cudaError_t e = cudaLaunchKernelEx(&cfg, gemv_step_kernel, p);
+    auto kern = mt == 1 ? gemv_step_kernel<1> : (mt == 2 ? gemv_step_kernel<2> : gemv_step_kernel<4>);
+    cudaError_t e = cudaLaunchKernelEx(&cfg, kern, p);
     if (e != cudaSuccess) return cuda_fail(e, "gemv step kernel launch");
     return TERN_OK;
 }
 
 }  // namespace
 
-tern_status launch_gemv_step(const MatDesc *md, int count, cudaStream_t stream) {
+tern_status launch_gemv_step(const MatDesc *md, int count, int M, cudaStream_t stream) {
     DeviceInfo dev;
     tern_status st = current_device(&dev);
     if (st != TERN_OK) return st;
-    if (!gemv_step_supports(md, count)) return fail(TERN_ERR_SHAPE, "step kernel: unsupported shapes");
-    if (!g_attr_step[dev.device]) {
-        cudaError_t e = cudaFuncSetAttribute(gemv_step_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if (!gemv_step_supports(md, count, M)) return fail(TERN_ERR_SHAPE, "step kernel: unsupported shapes");
+    const int mi = step_mt(M) == 1 ? 0 : (step_mt(M) == 2 ? 1 : 2);
+    if (!g_attr_step[dev.device][mi]) {
+        auto kern = mi == 0 ? gemv_step_kernel<1> : (mi == 1 ? gemv_step_kernel<2> : gemv_step_kernel<4>);
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              static_cast<int>(dev.max_smem_optin));
         if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(gemv step)");
-        g_attr_step[dev.device] = true;
+        g_attr_step[dev.device][mi] = true;
     }
     // Equal-sized launches of at most kMaxPer matrices each.
     const int launches = (count + kMaxPer - 1) / kMaxPer;
     int done = 0;
     for (int l = 0; l < launches; l++) {
         const int n = (count - done) / (launches - l);
-        st = launch_chunk(dev, md + done, n, stream);
+        st = launch_chunk(dev, md + done, n, M, stream);
         if (st != TERN_OK) return st;
         done += n;
     }

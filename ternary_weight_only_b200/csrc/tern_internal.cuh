@@ -94,9 +94,9 @@ tern_status read_gemm_status(bool reset, unsigned int *out);
 tern_status read_gemv_status(bool reset, unsigned int *out);
 tern_status read_gemvtc_status(bool reset, unsigned int *out);
 tern_status read_gemvpc_status(bool reset, unsigned int *out);
-// Persistent M = 1 launch over many matrices (K multiples of 1024).
-bool gemv_step_supports(const MatDesc *d, int count);
-tern_status launch_gemv_step(const MatDesc *d, int count, cudaStream_t stream);
+// Persistent launch over many matrices (M = 1..4, K multiples of 1024).
+bool gemv_step_supports(const MatDesc *d, int count, int M);
+tern_status launch_gemv_step(const MatDesc *d, int count, int M, cudaStream_t stream);
 tern_status read_gemvstep_status(bool reset, unsigned int *out);
 extern unsigned long long g_gemm_timeout_ns;
 extern int g_gemm_skip_loads;

@@ -67,7 +67,7 @@ _SIGS = {
     "tern_sync_status": ([_vp], _int),
     "tern_gemv_grouped_workspace_bytes": ([ctypes.POINTER(tern_gemv_desc), _i32, _i64], _sz),
     "tern_gemv_noalloc": ([_vp, _vp, _vp, _vp, _i64, _i64, _vp], _int),
-    "tern_gemv_step": ([ctypes.POINTER(tern_gemv_desc), _i32, _vp], _int),
+    "tern_gemv_step": ([ctypes.POINTER(tern_gemv_desc), _i32, _i64, _vp], _int),
 }
 for _name, (_args, _res) in _SIGS.items():
     _f = getattr(_L, _name)
@@ -253,9 +253,10 @@ def tern_gemv_grouped(mats: Sequence, M: int, stream=None, workspace=None):
     _check(_L.tern_gemv_grouped(arr, len(mats), M, wp, wn, st), "tern_gemv_grouped")
 
 
-def tern_gemv_step(mats: Sequence, stream=None):
-    """mats: sequence of (x [K], slots [N,K/4], scales [N,K/128], y [N]) CUDA
-    tensors, M = 1, every K a multiple of 1024: one persistent launch."""
+def tern_gemv_step(mats: Sequence, M: int = 1, stream=None):
+    """mats: sequence of (x [M,K] (or [K] for M = 1), slots [N,K/4],
+    scales [N,K/128], y [M,N] (or [N])) CUDA tensors, M in 1..4, every K a
+    multiple of 1024: one persistent launch."""
     arr = (tern_gemv_desc * len(mats))()
     for i, (x, s, sc, y) in enumerate(mats):
         arr[i].x = _dev(x, "x", torch.float16)
@@ -264,7 +265,7 @@ def tern_gemv_step(mats: Sequence, stream=None):
         arr[i].y = _dev(y, "y", torch.float16)
         arr[i].N = s.shape[0]
         arr[i].K = x.shape[-1]
-    _check(_L.tern_gemv_step(arr, len(mats), _stream(stream)), "tern_gemv_step")
+    _check(_L.tern_gemv_step(arr, len(mats), M, _stream(stream)), "tern_gemv_step")
 
 
 def tern_gemv_grouped_workspace_bytes(mats: Sequence, M: int) -> int:

@@ -139,22 +139,27 @@ def test_step_rejects(lib):
     arr = (tern.tern_gemv_desc * 3)()
     for d in arr:
         d.x, d.slots, d.scales, d.y, d.N, d.K = A, A, A, A, 16, 2048
-    assert lib.tern_gemv_step(None, 1, None) == 1
-    assert lib.tern_gemv_step(arr, 0, None) == 1
-    assert lib.tern_gemv_step(arr, tern.TERN_MAX_STEP + 1, None) == 1
+    assert lib.tern_gemv_step(None, 1, 1, None) == 1
+    assert lib.tern_gemv_step(arr, 0, 1, None) == 1
+    assert lib.tern_gemv_step(arr, tern.TERN_MAX_STEP + 1, 1, None) == 1
+    assert lib.tern_gemv_step(arr, 3, 0, None) == 3
+    assert lib.tern_gemv_step(arr, 3, 5, None) == 3
     arr[1].K = 1536                      # a multiple of 128 but not of 1024
-    assert lib.tern_gemv_step(arr, 3, None) == 3
+    assert lib.tern_gemv_step(arr, 3, 1, None) == 3
     arr[1].K = 1000                      # not a multiple of 128
-    assert lib.tern_gemv_step(arr, 3, None) == 3
+    assert lib.tern_gemv_step(arr, 3, 1, None) == 3
     arr[1].K = 2048
     arr[2].N = 0
-    assert lib.tern_gemv_step(arr, 3, None) == 3
+    assert lib.tern_gemv_step(arr, 3, 1, None) == 3
     arr[2].N = 16
     arr[2].slots = A + 8
-    assert lib.tern_gemv_step(arr, 3, None) == 2
+    assert lib.tern_gemv_step(arr, 3, 1, None) == 2
     arr[2].slots = A
     arr[0].x = None
-    assert lib.tern_gemv_step(arr, 3, None) == 1
+    assert lib.tern_gemv_step(arr, 3, 1, None) == 1
+    arr[0].x = A
+    arr[1].K = 40960                     # 4 x 40960 x 2 bytes of x do not fit beside the rings
+    assert lib.tern_gemv_step(arr, 3, 4, None) == 3
 
 
 def test_options(lib):

@@ -28,17 +28,19 @@ def T():
     tern.tern_set_option(tern.TERN_OPT_TEST_STALL_US, 0)
 
 
-def make_mats(orc, shapes, seed):
-    """Host inputs packed by the oracle; device copies; outputs pre-filled with NaN."""
+def make_mats(orc, shapes, seed, M=1):
+    """Host inputs packed by the oracle; device copies; outputs pre-filled with NaN.
+    M = 1 passes x [K] and y [N]; M > 1 passes x [M, K] and y [M, N]."""
     from ternary_weight_only_b200 import synth
     mats, refs = [], []
     for j, (K, N) in enumerate(shapes):
-        x, codes, scales = synth.case(1, K, N, seed=seed + 17 * j, codes="sparse", outlier_p=0.01)
+        x, codes, scales = synth.case(M, K, N, seed=seed + 17 * j, codes="sparse", outlier_p=0.01)
         xn, cn, sn = np_inputs(x, codes, scales)
         slots, sc, bad, _ = orc.pack(cn, sn)
         assert bad == 0
-        y = torch.full((N,), float("nan"), dtype=torch.float16, device="cuda")
-        mats.append((x[0].cuda(), torch.from_numpy(slots).cuda(), scales.cuda(), y))
+        y = torch.full((M, N), float("nan"), dtype=torch.float16, device="cuda")
+        xd = x.cuda()
+        mats.append((xd[0] if M == 1 else xd, torch.from_numpy(slots).cuda(), scales.cuda(), y[0] if M == 1 else y))
         refs.append((xn, slots, sc))
     return mats, refs
 
@@ -46,7 +48,8 @@ def make_mats(orc, shapes, seed):
 def check_all(orc, mats, refs, what):
     for j, ((xn, slots, sc), m) in enumerate(zip(refs, mats)):
         y_ref, bound = orc.matmul(xn, slots, sc, threads=NCPU)
-        check_close(m[3].view(1, -1), y_ref, bound, f"{what} matrix {j} (K={m[0].shape[0]}, N={m[1].shape[0]})")
+        check_close(m[3].reshape(y_ref.shape), y_ref, bound,
+                    f"{what} matrix {j} (K={m[0].shape[-1]}, N={m[1].shape[0]})")
 
 
 @pytest.mark.parametrize("grid", [0, 1, 3, 7, 40])
@@ -141,3 +144,29 @@ def test_timeout_reported_and_context_survives(T, orc):
     T.tern_gemv_step(mats)
     T.tern_sync_status()
     check_all(orc, mats, refs, "step after timeout")
+
+
+@pytest.mark.parametrize("M", [2, 3, 4])
+@pytest.mark.parametrize("grid", [0, 5])
+def test_verify_batch_mixed(T, orc, M, grid):
+    """M token rows (M = 3 runs padded to 4): every output of every token."""
+    shapes = [(1024, 1), (2048, 17), (5120, 100), (3072, 333), (6144, 64), (17408, 40), (4096, 129)]
+    mats, refs = make_mats(orc, shapes, seed=7500 + 10 * M + grid, M=M)
+    T.tern_set_option(T.TERN_OPT_GEMV_GRID, grid)
+    try:
+        T.tern_gemv_step(mats, M)
+        T.tern_sync_status()
+    finally:
+        T.tern_set_option(T.TERN_OPT_GEMV_GRID, 0)
+    check_all(orc, mats, refs, f"step M={M} grid={grid}")
+
+
+@pytest.mark.parametrize("M", [2, 4])
+def test_verify_layer(T, orc, M):
+    """The seven projections of a synthetic decode layer at M token rows."""
+    from ternary_weight_only_b200 import synth
+    shapes = [(K, N) for _, K, N in synth.LAYER_PROJ]
+    mats, refs = make_mats(orc, shapes, seed=7600 + M, M=M)
+    T.tern_gemv_step(mats, M)
+    T.tern_sync_status()
+    check_all(orc, mats, refs, f"step layer M={M}")
