@@ -171,6 +171,22 @@ tern_status launch_bandwidth(const MatDesc *d, int count, int M, void *workspace
     if ((g_opt.gemv_variant == kVarPc || g_opt.gemv_variant == kVarDefault || g_opt.gemv_variant == kVarPcTok) &&
         gemv_pc_supports(d, count, M, g_opt.gemv_variant == kVarPcTok))
         return launch_gemv_pc(d, count, M, g_opt.gemv_variant == kVarPcTok, s);
+    // M = 5..8 whose x does not fit the token-per-column kernel: two launches
+    // of the group-per-column kernel (4 + M - 4 token rows), each reading the
+    // weights once.
+    if (g_opt.gemv_variant == kVarDefault && M > 4 && gemv_pc_supports(d, count, 4, false) &&
+        count <= TERN_MAX_GROUP) {
+        MatDesc lo[TERN_MAX_GROUP], hi[TERN_MAX_GROUP];
+        for (int i = 0; i < count; i++) {
+            lo[i] = d[i];
+            hi[i] = d[i];
+            hi[i].x = d[i].x + static_cast<size_t>(4) * d[i].K;
+            hi[i].y = d[i].y + static_cast<size_t>(4) * d[i].N;
+        }
+        tern_status st = launch_gemv_pc(lo, count, 4, false, s);
+        if (st != TERN_OK) return st;
+        return launch_gemv_pc(hi, count, M - 4, false, s);
+    }
     return launch_gemv_tma(d, count, M, s);
 }
 

@@ -664,7 +664,9 @@ bool gemv_pc_supports(const MatDesc *md, int count, int M, bool token_columns) {
     }
     // x is staged whole per CTA; at least two ring stages must fit beside it.
     const bool gc = pc_mt(M) <= 4 && !token_columns;
-    return smem_bytes(2, pc_mt(M) * kmax, kmax, gc) <= kSmemBudget;
+    // (the group-per-column form refills a stage as soon as it is read, so
+    // one stage per warp still overlaps loads with the mmas)
+    return smem_bytes(gc ? 1 : 2, pc_mt(M) * kmax, kmax, gc) <= kSmemBudget;
 }
 
 tern_status launch_gemv_pc(const MatDesc *md, int count, int M, bool token_columns, cudaStream_t stream) {
@@ -685,7 +687,9 @@ tern_status launch_gemv_pc(const MatDesc *md, int count, int M, bool token_colum
     // The whole budget: every CTA sizes its rings (2..4 stages) from what its
     // own staged x leaves.
     const size_t smem = std::min(budget, smem_bytes(kMaxNS, MT * 1024, kmax, gc));
-    if (smem_bytes(2, xs_halves, kmax, gc) > smem) return fail(TERN_ERR_SHAPE, "needs %zu B of shared memory", smem_bytes(2, xs_halves, kmax, gc));
+    const int ns_min = gc ? 1 : 2;
+    if (smem_bytes(ns_min, xs_halves, kmax, gc) > smem)
+        return fail(TERN_ERR_SHAPE, "needs %zu B of shared memory", smem_bytes(ns_min, xs_halves, kmax, gc));
     if (!g_attr_pc[dev.device][mi]) {
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              static_cast<int>(dev.max_smem_optin));
