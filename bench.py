@@ -355,6 +355,25 @@ def pack_rows(T, peak_gbs):
                                 "frac": round(b / ms / 1e6 / peak_gbs, 4)}}
 
 
+def embed_rows(T, model, peak_gbs):
+    """tern_embed_gather from the head's table (tied weights, 151936 x 5120):
+    M = 1 (a decode token) and M = 2048 (a prompt); GB/s of slots + scales
+    read and fp16 rows written."""
+    out = {}
+    s = torch.cuda.Stream()
+    _, K, V, slots, sc = model.head
+    g = torch.Generator(device="cuda")
+    g.manual_seed(88)
+    for M in (1, 2048):
+        ids = torch.randint(0, V, (M,), generator=g, device="cuda", dtype=torch.int32)
+        o = torch.empty(M, K, dtype=torch.float16, device="cuda")
+        ms = graph_time([lambda ids=ids, o=o: T.tern_embed_gather(ids, slots, sc, K, out=o)] * 16, s, reps=5)
+        b = M * (K // 4 + 2 * (K // GROUP) + 2 * K) + 4 * M
+        out[f"embed_M{M}"] = {"us": round(ms * 1e3, 3), "GBps": round(b / ms / 1e6, 1),
+                              "frac": round(b / ms / 1e6 / peak_gbs, 4)}
+    return out
+
+
 def prefill_rows(T, peak_tf):
     """Prefill GEMM (tensor cores) at M = 2048 and 8192 for both shapes:
     TFLOP/s = 2*M*N*K / device time, against the measured dense fp16 peak."""
@@ -636,6 +655,7 @@ def run_tern(args):
     if rank == 0 and not args.no_rows:
         rows = proj_rows(T, model, peak_gbs, l2)
         rows.update(pack_rows(T, peak_gbs))
+        rows.update(embed_rows(T, model, peak_gbs))
         rows.update(prefill_rows(T, peak_tf))
 
     cpu = None

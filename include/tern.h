@@ -238,6 +238,31 @@ size_t tern_gemv_grouped_workspace_bytes(const tern_gemv_desc *descs, int32_t co
 tern_status tern_gemv_step(const tern_gemv_desc *descs, int32_t count, int64_t M, void *stream);
 
 /*
+ * tern_embed_gather -- ternary embedding lookup: rows of a ternary-g128
+ * matrix gathered by token id, written as fp16.  The pages count the
+ * embeddings among the ternary matrices ("Ternary-Bonsai-27B" model summary,
+ * aitrends.kr, section "Differentiators"; "Bonsai 27B ternary / 1-bit
+ * quantization", ThakiCloud blog, section "What it is"); with tied weights
+ * the output head's slots and scales are the table.
+ *   ids        int32 [M] token ids (device)
+ *   M          rows to gather, >= 1 (0 returns TERN_OK without a launch)
+ *   slots      uint8 [V][K/4], scales fp16 [V][K/128]: the table, as packed
+ *              by tern_pack_g128
+ *   V, K       table rows and row length (K a multiple of 128)
+ *   out        fp16 [M][K]: out[m][k] = s[id][k/128] * t[id][k], exact
+ *              (t is -1, 0 or +1; a zero keeps the sign of the scale, as
+ *              IEEE multiplication gives it); an invalid slot value 3 gives
+ *              an unspecified value
+ *   bad_count  nullable device int32: incremented once per id outside
+ *              [0, V); such rows are written as zeros
+ * All buffers are device memory owned by the caller; ids, bad_count 4-byte
+ * aligned, slots and out 16-byte aligned, scales 2-byte aligned.  Argument
+ * errors return before any launch.
+ */
+tern_status tern_embed_gather(const int32_t *ids, int64_t M, const uint8_t *slots, const uint16_t *scales,
+                              int64_t V, int64_t K, uint16_t *out, int32_t *bad_count, void *stream);
+
+/*
  * tern_sync_status -- wait for `stream`, then report whether any kernel of
  * this library on the current device gave up a bounded on-device wait since
  * the previous call (TERN_ERR_TIMEOUT), clearing that record.  No kernel of

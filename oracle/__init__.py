@@ -76,6 +76,8 @@ class Oracle:
         L.orc_matmul_at.restype = i32
         L.orc_matvec_rows.argtypes = [vp, i64, i64, vp, vp, i64, vp, vp, i32]
         L.orc_matvec_rows.restype = i32
+        L.orc_embed.argtypes = [vp, vp, i64, i64, vp, i64, vp]
+        L.orc_embed.restype = i64
         self.L = L
         self.threads_used = 1
 
@@ -171,6 +173,19 @@ class Oracle:
         self.threads_used = self.L.orc_matvec_rows(_ptr(x_bits), M, K, ps, pc, R, _ptr(y), _ptr(b),
                                                    int(threads))
         return y, b
+
+
+    # -- embedding lookup ------------------------------------------------
+    def embed(self, slots: np.ndarray, scales_bits: np.ndarray, K: int, ids: np.ndarray):
+        """Rows ids of the packed table -> (out fp64 [M,K] = s * t, count of ids
+        outside [0, V), whose rows are +0)."""
+        slots = np.ascontiguousarray(slots, dtype=np.uint8)
+        scales_bits = np.ascontiguousarray(scales_bits, dtype=np.uint16)
+        ids = np.ascontiguousarray(ids, dtype=np.int32)
+        V = slots.shape[0]
+        out = np.zeros((ids.size, K), dtype=np.float64)
+        bad = self.L.orc_embed(_ptr(slots), _ptr(scales_bits), V, K, _ptr(ids), ids.size, _ptr(out))
+        return out, int(bad)
 
 
 def load(mutant: int = 0) -> Oracle:

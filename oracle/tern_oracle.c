@@ -280,3 +280,25 @@ int orc_matvec_rows(const uint16_t *x, int64_t M, int64_t K, const uint8_t *cons
 #endif
     return used;
 }
+
+/* Embedding lookup: out[m][k] = s[id][k/128] * t[id][k] for the table row
+ * id = ids[m] (the same fp64 weight orc_weight gives, so the sign of a zero
+ * follows IEEE multiplication by the scale); an id outside [0, V) gives a row
+ * of +0.  Returns the number of such ids.  (Embeddings are among the ternary
+ * matrices: "Ternary-Bonsai-27B" model summary, aitrends.kr, section
+ * "Differentiators".) */
+int64_t orc_embed(const uint8_t *slots, const uint16_t *scales, int64_t V, int64_t K, const int32_t *ids,
+                  int64_t M, double *out)
+{
+    int64_t bad = 0;
+    for (int64_t m = 0; m < M; m++) {
+        int64_t id = ids[m];
+        if (id < 0 || id >= V) {
+            bad++;
+            for (int64_t k = 0; k < K; k++) out[m * K + k] = 0.0;
+            continue;
+        }
+        for (int64_t k = 0; k < K; k++) out[m * K + k] = orc_weight(slots, scales, K, id, k);
+    }
+    return bad;
+}

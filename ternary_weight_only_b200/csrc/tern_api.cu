@@ -334,6 +334,22 @@ tern_status tern_gemv_noalloc(const uint16_t *x, const uint8_t *slots, const uin
     return gemv_noalloc(mat(x, slots, scales, y, N, K), static_cast<cudaStream_t>(stream));
 }
 
+tern_status tern_embed_gather(const int32_t *ids, int64_t M, const uint8_t *slots, const uint16_t *scales,
+                              int64_t V, int64_t K, uint16_t *out, int32_t *bad_count, void *stream) {
+    clear_error();
+    if (M < 0) return fail(TERN_ERR_SHAPE, "M must be >= 0 (got %lld)", static_cast<long long>(M));
+    tern_status st = check_nk(V, K);
+    if (st != TERN_OK) return st;
+    if (V > 0x7FFFFFFFll || M > 0x7FFFFFFFll) return fail(TERN_ERR_SHAPE, "V and M must fit in int32");
+    if (!ids || !slots || !scales || !out) return fail(TERN_ERR_INVALID_ARG, "null buffer pointer");
+    if ((reinterpret_cast<uintptr_t>(ids) & 3u) || (reinterpret_cast<uintptr_t>(bad_count) & 3u))
+        return fail(TERN_ERR_ALIGN, "ids and bad_count must be 4-byte aligned");
+    if (!aligned16(slots) || !aligned16(out)) return fail(TERN_ERR_ALIGN, "slots and out must be 16-byte aligned");
+    if (reinterpret_cast<uintptr_t>(scales) & 1u) return fail(TERN_ERR_ALIGN, "scales are not 2-byte aligned");
+    if (M == 0) return TERN_OK;
+    return launch_embed(ids, M, slots, scales, V, K, out, bad_count, static_cast<cudaStream_t>(stream));
+}
+
 tern_status tern_gemv_step(const tern_gemv_desc *descs, int32_t count, int64_t M, void *stream) {
     clear_error();
     if (!descs) return fail(TERN_ERR_INVALID_ARG, "descs is NULL");

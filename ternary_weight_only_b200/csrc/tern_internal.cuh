@@ -94,6 +94,9 @@ tern_status read_gemm_status(bool reset, unsigned int *out);
 tern_status read_gemv_status(bool reset, unsigned int *out);
 tern_status read_gemvtc_status(bool reset, unsigned int *out);
 tern_status read_gemvpc_status(bool reset, unsigned int *out);
+// Ternary embedding rows gathered by id, written as fp16 s * t.
+tern_status launch_embed(const int32_t *ids, int64_t M, const uint8_t *slots, const uint16_t *scales, int64_t V,
+                         int64_t K, uint16_t *out, int32_t *bad_count, cudaStream_t stream);
 // Persistent launch over many matrices (M = 1..4, K multiples of 1024).
 bool gemv_step_supports(const MatDesc *d, int count, int M);
 tern_status launch_gemv_step(const MatDesc *d, int count, int M, cudaStream_t stream);

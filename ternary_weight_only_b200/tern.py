@@ -68,6 +68,7 @@ _SIGS = {
     "tern_gemv_grouped_workspace_bytes": ([ctypes.POINTER(tern_gemv_desc), _i32, _i64], _sz),
     "tern_gemv_noalloc": ([_vp, _vp, _vp, _vp, _i64, _i64, _vp], _int),
     "tern_gemv_step": ([ctypes.POINTER(tern_gemv_desc), _i32, _i64, _vp], _int),
+    "tern_embed_gather": ([_vp, _i64, _vp, _vp, _i64, _i64, _vp, _vp, _vp], _int),
 }
 for _name, (_args, _res) in _SIGS.items():
     _f = getattr(_L, _name)
@@ -251,6 +252,22 @@ def tern_gemv_grouped(mats: Sequence, M: int, stream=None, workspace=None):
     need = _L.tern_gemv_grouped_workspace_bytes(arr, len(mats), M) if workspace is None else 0
     wp, wn = _ws_args(workspace, need, mats[0][0].device, st)
     _check(_L.tern_gemv_grouped(arr, len(mats), M, wp, wn, st), "tern_gemv_grouped")
+
+
+def tern_embed_gather(ids: torch.Tensor, slots: torch.Tensor, scales: torch.Tensor, K: int,
+                      out: Optional[torch.Tensor] = None, bad_count: Optional[torch.Tensor] = None,
+                      stream=None) -> torch.Tensor:
+    """ids int32 [M]; slots uint8 [V,K/4]; scales fp16 [V,K/128] -> out fp16 [M,K]
+    (rows s * t of the ternary table); bad_count: optional int32 [1] counter."""
+    M = ids.shape[0]
+    V = slots.shape[0]
+    if out is None:
+        out = torch.empty((M, K), dtype=torch.float16, device=slots.device)
+    bc = None if bad_count is None else _dev(bad_count, "bad_count", torch.int32)
+    _check(_L.tern_embed_gather(_dev(ids, "ids", torch.int32), M, _dev(slots, "slots", torch.uint8),
+                                _dev(scales, "scales", torch.float16), V, K, _dev(out, "out", torch.float16),
+                                bc, _stream(stream)), "tern_embed_gather")
+    return out
 
 
 def tern_gemv_step(mats: Sequence, M: int = 1, stream=None):

@@ -29,7 +29,8 @@ def lib():
 def test_header_declares_the_boundary():
     names = _declared()
     for n in ["tern_pack_g128", "tern_unpack_g128", "tern_gemv", "tern_gemm",
-              "tern_gemv_grouped", "tern_gemv_step", "tern_workspace_bytes", "tern_slots_bytes",
+              "tern_gemv_grouped", "tern_gemv_step", "tern_embed_gather", "tern_workspace_bytes",
+              "tern_slots_bytes",
               "tern_scales_bytes", "tern_status_string", "tern_last_error", "tern_set_option",
               "tern_version"]:
         assert n in names
@@ -160,6 +161,20 @@ def test_step_rejects(lib):
     arr[0].x = A
     arr[1].K = 40960                     # 4 x 40960 x 2 bytes of x do not fit beside the rings
     assert lib.tern_gemv_step(arr, 3, 4, None) == 3
+
+
+def test_embed_rejects(lib):
+    """tern_embed_gather: argument errors return before any launch."""
+    assert lib.tern_embed_gather(None, 4, A, A, 100, 256, A, None, None) == 1
+    assert lib.tern_embed_gather(A, 4, A, A, 100, 200, A, None, None) == 3
+    assert lib.tern_embed_gather(A, 4, A, A, 0, 256, A, None, None) == 3
+    assert lib.tern_embed_gather(A, -1, A, A, 100, 256, A, None, None) == 3
+    assert lib.tern_embed_gather(A + 2, 4, A, A, 100, 256, A, None, None) == 2
+    assert lib.tern_embed_gather(A, 4, A + 8, A, 100, 256, A, None, None) == 2
+    assert lib.tern_embed_gather(A, 4, A, A + 1, 100, 256, A, None, None) == 2
+    assert lib.tern_embed_gather(A, 4, A, A, 100, 256, A + 8, None, None) == 2
+    assert lib.tern_embed_gather(A, 4, A, A, 100, 256, A, A + 2, None) == 2
+    assert lib.tern_embed_gather(A, 0, A, A, 100, 256, A, None, None) == 0
 
 
 def test_options(lib):

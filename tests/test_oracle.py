@@ -314,9 +314,30 @@ def pin_sampled_paths(o):
     assert np.array_equal(yr, y[:, rows]) and np.array_equal(br, b[:, rows])
 
 
+def pin_embed(o):
+    """Embedding rows equal codes[id] * s[id, k // 128] built with numpy from
+    the unpacked codes (values and the sign of zeros); ids outside [0, V)
+    give +0 rows and are counted."""
+    rng = _rng(31)
+    V, K = 57, 384
+    codes = rng.integers(-1, 2, size=(V, K)).astype(np.int8)
+    scales = _f16bits(rng.uniform(-0.05, 0.05, size=(V, K // 128)))  # negative scales too
+    slots, sc, _, _ = o.pack(codes, scales)
+    ids = np.array([0, V - 1, 3, 3, -1, V, 2 ** 31 - 1, 17, -5, 40], dtype=np.int32)
+    out, bad = o.embed(slots, sc, K, ids)
+    W = _np_dequant(codes, scales)
+    ok = (ids >= 0) & (ids < V)
+    assert bad == int((~ok).sum())
+    want = np.zeros((ids.size, K))
+    want[ok] = W[ids[ok]]
+    assert np.array_equal(out, want)
+    assert np.array_equal(np.signbit(out), np.signbit(want))
+    assert not np.signbit(out[~ok]).any()
+
+
 PINS = [pin_half_decode, pin_golden_bytes, pin_golden_matmul, pin_exhaustive_bytes,
         pin_roundtrip_random, pin_invalid_codes, pin_byte_count, pin_numpy_crosscheck,
-        pin_row_sums, pin_exact_cases, pin_brute_force, pin_sampled_paths]
+        pin_row_sums, pin_exact_cases, pin_brute_force, pin_sampled_paths, pin_embed]
 
 
 @pytest.mark.parametrize("pin", PINS, ids=lambda p: p.__name__)
