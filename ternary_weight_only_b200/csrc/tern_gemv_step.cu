@@ -210,7 +210,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_step_kernel(const __grid_con
     Cursor ic;
     ic.i = -1;
     if (T0 < T1 && !p.skip_loads) cursor_enter(ic, p, i0, T0, T1, warp);
-    long long issued = 0;
+    int issued = 0;
     // Lane 0 issues; all lanes keep the cursor (uniform).  Rows past N are
     // filled with zeros by the copy and never stored.
     auto issue = [&](int st) {
@@ -230,7 +230,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_step_kernel(const __grid_con
 
     int s = 0;
     uint32_t ph = 0;
-    long long consumed = 0;
+    int consumed = 0;
     bool dead = false;
     const int nthr = kThreads;
     for (int i = i0; T0 < T1 && i < p.count && p.d[i].tile0 < T1; i++) {
@@ -323,13 +323,15 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_step_kernel(const __grid_con
         const int tl_first = v0 / B;
         const bool first_partial = v0 - tl_first * B != 0;
         int tl = tl_first, kb = v0 - tl_first * B;
+        int to_end = B - kb;  // units until the current tile (or this warp's range) ends
+        if (to_end > v1 - v0) to_end = v1 - v0;
+        const uint8_t *stage = my_ring + s * kSlotStage;
+        const uint8_t *scs = my_scl + s * kScaleStage;
         for (int v = v0; v < v1; v++) {
             bool ok = !dead;
             if (ok) ok = __all_sync(0xffffffffu, step_wait(&my_full[s], ph, deadline));
             dead = dead || !ok;
             if (ok) {
-                const uint8_t *stage = my_ring + s * kSlotStage;
-                const uint8_t *scs = my_scl + s * kScaleStage;
                 uint32_t wd[kSG][4];
 #pragma unroll
                 for (int G8 = 0; G8 < kSG; G8++) {
@@ -386,11 +388,15 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_step_kernel(const __grid_con
                     acc[3] = fmaf(sb1, out[h][3] - on.y, acc[3]);
                 }
             }
+            stage += kSlotStage;
+            scs += kScaleStage;
             if (++s == ns) {
                 s = 0;
                 ph ^= 1;
+                stage = my_ring;
+                scs = my_scl;
             }
-            if (kb == B - 1 || v + 1 == v1) {
+            if (--to_end == 0) {
                 // ---- this warp's part of a tile is complete: sum the lanes q
                 // that hold other groups of the same tokens ----
                 if (MT == 1) {
@@ -414,6 +420,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_step_kernel(const __grid_con
                     if (lane == 0) rec_tile[warp * 2 + slot] = dead ? -2 : tile;
                 }
                 acc[0] = acc[1] = acc[2] = acc[3] = 0.f;
+                to_end = min(B, v1 - v - 1);
             }
             if (++kb == B) {
                 kb = 0;
@@ -454,7 +461,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_step_kernel(const __grid_con
     // must land before the CTA exits (bounded).
     if (dead) {
         const unsigned long long dl2 = globaltimer() + p.timeout_ns;
-        for (long long u = consumed; u < issued; u++) {
+        for (int u = consumed; u < issued; u++) {
             const int st = static_cast<int>(u % ns);
             const uint32_t phs = static_cast<uint32_t>((u / ns) & 1);
             step_wait(&my_full[st], phs, dl2);
