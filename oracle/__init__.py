@@ -78,6 +78,16 @@ class Oracle:
         L.orc_matvec_rows.restype = i32
         L.orc_embed.argtypes = [vp, vp, i64, i64, vp, i64, vp]
         L.orc_embed.restype = i64
+        L.orc_b1_slots_bytes.argtypes = [i64, i64]
+        L.orc_b1_slots_bytes.restype = i64
+        L.orc_pack_b1.argtypes = [vp, vp, i64, i64, vp, vp, ctypes.POINTER(i64)]
+        L.orc_pack_b1.restype = i64
+        L.orc_unpack_b1.argtypes = [vp, i64, i64, vp]
+        L.orc_unpack_b1.restype = i64
+        L.orc_b1_weight.argtypes = [vp, vp, i64, i64, i64]
+        L.orc_b1_weight.restype = dbl
+        L.orc_b1_matmul.argtypes = [vp, i64, i64, vp, vp, i64, vp, vp, i32]
+        L.orc_b1_matmul.restype = i32
         self.L = L
         self.threads_used = 1
 
@@ -186,6 +196,45 @@ class Oracle:
         out = np.zeros((ids.size, K), dtype=np.float64)
         bad = self.L.orc_embed(_ptr(slots), _ptr(scales_bits), V, K, _ptr(ids), ids.size, _ptr(out))
         return out, int(bad)
+
+
+    # -- the 1-bit variant ---------------------------------------------
+    def b1_slots_bytes(self, N: int, K: int) -> int:
+        return self.L.orc_b1_slots_bytes(N, K)
+
+    def b1_pack(self, codes: np.ndarray, scales_bits: np.ndarray):
+        """codes int8 [N,K] in {-1,+1}; scales uint16 [N,K/128] -> (bits uint8
+        [N,K/8], scales, invalid_count, first_bad_index)."""
+        codes = np.ascontiguousarray(codes, dtype=np.int8)
+        scales_bits = np.ascontiguousarray(scales_bits, dtype=np.uint16)
+        N, K = codes.shape
+        bits = np.zeros((N, max(K // 8, 0)), dtype=np.uint8)
+        sc = np.zeros((N, max(K // 128, 0)), dtype=np.uint16)
+        first = ctypes.c_int64(-1)
+        bad = self.L.orc_pack_b1(_ptr(codes), _ptr(scales_bits), N, K, _ptr(bits), _ptr(sc), ctypes.byref(first))
+        if bad < 0:
+            raise ValueError("oracle b1 pack: K must be a positive multiple of 128")
+        return bits, sc, int(bad), int(first.value)
+
+    def b1_unpack(self, bits: np.ndarray, K: int) -> np.ndarray:
+        bits = np.ascontiguousarray(bits, dtype=np.uint8)
+        N = bits.shape[0]
+        codes = np.zeros((N, K), dtype=np.int8)
+        if self.L.orc_unpack_b1(_ptr(bits), N, K, _ptr(codes)) < 0:
+            raise ValueError("oracle b1 unpack: K must be a positive multiple of 128")
+        return codes
+
+    def b1_matmul(self, x_bits: np.ndarray, bits: np.ndarray, scales_bits: np.ndarray, threads: int = 1):
+        x_bits = np.ascontiguousarray(x_bits, dtype=np.uint16)
+        bits = np.ascontiguousarray(bits, dtype=np.uint8)
+        scales_bits = np.ascontiguousarray(scales_bits, dtype=np.uint16)
+        M, K = x_bits.shape
+        N = bits.shape[0]
+        y = np.zeros((M, N), dtype=np.float64)
+        b = np.zeros((M, N), dtype=np.float64)
+        self.threads_used = self.L.orc_b1_matmul(_ptr(x_bits), M, K, _ptr(bits), _ptr(scales_bits), N,
+                                                 _ptr(y), _ptr(b), int(threads))
+        return y, b
 
 
 def load(mutant: int = 0) -> Oracle:

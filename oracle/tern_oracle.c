@@ -302,3 +302,101 @@ int64_t orc_embed(const uint8_t *slots, const uint16_t *scales, int64_t V, int64
     }
     return bad;
 }
+
+/* ------------------------------------------------------------------------
+ * The 1-bit variant ("Bonsai 27B ternary / 1-bit quantization", ThakiCloud
+ * blog, sections "What it is" and "How compression works": weights in
+ * {-1, +1} with one FP16 scale per 128 weights, 1 + 16/128 = 1.125
+ * bits/weight).  The pages give no bit layout; this library's: bit b =
+ * (t + 1) / 2 (0 -> -1, 1 -> +1), weight (n,k) in byte n*K/8 + k/8 at bit
+ * k%8 (least significant bit first); scales fp16 [N][K/128] as for the
+ * ternary slots.
+ * ------------------------------------------------------------------------ */
+
+int64_t orc_b1_slots_bytes(int64_t N, int64_t K) { return N * (K / 8); }
+
+/* Pack codes [N][K] (int8, -1 or +1) and scales into the 1-bit layout.  Any
+ * other input is stored as bit 0 and counted.  Returns the count (or -1 for
+ * a bad K); *first_bad receives the flat index of the first one (or -1). */
+int64_t orc_pack_b1(const int8_t *codes, const uint16_t *scales_in, int64_t N, int64_t K, uint8_t *bits,
+                    uint16_t *scales_out, int64_t *first_bad)
+{
+    int64_t bad = 0, first = -1;
+    if (K <= 0 || N <= 0 || K % ORC_GROUP != 0) return -1;
+    for (int64_t i = 0; i < N * (K / 8); i++) bits[i] = 0;
+    for (int64_t n = 0; n < N; n++) {
+        for (int64_t k = 0; k < K; k++) {
+            int t = codes[n * K + k];
+            int b = 0;
+            if (t == 1) {
+                b = 1;
+            } else if (t != -1) {
+                if (first < 0) first = n * K + k;
+                bad++;
+            }
+            bits[n * (K / 8) + k / 8] |= (uint8_t)(b << (k % 8));
+        }
+    }
+    for (int64_t i = 0; i < N * (K / ORC_GROUP); i++) scales_out[i] = scales_in[i];
+    if (first_bad) *first_bad = first;
+    return bad;
+}
+
+/* Bit of weight (n,k) -> t in {-1, +1}. */
+static int orc_b1_value(const uint8_t *bits, int64_t K, int64_t n, int64_t k)
+{
+#if ORC_MUTANT == 7
+    return ((bits[n * (K / 8) + k / 8] >> (7 - k % 8)) & 1) ? 1 : -1; /* planted: bits MSB first */
+#elif ORC_MUTANT == 8
+    return ((bits[n * (K / 8) + k / 8] >> (k % 8)) & 1) ? -1 : 1; /* planted: bit meaning swapped */
+#else
+    return ((bits[n * (K / 8) + k / 8] >> (k % 8)) & 1) ? 1 : -1;
+#endif
+}
+
+int64_t orc_unpack_b1(const uint8_t *bits, int64_t N, int64_t K, int8_t *codes_out)
+{
+    if (K <= 0 || N <= 0 || K % ORC_GROUP != 0) return -1;
+    for (int64_t n = 0; n < N; n++)
+        for (int64_t k = 0; k < K; k++) codes_out[n * K + k] = (int8_t)orc_b1_value(bits, K, n, k);
+    return 0;
+}
+
+/* w[n][k] = s[n][k/128] * t[n][k] in fp64 (exact). */
+double orc_b1_weight(const uint8_t *bits, const uint16_t *scales, int64_t K, int64_t n, int64_t k)
+{
+#if ORC_MUTANT == 9
+    return orc_half_to_double(scales[n * (K / ORC_GROUP)]) * (double)orc_b1_value(bits, K, n, k); /* planted: one scale per row */
+#else
+    return orc_half_to_double(scales[n * (K / ORC_GROUP) + k / ORC_GROUP]) * (double)orc_b1_value(bits, K, n, k);
+#endif
+}
+
+/* y[M][N] = x[M][K] * W^T with the 1-bit weights, naive fp64 in k order, and
+ * the bound sum_k |x*w|.  Returns the thread count used. */
+int orc_b1_matmul(const uint16_t *x, int64_t M, int64_t K, const uint8_t *bits, const uint16_t *scales,
+                  int64_t N, double *y, double *bound, int nthreads)
+{
+    int used = 1;
+#ifdef _OPENMP
+    if (nthreads < 1) nthreads = 1;
+#pragma omp parallel for num_threads(nthreads) schedule(static)
+#else
+    (void)nthreads;
+#endif
+    for (int64_t i = 0; i < M * N; i++) {
+#ifdef _OPENMP
+        if (i == 0) used = omp_get_num_threads();
+#endif
+        int64_t m = i / N, n = i % N;
+        double acc = 0.0, b = 0.0;
+        for (int64_t k = 0; k < K; k++) {
+            double p = orc_half_to_double(x[m * K + k]) * orc_b1_weight(bits, scales, K, n, k);
+            acc += p;
+            b += fabs(p);
+        }
+        y[i] = acc;
+        bound[i] = b;
+    }
+    return used;
+}

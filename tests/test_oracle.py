@@ -335,9 +335,62 @@ def pin_embed(o):
     assert not np.signbit(out[~ok]).any()
 
 
+def pin_b1_format(o):
+    """The 1-bit variant: the byte count is the closed form K*N/8 + 2*K*N/128
+    = 1.125 bits/weight, 16/1.125 = 14.2x smaller than fp16 (the figures the
+    ThakiCloud blog prints in "How compression works"); all 256 byte values
+    unpack to their bits (LSB first, 1 -> +1, 0 -> -1) and pack back; a
+    hand-worked row; random round trips; invalid inputs are counted."""
+    N, K = 3, 256
+    assert o.b1_slots_bytes(N, K) + o.scales_bytes(N, K) == K * N * 1.125 / 8
+    assert round(16 / 1.125, 1) == 14.2
+    # every byte value, 16 bytes per row of K = 128
+    bytes_ = np.arange(256, dtype=np.uint8).reshape(16, 16)
+    codes = o.b1_unpack(bytes_, 128)
+    want = np.where((bytes_[:, :, None] >> np.arange(8)) & 1, 1, -1).reshape(16, 128)
+    assert np.array_equal(codes, want)
+    back, _, bad, _ = o.b1_pack(codes, np.zeros((16, 1), np.uint16))
+    assert bad == 0 and np.array_equal(back, bytes_)
+    # hand-worked: codes +1,-1,-1,+1,+1,+1,-1,+1 -> bits 1,0,0,1,1,1,0,1 (LSB first) = 0b10111001 = 0xB9
+    row = np.full((1, 128), -1, dtype=np.int8)
+    row[0, :8] = [1, -1, -1, 1, 1, 1, -1, 1]
+    b, _, _, _ = o.b1_pack(row, np.zeros((1, 1), np.uint16))
+    assert b[0, 0] == 0xB9 and not b[0, 1:].any()
+    rng = _rng(41)
+    codes = rng.choice(np.array([-1, 1], dtype=np.int8), size=(7, 384))
+    b, _, bad, _ = o.b1_pack(codes, np.zeros((7, 3), np.uint16))
+    assert bad == 0 and np.array_equal(o.b1_unpack(b, 384), codes)
+    codes[2, 5] = 0
+    codes[6, 383] = 3
+    _, _, bad, first = o.b1_pack(codes, np.zeros((7, 3), np.uint16))
+    assert bad == 2 and first == 2 * 384 + 5
+
+
+def pin_b1_matmul(o):
+    """The 1-bit product equals numpy float64 x @ (s*t).T, and all-(+1) codes
+    with unit scales give row sums."""
+    rng = _rng(43)
+    M, K, N = 3, 384, 29
+    codes = rng.choice(np.array([-1, 1], dtype=np.int8), size=(N, K))
+    scales = _f16bits(rng.uniform(-0.05, 0.05, size=(N, K // 128)))
+    x = _f16bits(rng.standard_normal((M, K)))
+    bits, sc, _, _ = o.b1_pack(codes, scales)
+    y, b = o.b1_matmul(x, bits, sc)
+    W = _np_dequant(codes, scales)
+    X = x.view(np.float16).astype(np.float64)
+    ref = X @ W.T
+    assert np.allclose(y, ref, rtol=1e-12, atol=1e-12)
+    assert np.allclose(b, np.abs(X) @ np.abs(W).T, rtol=1e-12, atol=1e-12)
+    ones = np.ones((N, K), dtype=np.int8)
+    bits, sc, _, _ = o.b1_pack(ones, _f16bits(np.ones((N, K // 128))))
+    y, _ = o.b1_matmul(x, bits, sc)
+    assert np.array_equal(y, np.repeat(X.sum(axis=1, keepdims=True), N, axis=1))
+
+
 PINS = [pin_half_decode, pin_golden_bytes, pin_golden_matmul, pin_exhaustive_bytes,
         pin_roundtrip_random, pin_invalid_codes, pin_byte_count, pin_numpy_crosscheck,
-        pin_row_sums, pin_exact_cases, pin_brute_force, pin_sampled_paths, pin_embed]
+        pin_row_sums, pin_exact_cases, pin_brute_force, pin_sampled_paths, pin_embed, pin_b1_format,
+        pin_b1_matmul]
 
 
 @pytest.mark.parametrize("pin", PINS, ids=lambda p: p.__name__)
@@ -359,10 +412,11 @@ def test_rejects_bad_k(orc):
         orc.pack(np.zeros((1, 100), dtype=np.int8), np.zeros((1, 0), dtype=np.uint16))
 
 
-@pytest.mark.parametrize("mutant", [1, 2, 3, 4, 5, 6])
+@pytest.mark.parametrize("mutant", [1, 2, 3, 4, 5, 6, 7, 8, 9])
 def test_planted_mistakes_are_caught(mutant):
     """Each planted mistake in the oracle (bit order, code sign, group size,
-    transposed operand, dropped term, subnormal decode) fails at least one pin."""
+    transposed operand, dropped term, subnormal decode; in the 1-bit variant
+    bit order, bit meaning, scale group) fails at least one pin."""
     bad = oracle.Oracle(oracle.build(mutant))
     failed = []
     for pin in PINS:
