@@ -339,6 +339,58 @@ def proj_rows(T, model, peak_gbs, l2_bytes):
     return out
 
 
+def b1_rows(T, model, peak_gbs, sm_mhz=None):
+    """The 1-bit variant ({-1,+1} + fp16 scale per 128, 1.125 bits/weight)
+    over the same shapes: every projection of the 64 layers plus the head in
+    one tern_b1_gemv_step call, at M = 1 (decode) and M = 2, 4 (verify).
+    Weights are random signs; x and y are the decode model's buffers.  The
+    unpack costs as many integer instructions per weight as the ternary one
+    (one AND per pair of weights), over half the bytes, so the row also
+    reports the fraction of the integer-pipe bound (alu_frac): 2 logic
+    instructions per cycle per SM, 34 per 2048 weights."""
+    out = {}
+    s = torch.cuda.Stream()
+    mats, bmats = [], 0
+    for l in range(model.n_layers):
+        g = synth.gen(6000 + l, "cuda")
+        for i, (x, slots, sc, y) in enumerate(model.groups[l]):
+            _, K, N = synth.LAYER_PROJ[i]
+            codes = synth.codes_sign(N, K, g, device="cuda")
+            bits, bsc = T.tern_b1_pack(codes, synth.scales_uniform(N, K, g, device="cuda"))
+            del codes
+            mats.append((x, bits, bsc, y, K, N))
+    g = synth.gen(6000 + synth.N_LAYERS, "cuda")
+    _, K, N = synth.HEAD
+    codes = synth.codes_sign(N, K, g, device="cuda")
+    bits, bsc = T.tern_b1_pack(codes, synth.scales_uniform(N, K, g, device="cuda"))
+    del codes
+    mats.append((model.head_io[0], bits, bsc, model.head_io[1], K, N))
+    torch.cuda.synchronize()
+    nweights = sum(K * N for *_, K, N in mats)
+    props = torch.cuda.get_device_properties(torch.cuda.current_device())
+    mhz = sm_mhz or 1800.0
+    alu_weights_per_s = props.multi_processor_count * mhz * 1e6 * 2 / 34 * 2048
+    xbuf = torch.randn(4 * 17408, device="cuda").half()
+    for M in (1, 2, 4):
+        if M == 1:
+            run = [(x, b, sc, y) for x, b, sc, y, _, _ in mats]
+        else:
+            run = [(xbuf[:M * K].view(M, K), b, sc, torch.empty(M, N, dtype=torch.float16, device="cuda"))
+                   for _, b, sc, _, K, N in mats]
+        b = sum(N * K // 8 + 2 * N * (K // GROUP) + 2 * M * K + 2 * M * N for *_, K, N in mats)
+        ms = graph_time([lambda run=run, M=M: T.tern_b1_gemv_step(run, M)], s, reps=5)
+        wps = nweights / (ms * 1e-3)
+        out[f"b1_step_M{M}"] = {"ms": round(ms, 4), "GBps": round(b / ms / 1e6, 1),
+                                "frac": round(b / ms / 1e6 / peak_gbs, 4),
+                                "weights_per_s": float(f"{wps:.4g}"),
+                                "alu_frac": round(wps / alu_weights_per_s, 4),
+                                "products": len(run)}
+        del run
+    del mats
+    torch.cuda.empty_cache()
+    return out
+
+
 def pack_rows(T, peak_gbs):
     """tern_pack_g128 on a gate-sized matrix (17408 x 5120): int8 codes and
     fp16 scales in, 2-bit slots and scales out; GB/s of those bytes."""
@@ -656,6 +708,7 @@ def run_tern(args):
     if rank == 0 and not args.no_rows:
         rows = proj_rows(T, model, peak_gbs, l2)
         rows.update(pack_rows(T, peak_gbs))
+        rows.update(b1_rows(T, model, peak_gbs, (clocks.summary() or {}).get("sm_mhz")))
         rows.update(embed_rows(T, model, peak_gbs))
         rows.update(prefill_rows(T, peak_tf))
 

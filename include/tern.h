@@ -263,6 +263,47 @@ tern_status tern_embed_gather(const int32_t *ids, int64_t M, const uint8_t *slot
                               int64_t V, int64_t K, uint16_t *out, int32_t *bad_count, void *stream);
 
 /*
+ * The 1-bit variant.  Weights in {-1, +1} with the same fp16 scale per 128
+ * weights along K, w = s_g * t: 1 + 16/128 = 1.125 bits per weight, about
+ * 14.2x smaller than fp16 ("Bonsai 27B ternary / 1-bit quantization",
+ * ThakiCloud blog, sections "What it is" and "How compression works").  The
+ * pages fix no bit layout; this library's, for W with N rows and K columns:
+ *
+ *   bits    uint8 [N][K/8]   bit b = (t + 1) / 2 (0 -> -1, 1 -> +1) of weight
+ *                            (n,k) at bit k%8 of byte n*K/8 + k/8
+ *                            (least significant bit first);
+ *   scales  fp16  [N][K/128] as for the ternary slots.
+ *
+ * tern_b1_pack -- build the bit layout.
+ *   codes      int8 [N][K], each value -1 or +1                 (device, read)
+ *   scales_in  fp16 [N][K/128] raw 16-bit patterns              (device, read)
+ *   bits_out   uint8 [N][K/8]                                   (device, written)
+ *   scales_out fp16 [N][K/128], a bit-exact copy (may equal scales_in)
+ *   invalid_count  nullable device int32, incremented by the number of codes
+ *              other than -1 and +1; such a code is stored as bit 0 (-1).
+ * Alignment: codes and bits_out 16 bytes; scales 2 bytes; invalid_count 4.
+ */
+tern_status tern_b1_pack(const int8_t *codes, const uint16_t *scales_in, int64_t N, int64_t K, uint8_t *bits_out,
+                         uint16_t *scales_out, int32_t *invalid_count, void *stream);
+
+/*
+ * tern_b1_unpack -- inverse of the bit layout: codes_out int8 [N][K] gets -1
+ * or +1 (device, written).  bits and codes_out 16-byte aligned.
+ */
+tern_status tern_b1_unpack(const uint8_t *bits, int64_t N, int64_t K, int8_t *codes_out, void *stream);
+
+/*
+ * tern_b1_gemv_step -- tern_gemv_step for 1-bit matrices: y = x * W^T with
+ * w = s_g * t, t in {-1, +1}, for up to TERN_MAX_STEP matrices with the same
+ * M (1..4) in one persistent launch.  Each descriptor's `slots` field points
+ * to the bits (uint8 [N][K/8], as built by tern_b1_pack); everything else,
+ * including the shape rules (K a multiple of 1024, x in shared memory), the
+ * arithmetic (fp32 accumulation, fp16 output rounded to nearest even),
+ * argument checking and error reporting, is as for tern_gemv_step.
+ */
+tern_status tern_b1_gemv_step(const tern_gemv_desc *descs, int32_t count, int64_t M, void *stream);
+
+/*
  * tern_sync_status -- wait for `stream`, then report whether any kernel of
  * this library on the current device gave up a bounded on-device wait since
  * the previous call (TERN_ERR_TIMEOUT), clearing that record.  No kernel of

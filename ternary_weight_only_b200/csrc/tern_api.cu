@@ -350,26 +350,62 @@ tern_status tern_embed_gather(const int32_t *ids, int64_t M, const uint8_t *slot
     return launch_embed(ids, M, slots, scales, V, K, out, bad_count, static_cast<cudaStream_t>(stream));
 }
 
-tern_status tern_gemv_step(const tern_gemv_desc *descs, int32_t count, int64_t M, void *stream) {
+namespace {
+tern_status gemv_step_api(const tern_gemv_desc *descs, int32_t count, int64_t M, int fmt, const char *name,
+                          void *stream) {
     clear_error();
     if (!descs) return fail(TERN_ERR_INVALID_ARG, "descs is NULL");
     if (count < 1 || count > TERN_MAX_STEP)
         return fail(TERN_ERR_INVALID_ARG, "count must be 1..%d (got %d)", TERN_MAX_STEP, count);
-    if (M < 1 || M > 4) return fail(TERN_ERR_SHAPE, "tern_gemv_step takes M in 1..4 (got %lld)", static_cast<long long>(M));
+    if (M < 1 || M > 4) return fail(TERN_ERR_SHAPE, "%s takes M in 1..4 (got %lld)", name, static_cast<long long>(M));
     static MatDesc d[TERN_MAX_STEP];
     for (int i = 0; i < count; i++) {
         tern_status st = check_nk(descs[i].N, descs[i].K);
         if (st != TERN_OK) return st;
         if (descs[i].K % 1024 != 0)
-            return fail(TERN_ERR_SHAPE, "tern_gemv_step needs K a multiple of 1024 (descriptor %d has K=%lld)", i,
+            return fail(TERN_ERR_SHAPE, "%s needs K a multiple of 1024 (descriptor %d has K=%lld)", name, i,
                         static_cast<long long>(descs[i].K));
         st = check_mat(descs[i].x, descs[i].slots, descs[i].scales, descs[i].y);
         if (st != TERN_OK) return st;
         d[i] = mat(descs[i].x, descs[i].slots, descs[i].scales, descs[i].y, descs[i].N, descs[i].K);
     }
-    if (!gemv_step_supports(d, count, static_cast<int>(M)))
-        return fail(TERN_ERR_SHAPE, "tern_gemv_step: M x K too large for shared memory");
-    return launch_gemv_step(d, count, static_cast<int>(M), static_cast<cudaStream_t>(stream));
+    if (!gemv_step_supports(d, count, static_cast<int>(M), fmt))
+        return fail(TERN_ERR_SHAPE, "%s: M x K too large for shared memory", name);
+    return launch_gemv_step(d, count, static_cast<int>(M), fmt, static_cast<cudaStream_t>(stream));
+}
+}  // namespace
+
+tern_status tern_gemv_step(const tern_gemv_desc *descs, int32_t count, int64_t M, void *stream) {
+    return gemv_step_api(descs, count, M, 0, "tern_gemv_step", stream);
+}
+
+tern_status tern_b1_gemv_step(const tern_gemv_desc *descs, int32_t count, int64_t M, void *stream) {
+    return gemv_step_api(descs, count, M, 1, "tern_b1_gemv_step", stream);
+}
+
+tern_status tern_b1_pack(const int8_t *codes, const uint16_t *scales_in, int64_t N, int64_t K, uint8_t *bits_out,
+                         uint16_t *scales_out, int32_t *invalid_count, void *stream) {
+    clear_error();
+    tern_status st = check_nk(N, K);
+    if (st != TERN_OK) return st;
+    if (!codes || !scales_in || !bits_out || !scales_out) return fail(TERN_ERR_INVALID_ARG, "null buffer pointer");
+    if (!aligned16(codes)) return fail(TERN_ERR_ALIGN, "codes is not 16-byte aligned");
+    if (!aligned16(bits_out)) return fail(TERN_ERR_ALIGN, "bits_out is not 16-byte aligned");
+    if ((reinterpret_cast<uintptr_t>(scales_in) | reinterpret_cast<uintptr_t>(scales_out)) & 1u)
+        return fail(TERN_ERR_ALIGN, "scales are not 2-byte aligned");
+    if ((reinterpret_cast<uintptr_t>(invalid_count) & 3u) != 0)
+        return fail(TERN_ERR_ALIGN, "invalid_count is not 4-byte aligned");
+    return launch_pack_b1(codes, scales_in, N, K, bits_out, scales_out, invalid_count,
+                          static_cast<cudaStream_t>(stream));
+}
+
+tern_status tern_b1_unpack(const uint8_t *bits, int64_t N, int64_t K, int8_t *codes_out, void *stream) {
+    clear_error();
+    tern_status st = check_nk(N, K);
+    if (st != TERN_OK) return st;
+    if (!bits || !codes_out) return fail(TERN_ERR_INVALID_ARG, "null buffer pointer");
+    if (!aligned16(bits) || !aligned16(codes_out)) return fail(TERN_ERR_ALIGN, "bits and codes_out must be 16-byte aligned");
+    return launch_unpack_b1(bits, N, K, codes_out, static_cast<cudaStream_t>(stream));
 }
 
 tern_status tern_gemv_grouped(const tern_gemv_desc *descs, int32_t count, int64_t M,

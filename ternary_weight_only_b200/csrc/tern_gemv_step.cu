@@ -27,6 +27,13 @@
 // never depend on the preceding launch or piece.
 //
 // Arithmetic: the group-per-column mma.sync form (tern_unpack_mma.cuh).
+//
+// The same kernel serves the 1-bit variant (weights in {-1, +1}, one bit
+// each, fp16 scale per 128 weights: "Bonsai 27B ternary / 1-bit
+// quantization", ThakiCloud blog, sections "What it is" and "How compression
+// works"), template parameter F = 1: a stage's weights are one 128-byte-
+// swizzled box of 16 rows x 128 bytes (1024 k), the unpack is b1_slice, and
+// a group's sum is 2 D(bits) - D(all ones).
 #include <algorithm>
 #include <cstring>
 
@@ -45,9 +52,10 @@ constexpr int kThreads = kW * 32;
 constexpr int kRows = 16;                 // tile rows (mma M)
 constexpr int kSG = 8;                    // scale groups per unit (1024 k)
 constexpr int kBox = 128;                 // bytes per row of one slot box (512 k)
-constexpr int kSlotStage = kRows * kBox * 2;           // two boxes: 4096
 constexpr int kScaleStage = kRows * kSG * 2;           // 256
-constexpr int kStageBytes = kSlotStage + kScaleStage;  // 4352
+// weight bytes of one stage (16 rows x 1024 k): 2-bit slots (two boxes) or bits
+__host__ __device__ constexpr int slot_stage(int f) { return f ? kRows * kBox : kRows * kBox * 2; }
+__host__ __device__ constexpr int stage_bytes(int f) { return slot_stage(f) + kScaleStage; }
 constexpr int kMaxNS = 4;
 constexpr int kMaxCtas = 160;
 constexpr int kMaxPer = 96;               // matrices per launch (parameter space)
@@ -63,6 +71,7 @@ struct SDesc {
 
 struct alignas(64) SMaps {
     CUtensorMap smap;   // slots as uint8 [K/512][N][128], box 128 B x 16 rows x 2, 128-byte swizzle
+                        // (1-bit: bits as uint8 [N][K/8], box 128 B x 16 rows, 128-byte swizzle)
     CUtensorMap cmap;   // scales fp16 [N][K/128], box 8 x 16, no swizzle
 };
 
@@ -88,8 +97,8 @@ __host__ __device__ constexpr int d1_off() { return wmax_off() + kW * 4; }      
 __host__ __device__ constexpr int xs_off(int kmax) { return d1_off() + (kmax / 128) * 16 + 64; }
 // staged x: MT token rows (M real, the rest zero)
 __host__ __device__ constexpr int ring_off(int kmax, int mt) { return (xs_off(kmax) + kmax * 2 * mt + 1023) & ~1023; }
-size_t smem_bytes(int kmax, int mt, int ns) {
-    return 1024 + static_cast<size_t>(ring_off(kmax, mt)) + static_cast<size_t>(kW) * ns * kStageBytes;
+size_t smem_bytes(int kmax, int mt, int ns, int f) {
+    return 1024 + static_cast<size_t>(ring_off(kmax, mt)) + static_cast<size_t>(kW) * ns * stage_bytes(f);
 }
 
 __device__ __forceinline__ bool step_wait(uint64_t *bar, uint32_t parity, unsigned long long deadline) {
@@ -153,10 +162,13 @@ __device__ __forceinline__ void cursor_next(Cursor &c, const SParams &p, int T0,
 }
 
 // MT = token rows padded to 1, 2 or 4: the group-per-column form with
-// (group, token) pairs in the mma columns (gcm_slice).
-template <int MT>
+// (group, token) pairs in the mma columns (gcm_slice, or b1_slice for F = 1).
+template <int MT, int F>
 __global__ void __launch_bounds__(kThreads, 1) gemv_step_kernel(const __grid_constant__ SParams p) {
     constexpr int GPB = 8 / MT;  // groups per set
+    constexpr int kSlotStage = slot_stage(F);
+    constexpr int kStageBytes = stage_bytes(F);
+    constexpr int kWords = F ? 2 : 4;  // weight words of a group a lane holds
     extern __shared__ uint8_t smem_raw[];
     uint8_t *base = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     uint64_t *full = reinterpret_cast<uint64_t *>(base + bar_off());  // [kW][kMaxNS]
@@ -171,9 +183,17 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_step_kernel(const __grid_con
     const int row = tile_row(g);
     const float4 qm = make_float4(q == 0 ? 1.f : 0.f, q == 1 ? 1.f : 0.f, q == 2 ? 1.f : 0.f, q == 3 ? 1.f : 0.f);
     const float2 qh = make_float2(q < 2 ? 1.f : 0.f, q < 2 ? 0.f : 1.f);
-    uint32_t off[4];  // 128-byte-swizzled position of words 2q, 2q+1 of group j (0..3 in a box) of `row`
+    // 128-byte-swizzled position of the lane's words of group G in `row`:
+    // words 2q, 2q+1 of group G % 4 of box G / 4 (ternary), or word q of
+    // group G (1-bit: 16 bytes per group row)
+    uint32_t off[F ? 8 : 4];
+    if constexpr (F == 0) {
 #pragma unroll
-    for (int j = 0; j < 4; j++) off[j] = row * kBox + (((2 * j + (q >> 1)) ^ (row & 7)) << 4) + (q & 1) * 8;
+        for (int j = 0; j < 4; j++) off[j] = row * kBox + (((2 * j + (q >> 1)) ^ (row & 7)) << 4) + (q & 1) * 8;
+    } else {
+#pragma unroll
+        for (int G8 = 0; G8 < 8; G8++) off[G8] = row * kBox + ((G8 ^ (row & 7)) << 4) + 4 * q;
+    }
     const int T0 = p.cta_tile[blockIdx.x], T1 = p.cta_tile[blockIdx.x + 1];
     // first matrix with a tile at or after T0
     int i0 = 0;
@@ -217,7 +237,10 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_step_kernel(const __grid_con
         if (lane == 0) {
             uint8_t *stage = my_ring + st * kSlotStage;
             mbar_expect_tx(&my_full[st], kStageBytes);
-            tma_load_3d(stage, &p.m[ic.i].smap, 0, ic.tile * kRows, ic.kb * 2, &my_full[st]);
+            if constexpr (F == 0)
+                tma_load_3d(stage, &p.m[ic.i].smap, 0, ic.tile * kRows, ic.kb * 2, &my_full[st]);
+            else
+                tma_load_2d(stage, &p.m[ic.i].smap, ic.kb * kBox, ic.tile * kRows, &my_full[st]);
             tma_load_2d(my_scl + st * kScaleStage, &p.m[ic.i].cmap, ic.kb * kSG, ic.tile * kRows, &my_full[st]);
         }
         cursor_next(ic, p, T0, T1, warp);
@@ -256,8 +279,35 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_step_kernel(const __grid_con
 #pragma unroll
         for (int w = 0; w < kW; w++) mx = max(mx, wmax[w]);
         const int ex = max(static_cast<int>(mx >> 10), 1) - 15;
-        const int E = min(8, 15 - ex);
-        {
+        // the largest staged factor is 2^E: x * 2^E stays finite
+        const int E = min(F ? 7 : 8, 15 - ex);
+        if constexpr (F == 1) {
+            // factor of bit position p (0..15 in a half) is 2^(E - (p & 7));
+            // 8 consecutive x are positions p0 .. p0 + 7, p0 = 0 or 8
+            uint32_t fac2[4];
+#pragma unroll
+            for (int c = 0; c < 4; c++)
+                fac2[c] = (static_cast<uint32_t>(15 + E - 2 * c) << 10) |
+                          (static_cast<uint32_t>(15 + E - 2 * c - 1) << 26);
+            const int per_m = K / 8;
+            for (int idx = threadIdx.x; idx < MT * per_m; idx += nthr) {
+                const int m = idx / per_m, c8 = idx - m * per_m;
+                uint4 v = make_uint4(0u, 0u, 0u, 0u);
+                if (m < M) v = *reinterpret_cast<const uint4 *>(d.x + static_cast<size_t>(m) * K + c8 * 8);
+                const uint32_t pr[4] = {v.x, v.y, v.z, v.w};
+                const int kl = c8 * 8;
+                const int gk = kl >> 7;
+                unsigned short *dst = reinterpret_cast<unsigned short *>(
+                    xs + (gk / GPB) * 1024 + b1_xs_index((gk % GPB) * MT + m, kl & 127));
+#pragma unroll
+                for (int c = 0; c < 4; c++) {
+                    uint32_t h2;
+                    asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(h2) : "r"(pr[c]), "r"(fac2[c]));
+                    dst[(c >> 1) * 256 + (c & 1) * 4] = static_cast<unsigned short>(h2);
+                    dst[(c >> 1) * 256 + (c & 1) * 4 + 2] = static_cast<unsigned short>(h2 >> 16);
+                }
+            }
+        } else {
             uint32_t fac2[4];
 #pragma unroll
             for (int c = 0; c < 4; c++) {
@@ -290,7 +340,10 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_step_kernel(const __grid_con
         // one all-ones chain per set: d1[set * 8 + column]
         for (int sl = warp; sl < B * MT; sl += kW) {
             float c[4];
-            group_mma<8>(c, kOnes, kOnes, kOnes, kOnes, xlane + sl * 1024);
+            if constexpr (F == 0)
+                group_mma<8>(c, kOnes, kOnes, kOnes, kOnes, xlane + sl * 1024);
+            else
+                b1_ones_chain(c, xlane + sl * 1024);
             if (g == 0) *reinterpret_cast<float2 *>(d1 + sl * kSG + 2 * q) = make_float2(c[0], c[1]);
         }
         __syncthreads();
@@ -332,16 +385,21 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_step_kernel(const __grid_con
             if (ok) ok = __all_sync(0xffffffffu, step_wait(&my_full[s], ph, deadline));
             dead = dead || !ok;
             if (ok) {
-                uint32_t wd[kSG][4];
+                uint32_t wd[kSG][kWords];
 #pragma unroll
                 for (int G8 = 0; G8 < kSG; G8++) {
-                    const uint8_t *bx = stage + (G8 >> 2) * (kRows * kBox);
-                    const uint2 a = *reinterpret_cast<const uint2 *>(bx + off[G8 & 3]);
-                    const uint2 b = *reinterpret_cast<const uint2 *>(bx + off[G8 & 3] + 8 * kBox);
-                    wd[G8][0] = a.x;
-                    wd[G8][1] = b.x;
-                    wd[G8][2] = a.y;
-                    wd[G8][3] = b.y;
+                    if constexpr (F == 0) {
+                        const uint8_t *bx = stage + (G8 >> 2) * (kRows * kBox);
+                        const uint2 a = *reinterpret_cast<const uint2 *>(bx + off[G8 & 3]);
+                        const uint2 b = *reinterpret_cast<const uint2 *>(bx + off[G8 & 3] + 8 * kBox);
+                        wd[G8][0] = a.x;
+                        wd[G8][1] = b.x;
+                        wd[G8][2] = a.y;
+                        wd[G8][3] = b.y;
+                    } else {
+                        wd[G8][0] = *reinterpret_cast<const uint32_t *>(stage + off[G8]);
+                        wd[G8][1] = *reinterpret_cast<const uint32_t *>(stage + off[G8] + 8 * kBox);
+                    }
                 }
                 // scales of the lane's groups (rows `row`, `row` + 8): MT = 1
                 // groups 2q, 2q+1; otherwise one group per set h (4h + q, or
@@ -368,7 +426,10 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_step_kernel(const __grid_con
                     issue(s);
                 }
                 float out[MT][4];
-                gcm_slice<MT>(wd, xlane + kb * MT * 1024, qm, qh, out);
+                if constexpr (F == 0)
+                    gcm_slice<MT>(wd, xlane + kb * MT * 1024, qm, qh, out);
+                else
+                    b1_slice<MT>(wd, xlane + kb * MT * 1024, qm, qh, out);
                 // acc[0..1] = row g, columns 2q, 2q+1; acc[2..3] = row g+8
 #pragma unroll
                 for (int h = 0; h < MT; h++) {
@@ -382,10 +443,12 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_step_kernel(const __grid_con
                         sa0 = sa1 = f.x;
                         sb0 = sb1 = f.y;
                     }
-                    acc[0] = fmaf(sa0, out[h][0] - on.x, acc[0]);
-                    acc[1] = fmaf(sa1, out[h][1] - on.y, acc[1]);
-                    acc[2] = fmaf(sb0, out[h][2] - on.x, acc[2]);
-                    acc[3] = fmaf(sb1, out[h][3] - on.y, acc[3]);
+                    // t = c - 1 (ternary) or t = 2b - 1 (1-bit)
+                    constexpr float kMul = F ? 2.f : 1.f;
+                    acc[0] = fmaf(sa0, fmaf(kMul, out[h][0], -on.x), acc[0]);
+                    acc[1] = fmaf(sa1, fmaf(kMul, out[h][1], -on.y), acc[1]);
+                    acc[2] = fmaf(sb0, fmaf(kMul, out[h][2], -on.x), acc[2]);
+                    acc[3] = fmaf(sb1, fmaf(kMul, out[h][3], -on.y), acc[3]);
                 }
             }
             stage += kSlotStage;
@@ -469,13 +532,19 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_step_kernel(const __grid_con
     }
 }
 
-bool g_attr_step[64][3];
+bool g_attr_step[64][2][3];
+
+using StepKernel = void (*)(SParams);
+StepKernel step_kernel(int mt, int f) {
+    if (f == 0) return mt == 1 ? gemv_step_kernel<1, 0> : (mt == 2 ? gemv_step_kernel<2, 0> : gemv_step_kernel<4, 0>);
+    return mt == 1 ? gemv_step_kernel<1, 1> : (mt == 2 ? gemv_step_kernel<2, 1> : gemv_step_kernel<4, 1>);
+}
 
 int step_mt(int M) { return M == 1 ? 1 : (M == 2 ? 2 : 4); }
 
 }  // namespace
 
-bool gemv_step_supports(const MatDesc *md, int count, int M) {
+bool gemv_step_supports(const MatDesc *md, int count, int M, int fmt) {
     if (count < 1 || count > TERN_MAX_STEP || M < 1 || M > 4) return false;
     int kmax = 0;
     for (int i = 0; i < count; i++) {
@@ -483,13 +552,13 @@ bool gemv_step_supports(const MatDesc *md, int count, int M) {
         kmax = std::max(kmax, md[i].K);
     }
     // one ring stage per warp at least (refilled as soon as it is read)
-    return smem_bytes(kmax, step_mt(M), 1) <= kSmemBudget;
+    return smem_bytes(kmax, step_mt(M), 1, fmt) <= kSmemBudget;
 }
 
 namespace {
 
 // One launch over md[0..count) (count <= kMaxPer).
-tern_status launch_chunk(const DeviceInfo &dev, const MatDesc *md, int count, int M, cudaStream_t stream) {
+tern_status launch_chunk(const DeviceInfo &dev, const MatDesc *md, int count, int M, int fmt, cudaStream_t stream) {
     static SParams p;  // large (parameter space); filled on the host for each launch
     std::memset(&p, 0, sizeof(p));
     const int mt = step_mt(M);
@@ -507,14 +576,22 @@ tern_status launch_chunk(const DeviceInfo &dev, const MatDesc *md, int count, in
         tiles += d.ntile;
         total_units += static_cast<long long>(d.ntile) * (md[i].K / 1024);
         kmax = std::max(kmax, md[i].K);
-        // the slot matrix seen as [K/512 chunks][N rows][128 bytes]: one copy
-        // brings both 512-k boxes of a unit
-        const uint64_t sdims[3] = {static_cast<uint64_t>(kBox), static_cast<uint64_t>(md[i].N),
-                                   static_cast<uint64_t>(md[i].K / 512)};
-        const uint64_t sstr[2] = {static_cast<uint64_t>(md[i].K / 4), static_cast<uint64_t>(kBox)};
-        const uint32_t sbox[3] = {static_cast<uint32_t>(kBox), static_cast<uint32_t>(kRows), 2};
-        tern_status st = encode_tiled_3d(&p.m[i].smap, CU_TENSOR_MAP_DATA_TYPE_UINT8, md[i].slots, sdims, sstr, sbox,
-                                         CU_TENSOR_MAP_SWIZZLE_128B);
+        tern_status st;
+        if (fmt == 0) {
+            // the slot matrix seen as [K/512 chunks][N rows][128 bytes]: one
+            // copy brings both 512-k boxes of a unit
+            const uint64_t sdims[3] = {static_cast<uint64_t>(kBox), static_cast<uint64_t>(md[i].N),
+                                       static_cast<uint64_t>(md[i].K / 512)};
+            const uint64_t sstr[2] = {static_cast<uint64_t>(md[i].K / 4), static_cast<uint64_t>(kBox)};
+            const uint32_t sbox[3] = {static_cast<uint32_t>(kBox), static_cast<uint32_t>(kRows), 2};
+            st = encode_tiled_3d(&p.m[i].smap, CU_TENSOR_MAP_DATA_TYPE_UINT8, md[i].slots, sdims, sstr, sbox,
+                                 CU_TENSOR_MAP_SWIZZLE_128B);
+        } else {
+            // the bit matrix [N rows][K/8 bytes]: one 128-byte box is a unit's row
+            st = encode_tiled_2d(&p.m[i].smap, CU_TENSOR_MAP_DATA_TYPE_UINT8, md[i].slots,
+                                 static_cast<uint64_t>(md[i].K / 8), static_cast<uint64_t>(md[i].N),
+                                 static_cast<uint64_t>(md[i].K / 8), kBox, kRows, CU_TENSOR_MAP_SWIZZLE_128B);
+        }
         if (st != TERN_OK) return st;
         const int G = md[i].K / kGroup;
         st = encode_tiled_2d(&p.m[i].cmap, CU_TENSOR_MAP_DATA_TYPE_UINT16, md[i].scales, static_cast<uint64_t>(G),
@@ -524,9 +601,9 @@ tern_status launch_chunk(const DeviceInfo &dev, const MatDesc *md, int count, in
     }
     const size_t budget = std::min<size_t>(kSmemBudget, dev.max_smem_optin);
     // The whole budget: every CTA sizes its ring from what its own staged x leaves.
-    const size_t smem = std::min(budget, smem_bytes(kmax, mt, kMaxNS));
-    if (smem_bytes(kmax, mt, 1) > smem)
-        return fail(TERN_ERR_SHAPE, "step kernel needs %zu B of shared memory", smem_bytes(kmax, mt, 1));
+    const size_t smem = std::min(budget, smem_bytes(kmax, mt, kMaxNS, fmt));
+    if (smem_bytes(kmax, mt, 1, fmt) > smem)
+        return fail(TERN_ERR_SHAPE, "step kernel needs %zu B of shared memory", smem_bytes(kmax, mt, 1, fmt));
     int grid = std::min<int>(std::min(dev.sms, kMaxCtas), tiles);
     if (g_opt.gemv_grid > 0) grid = std::min(grid, g_opt.gemv_grid);
     // Cut the flat tile list into `grid` ranges of about equal units: CTA c
@@ -567,33 +644,32 @@ tern_status launch_chunk(const DeviceInfo &dev, const MatDesc *md, int count, in
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    auto kern = mt == 1 ? gemv_step_kernel<1> : (mt == 2 ? gemv_step_kernel<2> : gemv_step_kernel<4>);
-    cudaError_t e = cudaLaunchKernelEx(&cfg, kern, p);
+    cudaError_t e = cudaLaunchKernelEx(&cfg, step_kernel(mt, fmt), p);
     if (e != cudaSuccess) return cuda_fail(e, "gemv step kernel launch");
     return TERN_OK;
 }
 
 }  // namespace
 
-tern_status launch_gemv_step(const MatDesc *md, int count, int M, cudaStream_t stream) {
+tern_status launch_gemv_step(const MatDesc *md, int count, int M, int fmt, cudaStream_t stream) {
     DeviceInfo dev;
     tern_status st = current_device(&dev);
     if (st != TERN_OK) return st;
-    if (!gemv_step_supports(md, count, M)) return fail(TERN_ERR_SHAPE, "step kernel: unsupported shapes");
+    if (fmt != 0 && fmt != 1) return fail(TERN_ERR_INVALID_ARG, "step kernel: unknown weight format %d", fmt);
+    if (!gemv_step_supports(md, count, M, fmt)) return fail(TERN_ERR_SHAPE, "step kernel: unsupported shapes");
     const int mi = step_mt(M) == 1 ? 0 : (step_mt(M) == 2 ? 1 : 2);
-    if (!g_attr_step[dev.device][mi]) {
-        auto kern = mi == 0 ? gemv_step_kernel<1> : (mi == 1 ? gemv_step_kernel<2> : gemv_step_kernel<4>);
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if (!g_attr_step[dev.device][fmt][mi]) {
+        cudaError_t e = cudaFuncSetAttribute(step_kernel(step_mt(M), fmt), cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              static_cast<int>(dev.max_smem_optin));
         if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(gemv step)");
-        g_attr_step[dev.device][mi] = true;
+        g_attr_step[dev.device][fmt][mi] = true;
     }
     // Equal-sized launches of at most kMaxPer matrices each.
     const int launches = (count + kMaxPer - 1) / kMaxPer;
     int done = 0;
     for (int l = 0; l < launches; l++) {
         const int n = (count - done) / (launches - l);
-        st = launch_chunk(dev, md + done, n, M, stream);
+        st = launch_chunk(dev, md + done, n, M, fmt, stream);
         if (st != TERN_OK) return st;
         done += n;
     }

@@ -45,6 +45,10 @@ tern_status launch_pack(const int8_t *codes, const uint16_t *scales_in, int64_t 
                         cudaStream_t stream);
 tern_status launch_unpack(const uint8_t *slots, int64_t N, int64_t K, int8_t *codes,
                           cudaStream_t stream);
+// the 1-bit variant: bits uint8 [N][K/8], weight k at bit k % 8 of byte k / 8
+tern_status launch_pack_b1(const int8_t *codes, const uint16_t *scales_in, int64_t N, int64_t K, uint8_t *bits,
+                           uint16_t *scales_out, int32_t *invalid_count, cudaStream_t stream);
+tern_status launch_unpack_b1(const uint8_t *bits, int64_t N, int64_t K, int8_t *codes, cudaStream_t stream);
 
 struct MatDesc {
     const __half *x;
@@ -97,9 +101,10 @@ tern_status read_gemvpc_status(bool reset, unsigned int *out);
 // Ternary embedding rows gathered by id, written as fp16 s * t.
 tern_status launch_embed(const int32_t *ids, int64_t M, const uint8_t *slots, const uint16_t *scales, int64_t V,
                          int64_t K, uint16_t *out, int32_t *bad_count, cudaStream_t stream);
-// Persistent launch over many matrices (M = 1..4, K multiples of 1024).
-bool gemv_step_supports(const MatDesc *d, int count, int M);
-tern_status launch_gemv_step(const MatDesc *d, int count, int M, cudaStream_t stream);
+// Persistent launch over many matrices (M = 1..4, K multiples of 1024); fmt 0
+// = ternary slots, 1 = the 1-bit variant (MatDesc::slots holds the bits).
+bool gemv_step_supports(const MatDesc *d, int count, int M, int fmt);
+tern_status launch_gemv_step(const MatDesc *d, int count, int M, int fmt, cudaStream_t stream);
 tern_status read_gemvstep_status(bool reset, unsigned int *out);
 extern unsigned long long g_gemm_timeout_ns;
 extern int g_gemm_skip_loads;

@@ -10,6 +10,13 @@
 // Both kernels are plain streaming kernels: every thread turns 16 consecutive
 // int8 codes (one 16-byte load) into one 32-bit slot word, so code j of the
 // chunk lands at bit 2j of the word -- byte j/4, bit pair j%4.
+//
+// The 1-bit variant (weights in {-1, +1} with the same fp16 scale per 128
+// weights: "Bonsai 27B ternary / 1-bit quantization", ThakiCloud blog,
+// sections "What it is" and "How compression works") packs one bit
+// b = (t + 1) / 2 per weight, weight k of a row at bit k % 8 of byte k / 8:
+// a thread turns 32 codes (two 16-byte loads) into one 32-bit word, code j
+// at bit j.
 #include "tern_internal.cuh"
 
 namespace tern {
@@ -86,6 +93,66 @@ __global__ void __launch_bounds__(kPackThreads) unpack_kernel(const uint32_t *__
     }
 }
 
+__global__ void __launch_bounds__(kPackThreads) pack_b1_kernel(const int4 *__restrict__ codes,
+                                                               uint32_t *__restrict__ bits, int64_t nwords,
+                                                               const uint16_t *__restrict__ sc_in,
+                                                               uint16_t *__restrict__ sc_out, int64_t nscales,
+                                                               int32_t *invalid_count) {
+    int bad = 0;
+    const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+    for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < nwords; i += stride) {
+        const int4 v0 = codes[2 * i], v1 = codes[2 * i + 1];
+        const uint32_t w8[8] = {static_cast<uint32_t>(v0.x), static_cast<uint32_t>(v0.y),
+                                static_cast<uint32_t>(v0.z), static_cast<uint32_t>(v0.w),
+                                static_cast<uint32_t>(v1.x), static_cast<uint32_t>(v1.y),
+                                static_cast<uint32_t>(v1.z), static_cast<uint32_t>(v1.w)};
+        uint32_t out = 0;
+#pragma unroll
+        for (int b = 0; b < 8; b++) {
+#pragma unroll
+            for (int j = 0; j < 4; j++) {
+                const int t = static_cast<int8_t>((w8[b] >> (8 * j)) & 0xFF);
+                // +1 -> bit 1; -1 -> bit 0; anything else -> bit 0, counted
+                bad += (t == 1 || t == -1) ? 0 : 1;
+                out |= static_cast<uint32_t>(t == 1) << (4 * b + j);
+            }
+        }
+        bits[i] = out;
+    }
+    if (sc_out != nullptr) {
+        for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < nscales; i += stride)
+            sc_out[i] = sc_in[i];
+    }
+    if (invalid_count != nullptr) {
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) bad += __shfl_xor_sync(0xffffffffu, bad, o);
+        if ((threadIdx.x & 31) == 0 && bad != 0) atomicAdd(invalid_count, bad);
+    }
+}
+
+__global__ void __launch_bounds__(kPackThreads) unpack_b1_kernel(const uint32_t *__restrict__ bits,
+                                                                 int4 *__restrict__ codes, int64_t nwords) {
+    const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+    for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < nwords; i += stride) {
+        const uint32_t w = bits[i];
+        uint32_t o[8];
+#pragma unroll
+        for (int b = 0; b < 8; b++) {
+            uint32_t word = 0;
+#pragma unroll
+            for (int j = 0; j < 4; j++) {
+                const uint32_t t = ((w >> (4 * b + j)) & 1u) ? 0x01u : 0xFFu;  // +1 or -1 as int8
+                word |= t << (8 * j);
+            }
+            o[b] = word;
+        }
+        codes[2 * i] = make_int4(static_cast<int>(o[0]), static_cast<int>(o[1]), static_cast<int>(o[2]),
+                                 static_cast<int>(o[3]));
+        codes[2 * i + 1] = make_int4(static_cast<int>(o[4]), static_cast<int>(o[5]), static_cast<int>(o[6]),
+                                     static_cast<int>(o[7]));
+    }
+}
+
 int grid_for(int64_t work, int sms) {
     const int64_t want = (work + kPackThreads - 1) / kPackThreads;
     const int64_t cap = static_cast<int64_t>(sms) * 8;
@@ -119,6 +186,30 @@ tern_status launch_unpack(const uint8_t *slots, int64_t N, int64_t K, int8_t *co
     unpack_kernel<<<grid_for(nchunks, dev.sms), kPackThreads, 0, stream>>>(
         reinterpret_cast<const uint32_t *>(slots), reinterpret_cast<int4 *>(codes), nchunks);
     return cuda_fail(cudaGetLastError(), "unpack kernel launch");
+}
+
+tern_status launch_pack_b1(const int8_t *codes, const uint16_t *scales_in, int64_t N, int64_t K, uint8_t *bits,
+                           uint16_t *scales_out, int32_t *invalid_count, cudaStream_t stream) {
+    DeviceInfo dev;
+    tern_status st = current_device(&dev);
+    if (st != TERN_OK) return st;
+    const int64_t nwords = N * K / 32;
+    const int64_t nscales = N * (K / kGroup);
+    uint16_t *sout = (scales_in == scales_out) ? nullptr : scales_out;
+    pack_b1_kernel<<<grid_for(nwords, dev.sms), kPackThreads, 0, stream>>>(
+        reinterpret_cast<const int4 *>(codes), reinterpret_cast<uint32_t *>(bits), nwords, scales_in, sout, nscales,
+        invalid_count);
+    return cuda_fail(cudaGetLastError(), "1-bit pack kernel launch");
+}
+
+tern_status launch_unpack_b1(const uint8_t *bits, int64_t N, int64_t K, int8_t *codes, cudaStream_t stream) {
+    DeviceInfo dev;
+    tern_status st = current_device(&dev);
+    if (st != TERN_OK) return st;
+    const int64_t nwords = N * K / 32;
+    unpack_b1_kernel<<<grid_for(nwords, dev.sms), kPackThreads, 0, stream>>>(
+        reinterpret_cast<const uint32_t *>(bits), reinterpret_cast<int4 *>(codes), nwords);
+    return cuda_fail(cudaGetLastError(), "1-bit unpack kernel launch");
 }
 
 }  // namespace tern

@@ -138,6 +138,32 @@ __device__ __forceinline__ void gc_slice(uint32_t (&wd)[8][4], const uint4 (&xf)
     v3 = pick4(qm, dd[1][3], dd[3][3], dd[5][3], dd[7][3]);
 }
 
+// The lane's own columns of the eight per-group accumulators of a
+// group-per-column slice (dd[G] = group G's chain; the column map is the one
+// gcm_slice describes).
+template <int MG>
+__device__ __forceinline__ void gc_pick(const float (&dd)[8][4], const float4 &qm, const float2 &qh,
+                                        float (&out)[MG][4]) {
+    if (MG == 1) {
+#pragma unroll
+        for (int c = 0; c < 4; c++) {
+            const int o = c & 1;  // column 2q + o: group 2q + o
+            out[0][c] = pick4(qm, dd[o][c], dd[2 + o][c], dd[4 + o][c], dd[6 + o][c]);
+        }
+    } else if (MG == 2) {
+#pragma unroll
+        for (int h = 0; h < MG; h++)
+#pragma unroll
+            for (int c = 0; c < 4; c++)
+                out[h][c] = pick4(qm, dd[4 * h][c], dd[4 * h + 1][c], dd[4 * h + 2][c], dd[4 * h + 3][c]);
+    } else {
+#pragma unroll
+        for (int h = 0; h < MG; h++)
+#pragma unroll
+            for (int c = 0; c < 4; c++) out[h][c] = fmaf(qh.y, dd[(2 * h + 1) % 8][c], qh.x * dd[(2 * h) % 8][c]);
+    }
+}
+
 // Group-per-column slice for MG token rows (MG = 1, 2 or 4): the eight B
 // columns carry (group, token) pairs, column n = group n / MG of a "set",
 // token n % MG; a 1024-k slice has MG sets of 8 / MG groups, staged by
@@ -181,24 +207,99 @@ __device__ __forceinline__ void gcm_slice(uint32_t (&wd)[8][4], const __half *xs
                 mma_acc(dd[G8], wd[G8][0] & m, wd[G8][1] & m, wd[G8][2] & m, wd[G8][3] & m, b0, b1);
         }
     }
-    if (MG == 1) {
+    gc_pick<MG>(dd, qm, qh, out);
+}
+
+// ---- the 1-bit variant: weights in {-1, +1}, one bit b = (t + 1) / 2 each,
+// weight k of a row at bit k % 8 of byte k / 8 ("Bonsai 27B ternary / 1-bit
+// quantization", ThakiCloud blog, section "What it is") ----
+//
+// A 32-bit word holds 32 consecutive weights of one row; its "pair p"
+// (p = 0..15) is bit p of both 16-bit halves (weights p and p + 16).  One AND
+// with 0x00010001 << p' (p' = p for p < 8; the word shifted right by 8 and
+// p' = p - 8 otherwise) leaves an fp16 pair whose halves are the subnormals
+// b * 2^(p' - 24), exactly.  mma i (0..7) of a 16-row x 128-k group takes
+// pairs 2i (A registers a0, a1: rows g, g+8) and 2i + 1 (a2, a3) of the
+// lane's word q of rows g and g+8, so one mma sees the factors 2^(2i & 7)
+// and 2^((2i+1) & 7); the staged x carries their inverses (b1_xs_index).
+// With t = 2b - 1 a group's sum is 2 D(bits) - D(all ones), D(all ones)
+// from the very same chain on the all-ones word.
+
+// Index (in halves) of x at k = kl (0..127 inside the group) of column col
+// in the 1-bit staging area of one set: per mma pair (chunk c = mmas 2c,
+// 2c + 1) and lane (col, q) eight halves [mma & 1][pair & 1][half], so the
+// B fragments of two mmas are one 16-byte load, as for the ternary layout.
+__device__ __forceinline__ int b1_xs_index(int col, int kl) {
+    const int q = (kl >> 5) & 3;
+    const int hi = (kl >> 4) & 1;
+    const int p = kl & 15;
+    return (((p >> 2) * 8 + col) * 4 + q) * 8 + ((p >> 1) & 1) * 4 + (p & 1) * 2 + hi;
+}
+
+// The A registers of mma i from the lane's words (w0 = row g, w1 = row g+8),
+// already shifted right by 8 for i >= 4.
+__device__ __forceinline__ void b1_a_regs(int i, uint32_t w0, uint32_t w1, uint32_t (&a)[4]) {
+    const uint32_t m0 = 0x00010001u << ((2 * i) & 7), m1 = 0x00010001u << ((2 * i + 1) & 7);
+    a[0] = w0 & m0;
+    a[1] = w1 & m0;
+    a[2] = w0 & m1;
+    a[3] = w1 & m1;
+}
+
+// D(all ones) of one set's column: the eight-mma chain b1_slice runs for a
+// group, on the all-ones word (every A register is its mask), with the B
+// fragments at xb (the lane's eight halves of chunk 0; chunk c at + 256 c).
+__device__ __forceinline__ void b1_ones_chain(float (&c)[4], const __half *xb) {
+    uint4 xf[4];
+    load_xfrag<8>(xb, xf);
 #pragma unroll
-        for (int c = 0; c < 4; c++) {
-            const int o = c & 1;  // column 2q + o: group 2q + o
-            out[0][c] = pick4(qm, dd[o][c], dd[2 + o][c], dd[4 + o][c], dd[6 + o][c]);
-        }
-    } else if (MG == 2) {
-#pragma unroll
-        for (int h = 0; h < MG; h++)
-#pragma unroll
-            for (int c = 0; c < 4; c++)
-                out[h][c] = pick4(qm, dd[4 * h][c], dd[4 * h + 1][c], dd[4 * h + 2][c], dd[4 * h + 3][c]);
-    } else {
-#pragma unroll
-        for (int h = 0; h < MG; h++)
-#pragma unroll
-            for (int c = 0; c < 4; c++) out[h][c] = fmaf(qh.y, dd[(2 * h + 1) % 8][c], qh.x * dd[(2 * h) % 8][c]);
+    for (int i = 0; i < 8; i++) {
+        uint32_t a[4];
+        b1_a_regs(i, 0xFFFFFFFFu, 0xFFFFFFFFu, a);
+        const uint4 &xv = xf[i >> 1];
+        const uint32_t b0 = (i & 1) ? xv.z : xv.x, b1 = (i & 1) ? xv.w : xv.y;
+        if (i == 0)
+            mma_zero(c, a[0], a[1], a[2], a[3], b0, b1);
+        else
+            mma_acc(c, a[0], a[1], a[2], a[3], b0, b1);
     }
+}
+
+// The 1-bit group-per-column slice (same columns, sets and outputs as
+// gcm_slice): wd[G] = {row g word q, row g+8 word q} of group G
+// (overwritten).  The mmas go i outer, group inner: eight independent chains.
+template <int MG>
+__device__ __forceinline__ void b1_slice(uint32_t (&wd)[8][2], const __half *xs, const float4 &qm, const float2 &qh,
+                                         float (&out)[MG][4]) {
+    constexpr int GPB = 8 / MG;  // groups per set
+    float dd[8][4];
+    uint4 xq[MG];
+#pragma unroll
+    for (int i = 0; i < 8; i++) {
+        if ((i & 1) == 0) {
+#pragma unroll
+            for (int h = 0; h < MG; h++) xq[h] = *reinterpret_cast<const uint4 *>(xs + h * 1024 + (i >> 1) * 256);
+        }
+        if (i == 4) {
+#pragma unroll
+            for (int G8 = 0; G8 < 8; G8++) {
+                wd[G8][0] >>= 8;
+                wd[G8][1] >>= 8;
+            }
+        }
+#pragma unroll
+        for (int G8 = 0; G8 < 8; G8++) {
+            const uint4 &xv = xq[G8 / GPB];
+            const uint32_t b0 = (i & 1) ? xv.z : xv.x, b1 = (i & 1) ? xv.w : xv.y;
+            uint32_t a[4];
+            b1_a_regs(i, wd[G8][0], wd[G8][1], a);
+            if (i == 0)
+                mma_zero(dd[G8], a[0], a[1], a[2], a[3], b0, b1);
+            else
+                mma_acc(dd[G8], a[0], a[1], a[2], a[3], b0, b1);
+        }
+    }
+    gc_pick<MG>(dd, qm, qh, out);
 }
 
 }  // namespace tern

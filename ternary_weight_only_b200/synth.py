@@ -7,6 +7,7 @@ tensors feed the CUDA path and, in the tests, the CPU oracle.
 Distributions (one synthetic decoder layer at hidden size 5120, a 5120 ->
 151936 output head, and prefill blocks):
   * ternary codes: iid uniform over {-1,0,+1}, or P(0)=0.4, P(+-1)=0.3;
+  * 1-bit codes: iid uniform over {-1,+1};
   * group scales: fp32 U[0.005, 0.05] rounded to fp16 (round-to-nearest-even);
   * activations: fp32 N(0,1) rounded to fp16, optionally with each element
     independently multiplied by 20 with probability 0.01 (outliers).
@@ -56,6 +57,11 @@ def codes_sparse(N: int, K: int, g: torch.Generator, p0: float = 0.4, device="cp
     return out
 
 
+def codes_sign(N: int, K: int, g: torch.Generator, device="cpu") -> torch.Tensor:
+    """int8 [N,K], iid uniform over {-1,+1} (the 1-bit variant)."""
+    return (torch.randint(0, 2, (N, K), generator=g, device=device, dtype=torch.int8) * 2 - 1)
+
+
 def scales_uniform(N: int, K: int, g: torch.Generator, lo: float = 0.005, hi: float = 0.05,
                    device="cpu") -> torch.Tensor:
     """fp16 [N, K/128]: fp32 U[lo,hi] rounded to fp16."""
@@ -77,7 +83,12 @@ def case(M: int, K: int, N: int, seed: int, codes: str = "uniform", outlier_p: f
          device="cpu"):
     """(x fp16 [M,K], codes int8 [N,K], scales fp16 [N,K/128]) from one seed."""
     g = gen(seed, device)
-    c = codes_uniform(N, K, g, device) if codes == "uniform" else codes_sparse(N, K, g, device=device)
+    if codes == "uniform":
+        c = codes_uniform(N, K, g, device)
+    elif codes == "sign":
+        c = codes_sign(N, K, g, device)
+    else:
+        c = codes_sparse(N, K, g, device=device)
     s = scales_uniform(N, K, g, device=device)
     x = activations(M, K, g, outlier_p=outlier_p, device=device)
     return x, c, s

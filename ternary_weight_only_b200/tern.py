@@ -69,6 +69,9 @@ _SIGS = {
     "tern_gemv_noalloc": ([_vp, _vp, _vp, _vp, _i64, _i64, _vp], _int),
     "tern_gemv_step": ([ctypes.POINTER(tern_gemv_desc), _i32, _i64, _vp], _int),
     "tern_embed_gather": ([_vp, _i64, _vp, _vp, _i64, _i64, _vp, _vp, _vp], _int),
+    "tern_b1_pack": ([_vp, _vp, _i64, _i64, _vp, _vp, _vp, _vp], _int),
+    "tern_b1_unpack": ([_vp, _i64, _i64, _vp, _vp], _int),
+    "tern_b1_gemv_step": ([ctypes.POINTER(tern_gemv_desc), _i32, _i64, _vp], _int),
 }
 for _name, (_args, _res) in _SIGS.items():
     _f = getattr(_L, _name)
@@ -270,10 +273,7 @@ def tern_embed_gather(ids: torch.Tensor, slots: torch.Tensor, scales: torch.Tens
     return out
 
 
-def tern_gemv_step(mats: Sequence, M: int = 1, stream=None):
-    """mats: sequence of (x [M,K] (or [K] for M = 1), slots [N,K/4],
-    scales [N,K/128], y [M,N] (or [N])) CUDA tensors, M in 1..4, every K a
-    multiple of 1024: one persistent launch."""
+def _step_descs(mats: Sequence):
     arr = (tern_gemv_desc * len(mats))()
     for i, (x, s, sc, y) in enumerate(mats):
         arr[i].x = _dev(x, "x", torch.float16)
@@ -282,7 +282,46 @@ def tern_gemv_step(mats: Sequence, M: int = 1, stream=None):
         arr[i].y = _dev(y, "y", torch.float16)
         arr[i].N = s.shape[0]
         arr[i].K = x.shape[-1]
-    _check(_L.tern_gemv_step(arr, len(mats), M, _stream(stream)), "tern_gemv_step")
+    return arr
+
+
+def tern_gemv_step(mats: Sequence, M: int = 1, stream=None):
+    """mats: sequence of (x [M,K] (or [K] for M = 1), slots [N,K/4],
+    scales [N,K/128], y [M,N] (or [N])) CUDA tensors, M in 1..4, every K a
+    multiple of 1024: one persistent launch."""
+    _check(_L.tern_gemv_step(_step_descs(mats), len(mats), M, _stream(stream)), "tern_gemv_step")
+
+
+def tern_b1_pack(codes: torch.Tensor, scales: torch.Tensor, bits_out: Optional[torch.Tensor] = None,
+                 scales_out: Optional[torch.Tensor] = None,
+                 invalid_count: Optional[torch.Tensor] = None, stream=None):
+    """1-bit variant: codes int8 [N,K] in {-1,+1}, scales fp16 [N,K/128] ->
+    (bits uint8 [N,K/8], scales fp16 [N,K/128])."""
+    N, K = codes.shape
+    if bits_out is None:
+        bits_out = torch.empty((N, K // 8), dtype=torch.uint8, device=codes.device)
+    if scales_out is None:
+        scales_out = torch.empty_like(scales)
+    ic = None if invalid_count is None else _dev(invalid_count, "invalid_count", torch.int32)
+    _check(_L.tern_b1_pack(_dev(codes, "codes", torch.int8), _dev(scales, "scales", torch.float16), N, K,
+                           _dev(bits_out, "bits_out", torch.uint8), _dev(scales_out, "scales_out", torch.float16),
+                           ic, _stream(stream)), "tern_b1_pack")
+    return bits_out, scales_out
+
+
+def tern_b1_unpack(bits: torch.Tensor, K: int, codes_out: Optional[torch.Tensor] = None, stream=None):
+    N = bits.shape[0]
+    if codes_out is None:
+        codes_out = torch.empty((N, K), dtype=torch.int8, device=bits.device)
+    _check(_L.tern_b1_unpack(_dev(bits, "bits", torch.uint8), N, K, _dev(codes_out, "codes_out", torch.int8),
+                             _stream(stream)), "tern_b1_unpack")
+    return codes_out
+
+
+def tern_b1_gemv_step(mats: Sequence, M: int = 1, stream=None):
+    """1-bit variant of tern_gemv_step: mats as there with bits uint8 [N,K/8]
+    in place of the slots."""
+    _check(_L.tern_b1_gemv_step(_step_descs(mats), len(mats), M, _stream(stream)), "tern_b1_gemv_step")
 
 
 def tern_gemv_grouped_workspace_bytes(mats: Sequence, M: int) -> int:

@@ -30,6 +30,7 @@ def test_header_declares_the_boundary():
     names = _declared()
     for n in ["tern_pack_g128", "tern_unpack_g128", "tern_gemv", "tern_gemm",
               "tern_gemv_grouped", "tern_gemv_step", "tern_embed_gather", "tern_workspace_bytes",
+              "tern_b1_pack", "tern_b1_unpack", "tern_b1_gemv_step",
               "tern_slots_bytes",
               "tern_scales_bytes", "tern_status_string", "tern_last_error", "tern_set_option",
               "tern_version"]:
@@ -134,12 +135,17 @@ def test_grouped_rejects(lib):
     assert lib.tern_gemv_grouped(arr, 2, 1, None, 0, None) == 2
 
 
-def test_step_rejects(lib):
-    """tern_gemv_step: argument errors return before any launch."""
+@pytest.mark.parametrize("fn", ["tern_gemv_step", "tern_b1_gemv_step"])
+def test_step_rejects(lib, fn):
+    """tern_gemv_step and its 1-bit twin: argument errors return before any launch."""
     from ternary_weight_only_b200 import tern
     arr = (tern.tern_gemv_desc * 3)()
     for d in arr:
         d.x, d.slots, d.scales, d.y, d.N, d.K = A, A, A, A, 16, 2048
+
+    class _L:
+        tern_gemv_step = getattr(lib, fn)
+    lib = _L
     assert lib.tern_gemv_step(None, 1, 1, None) == 1
     assert lib.tern_gemv_step(arr, 0, 1, None) == 1
     assert lib.tern_gemv_step(arr, tern.TERN_MAX_STEP + 1, 1, None) == 1
@@ -161,6 +167,20 @@ def test_step_rejects(lib):
     arr[0].x = A
     arr[1].K = 40960                     # 4 x 40960 x 2 bytes of x do not fit beside the rings
     assert lib.tern_gemv_step(arr, 3, 4, None) == 3
+
+
+def test_b1_pack_rejects(lib):
+    """tern_b1_pack / tern_b1_unpack: argument errors return before any launch."""
+    assert lib.tern_b1_pack(None, A, 4, 256, A, A, None, None) == 1
+    assert lib.tern_b1_pack(A, A, 4, 200, A, A, None, None) == 3
+    assert lib.tern_b1_pack(A, A, 0, 256, A, A, None, None) == 3
+    assert lib.tern_b1_pack(A + 8, A, 4, 256, A, A, None, None) == 2
+    assert lib.tern_b1_pack(A, A, 4, 256, A + 8, A, None, None) == 2
+    assert lib.tern_b1_pack(A, A + 1, 4, 256, A, A, None, None) == 2
+    assert lib.tern_b1_pack(A, A, 4, 256, A, A, A + 2, None) == 2
+    assert lib.tern_b1_unpack(None, 4, 256, A, None) == 1
+    assert lib.tern_b1_unpack(A, 4, 100, A, None) == 3
+    assert lib.tern_b1_unpack(A + 4, 4, 256, A, None) == 2
 
 
 def test_embed_rejects(lib):
