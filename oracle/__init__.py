@@ -88,6 +88,16 @@ class Oracle:
         L.orc_b1_weight.restype = dbl
         L.orc_b1_matmul.argtypes = [vp, i64, i64, vp, vp, i64, vp, vp, i32]
         L.orc_b1_matmul.restype = i32
+        L.orc_t5_row_bytes.argtypes = [i64]
+        L.orc_t5_row_bytes.restype = i64
+        L.orc_pack_t5.argtypes = [vp, vp, i64, i64, vp, vp, ctypes.POINTER(i64)]
+        L.orc_pack_t5.restype = i64
+        L.orc_unpack_t5.argtypes = [vp, i64, i64, vp]
+        L.orc_unpack_t5.restype = i64
+        L.orc_t5_weight.argtypes = [vp, vp, i64, i64, i64]
+        L.orc_t5_weight.restype = dbl
+        L.orc_t5_matmul.argtypes = [vp, i64, i64, vp, vp, i64, vp, vp, i32]
+        L.orc_t5_matmul.restype = i32
         self.L = L
         self.threads_used = 1
 
@@ -233,6 +243,45 @@ class Oracle:
         y = np.zeros((M, N), dtype=np.float64)
         b = np.zeros((M, N), dtype=np.float64)
         self.threads_used = self.L.orc_b1_matmul(_ptr(x_bits), M, K, _ptr(bits), _ptr(scales_bits), N,
+                                                 _ptr(y), _ptr(b), int(threads))
+        return y, b
+
+
+    # -- five trits per byte -------------------------------------------
+    def t5_row_bytes(self, K: int) -> int:
+        return self.L.orc_t5_row_bytes(K)
+
+    def t5_pack(self, codes: np.ndarray, scales_bits: np.ndarray):
+        """codes int8 [N,K]; scales uint16 [N,K/128] -> (bytes uint8 [N,R],
+        scales, invalid_count, first_bad_index), R = t5_row_bytes(K)."""
+        codes = np.ascontiguousarray(codes, dtype=np.int8)
+        scales_bits = np.ascontiguousarray(scales_bits, dtype=np.uint16)
+        N, K = codes.shape
+        out = np.zeros((N, max(self.t5_row_bytes(K), 0)), dtype=np.uint8)
+        sc = np.zeros((N, max(K // 128, 0)), dtype=np.uint16)
+        first = ctypes.c_int64(-1)
+        bad = self.L.orc_pack_t5(_ptr(codes), _ptr(scales_bits), N, K, _ptr(out), _ptr(sc), ctypes.byref(first))
+        if bad < 0:
+            raise ValueError("oracle t5 pack: K must be a positive multiple of 128")
+        return out, sc, int(bad), int(first.value)
+
+    def t5_unpack(self, packed: np.ndarray, K: int) -> np.ndarray:
+        packed = np.ascontiguousarray(packed, dtype=np.uint8)
+        N = packed.shape[0]
+        codes = np.zeros((N, K), dtype=np.int8)
+        if self.L.orc_unpack_t5(_ptr(packed), N, K, _ptr(codes)) < 0:
+            raise ValueError("oracle t5 unpack: K must be a positive multiple of 128")
+        return codes
+
+    def t5_matmul(self, x_bits: np.ndarray, packed: np.ndarray, scales_bits: np.ndarray, threads: int = 1):
+        x_bits = np.ascontiguousarray(x_bits, dtype=np.uint16)
+        packed = np.ascontiguousarray(packed, dtype=np.uint8)
+        scales_bits = np.ascontiguousarray(scales_bits, dtype=np.uint16)
+        M, K = x_bits.shape
+        N = packed.shape[0]
+        y = np.zeros((M, N), dtype=np.float64)
+        b = np.zeros((M, N), dtype=np.float64)
+        self.threads_used = self.L.orc_t5_matmul(_ptr(x_bits), M, K, _ptr(packed), _ptr(scales_bits), N,
                                                  _ptr(y), _ptr(b), int(threads))
         return y, b
 

@@ -400,3 +400,134 @@ int orc_b1_matmul(const uint16_t *x, int64_t M, int64_t K, const uint8_t *bits, 
     }
     return used;
 }
+
+/* ------------------------------------------------------------------------
+ * Dense ternary packing, five trits per byte.  The pages expect a "native
+ * ternary" kernel near the log2(3) + 16/128 ~= 1.71 bits/weight ideal instead
+ * of 2-bit slots, without a layout ("Ternary-Bonsai-27B" model summary,
+ * aitrends.kr, sections "TL;DR" and "Technical features"; "Ternary
+ * quantization: 27B in 7 GB", devnsb blog, section "Limits").  Reading
+ * taken: 3^5 = 243 <= 256, so a byte holds five codes as base-3 digits,
+ *   byte value v = sum_{i=0..4} c_i * 3^i,  c = t + 1 (0 -> -1, 1 -> 0, 2 -> +1),
+ * weight k of a row is digit k % 5 of byte k / 5 of that row (row-continuous,
+ * least significant digit first); digits past K are 0; each row is padded
+ * with zero bytes to a multiple of 16 bytes (R = ceil(K/5) rounded up to 16);
+ * scales fp16 [N][K/128] as for the 2-bit slots.  1.6 + 16/128 = 1.725
+ * bits/weight for K a multiple of 80.  Byte values 243..255 are invalid.
+ * ------------------------------------------------------------------------ */
+
+int64_t orc_t5_row_bytes(int64_t K)
+{
+    if (K <= 0) return 0;
+#if ORC_MUTANT == 12
+    return (K + 4) / 5; /* planted: no padding to 16 bytes */
+#else
+    return ((K + 4) / 5 + 15) / 16 * 16;
+#endif
+}
+
+/* power of three of digit position d (0..4) */
+static int orc_pow3(int d)
+{
+    int p = 1;
+    for (int i = 0; i < d; i++) p *= 3;
+    return p;
+}
+
+/* Digit position of weight k inside its byte. */
+static int orc_t5_pos(int64_t k)
+{
+#if ORC_MUTANT == 10
+    return 4 - (int)(k % 5); /* planted: most significant digit first */
+#else
+    return (int)(k % 5);
+#endif
+}
+
+/* Code c of weight (n,k), or -1 for an invalid byte (243..255). */
+static int orc_t5_code(const uint8_t *bytes, int64_t K, int64_t n, int64_t k)
+{
+    int v = bytes[n * orc_t5_row_bytes(K) + k / 5];
+    if (v >= 243) return -1;
+#if ORC_MUTANT == 11
+    return (v >> (2 * orc_t5_pos(k))) & 3; /* planted: base 4 instead of 3 */
+#else
+    return (v / orc_pow3(orc_t5_pos(k))) % 3;
+#endif
+}
+
+/* Pack codes [N][K] (int8 in {-1,0,+1}) and scales.  Any other code is
+ * stored as digit 1 (t = 0) and counted; returns the count (or -1 for a bad
+ * K); *first_bad receives the flat index of the first one (or -1). */
+int64_t orc_pack_t5(const int8_t *codes, const uint16_t *scales_in, int64_t N, int64_t K, uint8_t *bytes,
+                    uint16_t *scales_out, int64_t *first_bad)
+{
+    int64_t bad = 0, first = -1;
+    if (K <= 0 || N <= 0 || K % ORC_GROUP != 0) return -1;
+    const int64_t R = orc_t5_row_bytes(K);
+    for (int64_t i = 0; i < N * R; i++) bytes[i] = 0;
+    for (int64_t n = 0; n < N; n++) {
+        for (int64_t k = 0; k < K; k++) {
+            int t = codes[n * K + k];
+            int c = t + 1;
+            if (t < -1 || t > 1) {
+                c = 1;
+                if (first < 0) first = n * K + k;
+                bad++;
+            }
+            bytes[n * R + k / 5] = (uint8_t)(bytes[n * R + k / 5] + c * orc_pow3(orc_t5_pos(k)));
+        }
+    }
+    for (int64_t i = 0; i < N * (K / ORC_GROUP); i++) scales_out[i] = scales_in[i];
+    if (first_bad) *first_bad = first;
+    return bad;
+}
+
+/* codes_out [N][K]: t = c - 1, or the sentinel 2 for weights of an invalid byte. */
+int64_t orc_unpack_t5(const uint8_t *bytes, int64_t N, int64_t K, int8_t *codes_out)
+{
+    if (K <= 0 || N <= 0 || K % ORC_GROUP != 0) return -1;
+    for (int64_t n = 0; n < N; n++)
+        for (int64_t k = 0; k < K; k++) {
+            int c = orc_t5_code(bytes, K, n, k);
+            codes_out[n * K + k] = (int8_t)(c < 0 ? 2 : c - 1);
+        }
+    return 0;
+}
+
+/* w[n][k] = s[n][k/128] * t[n][k] in fp64 (exact); an invalid byte gives 0. */
+double orc_t5_weight(const uint8_t *bytes, const uint16_t *scales, int64_t K, int64_t n, int64_t k)
+{
+    int c = orc_t5_code(bytes, K, n, k);
+    if (c < 0) return 0.0;
+    return orc_half_to_double(scales[n * (K / ORC_GROUP) + k / ORC_GROUP]) * (double)(c - 1);
+}
+
+/* y[M][N] = x[M][K] * W^T with the five-per-byte weights, naive fp64 in k
+ * order, and the bound sum_k |x*w|.  Returns the thread count used. */
+int orc_t5_matmul(const uint16_t *x, int64_t M, int64_t K, const uint8_t *bytes, const uint16_t *scales,
+                  int64_t N, double *y, double *bound, int nthreads)
+{
+    int used = 1;
+#ifdef _OPENMP
+    if (nthreads < 1) nthreads = 1;
+#pragma omp parallel for num_threads(nthreads) schedule(static)
+#else
+    (void)nthreads;
+#endif
+    for (int64_t i = 0; i < M * N; i++) {
+#ifdef _OPENMP
+        if (i == 0) used = omp_get_num_threads();
+#endif
+        int64_t m = i / N, n = i % N;
+        double acc = 0.0, b = 0.0;
+        for (int64_t k = 0; k < K; k++) {
+            double p = orc_half_to_double(x[m * K + k]) * orc_t5_weight(bytes, scales, K, n, k);
+            acc += p;
+            b += fabs(p);
+        }
+        y[i] = acc;
+        bound[i] = b;
+    }
+    return used;
+}

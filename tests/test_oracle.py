@@ -387,10 +387,69 @@ def pin_b1_matmul(o):
     assert np.array_equal(y, np.repeat(X.sum(axis=1, keepdims=True), N, axis=1))
 
 
+def pin_t5_format(o):
+    """Five trits per byte: the row length closed form and the size the pages'
+    arithmetic gives (1.6 + 16/128 = 1.725 bits/weight, within 1 % of the
+    log2(3) + 16/128 ~= 1.71 ideal of the ThakiCloud blog, "How compression
+    works"; 19 % below 2-bit slots); every valid byte value decodes to its
+    base-3 digits (numpy's base_repr), the invalid ones to the sentinel; a
+    hand-worked byte; digits continue across bytes and groups; round trips;
+    invalid codes are counted."""
+    assert [o.t5_row_bytes(K) for K in (128, 5120, 6144, 17408)] == [32, 1024, 1232, 3488]
+    K, N = 5120, 6
+    bpw = (o.t5_row_bytes(K) * N * 8 + o.scales_bytes(N, K) * 8) / (K * N)
+    assert bpw == 1.725 and abs(bpw / (np.log2(3) + 16 / 128) - 1) < 0.01
+    assert round(1 - 1.725 / 2.125, 3) == 0.188
+    # all byte values as the first byte of a row of K = 128 (weights 0..4)
+    rows = np.zeros((256, 32), dtype=np.uint8)
+    rows[:, 0] = np.arange(256)
+    codes = o.t5_unpack(rows, 128)
+    for v in range(256):
+        if v < 243:
+            digits = [int(ch) for ch in np.base_repr(v, 3).zfill(5)[::-1]]
+            assert list(codes[v, :5]) == [d - 1 for d in digits], v
+        else:
+            assert list(codes[v, :5]) == [2] * 5, v
+        assert not (codes[v, 5:] + 1).any()  # zero bytes: code 0, t = -1
+    # hand-worked: t = +1, 0, -1, +1, 0 -> digits 2, 1, 0, 2, 1 -> 2 + 3 + 0 + 54 + 81 = 140;
+    # weights 5..9 = -1 -> byte 1 = 0; weight 127 (byte 25, digit 2) = +1 -> 2 * 9 = 18
+    row = np.full((1, 128), -1, dtype=np.int8)
+    row[0, :5] = [1, 0, -1, 1, 0]
+    row[0, 125:128] = [-1, -1, 1]
+    b, _, _, _ = o.t5_pack(row, np.zeros((1, 1), np.uint16))
+    assert b.shape == (1, 32) and b[0, 0] == 140 and b[0, 25] == 18
+    assert not b[0, 1:25].any() and not b[0, 26:].any()
+    rng = _rng(47)
+    for K in (128, 384, 1152):
+        codes = rng.integers(-1, 2, size=(5, K), dtype=np.int8)
+        b, _, bad, _ = o.t5_pack(codes, np.zeros((5, K // 128), np.uint16))
+        assert bad == 0 and np.array_equal(o.t5_unpack(b, K), codes)
+        assert int(b.max()) < 243
+    codes[3, 7] = 5
+    codes[4, 1000] = -2
+    b, _, bad, first = o.t5_pack(codes, np.zeros((5, 9), np.uint16))
+    assert bad == 2 and first == 3 * 1152 + 7 and o.t5_unpack(b, 1152)[3, 7] == 0
+
+
+def pin_t5_matmul(o):
+    """The five-per-byte product equals numpy float64 x @ (s*t).T."""
+    rng = _rng(53)
+    M, K, N = 3, 640, 21
+    codes = rng.integers(-1, 2, size=(N, K), dtype=np.int8)
+    scales = _f16bits(rng.uniform(-0.05, 0.05, size=(N, K // 128)))
+    x = _f16bits(rng.standard_normal((M, K)))
+    b, sc, _, _ = o.t5_pack(codes, scales)
+    y, bound = o.t5_matmul(x, b, sc)
+    W = _np_dequant(codes, scales)
+    X = x.view(np.float16).astype(np.float64)
+    assert np.allclose(y, X @ W.T, rtol=1e-12, atol=1e-12)
+    assert np.allclose(bound, np.abs(X) @ np.abs(W).T, rtol=1e-12, atol=1e-12)
+
+
 PINS = [pin_half_decode, pin_golden_bytes, pin_golden_matmul, pin_exhaustive_bytes,
         pin_roundtrip_random, pin_invalid_codes, pin_byte_count, pin_numpy_crosscheck,
         pin_row_sums, pin_exact_cases, pin_brute_force, pin_sampled_paths, pin_embed, pin_b1_format,
-        pin_b1_matmul]
+        pin_b1_matmul, pin_t5_format, pin_t5_matmul]
 
 
 @pytest.mark.parametrize("pin", PINS, ids=lambda p: p.__name__)
@@ -412,11 +471,12 @@ def test_rejects_bad_k(orc):
         orc.pack(np.zeros((1, 100), dtype=np.int8), np.zeros((1, 0), dtype=np.uint16))
 
 
-@pytest.mark.parametrize("mutant", [1, 2, 3, 4, 5, 6, 7, 8, 9])
+@pytest.mark.parametrize("mutant", [1, 2, 3, 4, 5, 6, 7, 8, 9, 10, 11, 12])
 def test_planted_mistakes_are_caught(mutant):
     """Each planted mistake in the oracle (bit order, code sign, group size,
     transposed operand, dropped term, subnormal decode; in the 1-bit variant
-    bit order, bit meaning, scale group) fails at least one pin."""
+    bit order, bit meaning, scale group; in the five-per-byte packing digit
+    order, base, row padding) fails at least one pin."""
     bad = oracle.Oracle(oracle.build(mutant))
     failed = []
     for pin in PINS:
