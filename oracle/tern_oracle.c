@@ -409,20 +409,32 @@ int orc_b1_matmul(const uint16_t *x, int64_t M, int64_t K, const uint8_t *bits, 
  * quantization: 27B in 7 GB", devnsb blog, section "Limits").  Reading
  * taken: 3^5 = 243 <= 256, so a byte holds five codes as base-3 digits,
  *   byte value v = sum_{i=0..4} c_i * 3^i,  c = t + 1 (0 -> -1, 1 -> 0, 2 -> +1),
- * weight k of a row is digit k % 5 of byte k / 5 of that row (row-continuous,
- * least significant digit first); digits past K are 0; each row is padded
- * with zero bytes to a multiple of 16 bytes (R = ceil(K/5) rounded up to 16);
- * scales fp16 [N][K/128] as for the 2-bit slots.  1.6 + 16/128 = 1.725
- * bits/weight for K a multiple of 80.  Byte values 243..255 are invalid.
+ * least significant digit first, inside each 128-weight scale group: weight j
+ * of group g is digit j % 5 of byte 26 g + j / 5 of the row (25 full bytes
+ * and one byte holding weights 125..127, whose digits 3 and 4 are 0); each
+ * row is padded with zero bytes to a multiple of 16 bytes (R = 26 K / 128
+ * rounded up to 16); scales fp16 [N][K/128] as for the 2-bit slots.
+ * 26 * 8 / 128 + 16/128 = 1.75 bits/weight.  Byte values 243..255 are
+ * invalid.
  * ------------------------------------------------------------------------ */
 
 int64_t orc_t5_row_bytes(int64_t K)
 {
     if (K <= 0) return 0;
 #if ORC_MUTANT == 12
-    return (K + 4) / 5; /* planted: no padding to 16 bytes */
+    return 26 * (K / ORC_GROUP); /* planted: no padding to 16 bytes */
 #else
-    return ((K + 4) / 5 + 15) / 16 * 16;
+    return (26 * (K / ORC_GROUP) + 15) / 16 * 16;
+#endif
+}
+
+/* Byte of weight k inside its row. */
+static int64_t orc_t5_byte(int64_t k)
+{
+#if ORC_MUTANT == 13
+    return k / 5; /* planted: digits continue across groups */
+#else
+    return 26 * (k / ORC_GROUP) + (k % ORC_GROUP) / 5;
 #endif
 }
 
@@ -437,17 +449,20 @@ static int orc_pow3(int d)
 /* Digit position of weight k inside its byte. */
 static int orc_t5_pos(int64_t k)
 {
+    const int j = (int)(k % ORC_GROUP);
 #if ORC_MUTANT == 10
-    return 4 - (int)(k % 5); /* planted: most significant digit first */
-#else
+    return 4 - j % 5; /* planted: most significant digit first */
+#elif ORC_MUTANT == 13
     return (int)(k % 5);
+#else
+    return j % 5;
 #endif
 }
 
 /* Code c of weight (n,k), or -1 for an invalid byte (243..255). */
 static int orc_t5_code(const uint8_t *bytes, int64_t K, int64_t n, int64_t k)
 {
-    int v = bytes[n * orc_t5_row_bytes(K) + k / 5];
+    int v = bytes[n * orc_t5_row_bytes(K) + orc_t5_byte(k)];
     if (v >= 243) return -1;
 #if ORC_MUTANT == 11
     return (v >> (2 * orc_t5_pos(k))) & 3; /* planted: base 4 instead of 3 */
@@ -475,7 +490,7 @@ int64_t orc_pack_t5(const int8_t *codes, const uint16_t *scales_in, int64_t N, i
                 if (first < 0) first = n * K + k;
                 bad++;
             }
-            bytes[n * R + k / 5] = (uint8_t)(bytes[n * R + k / 5] + c * orc_pow3(orc_t5_pos(k)));
+            bytes[n * R + orc_t5_byte(k)] = (uint8_t)(bytes[n * R + orc_t5_byte(k)] + c * orc_pow3(orc_t5_pos(k)));
         }
     }
     for (int64_t i = 0; i < N * (K / ORC_GROUP); i++) scales_out[i] = scales_in[i];

@@ -388,18 +388,18 @@ def pin_b1_matmul(o):
 
 
 def pin_t5_format(o):
-    """Five trits per byte: the row length closed form and the size the pages'
-    arithmetic gives (1.6 + 16/128 = 1.725 bits/weight, within 1 % of the
-    log2(3) + 16/128 ~= 1.71 ideal of the ThakiCloud blog, "How compression
-    works"; 19 % below 2-bit slots); every valid byte value decodes to its
-    base-3 digits (numpy's base_repr), the invalid ones to the sentinel; a
-    hand-worked byte; digits continue across bytes and groups; round trips;
-    invalid codes are counted."""
-    assert [o.t5_row_bytes(K) for K in (128, 5120, 6144, 17408)] == [32, 1024, 1232, 3488]
+    """Five trits per byte: the row length closed form (26 bytes per group of
+    128) and the size against the pages' arithmetic (1.625 + 16/128 = 1.75
+    bits/weight, within 2.5 % of the log2(3) + 16/128 ~= 1.71 ideal of the
+    ThakiCloud blog, "How compression works"; 17.6 % below 2-bit slots);
+    every valid byte value decodes to its base-3 digits (numpy's base_repr),
+    the invalid ones to the sentinel; a hand-worked byte; each group starts a
+    new byte; round trips; invalid codes are counted."""
+    assert [o.t5_row_bytes(K) for K in (128, 5120, 6144, 17408)] == [32, 1040, 1248, 3536]
     K, N = 5120, 6
     bpw = (o.t5_row_bytes(K) * N * 8 + o.scales_bytes(N, K) * 8) / (K * N)
-    assert bpw == 1.725 and abs(bpw / (np.log2(3) + 16 / 128) - 1) < 0.01
-    assert round(1 - 1.725 / 2.125, 3) == 0.188
+    assert bpw == 1.75 and abs(bpw / (np.log2(3) + 16 / 128) - 1) < 0.025
+    assert round(1 - 1.75 / 2.125, 3) == 0.176
     # all byte values as the first byte of a row of K = 128 (weights 0..4)
     rows = np.zeros((256, 32), dtype=np.uint8)
     rows[:, 0] = np.arange(256)
@@ -419,6 +419,13 @@ def pin_t5_format(o):
     b, _, _, _ = o.t5_pack(row, np.zeros((1, 1), np.uint16))
     assert b.shape == (1, 32) and b[0, 0] == 140 and b[0, 25] == 18
     assert not b[0, 1:25].any() and not b[0, 26:].any()
+    # the second group starts at byte 26: weight 128 = +1, weight 133 = 0 -> bytes 26, 27 = 2, 1
+    row = np.full((1, 256), -1, dtype=np.int8)
+    row[0, 128] = 1
+    row[0, 133] = 0
+    b, _, _, _ = o.t5_pack(row, np.zeros((1, 2), np.uint16))
+    assert b.shape == (1, 64) and b[0, 26] == 2 and b[0, 27] == 1
+    assert not b[0, :26].any() and not b[0, 28:].any()
     rng = _rng(47)
     for K in (128, 384, 1152):
         codes = rng.integers(-1, 2, size=(5, K), dtype=np.int8)
@@ -471,12 +478,13 @@ def test_rejects_bad_k(orc):
         orc.pack(np.zeros((1, 100), dtype=np.int8), np.zeros((1, 0), dtype=np.uint16))
 
 
-@pytest.mark.parametrize("mutant", [1, 2, 3, 4, 5, 6, 7, 8, 9, 10, 11, 12])
+@pytest.mark.parametrize("mutant", [1, 2, 3, 4, 5, 6, 7, 8, 9, 10, 11, 12, 13])
 def test_planted_mistakes_are_caught(mutant):
     """Each planted mistake in the oracle (bit order, code sign, group size,
     transposed operand, dropped term, subnormal decode; in the 1-bit variant
     bit order, bit meaning, scale group; in the five-per-byte packing digit
-    order, base, row padding) fails at least one pin."""
+    order, base, row padding, digits running across groups) fails at least
+    one pin."""
     bad = oracle.Oracle(oracle.build(mutant))
     failed = []
     for pin in PINS:
