@@ -391,6 +391,51 @@ def b1_rows(T, model, peak_gbs, sm_mhz=None):
     return out
 
 
+def t5_rows(T, model, peak_gbs):
+    """Five trits per byte (26 bytes per 128-weight group, 1.75 bits/weight)
+    over the same shapes and codes distribution as the decode step (P(0) =
+    0.4): every projection of the 64 layers plus the head in one
+    tern_t5_gemv_step call, at M = 1 and M = 2 (M = 4 does not fit beside
+    the decode table at K = 17408).  weights_per_s compares the decode rate
+    with the 2-bit slots' (decode_step in the main line)."""
+    out = {}
+    s = torch.cuda.Stream()
+    mats = []
+    for l in range(model.n_layers):
+        g = synth.gen(7000 + l, "cuda")
+        for i, (x, slots, sc, y) in enumerate(model.groups[l]):
+            _, K, N = synth.LAYER_PROJ[i]
+            codes = synth.codes_sparse(N, K, g, device="cuda")
+            packed, psc = T.tern_t5_pack(codes, synth.scales_uniform(N, K, g, device="cuda"))
+            del codes
+            mats.append((x, packed, psc, y, K, N))
+    g = synth.gen(7000 + synth.N_LAYERS, "cuda")
+    _, K, N = synth.HEAD
+    codes = synth.codes_sparse(N, K, g, device="cuda")
+    packed, psc = T.tern_t5_pack(codes, synth.scales_uniform(N, K, g, device="cuda"))
+    del codes
+    mats.append((model.head_io[0], packed, psc, model.head_io[1], K, N))
+    torch.cuda.synchronize()
+    nweights = sum(K * N for *_, K, N in mats)
+    xbuf = torch.randn(2 * 17408, device="cuda").half()
+    for M in (1, 2):
+        if M == 1:
+            run = [(x, b, sc, y) for x, b, sc, y, _, _ in mats]
+        else:
+            run = [(xbuf[:M * K].view(M, K), b, sc, torch.empty(M, N, dtype=torch.float16, device="cuda"))
+                   for _, b, sc, _, K, N in mats]
+        b = sum(N * (26 * K // GROUP) + 2 * N * (K // GROUP) + 2 * M * K + 2 * M * N for *_, K, N in mats)
+        ms = graph_time([lambda run=run, M=M: T.tern_t5_gemv_step(run, M)], s, reps=5)
+        out[f"t5_step_M{M}"] = {"ms": round(ms, 4), "GBps": round(b / ms / 1e6, 1),
+                                "frac": round(b / ms / 1e6 / peak_gbs, 4),
+                                "weights_per_s": float(f"{nweights / (ms * 1e-3):.4g}"),
+                                "products": len(run)}
+        del run
+    del mats
+    torch.cuda.empty_cache()
+    return out
+
+
 def pack_rows(T, peak_gbs):
     """tern_pack_g128 on a gate-sized matrix (17408 x 5120): int8 codes and
     fp16 scales in, 2-bit slots and scales out; GB/s of those bytes."""
@@ -709,6 +754,7 @@ def run_tern(args):
         rows = proj_rows(T, model, peak_gbs, l2)
         rows.update(pack_rows(T, peak_gbs))
         rows.update(b1_rows(T, model, peak_gbs, (clocks.summary() or {}).get("sm_mhz")))
+        rows.update(t5_rows(T, model, peak_gbs))
         rows.update(embed_rows(T, model, peak_gbs))
         rows.update(prefill_rows(T, peak_tf))
 

@@ -304,6 +304,58 @@ tern_status tern_b1_unpack(const uint8_t *bits, int64_t N, int64_t K, int8_t *co
 tern_status tern_b1_gemv_step(const tern_gemv_desc *descs, int32_t count, int64_t M, void *stream);
 
 /*
+ * Five trits per byte: a denser ternary storage, the "native ternary" packing
+ * the pages expect closer to the log2(3) + 16/128 ~= 1.71 bits/weight ideal
+ * than 2-bit slots ("Ternary-Bonsai-27B" model summary, aitrends.kr, sections
+ * "TL;DR" and "Technical features"; "Ternary quantization: 27B in 7 GB",
+ * devnsb blog, section "Limits").  The pages fix no layout; this library's,
+ * for W with N rows and K columns (K a multiple of 128):
+ *
+ *   bytes   uint8 [N][R], R = 26 K / 128 rounded up to a multiple of 16: in
+ *           each 128-weight group g of a row, weight j (0..127) is base-3
+ *           digit j % 5 (least significant first) of byte 26 g + j / 5, the
+ *           digit being the code c = t + 1 (0 -> -1, 1 -> 0, 2 -> +1); byte
+ *           25 of a group holds weights 125..127 (digits 3, 4 are 0); the
+ *           row padding is zero.  Byte values 243..255 are invalid.
+ *   scales  fp16 [N][K/128] as for the 2-bit slots.
+ *
+ * 26 * 8 / 128 + 16 / 128 = 1.75 bits per weight (2-bit slots: 2.125).
+ *
+ * tern_t5_bytes -- N * R, or 0 for invalid arguments.
+ */
+size_t tern_t5_bytes(int64_t N, int64_t K);
+
+/*
+ * tern_t5_pack -- build the five-per-byte layout.
+ *   codes      int8 [N][K] in {-1, 0, +1}                        (device, read)
+ *   scales_in  fp16 [N][K/128] raw 16-bit patterns               (device, read)
+ *   bytes_out  uint8 [N][R], R as above (tern_t5_bytes / N)      (device, written)
+ *   scales_out fp16 [N][K/128], a bit-exact copy (may equal scales_in)
+ *   invalid_count  nullable device int32, incremented by the number of codes
+ *              outside {-1, 0, +1}; such a code is stored as t = 0.
+ * Alignment: codes and bytes_out 16 bytes; scales 2 bytes; invalid_count 4.
+ */
+tern_status tern_t5_pack(const int8_t *codes, const uint16_t *scales_in, int64_t N, int64_t K, uint8_t *bytes_out,
+                         uint16_t *scales_out, int32_t *invalid_count, void *stream);
+
+/*
+ * tern_t5_unpack -- inverse: codes_out int8 [N][K] gets t = c - 1, or the
+ * sentinel 2 for the five weights of an invalid byte.  16-byte alignment.
+ */
+tern_status tern_t5_unpack(const uint8_t *bytes, int64_t N, int64_t K, int8_t *codes_out, void *stream);
+
+/*
+ * tern_t5_gemv_step -- tern_gemv_step for five-per-byte matrices: each
+ * descriptor's `slots` field points to the bytes (uint8 [N][R]); shapes
+ * (K a multiple of 1024, M in 1..4), arithmetic, argument checks and error
+ * reporting as for tern_gemv_step.  The kernel keeps a 32 KiB decode table
+ * in shared memory, so the largest M x K it accepts is smaller than for
+ * tern_gemv_step (TERN_ERR_SHAPE beyond it; M = 4 at K = 17408 does not fit).
+ * An invalid byte contributes an unspecified finite value for its weights.
+ */
+tern_status tern_t5_gemv_step(const tern_gemv_desc *descs, int32_t count, int64_t M, void *stream);
+
+/*
  * tern_sync_status -- wait for `stream`, then report whether any kernel of
  * this library on the current device gave up a bounded on-device wait since
  * the previous call (TERN_ERR_TIMEOUT), clearing that record.  No kernel of

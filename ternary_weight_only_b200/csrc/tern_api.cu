@@ -383,6 +383,40 @@ tern_status tern_b1_gemv_step(const tern_gemv_desc *descs, int32_t count, int64_
     return gemv_step_api(descs, count, M, 1, "tern_b1_gemv_step", stream);
 }
 
+tern_status tern_t5_gemv_step(const tern_gemv_desc *descs, int32_t count, int64_t M, void *stream) {
+    return gemv_step_api(descs, count, M, 2, "tern_t5_gemv_step", stream);
+}
+
+size_t tern_t5_bytes(int64_t N, int64_t K) {
+    if (N < 1 || K < kGroup || K % kGroup != 0) return 0;
+    return static_cast<size_t>(N) * static_cast<size_t>(t5_row_bytes(K));
+}
+
+tern_status tern_t5_pack(const int8_t *codes, const uint16_t *scales_in, int64_t N, int64_t K, uint8_t *bytes_out,
+                         uint16_t *scales_out, int32_t *invalid_count, void *stream) {
+    clear_error();
+    tern_status st = check_nk(N, K);
+    if (st != TERN_OK) return st;
+    if (!codes || !scales_in || !bytes_out || !scales_out) return fail(TERN_ERR_INVALID_ARG, "null buffer pointer");
+    if (!aligned16(codes)) return fail(TERN_ERR_ALIGN, "codes is not 16-byte aligned");
+    if (!aligned16(bytes_out)) return fail(TERN_ERR_ALIGN, "bytes_out is not 16-byte aligned");
+    if ((reinterpret_cast<uintptr_t>(scales_in) | reinterpret_cast<uintptr_t>(scales_out)) & 1u)
+        return fail(TERN_ERR_ALIGN, "scales are not 2-byte aligned");
+    if ((reinterpret_cast<uintptr_t>(invalid_count) & 3u) != 0)
+        return fail(TERN_ERR_ALIGN, "invalid_count is not 4-byte aligned");
+    return launch_pack_t5(codes, scales_in, N, K, bytes_out, scales_out, invalid_count,
+                          static_cast<cudaStream_t>(stream));
+}
+
+tern_status tern_t5_unpack(const uint8_t *bytes, int64_t N, int64_t K, int8_t *codes_out, void *stream) {
+    clear_error();
+    tern_status st = check_nk(N, K);
+    if (st != TERN_OK) return st;
+    if (!bytes || !codes_out) return fail(TERN_ERR_INVALID_ARG, "null buffer pointer");
+    if (!aligned16(bytes) || !aligned16(codes_out)) return fail(TERN_ERR_ALIGN, "bytes and codes_out must be 16-byte aligned");
+    return launch_unpack_t5(bytes, N, K, codes_out, static_cast<cudaStream_t>(stream));
+}
+
 tern_status tern_b1_pack(const int8_t *codes, const uint16_t *scales_in, int64_t N, int64_t K, uint8_t *bits_out,
                          uint16_t *scales_out, int32_t *invalid_count, void *stream) {
     clear_error();

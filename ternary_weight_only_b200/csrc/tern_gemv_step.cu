@@ -34,6 +34,16 @@
 // works"), template parameter F = 1: a stage's weights are one 128-byte-
 // swizzled box of 16 rows x 128 bytes (1024 k), the unpack is b1_slice, and
 // a group's sum is 2 D(bits) - D(all ones).
+//
+// F = 2 serves the five-per-byte packing (base-3 digits, 26 bytes per
+// 128-weight group; tern.h): a stage is one box of 16 rows x 208 bytes (1024
+// k, no swizzle), and every lane turns its bytes into the 2-bit codes of the
+// ternary slot words in registers -- an 8-byte window per group and row (the
+// lane's 32 weights start at byte 0, 6, 12 or 19 of the group, digit 0, 2, 4
+// or 1), each byte through a 256-entry table of its five codes (replicated
+// per lane so that the 32 lookups of a warp hit 32 distinct banks), the eight
+// 10-bit results joined and shifted by the digit offset -- after which the
+// ternary arithmetic runs unchanged.
 #include <algorithm>
 #include <cstring>
 
@@ -53,8 +63,13 @@ constexpr int kRows = 16;                 // tile rows (mma M)
 constexpr int kSG = 8;                    // scale groups per unit (1024 k)
 constexpr int kBox = 128;                 // bytes per row of one slot box (512 k)
 constexpr int kScaleStage = kRows * kSG * 2;           // 256
-// weight bytes of one stage (16 rows x 1024 k): 2-bit slots (two boxes) or bits
-__host__ __device__ constexpr int slot_stage(int f) { return f ? kRows * kBox : kRows * kBox * 2; }
+constexpr int kT5Row = 208;              // five-per-byte bytes of one row of a unit (8 x 26)
+// weight bytes of one stage (16 rows x 1024 k): 2-bit slots (two boxes), bits, or base-3 bytes
+__host__ __device__ constexpr int slot_stage(int f) {
+    return f == 0 ? kRows * kBox * 2 : (f == 1 ? kRows * kBox : kRows * kT5Row);
+}
+// the five-per-byte code table: 256 entries x 32 lanes x 4 bytes
+__host__ __device__ constexpr int lut_bytes(int f) { return f == 2 ? 256 * 32 * 4 : 0; }
 __host__ __device__ constexpr int stage_bytes(int f) { return slot_stage(f) + kScaleStage; }
 constexpr int kMaxNS = 4;
 constexpr int kMaxCtas = 160;
@@ -71,7 +86,8 @@ struct SDesc {
 
 struct alignas(64) SMaps {
     CUtensorMap smap;   // slots as uint8 [K/512][N][128], box 128 B x 16 rows x 2, 128-byte swizzle
-                        // (1-bit: bits as uint8 [N][K/8], box 128 B x 16 rows, 128-byte swizzle)
+                        // (1-bit: bits as uint8 [N][K/8], box 128 B x 16 rows, 128-byte swizzle;
+                        //  five-per-byte: uint8 [N][R], box 208 B x 16 rows, no swizzle)
     CUtensorMap cmap;   // scales fp16 [N][K/128], box 8 x 16, no swizzle
 };
 
@@ -94,11 +110,48 @@ __host__ __device__ constexpr int rtile_off() { return rec_off() + kW * 2 * 16 *
 __host__ __device__ constexpr int wmax_off() { return rtile_off() + kW * 2 * 4; }     // [kW] uint
 __host__ __device__ constexpr int d1_off() { return wmax_off() + kW * 4; }            // [kmax / 128] float
 // d1 holds one float per (set, column): kmax / 128 * MT floats, MT <= 4
-__host__ __device__ constexpr int xs_off(int kmax) { return d1_off() + (kmax / 128) * 16 + 64; }
+__host__ __device__ constexpr int lut_off(int kmax) { return d1_off() + (kmax / 128) * 16 + 64; }
+__host__ __device__ constexpr int xs_off(int kmax, int f) { return lut_off(kmax) + lut_bytes(f); }
 // staged x: MT token rows (M real, the rest zero)
-__host__ __device__ constexpr int ring_off(int kmax, int mt) { return (xs_off(kmax) + kmax * 2 * mt + 1023) & ~1023; }
+__host__ __device__ constexpr int ring_off(int kmax, int mt, int f) {
+    return (xs_off(kmax, f) + kmax * 2 * mt + 1023) & ~1023;
+}
 size_t smem_bytes(int kmax, int mt, int ns, int f) {
-    return 1024 + static_cast<size_t>(ring_off(kmax, mt)) + static_cast<size_t>(kW) * ns * stage_bytes(f);
+    return 1024 + static_cast<size_t>(ring_off(kmax, mt, f)) + static_cast<size_t>(kW) * ns * stage_bytes(f);
+}
+
+// The 2-bit codes (c = digit, code i at bits 2i) of the five base-3 digits of
+// byte v; an invalid byte (243..255) gives code 1 (t = 0) five times.
+__device__ __forceinline__ uint32_t t5_codes(uint32_t v) {
+    if (v >= 243u) return 0x155u;
+    uint32_t out = 0;
+#pragma unroll
+    for (int i = 0; i < 5; i++) {
+        out |= (v % 3u) << (2 * i);
+        v /= 3u;
+    }
+    return out;
+}
+
+// Slot words 2q, 2q+1 (codes of the lane's 32 weights) from its 8-byte
+// window at p (4-byte aligned, the window starting sh bits in), the table
+// entries of this lane at lutl (entry v at lutl[32 v]) and the digit offset
+// times two, dd.
+__device__ __forceinline__ void t5_words(const uint8_t *p, uint32_t sh, const uint32_t *lutl, uint32_t dd,
+                                         uint32_t &lo, uint32_t &hi) {
+    const uint32_t w0 = *reinterpret_cast<const uint32_t *>(p);
+    const uint32_t w1 = *reinterpret_cast<const uint32_t *>(p + 4);
+    const uint32_t w2 = *reinterpret_cast<const uint32_t *>(p + 8);
+    const uint32_t b03 = __funnelshift_r(w0, w1, sh), b47 = __funnelshift_r(w1, w2, sh);
+    uint32_t l[8];
+#pragma unroll
+    for (int i = 0; i < 8; i++) l[i] = lutl[32u * __byte_perm(i < 4 ? b03 : b47, 0u, 0x4440u + (i & 3))];
+    // the 80-bit string of the eight 10-bit code groups, as three words
+    const uint32_t s0 = l[0] + (l[1] << 10) + (l[2] << 20) + (l[3] << 30);
+    const uint32_t s1 = (l[3] >> 2) + (l[4] << 8) + (l[5] << 18) + (l[6] << 28);
+    const uint32_t s2 = (l[6] >> 4) + (l[7] << 6);
+    lo = __funnelshift_r(s0, s1, dd);
+    hi = __funnelshift_r(s1, s2, dd);
 }
 
 __device__ __forceinline__ bool step_wait(uint64_t *bar, uint32_t parity, unsigned long long deadline) {
@@ -168,7 +221,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_step_kernel(const __grid_con
     constexpr int GPB = 8 / MT;  // groups per set
     constexpr int kSlotStage = slot_stage(F);
     constexpr int kStageBytes = stage_bytes(F);
-    constexpr int kWords = F ? 2 : 4;  // weight words of a group a lane holds
+    constexpr int kWords = F == 1 ? 2 : 4;  // weight words of a group a lane holds
     extern __shared__ uint8_t smem_raw[];
     uint8_t *base = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     uint64_t *full = reinterpret_cast<uint64_t *>(base + bar_off());  // [kW][kMaxNS]
@@ -176,7 +229,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_step_kernel(const __grid_con
     int *rec_tile = reinterpret_cast<int *>(base + rtile_off());
     unsigned int *wmax = reinterpret_cast<unsigned int *>(base + wmax_off());
     float *d1 = reinterpret_cast<float *>(base + d1_off());
-    __half *xs = reinterpret_cast<__half *>(base + xs_off(p.kmax));
+    __half *xs = reinterpret_cast<__half *>(base + xs_off(p.kmax, F));
+    uint32_t *lut = reinterpret_cast<uint32_t *>(base + lut_off(p.kmax));
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int g = lane >> 2, q = lane & 3;
@@ -186,14 +240,26 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_step_kernel(const __grid_con
     // 128-byte-swizzled position of the lane's words of group G in `row`:
     // words 2q, 2q+1 of group G % 4 of box G / 4 (ternary), or word q of
     // group G (1-bit: 16 bytes per group row)
-    uint32_t off[F ? 8 : 4];
+    uint32_t off[F == 1 ? 8 : 4];
     if constexpr (F == 0) {
 #pragma unroll
         for (int j = 0; j < 4; j++) off[j] = row * kBox + (((2 * j + (q >> 1)) ^ (row & 7)) << 4) + (q & 1) * 8;
-    } else {
+    } else if constexpr (F == 1) {
 #pragma unroll
         for (int G8 = 0; G8 < 8; G8++) off[G8] = row * kBox + ((G8 ^ (row & 7)) << 4) + 4 * q;
+    } else {
+        // five-per-byte: the lane's window in group G of `row` starts at byte
+        // 26 G + sq (sq = 0, 6, 12, 19) at digit 0, 2, 4, 1.  off[0] / off[1]:
+        // 4-byte-aligned window offsets for even / odd G (add 52 (G / 2));
+        // off[2] / off[3]: the matching shifts in bits.
+        const int sq = q == 0 ? 0 : (q == 1 ? 6 : (q == 2 ? 12 : 19));
+        off[0] = row * kT5Row + (sq & ~3);
+        off[1] = row * kT5Row + 26 + sq - ((sq + 2) & 3);
+        off[2] = (sq & 3) * 8;
+        off[3] = ((sq + 2) & 3) * 8;
     }
+    const uint32_t t5dd = 2u * (q == 0 ? 0u : (q == 1 ? 2u : (q == 2 ? 4u : 1u)));
+    const uint32_t *lutl = lut + lane;
     const int T0 = p.cta_tile[blockIdx.x], T1 = p.cta_tile[blockIdx.x + 1];
     // first matrix with a tile at or after T0
     int i0 = 0;
@@ -208,7 +274,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_step_kernel(const __grid_con
     // The ring takes what this CTA's largest staged x leaves (2..4 stages).
     int kcta = 1024;
     for (int i = i0; T0 < T1 && i < p.count && p.d[i].tile0 < T1; i++) kcta = max(kcta, p.d[i].K);
-    const uint32_t roff = (static_cast<uint32_t>(xs_off(p.kmax)) + 2u * MT * kcta + 1023u) & ~1023u;
+    const uint32_t roff = (static_cast<uint32_t>(xs_off(p.kmax, F)) + 2u * MT * kcta + 1023u) & ~1023u;
     const int ns = min(kMaxNS, static_cast<int>((p.smem_usable - roff) / (kW * kStageBytes)));
     const int M = p.M;
     uint8_t *ring = base + roff;
@@ -216,6 +282,9 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_step_kernel(const __grid_con
     if (threadIdx.x == 0) {
         for (int i = 0; i < kW * kMaxNS; i++) mbar_init(&full[i], 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if constexpr (F == 2) {
+        for (int i = threadIdx.x; i < 256 * 32; i += kThreads) lut[i] = t5_codes(static_cast<uint32_t>(i >> 5));
     }
     __syncthreads();
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
@@ -239,8 +308,10 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_step_kernel(const __grid_con
             mbar_expect_tx(&my_full[st], kStageBytes);
             if constexpr (F == 0)
                 tma_load_3d(stage, &p.m[ic.i].smap, 0, ic.tile * kRows, ic.kb * 2, &my_full[st]);
-            else
+            else if constexpr (F == 1)
                 tma_load_2d(stage, &p.m[ic.i].smap, ic.kb * kBox, ic.tile * kRows, &my_full[st]);
+            else
+                tma_load_2d(stage, &p.m[ic.i].smap, ic.kb * kT5Row, ic.tile * kRows, &my_full[st]);
             tma_load_2d(my_scl + st * kScaleStage, &p.m[ic.i].cmap, ic.kb * kSG, ic.tile * kRows, &my_full[st]);
         }
         cursor_next(ic, p, T0, T1, warp);
@@ -280,7 +351,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_step_kernel(const __grid_con
         for (int w = 0; w < kW; w++) mx = max(mx, wmax[w]);
         const int ex = max(static_cast<int>(mx >> 10), 1) - 15;
         // the largest staged factor is 2^E: x * 2^E stays finite
-        const int E = min(F ? 7 : 8, 15 - ex);
+        const int E = min(F == 1 ? 7 : 8, 15 - ex);
         if constexpr (F == 1) {
             // factor of bit position p (0..15 in a half) is 2^(E - (p & 7));
             // 8 consecutive x are positions p0 .. p0 + 7, p0 = 0 or 8
@@ -340,7 +411,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_step_kernel(const __grid_con
         // one all-ones chain per set: d1[set * 8 + column]
         for (int sl = warp; sl < B * MT; sl += kW) {
             float c[4];
-            if constexpr (F == 0)
+            if constexpr (F != 1)
                 group_mma<8>(c, kOnes, kOnes, kOnes, kOnes, xlane + sl * 1024);
             else
                 b1_ones_chain(c, xlane + sl * 1024);
@@ -388,7 +459,12 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_step_kernel(const __grid_con
                 uint32_t wd[kSG][kWords];
 #pragma unroll
                 for (int G8 = 0; G8 < kSG; G8++) {
-                    if constexpr (F == 0) {
+                    if constexpr (F == 2) {
+                        const uint8_t *pw = stage + off[G8 & 1] + 52 * (G8 >> 1);
+                        const uint32_t sh = off[2 + (G8 & 1)];
+                        t5_words(pw, sh, lutl, t5dd, wd[G8][0], wd[G8][2]);
+                        t5_words(pw + 8 * kT5Row, sh, lutl, t5dd, wd[G8][1], wd[G8][3]);
+                    } else if constexpr (F == 0) {
                         const uint8_t *bx = stage + (G8 >> 2) * (kRows * kBox);
                         const uint2 a = *reinterpret_cast<const uint2 *>(bx + off[G8 & 3]);
                         const uint2 b = *reinterpret_cast<const uint2 *>(bx + off[G8 & 3] + 8 * kBox);
@@ -426,7 +502,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_step_kernel(const __grid_con
                     issue(s);
                 }
                 float out[MT][4];
-                if constexpr (F == 0)
+                if constexpr (F != 1)
                     gcm_slice<MT>(wd, xlane + kb * MT * 1024, qm, qh, out);
                 else
                     b1_slice<MT>(wd, xlane + kb * MT * 1024, qm, qh, out);
@@ -444,7 +520,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_step_kernel(const __grid_con
                         sb0 = sb1 = f.y;
                     }
                     // t = c - 1 (ternary) or t = 2b - 1 (1-bit)
-                    constexpr float kMul = F ? 2.f : 1.f;
+                    constexpr float kMul = F == 1 ? 2.f : 1.f;
                     acc[0] = fmaf(sa0, fmaf(kMul, out[h][0], -on.x), acc[0]);
                     acc[1] = fmaf(sa1, fmaf(kMul, out[h][1], -on.y), acc[1]);
                     acc[2] = fmaf(sb0, fmaf(kMul, out[h][2], -on.x), acc[2]);
@@ -532,12 +608,13 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_step_kernel(const __grid_con
     }
 }
 
-bool g_attr_step[64][2][3];
+bool g_attr_step[64][3][3];
 
 using StepKernel = void (*)(SParams);
 StepKernel step_kernel(int mt, int f) {
     if (f == 0) return mt == 1 ? gemv_step_kernel<1, 0> : (mt == 2 ? gemv_step_kernel<2, 0> : gemv_step_kernel<4, 0>);
-    return mt == 1 ? gemv_step_kernel<1, 1> : (mt == 2 ? gemv_step_kernel<2, 1> : gemv_step_kernel<4, 1>);
+    if (f == 1) return mt == 1 ? gemv_step_kernel<1, 1> : (mt == 2 ? gemv_step_kernel<2, 1> : gemv_step_kernel<4, 1>);
+    return mt == 1 ? gemv_step_kernel<1, 2> : (mt == 2 ? gemv_step_kernel<2, 2> : gemv_step_kernel<4, 2>);
 }
 
 int step_mt(int M) { return M == 1 ? 1 : (M == 2 ? 2 : 4); }
@@ -586,11 +663,17 @@ tern_status launch_chunk(const DeviceInfo &dev, const MatDesc *md, int count, in
             const uint32_t sbox[3] = {static_cast<uint32_t>(kBox), static_cast<uint32_t>(kRows), 2};
             st = encode_tiled_3d(&p.m[i].smap, CU_TENSOR_MAP_DATA_TYPE_UINT8, md[i].slots, sdims, sstr, sbox,
                                  CU_TENSOR_MAP_SWIZZLE_128B);
-        } else {
+        } else if (fmt == 1) {
             // the bit matrix [N rows][K/8 bytes]: one 128-byte box is a unit's row
             st = encode_tiled_2d(&p.m[i].smap, CU_TENSOR_MAP_DATA_TYPE_UINT8, md[i].slots,
                                  static_cast<uint64_t>(md[i].K / 8), static_cast<uint64_t>(md[i].N),
                                  static_cast<uint64_t>(md[i].K / 8), kBox, kRows, CU_TENSOR_MAP_SWIZZLE_128B);
+        } else {
+            // the base-3 bytes [N rows][R bytes], R = 208 K / 1024: one
+            // 208-byte box is a unit's row (a multiple of 16 bytes)
+            const uint64_t R = static_cast<uint64_t>(md[i].K / 1024) * kT5Row;
+            st = encode_tiled_2d(&p.m[i].smap, CU_TENSOR_MAP_DATA_TYPE_UINT8, md[i].slots, R,
+                                 static_cast<uint64_t>(md[i].N), R, kT5Row, kRows, CU_TENSOR_MAP_SWIZZLE_NONE);
         }
         if (st != TERN_OK) return st;
         const int G = md[i].K / kGroup;
@@ -655,7 +738,7 @@ tern_status launch_gemv_step(const MatDesc *md, int count, int M, int fmt, cudaS
     DeviceInfo dev;
     tern_status st = current_device(&dev);
     if (st != TERN_OK) return st;
-    if (fmt != 0 && fmt != 1) return fail(TERN_ERR_INVALID_ARG, "step kernel: unknown weight format %d", fmt);
+    if (fmt < 0 || fmt > 2) return fail(TERN_ERR_INVALID_ARG, "step kernel: unknown weight format %d", fmt);
     if (!gemv_step_supports(md, count, M, fmt)) return fail(TERN_ERR_SHAPE, "step kernel: unsupported shapes");
     const int mi = step_mt(M) == 1 ? 0 : (step_mt(M) == 2 ? 1 : 2);
     if (!g_attr_step[dev.device][fmt][mi]) {

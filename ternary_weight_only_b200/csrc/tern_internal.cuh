@@ -49,6 +49,11 @@ tern_status launch_unpack(const uint8_t *slots, int64_t N, int64_t K, int8_t *co
 tern_status launch_pack_b1(const int8_t *codes, const uint16_t *scales_in, int64_t N, int64_t K, uint8_t *bits,
                            uint16_t *scales_out, int32_t *invalid_count, cudaStream_t stream);
 tern_status launch_unpack_b1(const uint8_t *bits, int64_t N, int64_t K, int8_t *codes, cudaStream_t stream);
+// five trits per byte: uint8 [N][t5_row_bytes(K)], 26 bytes per 128-weight group
+int64_t t5_row_bytes(int64_t K);
+tern_status launch_pack_t5(const int8_t *codes, const uint16_t *scales_in, int64_t N, int64_t K, uint8_t *out,
+                           uint16_t *scales_out, int32_t *invalid_count, cudaStream_t stream);
+tern_status launch_unpack_t5(const uint8_t *in, int64_t N, int64_t K, int8_t *codes, cudaStream_t stream);
 
 struct MatDesc {
     const __half *x;
@@ -102,7 +107,8 @@ tern_status read_gemvpc_status(bool reset, unsigned int *out);
 tern_status launch_embed(const int32_t *ids, int64_t M, const uint8_t *slots, const uint16_t *scales, int64_t V,
                          int64_t K, uint16_t *out, int32_t *bad_count, cudaStream_t stream);
 // Persistent launch over many matrices (M = 1..4, K multiples of 1024); fmt 0
-// = ternary slots, 1 = the 1-bit variant (MatDesc::slots holds the bits).
+// = ternary slots, 1 = the 1-bit variant (MatDesc::slots holds the bits), 2 =
+// five trits per byte (MatDesc::slots holds the base-3 bytes).
 bool gemv_step_supports(const MatDesc *d, int count, int M, int fmt);
 tern_status launch_gemv_step(const MatDesc *d, int count, int M, int fmt, cudaStream_t stream);
 tern_status read_gemvstep_status(bool reset, unsigned int *out);

@@ -72,6 +72,10 @@ _SIGS = {
     "tern_b1_pack": ([_vp, _vp, _i64, _i64, _vp, _vp, _vp, _vp], _int),
     "tern_b1_unpack": ([_vp, _i64, _i64, _vp, _vp], _int),
     "tern_b1_gemv_step": ([ctypes.POINTER(tern_gemv_desc), _i32, _i64, _vp], _int),
+    "tern_t5_bytes": ([_i64, _i64], _sz),
+    "tern_t5_pack": ([_vp, _vp, _i64, _i64, _vp, _vp, _vp, _vp], _int),
+    "tern_t5_unpack": ([_vp, _i64, _i64, _vp, _vp], _int),
+    "tern_t5_gemv_step": ([ctypes.POINTER(tern_gemv_desc), _i32, _i64, _vp], _int),
 }
 for _name, (_args, _res) in _SIGS.items():
     _f = getattr(_L, _name)
@@ -330,3 +334,36 @@ def tern_gemv_grouped_workspace_bytes(mats: Sequence, M: int) -> int:
         arr[i].N = s.shape[0]
         arr[i].K = x.shape[-1]
     return _L.tern_gemv_grouped_workspace_bytes(arr, len(mats), M)
+
+
+def tern_t5_pack(codes: torch.Tensor, scales: torch.Tensor, bytes_out: Optional[torch.Tensor] = None,
+                 scales_out: Optional[torch.Tensor] = None,
+                 invalid_count: Optional[torch.Tensor] = None, stream=None):
+    """Five trits per byte: codes int8 [N,K], scales fp16 [N,K/128] ->
+    (bytes uint8 [N,R], scales fp16 [N,K/128]), R = tern_t5_bytes(N, K) / N."""
+    N, K = codes.shape
+    if bytes_out is None:
+        R = _L.tern_t5_bytes(N, K) // max(N, 1)
+        bytes_out = torch.empty((N, R), dtype=torch.uint8, device=codes.device)
+    if scales_out is None:
+        scales_out = torch.empty_like(scales)
+    ic = None if invalid_count is None else _dev(invalid_count, "invalid_count", torch.int32)
+    _check(_L.tern_t5_pack(_dev(codes, "codes", torch.int8), _dev(scales, "scales", torch.float16), N, K,
+                           _dev(bytes_out, "bytes_out", torch.uint8), _dev(scales_out, "scales_out", torch.float16),
+                           ic, _stream(stream)), "tern_t5_pack")
+    return bytes_out, scales_out
+
+
+def tern_t5_unpack(packed: torch.Tensor, K: int, codes_out: Optional[torch.Tensor] = None, stream=None):
+    N = packed.shape[0]
+    if codes_out is None:
+        codes_out = torch.empty((N, K), dtype=torch.int8, device=packed.device)
+    _check(_L.tern_t5_unpack(_dev(packed, "bytes", torch.uint8), N, K, _dev(codes_out, "codes_out", torch.int8),
+                             _stream(stream)), "tern_t5_unpack")
+    return codes_out
+
+
+def tern_t5_gemv_step(mats: Sequence, M: int = 1, stream=None):
+    """Five-per-byte variant of tern_gemv_step: mats as there with the bytes
+    uint8 [N,R] in place of the slots."""
+    _check(_L.tern_t5_gemv_step(_step_descs(mats), len(mats), M, _stream(stream)), "tern_t5_gemv_step")

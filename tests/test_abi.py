@@ -30,7 +30,8 @@ def test_header_declares_the_boundary():
     names = _declared()
     for n in ["tern_pack_g128", "tern_unpack_g128", "tern_gemv", "tern_gemm",
               "tern_gemv_grouped", "tern_gemv_step", "tern_embed_gather", "tern_workspace_bytes",
-              "tern_b1_pack", "tern_b1_unpack", "tern_b1_gemv_step",
+              "tern_b1_pack", "tern_b1_unpack", "tern_b1_gemv_step", "tern_t5_bytes", "tern_t5_pack",
+              "tern_t5_unpack", "tern_t5_gemv_step",
               "tern_slots_bytes",
               "tern_scales_bytes", "tern_status_string", "tern_last_error", "tern_set_option",
               "tern_version"]:
@@ -135,7 +136,7 @@ def test_grouped_rejects(lib):
     assert lib.tern_gemv_grouped(arr, 2, 1, None, 0, None) == 2
 
 
-@pytest.mark.parametrize("fn", ["tern_gemv_step", "tern_b1_gemv_step"])
+@pytest.mark.parametrize("fn", ["tern_gemv_step", "tern_b1_gemv_step", "tern_t5_gemv_step"])
 def test_step_rejects(lib, fn):
     """tern_gemv_step and its 1-bit twin: argument errors return before any launch."""
     from ternary_weight_only_b200 import tern
@@ -181,6 +182,25 @@ def test_b1_pack_rejects(lib):
     assert lib.tern_b1_unpack(None, 4, 256, A, None) == 1
     assert lib.tern_b1_unpack(A, 4, 100, A, None) == 3
     assert lib.tern_b1_unpack(A + 4, 4, 256, A, None) == 2
+
+
+def test_t5_sizes_and_rejects(lib):
+    """tern_t5_bytes: 26 bytes per 128-weight group, rows padded to 16 bytes;
+    tern_t5_pack / tern_t5_unpack argument errors return before any launch."""
+    assert lib.tern_t5_bytes(3, 128) == 3 * 32
+    assert lib.tern_t5_bytes(2, 5120) == 2 * 1040
+    assert lib.tern_t5_bytes(151936, 5120) + lib.tern_scales_bytes(151936, 5120) == 151936 * 5120 * 7 // 32
+    for bad in [(0, 128), (4, 0), (4, 100), (-1, 128)]:
+        assert lib.tern_t5_bytes(*bad) == 0
+    assert lib.tern_t5_pack(None, A, 4, 256, A, A, None, None) == 1
+    assert lib.tern_t5_pack(A, A, 4, 200, A, A, None, None) == 3
+    assert lib.tern_t5_pack(A + 8, A, 4, 256, A, A, None, None) == 2
+    assert lib.tern_t5_pack(A, A, 4, 256, A + 8, A, None, None) == 2
+    assert lib.tern_t5_pack(A, A + 1, 4, 256, A, A, None, None) == 2
+    assert lib.tern_t5_pack(A, A, 4, 256, A, A, A + 2, None) == 2
+    assert lib.tern_t5_unpack(None, 4, 256, A, None) == 1
+    assert lib.tern_t5_unpack(A, 4, 100, A, None) == 3
+    assert lib.tern_t5_unpack(A + 4, 4, 256, A, None) == 2
 
 
 def test_embed_rejects(lib):
