@@ -100,6 +100,7 @@ struct SParams {
     unsigned int smem_usable;     // dynamic shared memory past the 1024-byte alignment
     int kmax;
     int skip_loads;               // test only: issue no copies (exercises the timeout path)
+    int first;                    // 1 for the first launch of a call, 0 for the later ones
     unsigned long long timeout_ns;
 };
 
@@ -287,7 +288,15 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_step_kernel(const __grid_con
         for (int i = threadIdx.x; i < 256 * 32; i += kThreads) lut[i] = t5_codes(static_cast<uint32_t>(i >> 5));
     }
     __syncthreads();
-    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    // Ordering between launches (programmatic dependent launch).  The inputs
+    // of a call may come from the kernel before it, so its first launch waits
+    // for that kernel before anything reads x, and only then lets the next
+    // launch start.  The later launches of the same call read inputs that were
+    // complete before the first launch went past its wait, so they start their
+    // successors at once and do not wait before reading; they wait at the end
+    // instead, so that every launch still completes after the one before it
+    // (a kernel after the call that waits for its last launch sees all outputs).
+    if (!p.first) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     const unsigned long long deadline = globaltimer() + p.timeout_ns;
     uint64_t *my_full = full + warp * kMaxNS;
     // slot stages (4096 bytes, 1024-aligned: the 128-byte swizzle pattern is
@@ -319,8 +328,10 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_step_kernel(const __grid_con
     };
     for (int st = 0; st < ns && ic.i >= 0; st++) issue(st);
 
-    // x may be the output of the preceding launch: wait for it to finish.
-    asm volatile("griddepcontrol.wait;" ::: "memory");
+    if (p.first) {
+        asm volatile("griddepcontrol.wait;" ::: "memory");
+        asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    }
 
     int s = 0;
     uint32_t ph = 0;
@@ -606,6 +617,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_step_kernel(const __grid_con
             step_wait(&my_full[st], phs, dl2);
         }
     }
+    if (!p.first) asm volatile("griddepcontrol.wait;" ::: "memory");
 }
 
 bool g_attr_step[64][3][3];
@@ -635,7 +647,8 @@ bool gemv_step_supports(const MatDesc *md, int count, int M, int fmt) {
 namespace {
 
 // One launch over md[0..count) (count <= kMaxPer).
-tern_status launch_chunk(const DeviceInfo &dev, const MatDesc *md, int count, int M, int fmt, cudaStream_t stream) {
+tern_status launch_chunk(const DeviceInfo &dev, const MatDesc *md, int count, int M, int fmt, bool first,
+                         cudaStream_t stream) {
     static SParams p;  // large (parameter space); filled on the host for each launch
     std::memset(&p, 0, sizeof(p));
     const int mt = step_mt(M);
@@ -715,6 +728,7 @@ tern_status launch_chunk(const DeviceInfo &dev, const MatDesc *md, int count, in
     p.smem_usable = static_cast<unsigned int>(smem - 1024);
     p.kmax = kmax;
     p.skip_loads = g_gemm_skip_loads;
+    p.first = first ? 1 : 0;
     p.timeout_ns = g_gemm_timeout_ns;
     cudaLaunchConfig_t cfg;
     std::memset(&cfg, 0, sizeof(cfg));
@@ -752,7 +766,7 @@ tern_status launch_gemv_step(const MatDesc *md, int count, int M, int fmt, cudaS
     int done = 0;
     for (int l = 0; l < launches; l++) {
         const int n = (count - done) / (launches - l);
-        st = launch_chunk(dev, md + done, n, M, fmt, stream);
+        st = launch_chunk(dev, md + done, n, M, fmt, l == 0, stream);
         if (st != TERN_OK) return st;
         done += n;
     }

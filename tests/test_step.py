@@ -170,3 +170,53 @@ def test_verify_layer(T, orc, M):
     T.tern_gemv_step(mats, M)
     T.tern_sync_status()
     check_all(orc, mats, refs, f"step layer M={M}")
+
+
+def test_chained_calls_see_complete_inputs(T):
+    """Calls of more than 96 products run as several launches that may
+    overlap; a call whose inputs are the outputs of the previous call must
+    still read them complete.  Three chained calls of 200 products (three
+    launches each; large matrices first, so the later launches of a call
+    finish early): every output equals the same call repeated after a full
+    synchronisation (the kernel is deterministic)."""
+    from ternary_weight_only_b200 import synth
+    g = synth.gen(7700, "cuda")
+    count = 200
+
+    def layer(N_of):
+        mats = []
+        for j in range(count):
+            N = N_of(j)
+            codes = synth.codes_sparse(N, 1024, g, device="cuda")
+            slots, sc = T.tern_pack_g128(codes, synth.scales_uniform(N, 1024, g, device="cuda"))
+            mats.append((slots, sc))
+        return mats
+
+    # A: x0 -> ya, B: ya -> yb, C: yb -> yc; C's first 20 products have four
+    # times the rows, so its first launch runs longest
+    A = layer(lambda j: 1024)
+    B = layer(lambda j: 1024)
+    C = layer(lambda j: 4096 if j < 20 else 1024)
+    x0 = [synth.activations(1, 1024, g, device="cuda")[0] for _ in range(count)]
+    ya = [torch.empty(1024, dtype=torch.float16, device="cuda") for _ in range(count)]
+    yb = [torch.empty(1024, dtype=torch.float16, device="cuda") for _ in range(count)]
+    yc = [torch.empty(C[j][0].shape[0], dtype=torch.float16, device="cuda") for j in range(count)]
+    stream = torch.cuda.Stream()
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            T.tern_gemv_step([(x0[j], A[j][0], A[j][1], ya[j]) for j in range(count)], stream=stream)
+            T.tern_gemv_step([(ya[j], B[j][0], B[j][1], yb[j]) for j in range(count)], stream=stream)
+            T.tern_gemv_step([(yb[j], C[j][0], C[j][1], yc[j]) for j in range(count)], stream=stream)
+    T.tern_sync_status(stream)
+    got = [t.clone() for t in ya + yb + yc]
+    # the same calls one at a time, each after a full synchronisation
+    for mats_fn in (
+            lambda: [(x0[j], A[j][0], A[j][1], ya[j]) for j in range(count)],
+            lambda: [(ya[j], B[j][0], B[j][1], yb[j]) for j in range(count)],
+            lambda: [(yb[j], C[j][0], C[j][1], yc[j]) for j in range(count)]):
+        torch.cuda.synchronize()
+        T.tern_gemv_step(mats_fn())
+        T.tern_sync_status()
+    want = ya + yb + yc
+    for i, (a, b) in enumerate(zip(got, want)):
+        assert torch.equal(a, b), i
