@@ -206,26 +206,38 @@ class DecodeModel:
         one tern_gemv_step call (the inputs are independent)."""
         self.T.tern_gemv_step(self.all_mats())
 
-    def e2e_chunks(self, n):
-        """The step's products in n chunks of consecutive layers (the head
-        with the last): (products, x range, y range) with the ranges as
-        element offsets into x_all / y_all (each chunk's inputs and outputs
-        are contiguous)."""
+    def e2e_chunks(self, frac=(8 / 64, 60 / 64)):
+        """The step's products in chunks of consecutive layers cut at the
+        given fractions of the layer count, the head in the first chunk.  Only
+        the first chunk's copy in and the last chunk's copy out are not hidden
+        behind products, so both are small: the first chunk holds the head
+        (10 KB of x; its 304 KB of y go back while the rest runs) and eight
+        layers, the last four layers (0.4 MB of y).  Every further chunk costs
+        a call boundary (~12 us), so there are three.  (Measured on B200 over
+        ten cuttings: this one 1.407 ms per step end to end, five equal chunks
+        with the head last 1.453 ms; the copies alone take 0.139 ms.)
+        Returns (products, x ranges, y ranges), ranges as element offsets into
+        x_all / y_all."""
         per_x = 5120 + 6144 + 17408
         per_y = sum(N for _, _, N in synth.LAYER_PROJ)
-        out = []
-        bounds = [round(i * self.n_layers / n) for i in range(n + 1)]
+        L = self.n_layers
         _, K, N, slots, sc = self.head
-        for c in range(n):
-            l0, l1 = bounds[c], bounds[c + 1]
+        head = (self.head_io[0], slots, sc, self.head_io[1])
+        hx = (L * per_x, L * per_x + 5120)
+        hy = (L * per_y, L * per_y + N)
+        cuts = [0] + [round(f * L) for f in frac] + [L]
+        out = []
+        for c in range(len(cuts) - 1):
+            l0, l1 = cuts[c], cuts[c + 1]
+            if l1 <= l0 and c != 0:
+                continue
             mats = [m for grp in self.groups[l0:l1] for m in grp]
-            xr = [l0 * per_x, l1 * per_x]
-            yr = [l0 * per_y, l1 * per_y]
-            if c == n - 1:
-                mats.append((self.head_io[0], slots, sc, self.head_io[1]))
-                xr[1] += 5120
-                yr[1] += N
-            out.append((mats, tuple(xr), tuple(yr)))
+            xr = [(l0 * per_x, l1 * per_x)] if l1 > l0 else []
+            yr = [(l0 * per_y, l1 * per_y)] if l1 > l0 else []
+            if c == 0:
+                mats = [head] + mats
+                xr, yr = [hx] + xr, [hy] + yr
+            out.append((mats, xr, yr))
         return out
 
     def step_per_layer(self):
@@ -640,6 +652,24 @@ def run_profile(args):
         T.tern_set_option(T.TERN_OPT_GEMV_VARIANT, args.gemv_variant)
     model = DecodeModel(T, n_layers=args.profile_layers)
     _, hK, hN, hslots, hsc = model.head
+    if args.profile_format != "tern":
+        # the same products with 1-bit or five-per-byte weights, one step call
+        pack = T.tern_b1_pack if args.profile_format == "b1" else T.tern_t5_pack
+        draw = synth.codes_sign if args.profile_format == "b1" else synth.codes_sparse
+        g = synth.gen(8800, "cuda")
+        mats, nbytes = [], 0
+        for x, slots, sc, y in model.all_mats():
+            N, K = slots.shape[0], x.shape[-1]
+            w, wsc = pack(draw(N, K, g, device="cuda"), synth.scales_uniform(N, K, g, device="cuda"))
+            mats.append((x, w, wsc, y))
+            nbytes += w.numel() + 2 * wsc.numel() + 2 * K + 2 * N
+        step = T.tern_b1_gemv_step if args.profile_format == "b1" else T.tern_t5_gemv_step
+        for _ in range(3):
+            step(mats)
+        torch.cuda.synchronize()
+        print(json.dumps({"profile_layers": args.profile_layers, "profile_format": args.profile_format,
+                          "bytes_per_launch": nbytes}))
+        return 0
     for _ in range(3):
         if args.profile_step:
             model.step()
@@ -700,15 +730,16 @@ def run_tern(args):
     value = ws * total_bytes / (ms * 1e-3) / 1e9  # GB/s over all ranks (weak scaling)
 
     # ---- e2e: host inputs -> device, step, outputs -> host, every step ----
-    # The step's products go in five chunks of consecutive layers (the head
-    # with the last); per chunk: copy its inputs in (copy stream), run it
-    # (tern_gemv_step on the compute stream), copy its outputs back (second
-    # copy stream), so that the copies of one chunk overlap the products of
-    # the others.  One step is captured as one CUDA graph.
+    # The step's products go in three chunks of consecutive layers (the head
+    # with the first; DecodeModel.e2e_chunks); per chunk: copy its inputs in
+    # (copy stream), run it (tern_gemv_step on the compute stream), copy its
+    # outputs back (second copy stream), so that the copies of one chunk
+    # overlap the products of the others.  One step is captured as one CUDA
+    # graph.
     x_host = torch.empty(model.x_all.shape, dtype=torch.float16, pin_memory=True)
     x_host.copy_(model.x_all.cpu())
     y_host = torch.empty(model.y_all.shape, dtype=torch.float16, pin_memory=True)
-    chunks = model.e2e_chunks(5)
+    chunks = model.e2e_chunks()
     s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
 
     def e2e_body():
@@ -716,7 +747,8 @@ def run_tern(args):
         for (mats, xr, yr) in chunks:
             s_in.wait_stream(stream)
             with torch.cuda.stream(s_in):
-                model.x_all[xr[0]:xr[1]].copy_(x_host[xr[0]:xr[1]], non_blocking=True)
+                for a, b in xr:
+                    model.x_all[a:b].copy_(x_host[a:b], non_blocking=True)
                 e = torch.cuda.Event()
                 e.record(s_in)
                 ev_in.append(e)
@@ -727,7 +759,8 @@ def run_tern(args):
             d.record(stream)
             s_out.wait_event(d)
             with torch.cuda.stream(s_out):
-                y_host[yr[0]:yr[1]].copy_(model.y_all[yr[0]:yr[1]], non_blocking=True)
+                for a, b in yr:
+                    y_host[a:b].copy_(model.y_all[a:b], non_blocking=True)
         stream.wait_stream(s_out)
         stream.wait_stream(s_in)
 
@@ -816,6 +849,9 @@ def main():
                     help="profiling case: build this many layers, run their grouped launches 3x, exit")
     ap.add_argument("--profile-step", action="store_true",
                     help="profiling case: run the layers and the head as tern_gemv_step calls 3x")
+    ap.add_argument("--profile-format", choices=["tern", "b1", "t5"], default="tern",
+                    help="profiling case with --profile-layers: the step's products as 1-bit or five-per-byte "
+                         "matrices in one step call (run 3x)")
     ap.add_argument("--profile-head", action="store_true",
                     help="profiling case: run the 5120x151936 head launch 3x instead of the layers")
     ap.add_argument("--gemv-variant", type=int, default=0,
