@@ -315,9 +315,10 @@ def proj_rows(T, model, peak_gbs, l2_bytes):
         b = sum(wbytes(K, N) + 2 * M * K + 2 * M * N for _, K, N in synth.LAYER_PROJ)
         out[f"layer_M{M}"] = {"us": round(ms * 1e3, 3), "GBps": round(b / ms / 1e6, 1),
                               "frac": round(b / ms / 1e6 / peak_gbs, 4)}
-    # the verify step: every projection of all layers at M = 2, 4 token rows,
-    # one tern_gemv_step call (5 launches)
-    for M in (2, 4):
+    # the verify step: every projection of all layers at M = 2, 4, 8 token
+    # rows, one tern_gemv_step call (5 launches; at M = 8 the down
+    # projections, whose eight rows of x do not fit, run as two passes)
+    for M in (2, 4, 8):
         mats, b = [], 0
         for l in range(synth.N_LAYERS):
             for i, (x, slots, sc, y) in enumerate(model.groups[l]):

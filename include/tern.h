@@ -213,7 +213,7 @@ size_t tern_gemv_grouped_workspace_bytes(const tern_gemv_desc *descs, int32_t co
 
 /*
  * tern_gemv_step -- products of up to TERN_MAX_STEP independent matrices with
- * the same M (1..4 token rows: a decode step, M = 1, or a speculative-verify
+ * the same M (1..8 token rows: a decode step, M = 1, or a speculative-verify
  * step) in ONE persistent launch, e.g. every projection of every layer plus
  * the output head of one step whose inputs do not depend on each other.
  * Generation speed is set by the bytes of weights read per token ("Bonsai
@@ -225,10 +225,13 @@ size_t tern_gemv_grouped_workspace_bytes(const tern_gemv_desc *descs, int32_t co
  *           buffers owned by the caller, 16-byte aligned; read on the host
  *           during the call (the array need not outlive it)
  *   count   1..TERN_MAX_STEP
- *   M       1..4 (TERN_ERR_SHAPE otherwise)
+ *   M       1..8 (TERN_ERR_SHAPE otherwise)
  * Every K must be a multiple of 1024, and M x (largest K) x 2 bytes of x
  * must fit in shared memory beside the weight rings (TERN_ERR_SHAPE
- * otherwise; use tern_gemv_grouped then).  Results are those of tern_gemv /
+ * otherwise; use tern_gemv_grouped then).  With M = 5..8 the products whose
+ * eight rows of x do not fit (K above ~12000) run instead as two passes of 4
+ * and M - 4 rows, in launches of their own after the others; M = 4 at
+ * K = 17408 still fits.  Results are those of tern_gemv /
  * tern_gemm for each matrix (same arithmetic, fixed summation order per tile);
  * outputs must not overlap inputs or each other.  Argument errors return
  * before any launch; a device wait that gives up is reported by
@@ -347,7 +350,7 @@ tern_status tern_t5_unpack(const uint8_t *bytes, int64_t N, int64_t K, int8_t *c
 /*
  * tern_t5_gemv_step -- tern_gemv_step for five-per-byte matrices: each
  * descriptor's `slots` field points to the bytes (uint8 [N][R]); shapes
- * (K a multiple of 1024, M in 1..4), arithmetic, argument checks and error
+ * (K a multiple of 1024, M in 1..8), arithmetic, argument checks and error
  * reporting as for tern_gemv_step.  The kernel keeps a 32 KiB decode table
  * in shared memory, so the largest M x K it accepts is smaller than for
  * tern_gemv_step (TERN_ERR_SHAPE beyond it; M = 4 at K = 17408 does not fit).

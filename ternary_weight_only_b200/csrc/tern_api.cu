@@ -357,7 +357,9 @@ tern_status gemv_step_api(const tern_gemv_desc *descs, int32_t count, int64_t M,
     if (!descs) return fail(TERN_ERR_INVALID_ARG, "descs is NULL");
     if (count < 1 || count > TERN_MAX_STEP)
         return fail(TERN_ERR_INVALID_ARG, "count must be 1..%d (got %d)", TERN_MAX_STEP, count);
-    if (M < 1 || M > 4) return fail(TERN_ERR_SHAPE, "%s takes M in 1..4 (got %lld)", name, static_cast<long long>(M));
+    const int mmax = fmt == 1 ? 4 : 8;
+    if (M < 1 || M > mmax)
+        return fail(TERN_ERR_SHAPE, "%s takes M in 1..%d (got %lld)", name, mmax, static_cast<long long>(M));
     static MatDesc d[TERN_MAX_STEP];
     for (int i = 0; i < count; i++) {
         tern_status st = check_nk(descs[i].N, descs[i].K);
@@ -369,9 +371,39 @@ tern_status gemv_step_api(const tern_gemv_desc *descs, int32_t count, int64_t M,
         if (st != TERN_OK) return st;
         d[i] = mat(descs[i].x, descs[i].slots, descs[i].scales, descs[i].y, descs[i].N, descs[i].K);
     }
-    if (!gemv_step_supports(d, count, static_cast<int>(M), fmt))
+    const int m = static_cast<int>(M);
+    cudaStream_t st_ = static_cast<cudaStream_t>(stream);
+    if (m <= 4 || gemv_step_supports(d, count, m, fmt)) {
+        if (!gemv_step_supports(d, count, m, fmt))
+            return fail(TERN_ERR_SHAPE, "%s: M x K too large for shared memory", name);
+        return launch_gemv_step(d, count, m, fmt, st_);
+    }
+    // M = 5..8: the products whose M x K of x fit run in one pass of eight
+    // token rows; the others in two passes of 4 and M - 4 rows (each reading
+    // the weights once).
+    static MatDesc one[TERN_MAX_STEP], lo[TERN_MAX_STEP], hi[TERN_MAX_STEP];
+    int n1 = 0, n2 = 0;
+    for (int i = 0; i < count; i++) {
+        if (gemv_step_fits(d[i].K, m, fmt)) {
+            one[n1++] = d[i];
+        } else {
+            lo[n2] = d[i];
+            hi[n2] = d[i];
+            hi[n2].x = d[i].x + static_cast<size_t>(4) * d[i].K;
+            hi[n2].y = d[i].y + static_cast<size_t>(4) * d[i].N;
+            n2++;
+        }
+    }
+    if ((n2 > 0 && (!gemv_step_supports(lo, n2, 4, fmt) || !gemv_step_supports(hi, n2, m - 4, fmt))))
         return fail(TERN_ERR_SHAPE, "%s: M x K too large for shared memory", name);
-    return launch_gemv_step(d, count, static_cast<int>(M), fmt, static_cast<cudaStream_t>(stream));
+    tern_status st;
+    if (n1 > 0) {
+        st = launch_gemv_step(one, n1, m, fmt, st_);
+        if (st != TERN_OK) return st;
+    }
+    st = launch_gemv_step(lo, n2, 4, fmt, st_);
+    if (st != TERN_OK) return st;
+    return launch_gemv_step(hi, n2, m - 4, fmt, st_);
 }
 }  // namespace
 

@@ -106,12 +106,12 @@ struct SParams {
 
 // Shared memory layout (bytes from the 128-aligned base).
 __host__ __device__ constexpr int bar_off() { return 0; }
-__host__ __device__ constexpr int rec_off() { return kW * kMaxNS * 8; }               // [kW][2][8][2] float4
-__host__ __device__ constexpr int rtile_off() { return rec_off() + kW * 2 * 16 * 16; }  // [kW][2] int
+__host__ __device__ constexpr int rec_off() { return kW * kMaxNS * 8; }               // [kW][2][8][4] float4
+__host__ __device__ constexpr int rtile_off() { return rec_off() + kW * 2 * 8 * 4 * 16; }  // [kW][2] int
 __host__ __device__ constexpr int wmax_off() { return rtile_off() + kW * 2 * 4; }     // [kW] uint
-__host__ __device__ constexpr int d1_off() { return wmax_off() + kW * 4; }            // [kmax / 128] float
-// d1 holds one float per (set, column): kmax / 128 * MT floats, MT <= 4
-__host__ __device__ constexpr int lut_off(int kmax) { return d1_off() + (kmax / 128) * 16 + 64; }
+__host__ __device__ constexpr int d1_off() { return wmax_off() + kW * 4; }            // [kmax / 128 * 8] float
+// d1 holds one float per (set, column): kmax / 1024 * MT sets of 8, MT <= 8
+__host__ __device__ constexpr int lut_off(int kmax) { return d1_off() + (kmax / 128) * 32 + 64; }
 __host__ __device__ constexpr int xs_off(int kmax, int f) { return lut_off(kmax) + lut_bytes(f); }
 // staged x: MT token rows (M real, the rest zero)
 __host__ __device__ constexpr int ring_off(int kmax, int mt, int f) {
@@ -217,6 +217,9 @@ __device__ __forceinline__ void cursor_next(Cursor &c, const SParams &p, int T0,
 
 // MT = token rows padded to 1, 2 or 4: the group-per-column form with
 // (group, token) pairs in the mma columns (gcm_slice, or b1_slice for F = 1).
+// MT = 8 (5..8 token rows; not for F = 1): the eight columns are the eight
+// tokens of one group, so a slice is eight sets of one group, each group's
+// eight-mma chain (group_mma) taken in turn, group by group.
 template <int MT, int F>
 __global__ void __launch_bounds__(kThreads, 1) gemv_step_kernel(const __grid_constant__ SParams p) {
     constexpr int GPB = 8 / MT;  // groups per set
@@ -434,11 +437,12 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_step_kernel(const __grid_con
         // reduction; lane (g, q) stores v = (row g: tokens t0, t1; row g+8:
         // tokens t0, t1), t0 = 2q, t1 = 2q + 1 (MT = 4), 0, 1 (MT = 2), or
         // token 0 only from v.x, v.z (MT = 1).
-        constexpr int kGcLanes = MT == 4 ? 2 : 1;
+        // MT = 8: every lane holds its own tokens 2q, 2q + 1.
+        constexpr int kGcLanes = MT == 8 ? 4 : (MT == 4 ? 2 : 1);
         auto gc_store = [&](int tile, float4 v) {
             if (q >= kGcLanes) return;
             const int n0 = tile * kRows + row, n1 = n0 + 8;
-            const int t0 = MT == 4 ? 2 * q : 0, t1 = t0 + 1;
+            const int t0 = MT >= 4 ? 2 * q : 0, t1 = t0 + 1;
             if (n0 < N) {
                 if (t0 < M) d.y[static_cast<size_t>(t0) * N + n0] = __float2half_rn(v.x);
                 if (MT > 1 && t1 < M) d.y[static_cast<size_t>(t1) * N + n0] = __float2half_rn(v.y);
@@ -489,10 +493,14 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_step_kernel(const __grid_con
                     }
                 }
                 // scales of the lane's groups (rows `row`, `row` + 8): MT = 1
-                // groups 2q, 2q+1; otherwise one group per set h (4h + q, or
-                // 2h + q/2)
-                __half2 sh[MT == 1 ? 2 : MT];
-                if (MT == 1) {
+                // groups 2q, 2q+1; MT = 2, 4: one group per set h (4h + q, or
+                // 2h + q/2); MT = 8: all eight groups of both rows
+                __half2 sh[MT == 1 ? 2 : (MT == 8 ? 1 : MT)];
+                uint4 s8a, s8b;
+                if constexpr (MT == 8) {
+                    s8a = *reinterpret_cast<const uint4 *>(scs + row * 16);
+                    s8b = *reinterpret_cast<const uint4 *>(scs + (row + 8) * 16);
+                } else if (MT == 1) {
                     sh[0] = *reinterpret_cast<const __half2 *>(scs + row * 16 + 4 * q);
                     sh[MT == 1 ? 1 : 0] = *reinterpret_cast<const __half2 *>(scs + (row + 8) * 16 + 4 * q);
                 } else {
@@ -512,6 +520,25 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_step_kernel(const __grid_con
                     if (lane == 0) asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
                     issue(s);
                 }
+                if constexpr (MT == 8) {
+                    // group by group: acc[0..1] = row g, tokens 2q, 2q+1;
+                    // acc[2..3] = row g+8
+                    const uint32_t sw[2][4] = {{s8a.x, s8a.y, s8a.z, s8a.w}, {s8b.x, s8b.y, s8b.z, s8b.w}};
+#pragma unroll
+                    for (int G8 = 0; G8 < kSG; G8++) {
+                        float c[4];
+                        group_mma<8>(c, wd[G8][0], wd[G8][2], wd[G8][1], wd[G8][3], xlane + (kb * 8 + G8) * 1024);
+                        const float2 on = *reinterpret_cast<const float2 *>(d1 + (kb * 8 + G8) * kSG + 2 * q);
+                        const float sa = __half2float(__ushort_as_half(
+                            static_cast<unsigned short>(sw[0][G8 >> 1] >> (16 * (G8 & 1)))));
+                        const float sb = __half2float(__ushort_as_half(
+                            static_cast<unsigned short>(sw[1][G8 >> 1] >> (16 * (G8 & 1)))));
+                        acc[0] = fmaf(sa, c[0] - on.x, acc[0]);
+                        acc[1] = fmaf(sa, c[1] - on.y, acc[1]);
+                        acc[2] = fmaf(sb, c[2] - on.x, acc[2]);
+                        acc[3] = fmaf(sb, c[3] - on.y, acc[3]);
+                    }
+                } else {
                 float out[MT][4];
                 if constexpr (F != 1)
                     gcm_slice<MT>(wd, xlane + kb * MT * 1024, qm, qh, out);
@@ -537,6 +564,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_step_kernel(const __grid_con
                     acc[2] = fmaf(sb0, fmaf(kMul, out[h][2], -on.x), acc[2]);
                     acc[3] = fmaf(sb1, fmaf(kMul, out[h][3], -on.y), acc[3]);
                 }
+                }
             }
             stage += kSlotStage;
             scs += kScaleStage;
@@ -557,7 +585,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_step_kernel(const __grid_con
 #pragma unroll
                 for (int c = 0; c < 4; c++) {
                     if (MT <= 2) acc[c] += __shfl_xor_sync(0xffffffffu, acc[c], 1);
-                    acc[c] += __shfl_xor_sync(0xffffffffu, acc[c], 2);
+                    if (MT <= 4) acc[c] += __shfl_xor_sync(0xffffffffu, acc[c], 2);
                 }
                 const int tile = tbeg + tl;
                 const bool whole = kb == B - 1 && (tl != tl_first || !first_partial);
@@ -566,7 +594,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_step_kernel(const __grid_con
                     if (!dead) gc_store(tile, vv);
                 } else {
                     const int slot = (tl == tl_first) ? 0 : 1;
-                    if (q < kGcLanes) *reinterpret_cast<float4 *>(rec + (((warp * 2 + slot) * 8 + g) * 2 + q) * 4) = vv;
+                    if (q < kGcLanes) *reinterpret_cast<float4 *>(rec + (((warp * 2 + slot) * 8 + g) * 4 + q) * 4) = vv;
                     if (lane == 0) rec_tile[warp * 2 + slot] = dead ? -2 : tile;
                 }
                 acc[0] = acc[1] = acc[2] = acc[3] = 0.f;
@@ -597,7 +625,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_step_kernel(const __grid_con
                 for (int w2 = warp; w2 < kW; w2++)
                     for (int s2i = 0; s2i < 2; s2i++) {
                         if (rec_tile[w2 * 2 + s2i] != tile) continue;
-                        const float4 o = *reinterpret_cast<const float4 *>(rec + (((w2 * 2 + s2i) * 8 + g) * 2 + q) * 4);
+                        const float4 o = *reinterpret_cast<const float4 *>(rec + (((w2 * 2 + s2i) * 8 + g) * 4 + q) * 4);
                         sum.x += o.x;
                         sum.y += o.y;
                         sum.z += o.z;
@@ -620,21 +648,29 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_step_kernel(const __grid_con
     if (!p.first) asm volatile("griddepcontrol.wait;" ::: "memory");
 }
 
-bool g_attr_step[64][3][3];
+bool g_attr_step[64][3][4];
 
 using StepKernel = void (*)(SParams);
 StepKernel step_kernel(int mt, int f) {
-    if (f == 0) return mt == 1 ? gemv_step_kernel<1, 0> : (mt == 2 ? gemv_step_kernel<2, 0> : gemv_step_kernel<4, 0>);
+    if (f == 0)
+        return mt == 1 ? gemv_step_kernel<1, 0>
+                       : (mt == 2 ? gemv_step_kernel<2, 0> : (mt == 4 ? gemv_step_kernel<4, 0> : gemv_step_kernel<8, 0>));
     if (f == 1) return mt == 1 ? gemv_step_kernel<1, 1> : (mt == 2 ? gemv_step_kernel<2, 1> : gemv_step_kernel<4, 1>);
-    return mt == 1 ? gemv_step_kernel<1, 2> : (mt == 2 ? gemv_step_kernel<2, 2> : gemv_step_kernel<4, 2>);
+    return mt == 1 ? gemv_step_kernel<1, 2>
+                   : (mt == 2 ? gemv_step_kernel<2, 2> : (mt == 4 ? gemv_step_kernel<4, 2> : gemv_step_kernel<8, 2>));
 }
 
-int step_mt(int M) { return M == 1 ? 1 : (M == 2 ? 2 : 4); }
+int step_mt(int M) { return M == 1 ? 1 : (M == 2 ? 2 : (M <= 4 ? 4 : 8)); }
+int mt_index(int mt) { return mt == 1 ? 0 : (mt == 2 ? 1 : (mt == 4 ? 2 : 3)); }
 
 }  // namespace
 
+bool gemv_step_fits(int K, int M, int fmt) {
+    return K % 1024 == 0 && M >= 1 && M <= (fmt == 1 ? 4 : 8) && smem_bytes(K, step_mt(M), 1, fmt) <= kSmemBudget;
+}
+
 bool gemv_step_supports(const MatDesc *md, int count, int M, int fmt) {
-    if (count < 1 || count > TERN_MAX_STEP || M < 1 || M > 4) return false;
+    if (count < 1 || count > TERN_MAX_STEP || M < 1 || M > (fmt == 1 ? 4 : 8)) return false;
     int kmax = 0;
     for (int i = 0; i < count; i++) {
         if (md[i].K % 1024 != 0) return false;
@@ -754,7 +790,7 @@ tern_status launch_gemv_step(const MatDesc *md, int count, int M, int fmt, cudaS
     if (st != TERN_OK) return st;
     if (fmt < 0 || fmt > 2) return fail(TERN_ERR_INVALID_ARG, "step kernel: unknown weight format %d", fmt);
     if (!gemv_step_supports(md, count, M, fmt)) return fail(TERN_ERR_SHAPE, "step kernel: unsupported shapes");
-    const int mi = step_mt(M) == 1 ? 0 : (step_mt(M) == 2 ? 1 : 2);
+    const int mi = mt_index(step_mt(M));
     if (!g_attr_step[dev.device][fmt][mi]) {
         cudaError_t e = cudaFuncSetAttribute(step_kernel(step_mt(M), fmt), cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              static_cast<int>(dev.max_smem_optin));

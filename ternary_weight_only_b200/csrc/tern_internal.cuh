@@ -106,10 +106,12 @@ tern_status read_gemvpc_status(bool reset, unsigned int *out);
 // Ternary embedding rows gathered by id, written as fp16 s * t.
 tern_status launch_embed(const int32_t *ids, int64_t M, const uint8_t *slots, const uint16_t *scales, int64_t V,
                          int64_t K, uint16_t *out, int32_t *bad_count, cudaStream_t stream);
-// Persistent launch over many matrices (M = 1..4, K multiples of 1024); fmt 0
+// Persistent launch over many matrices (M = 1..8, 1..4 for fmt 1; K multiples of 1024); fmt 0
 // = ternary slots, 1 = the 1-bit variant (MatDesc::slots holds the bits), 2 =
 // five trits per byte (MatDesc::slots holds the base-3 bytes).
 bool gemv_step_supports(const MatDesc *d, int count, int M, int fmt);
+// whether one product of depth K at M token rows fits the step kernel
+bool gemv_step_fits(int K, int M, int fmt);
 tern_status launch_gemv_step(const MatDesc *d, int count, int M, int fmt, cudaStream_t stream);
 tern_status read_gemvstep_status(bool reset, unsigned int *out);
 extern unsigned long long g_gemm_timeout_ns;

@@ -291,7 +291,7 @@ def _step_descs(mats: Sequence):
 
 def tern_gemv_step(mats: Sequence, M: int = 1, stream=None):
     """mats: sequence of (x [M,K] (or [K] for M = 1), slots [N,K/4],
-    scales [N,K/128], y [M,N] (or [N])) CUDA tensors, M in 1..4, every K a
+    scales [N,K/128], y [M,N] (or [N])) CUDA tensors, M in 1..8, every K a
     multiple of 1024: one persistent launch."""
     _check(_L.tern_gemv_step(_step_descs(mats), len(mats), M, _stream(stream)), "tern_gemv_step")
 

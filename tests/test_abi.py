@@ -147,11 +147,12 @@ def test_step_rejects(lib, fn):
     class _L:
         tern_gemv_step = getattr(lib, fn)
     lib = _L
+    mmax = 4 if fn == "tern_b1_gemv_step" else 8
     assert lib.tern_gemv_step(None, 1, 1, None) == 1
     assert lib.tern_gemv_step(arr, 0, 1, None) == 1
     assert lib.tern_gemv_step(arr, tern.TERN_MAX_STEP + 1, 1, None) == 1
     assert lib.tern_gemv_step(arr, 3, 0, None) == 3
-    assert lib.tern_gemv_step(arr, 3, 5, None) == 3
+    assert lib.tern_gemv_step(arr, 3, mmax + 1, None) == 3
     arr[1].K = 1536                      # a multiple of 128 but not of 1024
     assert lib.tern_gemv_step(arr, 3, 1, None) == 3
     arr[1].K = 1000                      # not a multiple of 128

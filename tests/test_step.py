@@ -146,10 +146,12 @@ def test_timeout_reported_and_context_survives(T, orc):
     check_all(orc, mats, refs, "step after timeout")
 
 
-@pytest.mark.parametrize("M", [2, 3, 4])
+@pytest.mark.parametrize("M", [2, 3, 4, 5, 6, 8])
 @pytest.mark.parametrize("grid", [0, 5])
 def test_verify_batch_mixed(T, orc, M, grid):
-    """M token rows (M = 3 runs padded to 4): every output of every token."""
+    """M token rows (M = 3 runs padded to 4, 5..8 padded to 8; at M > 4 the
+    K = 17408 product does not fit eight rows of x and runs as two passes of
+    4 and M - 4 rows): every output of every token."""
     shapes = [(1024, 1), (2048, 17), (5120, 100), (3072, 333), (6144, 64), (17408, 40), (4096, 129)]
     mats, refs = make_mats(orc, shapes, seed=7500 + 10 * M + grid, M=M)
     T.tern_set_option(T.TERN_OPT_GEMV_GRID, grid)
@@ -161,7 +163,7 @@ def test_verify_batch_mixed(T, orc, M, grid):
     check_all(orc, mats, refs, f"step M={M} grid={grid}")
 
 
-@pytest.mark.parametrize("M", [2, 4])
+@pytest.mark.parametrize("M", [2, 4, 8])
 def test_verify_layer(T, orc, M):
     """The seven projections of a synthetic decode layer at M token rows."""
     from ternary_weight_only_b200 import synth

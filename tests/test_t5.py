@@ -123,7 +123,7 @@ def test_decode_layer_and_head(T, orc):
     check_all(orc, mats, refs, "t5 step layer+head")
 
 
-@pytest.mark.parametrize("M", [2, 3, 4])
+@pytest.mark.parametrize("M", [2, 3, 4, 8])
 @pytest.mark.parametrize("grid", [0, 5])
 def test_verify_batch_mixed(T, orc, M, grid):
     shapes = [(1024, 1), (2048, 17), (5120, 100), (3072, 333), (6144, 64), (4096, 129)]
