@@ -317,7 +317,7 @@ def proj_rows(T, model, peak_gbs, l2_bytes):
                               "frac": round(b / ms / 1e6 / peak_gbs, 4)}
     # the verify step: every projection of all layers at M = 2, 4, 8 token
     # rows, one tern_gemv_step call (5 launches; at M = 8 the down
-    # projections, whose eight rows of x do not fit, run as two passes)
+    # projections, whose eight rows of x do not fit, run as two K segments)
     for M in (2, 4, 8):
         mats, b = [], 0
         for l in range(synth.N_LAYERS):

@@ -226,13 +226,15 @@ size_t tern_gemv_grouped_workspace_bytes(const tern_gemv_desc *descs, int32_t co
  *           during the call (the array need not outlive it)
  *   count   1..TERN_MAX_STEP
  *   M       1..8 (TERN_ERR_SHAPE otherwise)
- * Every K must be a multiple of 1024, and M x (largest K) x 2 bytes of x
- * must fit in shared memory beside the weight rings (TERN_ERR_SHAPE
- * otherwise; use tern_gemv_grouped then).  With M = 5..8 the products whose
- * eight rows of x do not fit (K above ~12000) run instead as two passes of 4
- * and M - 4 rows, in launches of their own after the others; M = 4 at
- * K = 17408 still fits.  Results are those of tern_gemv /
- * tern_gemm for each matrix (same arithmetic, fixed summation order per tile);
+ * Every K must be a multiple of 1024.  The M rows of a product's x are
+ * staged in shared memory beside the weight rings; a product whose x does
+ * not fit (at M = 8 above K ~ 8900, at M = 4 above K ~ 17900) runs as up to
+ * eight K segments of whole 1024-k units, in launches of their own after the
+ * others: the first writes y, each later one adds its fp16-rounded partial
+ * sum to y (one extra rounding, within the tolerance below); beyond eight
+ * segments TERN_ERR_SHAPE.  Each weight is read once either way.  Results are
+ * within |y - y_ref| <= 2e-3 sum_k |x_k w_k| + 1e-5 of the exact product, as
+ * for tern_gemv / tern_gemm (fixed summation order per tile);
  * outputs must not overlap inputs or each other.  Argument errors return
  * before any launch; a device wait that gives up is reported by
  * tern_sync_status.  Internally a list longer than 96 matrices becomes a few
@@ -352,8 +354,8 @@ tern_status tern_t5_unpack(const uint8_t *bytes, int64_t N, int64_t K, int8_t *c
  * descriptor's `slots` field points to the bytes (uint8 [N][R]); shapes
  * (K a multiple of 1024, M in 1..8), arithmetic, argument checks and error
  * reporting as for tern_gemv_step.  The kernel keeps a 32 KiB decode table
- * in shared memory, so the largest M x K it accepts is smaller than for
- * tern_gemv_step (TERN_ERR_SHAPE beyond it; M = 4 at K = 17408 does not fit).
+ * in shared memory, so products are cut into K segments at a smaller K than
+ * for tern_gemv_step (M = 4 at K = 17408 runs as two).
  * An invalid byte contributes an unspecified finite value for its weights.
  */
 tern_status tern_t5_gemv_step(const tern_gemv_desc *descs, int32_t count, int64_t M, void *stream);

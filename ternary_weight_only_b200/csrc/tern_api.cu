@@ -373,37 +373,49 @@ tern_status gemv_step_api(const tern_gemv_desc *descs, int32_t count, int64_t M,
     }
     const int m = static_cast<int>(M);
     cudaStream_t st_ = static_cast<cudaStream_t>(stream);
-    if (m <= 4 || gemv_step_supports(d, count, m, fmt)) {
-        if (!gemv_step_supports(d, count, m, fmt))
-            return fail(TERN_ERR_SHAPE, "%s: M x K too large for shared memory", name);
-        return launch_gemv_step(d, count, m, fmt, st_);
-    }
-    // M = 5..8: the products whose M x K of x fit run in one pass of eight
-    // token rows; the others in two passes of 4 and M - 4 rows (each reading
-    // the weights once).
-    static MatDesc one[TERN_MAX_STEP], lo[TERN_MAX_STEP], hi[TERN_MAX_STEP];
-    int n1 = 0, n2 = 0;
+    if (gemv_step_supports(d, count, m, fmt)) return launch_gemv_step(d, count, m, fmt, st_);
+    // Products whose M rows of x do not fit in shared memory beside the
+    // rings run as K segments of whole 1024-k units that do, in calls of
+    // their own: segment 0 (with every product that fits) writes y, each
+    // later segment adds its sum to y.  Each weight is still read once.
+    static MatDesc seg[8][TERN_MAX_STEP];
+    int nseg_max = 1, n[8] = {0};
+    const int unit_bytes = fmt == 0 ? 256 : (fmt == 1 ? 128 : 208);  // weight bytes of one 1024-k row unit
     for (int i = 0; i < count; i++) {
         if (gemv_step_fits(d[i].K, m, fmt)) {
-            one[n1++] = d[i];
-        } else {
-            lo[n2] = d[i];
-            hi[n2] = d[i];
-            hi[n2].x = d[i].x + static_cast<size_t>(4) * d[i].K;
-            hi[n2].y = d[i].y + static_cast<size_t>(4) * d[i].N;
-            n2++;
+            seg[0][n[0]++] = d[i];
+            continue;
+        }
+        const int B = d[i].K / 1024;
+        int bfit = B - 1;
+        while (bfit > 0 && !gemv_step_fits(bfit * 1024, m, fmt)) bfit--;
+        if (bfit == 0) return fail(TERN_ERR_SHAPE, "%s: M x 1024 too large for shared memory", name);
+        const int nseg = (B + bfit - 1) / bfit;
+        if (nseg > 8) return fail(TERN_ERR_SHAPE, "%s: K=%d needs more than 8 segments at M=%d", name, d[i].K, m);
+        nseg_max = std::max(nseg_max, nseg);
+        for (int sgi = 0; sgi < nseg; sgi++) {
+            const int u0 = sgi * B / nseg, u1 = (sgi + 1) * B / nseg;
+            MatDesc e = d[i];
+            e.x = d[i].x + static_cast<size_t>(u0) * 1024;
+            e.slots = d[i].slots + static_cast<size_t>(u0) * unit_bytes;
+            e.scales = d[i].scales + static_cast<size_t>(u0) * (1024 / kGroup);
+            e.K = (u1 - u0) * 1024;
+            e.kfull = d[i].K;
+            e.accum = sgi > 0;
+            seg[sgi][n[sgi]++] = e;
         }
     }
-    if ((n2 > 0 && (!gemv_step_supports(lo, n2, 4, fmt) || !gemv_step_supports(hi, n2, m - 4, fmt))))
-        return fail(TERN_ERR_SHAPE, "%s: M x K too large for shared memory", name);
-    tern_status st;
-    if (n1 > 0) {
-        st = launch_gemv_step(one, n1, m, fmt, st_);
+    for (int sgi = 0; sgi < nseg_max; sgi++) {
+        if (n[sgi] == 0) continue;
+        if (!gemv_step_supports(seg[sgi], n[sgi], m, fmt))
+            return fail(TERN_ERR_SHAPE, "%s: M x K too large for shared memory", name);
+    }
+    for (int sgi = 0; sgi < nseg_max; sgi++) {
+        if (n[sgi] == 0) continue;
+        tern_status st = launch_gemv_step(seg[sgi], n[sgi], m, fmt, st_);
         if (st != TERN_OK) return st;
     }
-    st = launch_gemv_step(lo, n2, 4, fmt, st_);
-    if (st != TERN_OK) return st;
-    return launch_gemv_step(hi, n2, m - 4, fmt, st_);
+    return TERN_OK;
 }
 }  // namespace
 

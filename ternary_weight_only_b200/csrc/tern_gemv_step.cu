@@ -82,6 +82,8 @@ struct SDesc {
     int N, K;
     int tile0;   // first tile of this matrix in the flat tile list
     int ntile;   // ceil(N / 16)
+    int xs;      // row stride of x (elements): K, or the full row of a K segment
+    int accum;   // add the result to y (a K segment after the first) instead of writing it
 };
 
 struct alignas(64) SMaps {
@@ -348,8 +350,10 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_step_kernel(const __grid_con
         __syncthreads();  // the previous piece is finished with xs, d1, rec
         {
             unsigned int mx = 0;
-            for (int idx = threadIdx.x; idx < M * K / 8; idx += nthr) {
-                const uint4 v = *reinterpret_cast<const uint4 *>(d.x + static_cast<size_t>(idx) * 8);
+            const int per_row = K / 8;
+            for (int idx = threadIdx.x; idx < M * per_row; idx += nthr) {
+                const int m = idx / per_row, c8 = idx - m * per_row;
+                const uint4 v = *reinterpret_cast<const uint4 *>(d.x + static_cast<size_t>(m) * d.xs + c8 * 8);
                 const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
                 for (int e = 0; e < 4; e++) mx = __vmaxu2(mx, __vminu2(wv[e] & 0x7FFF7FFFu, 0x7BFF7BFFu));
@@ -378,7 +382,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_step_kernel(const __grid_con
             for (int idx = threadIdx.x; idx < MT * per_m; idx += nthr) {
                 const int m = idx / per_m, c8 = idx - m * per_m;
                 uint4 v = make_uint4(0u, 0u, 0u, 0u);
-                if (m < M) v = *reinterpret_cast<const uint4 *>(d.x + static_cast<size_t>(m) * K + c8 * 8);
+                if (m < M) v = *reinterpret_cast<const uint4 *>(d.x + static_cast<size_t>(m) * d.xs + c8 * 8);
                 const uint32_t pr[4] = {v.x, v.y, v.z, v.w};
                 const int kl = c8 * 8;
                 const int gk = kl >> 7;
@@ -405,7 +409,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_step_kernel(const __grid_con
             for (int idx = threadIdx.x; idx < MT * per_m; idx += nthr) {
                 const int m = idx / per_m, c8 = idx - m * per_m;
                 uint4 v = make_uint4(0u, 0u, 0u, 0u);
-                if (m < M) v = *reinterpret_cast<const uint4 *>(d.x + static_cast<size_t>(m) * K + c8 * 8);
+                if (m < M) v = *reinterpret_cast<const uint4 *>(d.x + static_cast<size_t>(m) * d.xs + c8 * 8);
                 const uint32_t pr[4] = {v.x, v.y, v.z, v.w};
                 const int kl = c8 * 8;
                 const int gk = kl >> 7;
@@ -439,17 +443,24 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_step_kernel(const __grid_con
         // token 0 only from v.x, v.z (MT = 1).
         // MT = 8: every lane holds its own tokens 2q, 2q + 1.
         constexpr int kGcLanes = MT == 8 ? 4 : (MT == 4 ? 2 : 1);
+        // A K segment after the first adds its sum to the fp16 y of the ones
+        // before it (one more rounding of the partial sum).
+        const bool accum = d.accum != 0;
+        auto put = [&](size_t idx, float v) {
+            if (accum) v += __half2float(d.y[idx]);
+            d.y[idx] = __float2half_rn(v);
+        };
         auto gc_store = [&](int tile, float4 v) {
             if (q >= kGcLanes) return;
             const int n0 = tile * kRows + row, n1 = n0 + 8;
             const int t0 = MT >= 4 ? 2 * q : 0, t1 = t0 + 1;
             if (n0 < N) {
-                if (t0 < M) d.y[static_cast<size_t>(t0) * N + n0] = __float2half_rn(v.x);
-                if (MT > 1 && t1 < M) d.y[static_cast<size_t>(t1) * N + n0] = __float2half_rn(v.y);
+                if (t0 < M) put(static_cast<size_t>(t0) * N + n0, v.x);
+                if (MT > 1 && t1 < M) put(static_cast<size_t>(t1) * N + n0, v.y);
             }
             if (n1 < N) {
-                if (t0 < M) d.y[static_cast<size_t>(t0) * N + n1] = __float2half_rn(v.z);
-                if (MT > 1 && t1 < M) d.y[static_cast<size_t>(t1) * N + n1] = __float2half_rn(v.w);
+                if (t0 < M) put(static_cast<size_t>(t0) * N + n1, v.z);
+                if (MT > 1 && t1 < M) put(static_cast<size_t>(t1) * N + n1, v.w);
             }
         };
 
@@ -699,6 +710,9 @@ tern_status launch_chunk(const DeviceInfo &dev, const MatDesc *md, int count, in
         d.K = md[i].K;
         d.tile0 = tiles;
         d.ntile = (md[i].N + kRows - 1) / kRows;
+        const int kfull = md[i].kfull > 0 ? md[i].kfull : md[i].K;
+        d.xs = kfull;
+        d.accum = md[i].accum;
         tiles += d.ntile;
         total_units += static_cast<long long>(d.ntile) * (md[i].K / 1024);
         kmax = std::max(kmax, md[i].K);
@@ -708,7 +722,7 @@ tern_status launch_chunk(const DeviceInfo &dev, const MatDesc *md, int count, in
             // copy brings both 512-k boxes of a unit
             const uint64_t sdims[3] = {static_cast<uint64_t>(kBox), static_cast<uint64_t>(md[i].N),
                                        static_cast<uint64_t>(md[i].K / 512)};
-            const uint64_t sstr[2] = {static_cast<uint64_t>(md[i].K / 4), static_cast<uint64_t>(kBox)};
+            const uint64_t sstr[2] = {static_cast<uint64_t>(kfull / 4), static_cast<uint64_t>(kBox)};
             const uint32_t sbox[3] = {static_cast<uint32_t>(kBox), static_cast<uint32_t>(kRows), 2};
             st = encode_tiled_3d(&p.m[i].smap, CU_TENSOR_MAP_DATA_TYPE_UINT8, md[i].slots, sdims, sstr, sbox,
                                  CU_TENSOR_MAP_SWIZZLE_128B);
@@ -716,18 +730,19 @@ tern_status launch_chunk(const DeviceInfo &dev, const MatDesc *md, int count, in
             // the bit matrix [N rows][K/8 bytes]: one 128-byte box is a unit's row
             st = encode_tiled_2d(&p.m[i].smap, CU_TENSOR_MAP_DATA_TYPE_UINT8, md[i].slots,
                                  static_cast<uint64_t>(md[i].K / 8), static_cast<uint64_t>(md[i].N),
-                                 static_cast<uint64_t>(md[i].K / 8), kBox, kRows, CU_TENSOR_MAP_SWIZZLE_128B);
+                                 static_cast<uint64_t>(kfull / 8), kBox, kRows, CU_TENSOR_MAP_SWIZZLE_128B);
         } else {
             // the base-3 bytes [N rows][R bytes], R = 208 K / 1024: one
             // 208-byte box is a unit's row (a multiple of 16 bytes)
             const uint64_t R = static_cast<uint64_t>(md[i].K / 1024) * kT5Row;
+            const uint64_t Rfull = static_cast<uint64_t>(kfull / 1024) * kT5Row;
             st = encode_tiled_2d(&p.m[i].smap, CU_TENSOR_MAP_DATA_TYPE_UINT8, md[i].slots, R,
-                                 static_cast<uint64_t>(md[i].N), R, kT5Row, kRows, CU_TENSOR_MAP_SWIZZLE_NONE);
+                                 static_cast<uint64_t>(md[i].N), Rfull, kT5Row, kRows, CU_TENSOR_MAP_SWIZZLE_NONE);
         }
         if (st != TERN_OK) return st;
         const int G = md[i].K / kGroup;
         st = encode_tiled_2d(&p.m[i].cmap, CU_TENSOR_MAP_DATA_TYPE_UINT16, md[i].scales, static_cast<uint64_t>(G),
-                             static_cast<uint64_t>(md[i].N), static_cast<uint64_t>(G) * 2, kSG, kRows,
+                             static_cast<uint64_t>(md[i].N), static_cast<uint64_t>(kfull / kGroup) * 2, kSG, kRows,
                              CU_TENSOR_MAP_SWIZZLE_NONE);
         if (st != TERN_OK) return st;
     }

@@ -61,6 +61,11 @@ struct MatDesc {
     const __half *scales;
     __half *y;
     int N, K;
+    // Step kernel only: the full row length of x, slots and scales when the
+    // product covers a K segment of a wider matrix (0: K), and whether the
+    // result is added to y instead of written.
+    int kfull = 0;
+    int accum = 0;
 };
 // Bandwidth-bound product for M in [1,8] over `count` matrices in one launch:
 // TMA-staged kernel (default) and the register-ring kernel (variant 1).

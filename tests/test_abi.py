@@ -167,8 +167,8 @@ def test_step_rejects(lib, fn):
     arr[0].x = None
     assert lib.tern_gemv_step(arr, 3, 1, None) == 1
     arr[0].x = A
-    arr[1].K = 40960                     # 4 x 40960 x 2 bytes of x do not fit beside the rings
-    assert lib.tern_gemv_step(arr, 3, 4, None) == 3
+    arr[1].K = 204800                    # x beyond eight K segments that fit shared memory
+    assert lib.tern_gemv_step(arr, 3, mmax, None) == 3
 
 
 def test_b1_pack_rejects(lib):

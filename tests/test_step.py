@@ -150,8 +150,8 @@ def test_timeout_reported_and_context_survives(T, orc):
 @pytest.mark.parametrize("grid", [0, 5])
 def test_verify_batch_mixed(T, orc, M, grid):
     """M token rows (M = 3 runs padded to 4, 5..8 padded to 8; at M > 4 the
-    K = 17408 product does not fit eight rows of x and runs as two passes of
-    4 and M - 4 rows): every output of every token."""
+    K = 17408 product does not fit eight rows of x and runs as K segments
+    whose sums are added to y): every output of every token."""
     shapes = [(1024, 1), (2048, 17), (5120, 100), (3072, 333), (6144, 64), (17408, 40), (4096, 129)]
     mats, refs = make_mats(orc, shapes, seed=7500 + 10 * M + grid, M=M)
     T.tern_set_option(T.TERN_OPT_GEMV_GRID, grid)
@@ -222,3 +222,16 @@ def test_chained_calls_see_complete_inputs(T):
     want = ya + yb + yc
     for i, (a, b) in enumerate(zip(got, want)):
         assert torch.equal(a, b), i
+
+
+@pytest.mark.parametrize("M", [1, 4, 8])
+def test_long_rows_run_as_k_segments(T, orc, M):
+    """Rows far longer than the staged x allows (K = 65536 at M = 1 and 4,
+    K = 40960 at M = 8) run as K segments; mixed with short products in one
+    call; every output."""
+    K = 65536 if M < 8 else 40960
+    shapes = [(K, 48), (2048, 33), (K, 17)]
+    mats, refs = make_mats(orc, shapes, seed=7800 + M, M=M)
+    T.tern_gemv_step(mats, M)
+    T.tern_sync_status()
+    check_all(orc, mats, refs, f"step K segments M={M}")

@@ -126,9 +126,7 @@ def test_decode_layer_and_head(T, orc):
 @pytest.mark.parametrize("M", [2, 3, 4, 8])
 @pytest.mark.parametrize("grid", [0, 5])
 def test_verify_batch_mixed(T, orc, M, grid):
-    shapes = [(1024, 1), (2048, 17), (5120, 100), (3072, 333), (6144, 64), (4096, 129)]
-    if M == 2:
-        shapes.append((17408, 40))
+    shapes = [(1024, 1), (2048, 17), (5120, 100), (3072, 333), (6144, 64), (4096, 129), (17408, 40)]
     mats, refs = make_mats(orc, shapes, seed=9500 + 10 * M + grid, M=M)
     T.tern_set_option(T.TERN_OPT_GEMV_GRID, grid)
     try:
@@ -140,15 +138,15 @@ def test_verify_batch_mixed(T, orc, M, grid):
 
 
 def test_shared_memory_limit_is_a_shape_error(T):
-    """M = 4 at K = 17408 leaves no room beside the decode table: refused
-    before any launch."""
-    K, N = 17408, 16
-    x = torch.zeros(4, K, dtype=torch.float16, device="cuda")
-    packed = torch.zeros(N, 3536, dtype=torch.uint8, device="cuda")
+    """A row so long that even eight K segments leave x too large for the
+    room beside the decode table is refused before any launch."""
+    K, N = 204800, 16
+    x = torch.zeros(8, K, dtype=torch.float16, device="cuda")
+    packed = torch.zeros(N, 208 * K // 1024, dtype=torch.uint8, device="cuda")
     sc = torch.zeros(N, K // 128, dtype=torch.float16, device="cuda")
-    y = torch.zeros(4, N, dtype=torch.float16, device="cuda")
+    y = torch.zeros(8, N, dtype=torch.float16, device="cuda")
     with pytest.raises(T.TernError) as ei:
-        T.tern_t5_gemv_step([(x, packed, sc, y)], 4)
+        T.tern_t5_gemv_step([(x, packed, sc, y)], 8)
     assert ei.value.status == T.TERN_ERR_SHAPE
 
 
