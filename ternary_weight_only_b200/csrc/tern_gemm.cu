@@ -9,19 +9,22 @@
 // section "Technical features").
 //
 // Design.  The MMA computes the transposed tile D[n][m] = sum_k W[n][k] x[m][k]:
-//  * A operand = 128 weight rows x 64 k per step, held in TENSOR MEMORY.  Each
-//    of the 128 unpack threads owns one weight row: one 16-byte load brings
-//    the row's 64 codes, two instructions per pair turn them into exact fp16
-//    t (the LOP3/HFMA2 construction of the bandwidth kernel), a byte permute
-//    puts them in k order, one HMUL2 applies the row's fp16 group scale (s*t
-//    is exact: t is -1, 0 or +1), and one tcgen05.st writes the 32 columns.
-//    The unpacked weights never touch shared memory or HBM.
+//  * A operand = 128 weight rows x 64 k per step, held in TENSOR MEMORY.  Two
+//    of the 256 unpack threads share a weight row, one half of the step each:
+//    one 8-byte load brings 32 codes, two instructions per pair turn them
+//    into exact fp16 t (the LOP3/HFMA2 construction of the bandwidth kernel),
+//    a byte permute puts them in k order, one HMUL2 applies the row's fp16
+//    group scale (s*t is exact: t is -1, 0 or +1), and one tcgen05.st writes
+//    16 columns.  Two unpack warps per tensor-memory lane quarter (one per
+//    half) let one hide the other's latencies.  The unpacked weights never
+//    touch shared memory or HBM.
 //  * B operand = 256 token rows x 64 k of x, brought by TMA into shared memory
 //    in the 128-byte-swizzled K-major layout the MMA reads directly.
 //  * D = 128 x 256 fp32 accumulator in tensor memory; one thread issues
 //    tcgen05.mma (M=128, N=256, K=16) four times per k step.
 //  * Producer (TMA), MMA issuer and unpack warps run a 4-stage mbarrier
-//    pipeline; the unpack warps then drain D with tcgen05.ld and write fp16.
+//    pipeline; the unpack warps then drain D with tcgen05.ld and write fp16
+//    (the two warps of a lane quarter take 128 token columns each).
 //  * Every wait is bounded: past the limit the waiting thread records
 //    TERN_ERR_TIMEOUT in a device-side status word, the CTA stops issuing
 //    work, waits (bounded) for its own copies and MMAs in flight, releases its
@@ -42,7 +45,8 @@ constexpr int kTN = 128;       // weight rows per tile (MMA M)
 constexpr int kTM = 256;       // token rows per tile (MMA N)
 constexpr int kBK = 64;        // k per pipeline step (one 128-byte swizzle row of fp16)
 constexpr int kStages = 4;
-constexpr int kThreads = 192;  // warp 0: TMA, warp 1: MMA + TMEM owner, warps 2..5: unpack + epilogue
+constexpr int kThreads = 320;  // warp 0: TMA, warp 1: MMA + TMEM owner, warps 2..9: unpack + epilogue
+constexpr int kUnpackWarps = 8;
 constexpr int kXStageBytes = kTM * kBK * 2;  // 32 KB
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kDCol = 0;        // accumulator: columns [0, 256)
@@ -101,14 +105,12 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t addr) {
            (static_cast<uint64_t>(2) << 61);
 }
 
-__device__ __forceinline__ void tmem_st_x32(uint32_t taddr, const uint32_t (&v)[32]) {
+__device__ __forceinline__ void tmem_st_x16(uint32_t taddr, const uint32_t (&v)[16]) {
     asm volatile(
-        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, "
-        "%13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};"
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, "
+        "%13, %14, %15, %16};"
         ::"r"(taddr), "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]),
-        "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15]),
-        "r"(v[16]), "r"(v[17]), "r"(v[18]), "r"(v[19]), "r"(v[20]), "r"(v[21]), "r"(v[22]), "r"(v[23]),
-        "r"(v[24]), "r"(v[25]), "r"(v[26]), "r"(v[27]), "r"(v[28]), "r"(v[29]), "r"(v[30]), "r"(v[31])
+        "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
         : "memory");
 }
 
@@ -170,7 +172,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; s++) {
             mbar_init(&full_x[s], 1);
-            mbar_init(&full_a[s], 4);
+            mbar_init(&full_a[s], kUnpackWarps);
             mbar_init(&empty[s], 1);
         }
         mbar_init(d_full, 1);
@@ -239,7 +241,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__
         }
     } else {
         // ---------------- unpack (A producer), then epilogue ----------------
-        const int q = warp & 3;  // tensor-memory lane quarter this warp may access
+        const int q = warp & 3;         // tensor-memory lane quarter this warp may access
+        const int hh = (warp - 2) >> 2;  // which half of a k step (32 codes, 16 columns) it unpacks
         const int row = q * 32 + lane;
         const int n = n0 + row;
         const int nld = n < p.N ? n : p.N - 1;
@@ -247,12 +250,13 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__
         const int G = p.K / kGroup;
         const uint8_t *srow = p.slots + static_cast<size_t>(nld) * K4;
         const unsigned short *scrow = reinterpret_cast<const unsigned short *>(p.scales) + static_cast<size_t>(nld) * G;
-        uint4 ring[kRingK];
+        uint2 ring[kRingK];
         uint32_t sring[kRingK];
+        const uint8_t *hrow = srow + hh * 8;
 #pragma unroll
         for (int u = 0; u < kRingK; u++) {
             if (u < nk) {
-                ring[u] = __ldg(reinterpret_cast<const uint4 *>(srow + u * 16));
+                ring[u] = __ldg(reinterpret_cast<const uint2 *>(hrow + u * 16));
                 sring[u] = __ldg(scrow + (u * kBK) / kGroup);
             }
         }
@@ -265,23 +269,21 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__
                 if (i < nk && ok) {
                     const int s = i % kStages;
                     const uint32_t ph = (i / kStages) & 1;
-                    const uint4 wv = ring[u];
+                    const uint2 wv = ring[u];
                     const uint32_t sc = sring[u];
                     if (i + kRingK < nk) {
-                        ring[u] = __ldg(reinterpret_cast<const uint4 *>(srow + (i + kRingK) * 16));
+                        ring[u] = __ldg(reinterpret_cast<const uint2 *>(hrow + (i + kRingK) * 16));
                         sring[u] = __ldg(scrow + ((i + kRingK) * kBK) / kGroup);
                     }
-                    uint32_t v[32];
+                    uint32_t v[16];
                     const uint32_t s2 = sc | (sc << 16);
                     unpack_word_scaled(wv.x, s2, v);
                     unpack_word_scaled(wv.y, s2, v + 8);
-                    unpack_word_scaled(wv.z, s2, v + 16);
-                    unpack_word_scaled(wv.w, s2, v + 24);
                     // tcgen05.st is warp-collective: take the decision warp-wide.
                     ok = __all_sync(0xffffffffu, mbar_wait(&empty[s], ph ^ 1, deadline, abort_flag));
                     if (ok) {
                         tc_fence_after();
-                        tmem_st_x32(tmem + lane_base + kACol + s * (kBK / 2), v);
+                        tmem_st_x16(tmem + lane_base + kACol + s * (kBK / 2) + hh * 16, v);
                         asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
                         tc_fence_before();
                         __syncwarp();
@@ -295,7 +297,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__
         if (ok) {
             tc_fence_after();
 #pragma unroll 1
-            for (int c0 = 0; c0 < kTM; c0 += 32) {
+            for (int c0 = hh * (kTM / 2); c0 < (hh + 1) * (kTM / 2); c0 += 32) {
                 uint32_t v[32];
                 tmem_ld_x32(tmem + lane_base + kDCol + c0, v);
                 asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
