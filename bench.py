@@ -783,8 +783,9 @@ def run_tern(args):
     e2e_value = ws * total_bytes / (e2e_ms * 1e-3) / 1e9
 
     # ---- per-shape breakdown (rank 0 only, outside the timed region) ----
+    # (one GPU only: under torchrun the other GPUs would sit idle meanwhile)
     rows = None
-    if rank == 0 and not args.no_rows:
+    if rank == 0 and ws == 1 and not args.no_rows:
         rows = proj_rows(T, model, peak_gbs, l2)
         rows.update(pack_rows(T, peak_gbs))
         rows.update(b1_rows(T, model, peak_gbs, (clocks.summary() or {}).get("sm_mhz")))
