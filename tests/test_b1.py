@@ -177,3 +177,14 @@ def test_timeout_reported_and_context_survives(T, orc):
     T.tern_b1_gemv_step(mats)
     T.tern_sync_status()
     check_all(orc, mats, refs, "b1 step after timeout")
+
+
+@pytest.mark.parametrize("M", [1, 4])
+def test_long_rows_run_as_k_segments(T, orc, M):
+    """Rows longer than the staged x allows run as K segments whose sums are
+    added to y; mixed with a short product in one call; every output."""
+    shapes = [(98304, 40), (2048, 33)]
+    mats, refs = make_mats(orc, shapes, seed=8700 + M, M=M)
+    T.tern_b1_gemv_step(mats, M)
+    T.tern_sync_status()
+    check_all(orc, mats, refs, f"b1 step K segments M={M}")

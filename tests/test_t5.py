@@ -191,3 +191,15 @@ def test_timeout_reported_and_context_survives(T, orc):
     T.tern_t5_gemv_step(mats)
     T.tern_sync_status()
     check_all(orc, mats, refs, "t5 step after timeout")
+
+
+@pytest.mark.parametrize("M", [1, 8])
+def test_long_rows_run_as_k_segments(T, orc, M):
+    """Rows longer than the staged x and the decode table allow run as K
+    segments whose sums are added to y; every output."""
+    K = 65536 if M == 1 else 24576
+    shapes = [(K, 40), (2048, 33)]
+    mats, refs = make_mats(orc, shapes, seed=9700 + M, M=M)
+    T.tern_t5_gemv_step(mats, M)
+    T.tern_sync_status()
+    check_all(orc, mats, refs, f"t5 step K segments M={M}")
