@@ -41,6 +41,17 @@ tern_status current_device(DeviceInfo *out) {
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
     if (dev < 0 || dev >= 64) return fail(TERN_ERR_DEVICE, "device ordinal %d out of range", dev);
+    // The tensor maps are encoded through the driver API, which needs a
+    // context current in the calling thread; a host thread whose first CUDA
+    // call is one of ours has none yet.  cudaFree(nullptr) binds the device's
+    // primary context when no context is current (and leaves a current one
+    // alone), once per thread and device.
+    thread_local bool t_bound[64] = {};
+    if (!t_bound[dev]) {
+        e = cudaFree(nullptr);
+        if (e != cudaSuccess) return cuda_fail(e, "binding the device context");
+        t_bound[dev] = true;
+    }
     std::lock_guard<std::mutex> lock(g_dev_mu);
     if (!g_dev_valid[dev]) {
         DeviceInfo d;
@@ -360,7 +371,7 @@ tern_status gemv_step_api(const tern_gemv_desc *descs, int32_t count, int64_t M,
     const int mmax = fmt == 1 ? 4 : 8;
     if (M < 1 || M > mmax)
         return fail(TERN_ERR_SHAPE, "%s takes M in 1..%d (got %lld)", name, mmax, static_cast<long long>(M));
-    static MatDesc d[TERN_MAX_STEP];
+    thread_local MatDesc d[TERN_MAX_STEP];  // per host thread: calls may run concurrently
     for (int i = 0; i < count; i++) {
         tern_status st = check_nk(descs[i].N, descs[i].K);
         if (st != TERN_OK) return st;
@@ -378,7 +389,7 @@ tern_status gemv_step_api(const tern_gemv_desc *descs, int32_t count, int64_t M,
     // rings run as K segments of whole 1024-k units that do, in calls of
     // their own: segment 0 (with every product that fits) writes y, each
     // later segment adds its sum to y.  Each weight is still read once.
-    static MatDesc seg[8][TERN_MAX_STEP];
+    thread_local MatDesc seg[8][TERN_MAX_STEP];
     int nseg_max = 1, n[8] = {0};
     const int unit_bytes = fmt == 0 ? 256 : (fmt == 1 ? 128 : 208);  // weight bytes of one 1024-k row unit
     for (int i = 0; i < count; i++) {

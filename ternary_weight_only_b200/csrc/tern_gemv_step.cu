@@ -696,7 +696,7 @@ namespace {
 // One launch over md[0..count) (count <= kMaxPer).
 tern_status launch_chunk(const DeviceInfo &dev, const MatDesc *md, int count, int M, int fmt, bool first,
                          cudaStream_t stream) {
-    static SParams p;  // large (parameter space); filled on the host for each launch
+    thread_local SParams p;  // large (parameter space); filled on the host for each launch, per host thread
     std::memset(&p, 0, sizeof(p));
     const int mt = step_mt(M);
     int kmax = 0;

@@ -235,3 +235,53 @@ def test_long_rows_run_as_k_segments(T, orc, M):
     T.tern_gemv_step(mats, M)
     T.tern_sync_status()
     check_all(orc, mats, refs, f"step K segments M={M}")
+
+
+def test_concurrent_calls_from_two_host_threads(T):
+    """Two host threads call tern_gemv_step at the same time on their own
+    streams (120 products each, two launches per call); every output equals
+    the same call made alone."""
+    import threading
+    from ternary_weight_only_b200 import synth
+    g = synth.gen(7900, "cuda")
+    sets = []
+    for t in range(2):
+        mats = []
+        for j in range(120):
+            N = 64 + 16 * ((j + t) % 5)
+            codes = synth.codes_sparse(N, 1024 * (1 + j % 3), g, device="cuda")
+            slots, sc = T.tern_pack_g128(codes, synth.scales_uniform(N, codes.shape[1], g, device="cuda"))
+            x = synth.activations(1, codes.shape[1], g, device="cuda")[0]
+            mats.append((x, slots, sc, torch.empty(N, dtype=torch.float16, device="cuda")))
+        sets.append(mats)
+    torch.cuda.synchronize()
+    # alone, one after the other
+    want = []
+    for mats in sets:
+        T.tern_gemv_step(mats)
+        T.tern_sync_status()
+        want.append([m[3].clone() for m in mats])
+        for m in mats:
+            m[3].fill_(float("nan"))
+    torch.cuda.synchronize()
+    streams = [torch.cuda.Stream() for _ in sets]
+    errors = []
+
+    def worker(i):
+        try:
+            for _ in range(20):
+                T.tern_gemv_step(sets[i], stream=streams[i])
+            streams[i].synchronize()
+        except Exception as e:  # reported below
+            errors.append(e)
+
+    threads = [threading.Thread(target=worker, args=(i,)) for i in range(2)]
+    for th in threads:
+        th.start()
+    for th in threads:
+        th.join()
+    assert not errors, errors
+    T.tern_sync_status()
+    for mats, w in zip(sets, want):
+        for m, y in zip(mats, w):
+            assert torch.equal(m[3], y)
