@@ -666,7 +666,9 @@ StepKernel step_kernel(int mt, int f) {
     if (f == 0)
         return mt == 1 ? gemv_step_kernel<1, 0>
                        : (mt == 2 ? gemv_step_kernel<2, 0> : (mt == 4 ? gemv_step_kernel<4, 0> : gemv_step_kernel<8, 0>));
-    if (f == 1) return mt == 1 ? gemv_step_kernel<1, 1> : (mt == 2 ? gemv_step_kernel<2, 1> : gemv_step_kernel<4, 1>);
+    if (f == 1)  // no eight-token form for the 1-bit weights
+        return mt == 1 ? gemv_step_kernel<1, 1>
+                       : (mt == 2 ? gemv_step_kernel<2, 1> : (mt == 4 ? gemv_step_kernel<4, 1> : nullptr));
     return mt == 1 ? gemv_step_kernel<1, 2>
                    : (mt == 2 ? gemv_step_kernel<2, 2> : (mt == 4 ? gemv_step_kernel<4, 2> : gemv_step_kernel<8, 2>));
 }
@@ -804,7 +806,8 @@ tern_status launch_gemv_step(const MatDesc *md, int count, int M, int fmt, cudaS
     tern_status st = current_device(&dev);
     if (st != TERN_OK) return st;
     if (fmt < 0 || fmt > 2) return fail(TERN_ERR_INVALID_ARG, "step kernel: unknown weight format %d", fmt);
-    if (!gemv_step_supports(md, count, M, fmt)) return fail(TERN_ERR_SHAPE, "step kernel: unsupported shapes");
+    if (!gemv_step_supports(md, count, M, fmt) || step_kernel(step_mt(M), fmt) == nullptr)
+        return fail(TERN_ERR_SHAPE, "step kernel: unsupported shapes");
     const int mi = mt_index(step_mt(M));
     if (!g_attr_step[dev.device][fmt][mi]) {
         cudaError_t e = cudaFuncSetAttribute(step_kernel(step_mt(M), fmt), cudaFuncAttributeMaxDynamicSharedMemorySize,
