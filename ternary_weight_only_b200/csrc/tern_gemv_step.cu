@@ -108,16 +108,18 @@ struct SParams {
 
 // Shared memory layout (bytes from the 128-aligned base).
 __host__ __device__ constexpr int bar_off() { return 0; }
-__host__ __device__ constexpr int rec_off() { return kW * kMaxNS * 8; }               // [kW][2][8][4] float4
-__host__ __device__ constexpr int rtile_off() { return rec_off() + kW * 2 * 8 * 4 * 16; }  // [kW][2] int
-__host__ __device__ constexpr int wmax_off() { return rtile_off() + kW * 2 * 4; }     // [kW] uint
-__host__ __device__ constexpr int d1_off() { return wmax_off() + kW * 4; }            // [kmax / 128 * 8] float
-// d1 holds one float per (set, column): kmax / 1024 * MT sets of 8, MT <= 8
-__host__ __device__ constexpr int lut_off(int kmax) { return d1_off() + (kmax / 128) * 32 + 64; }
-__host__ __device__ constexpr int xs_off(int kmax, int f) { return lut_off(kmax) + lut_bytes(f); }
+// Lanes of a quad that hold distinct tokens after a tile's lane reduction.
+__host__ __device__ constexpr int gc_lanes(int mt) { return mt == 8 ? 4 : (mt == 4 ? 2 : 1); }
+__host__ __device__ constexpr int rec_off() { return kW * kMaxNS * 8; }  // [kW][2][8][gc_lanes] float4
+__host__ __device__ constexpr int rtile_off(int mt) { return rec_off() + kW * 2 * 8 * gc_lanes(mt) * 16; }  // [kW][2] int
+__host__ __device__ constexpr int wmax_off(int mt) { return rtile_off(mt) + kW * 2 * 4; }  // [kW] uint
+__host__ __device__ constexpr int d1_off(int mt) { return wmax_off(mt) + kW * 4; }
+// d1 holds one float per (set, column): kmax / 1024 * mt sets of 8 columns
+__host__ __device__ constexpr int lut_off(int kmax, int mt) { return d1_off(mt) + kmax / 32 * mt + 64; }
+__host__ __device__ constexpr int xs_off(int kmax, int mt, int f) { return lut_off(kmax, mt) + lut_bytes(f); }
 // staged x: MT token rows (M real, the rest zero)
 __host__ __device__ constexpr int ring_off(int kmax, int mt, int f) {
-    return (xs_off(kmax, f) + kmax * 2 * mt + 1023) & ~1023;
+    return (xs_off(kmax, mt, f) + kmax * 2 * mt + 1023) & ~1023;
 }
 size_t smem_bytes(int kmax, int mt, int ns, int f) {
     return 1024 + static_cast<size_t>(ring_off(kmax, mt, f)) + static_cast<size_t>(kW) * ns * stage_bytes(f);
@@ -232,11 +234,11 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_step_kernel(const __grid_con
     uint8_t *base = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     uint64_t *full = reinterpret_cast<uint64_t *>(base + bar_off());  // [kW][kMaxNS]
     float *rec = reinterpret_cast<float *>(base + rec_off());
-    int *rec_tile = reinterpret_cast<int *>(base + rtile_off());
-    unsigned int *wmax = reinterpret_cast<unsigned int *>(base + wmax_off());
-    float *d1 = reinterpret_cast<float *>(base + d1_off());
-    __half *xs = reinterpret_cast<__half *>(base + xs_off(p.kmax, F));
-    uint32_t *lut = reinterpret_cast<uint32_t *>(base + lut_off(p.kmax));
+    int *rec_tile = reinterpret_cast<int *>(base + rtile_off(MT));
+    unsigned int *wmax = reinterpret_cast<unsigned int *>(base + wmax_off(MT));
+    float *d1 = reinterpret_cast<float *>(base + d1_off(MT));
+    __half *xs = reinterpret_cast<__half *>(base + xs_off(p.kmax, MT, F));
+    uint32_t *lut = reinterpret_cast<uint32_t *>(base + lut_off(p.kmax, MT));
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int g = lane >> 2, q = lane & 3;
@@ -280,7 +282,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_step_kernel(const __grid_con
     // The ring takes what this CTA's largest staged x leaves (2..4 stages).
     int kcta = 1024;
     for (int i = i0; T0 < T1 && i < p.count && p.d[i].tile0 < T1; i++) kcta = max(kcta, p.d[i].K);
-    const uint32_t roff = (static_cast<uint32_t>(xs_off(p.kmax, F)) + 2u * MT * kcta + 1023u) & ~1023u;
+    const uint32_t roff = (static_cast<uint32_t>(xs_off(p.kmax, MT, F)) + 2u * MT * kcta + 1023u) & ~1023u;
     const int ns = min(kMaxNS, static_cast<int>((p.smem_usable - roff) / (kW * kStageBytes)));
     const int M = p.M;
     uint8_t *ring = base + roff;
@@ -442,7 +444,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_step_kernel(const __grid_con
         // tokens t0, t1), t0 = 2q, t1 = 2q + 1 (MT = 4), 0, 1 (MT = 2), or
         // token 0 only from v.x, v.z (MT = 1).
         // MT = 8: every lane holds its own tokens 2q, 2q + 1.
-        constexpr int kGcLanes = MT == 8 ? 4 : (MT == 4 ? 2 : 1);
+        constexpr int kGcLanes = gc_lanes(MT);
         // A K segment after the first adds its sum to the fp16 y of the ones
         // before it (one more rounding of the partial sum).
         const bool accum = d.accum != 0;
@@ -605,7 +607,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_step_kernel(const __grid_con
                     if (!dead) gc_store(tile, vv);
                 } else {
                     const int slot = (tl == tl_first) ? 0 : 1;
-                    if (q < kGcLanes) *reinterpret_cast<float4 *>(rec + (((warp * 2 + slot) * 8 + g) * 4 + q) * 4) = vv;
+                    if (q < kGcLanes)
+                        *reinterpret_cast<float4 *>(rec + (((warp * 2 + slot) * 8 + g) * kGcLanes + q) * 4) = vv;
                     if (lane == 0) rec_tile[warp * 2 + slot] = dead ? -2 : tile;
                 }
                 acc[0] = acc[1] = acc[2] = acc[3] = 0.f;
@@ -636,7 +639,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_step_kernel(const __grid_con
                 for (int w2 = warp; w2 < kW; w2++)
                     for (int s2i = 0; s2i < 2; s2i++) {
                         if (rec_tile[w2 * 2 + s2i] != tile) continue;
-                        const float4 o = *reinterpret_cast<const float4 *>(rec + (((w2 * 2 + s2i) * 8 + g) * 4 + q) * 4);
+                        const float4 o =
+                            *reinterpret_cast<const float4 *>(rec + (((w2 * 2 + s2i) * 8 + g) * kGcLanes + q) * 4);
                         sum.x += o.x;
                         sum.y += o.y;
                         sum.z += o.z;
