@@ -16,7 +16,8 @@
 //    a byte permute puts them in k order, one HMUL2 applies the row's fp16
 //    group scale (s*t is exact: t is -1, 0 or +1), and one tcgen05.st writes
 //    16 columns.  Two unpack warps per tensor-memory lane quarter (one per
-//    half) let one hide the other's latencies.  The unpacked weights never
+//    half) let one hide the other's latencies, and a warp announces a stage
+//    one k step late, so that its store completes while it unpacks the next.  The unpacked weights never
 //    touch shared memory or HBM.
 //  * B operand = 256 token rows x 64 k of x, brought by TMA into shared memory
 //    in the 128-byte-swizzled K-major layout the MMA reads directly.
@@ -262,6 +263,19 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__
         }
         const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
         bool ok = true;
+        // A stage is announced to the MMA issuer one k step late: the store
+        // into tensor memory of step i completes while step i + 1 is
+        // unpacked, then the warp waits for it and arrives on step i's
+        // barrier (before waiting for step i + 1's stage to be free).
+        int pending = -1;
+        auto announce = [&]() {
+            if (pending < 0) return;
+            asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&full_a[pending]);
+            pending = -1;
+        };
         for (int ib = 0; ib < nk && ok; ib += kRingK) {
 #pragma unroll
             for (int u = 0; u < kRingK; u++) {
@@ -279,18 +293,21 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__
                     const uint32_t s2 = sc | (sc << 16);
                     unpack_word_scaled(wv.x, s2, v);
                     unpack_word_scaled(wv.y, s2, v + 8);
+                    announce();
                     // tcgen05.st is warp-collective: take the decision warp-wide.
                     ok = __all_sync(0xffffffffu, mbar_wait(&empty[s], ph ^ 1, deadline, abort_flag));
                     if (ok) {
                         tc_fence_after();
                         tmem_st_x16(tmem + lane_base + kACol + s * (kBK / 2) + hh * 16, v);
-                        asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
-                        tc_fence_before();
-                        __syncwarp();
-                        if (lane == 0) mbar_arrive(&full_a[s]);
+                        pending = s;
                     }
                 }
             }
+        }
+        if (ok) {
+            announce();
+        } else {
+            asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");  // no store left in flight
         }
         // Epilogue: D[row][token] -> y[m0 + token][n]
         if (ok) ok = __all_sync(0xffffffffu, mbar_wait(d_full, 0, deadline, abort_flag) && !*abort_flag);
