@@ -146,7 +146,7 @@ def test_timeout_reported_and_context_survives(T, orc):
     check_all(orc, mats, refs, "step after timeout")
 
 
-@pytest.mark.parametrize("M", [2, 3, 4, 5, 6, 8])
+@pytest.mark.parametrize("M", [2, 3, 4, 5, 6, 7, 8])
 @pytest.mark.parametrize("grid", [0, 5])
 def test_verify_batch_mixed(T, orc, M, grid):
     """M token rows (M = 3 runs padded to 4, 5..8 padded to 8; at M > 4 the

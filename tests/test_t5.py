@@ -203,3 +203,25 @@ def test_long_rows_run_as_k_segments(T, orc, M):
     T.tern_t5_gemv_step(mats, M)
     T.tern_sync_status()
     check_all(orc, mats, refs, f"t5 step K segments M={M}")
+
+
+def test_invalid_bytes_give_finite_values_and_spare_other_rows(T, orc):
+    """Bytes 243..255 are invalid: the rows holding them get some finite
+    value, every other row is computed as the oracle computes it."""
+    from ternary_weight_only_b200 import synth
+    K, N = 2048, 64
+    x, codes, scales = synth.case(1, K, N, seed=9800, codes="sparse")
+    xn, cn, sn = np_inputs(x, codes, scales)
+    packed, sc, _, _ = orc.t5_pack(cn, sn)
+    bad_rows = [3, 17, 40]
+    for r, b in zip(bad_rows, (243, 250, 255)):
+        packed[r, 7] = b
+        packed[r, 26 * 9 + 25] = b
+    y = torch.full((N,), float("nan"), dtype=torch.float16, device="cuda")
+    T.tern_t5_gemv_step([(x[0].cuda(), torch.from_numpy(packed).cuda(), scales.cuda(), y)])
+    T.tern_sync_status()
+    got = y.float().cpu().double().numpy()
+    assert np.all(np.isfinite(got))
+    good = [n for n in range(N) if n not in bad_rows]
+    y_ref, bound = orc.t5_matmul(xn, packed[good], sc[good], threads=NCPU)
+    check_close(y[good].view(1, -1), y_ref, bound, "t5 rows without invalid bytes")
