@@ -453,10 +453,35 @@ def pin_t5_matmul(o):
     assert np.allclose(bound, np.abs(X) @ np.abs(W).T, rtol=1e-12, atol=1e-12)
 
 
+def pin_formats_agree(o):
+    """The same weights give bit-identical fp64 products whatever the
+    storage: ternary codes as 2-bit slots and as five trits per byte; +-1
+    codes as 2-bit slots, five per byte and 1-bit signs (the three oracle
+    paths share no packing code, so a slip in one shows as a difference)."""
+    rng = _rng(59)
+    M, K, N = 2, 384, 13
+    x = _f16bits(rng.standard_normal((M, K)))
+    scales = _f16bits(rng.uniform(-0.05, 0.05, size=(N, K // 128)))
+    tern = rng.integers(-1, 2, size=(N, K), dtype=np.int8)
+    sgn = rng.choice(np.array([-1, 1], dtype=np.int8), size=(N, K))
+    s2, sc2, _, _ = o.pack(tern, scales)
+    t5, sc5, _, _ = o.t5_pack(tern, scales)
+    y2, b2 = o.matmul(x, s2, sc2)
+    y5, b5 = o.t5_matmul(x, t5, sc5)
+    assert np.array_equal(y2, y5) and np.array_equal(b2, b5)
+    s2, sc2, _, _ = o.pack(sgn, scales)
+    t5, sc5, _, _ = o.t5_pack(sgn, scales)
+    b1, sc1, _, _ = o.b1_pack(sgn, scales)
+    ya, _ = o.matmul(x, s2, sc2)
+    yb, _ = o.t5_matmul(x, t5, sc5)
+    yc, _ = o.b1_matmul(x, b1, sc1)
+    assert np.array_equal(ya, yb) and np.array_equal(ya, yc)
+
+
 PINS = [pin_half_decode, pin_golden_bytes, pin_golden_matmul, pin_exhaustive_bytes,
         pin_roundtrip_random, pin_invalid_codes, pin_byte_count, pin_numpy_crosscheck,
         pin_row_sums, pin_exact_cases, pin_brute_force, pin_sampled_paths, pin_embed, pin_b1_format,
-        pin_b1_matmul, pin_t5_format, pin_t5_matmul]
+        pin_b1_matmul, pin_t5_format, pin_t5_matmul, pin_formats_agree]
 
 
 @pytest.mark.parametrize("pin", PINS, ids=lambda p: p.__name__)
