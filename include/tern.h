@@ -408,6 +408,12 @@ tern_status tern_sync_status(void *stream);
  *                          kernel, in 16-row x 1024-k units per consumer warp;
  *                          0 or n <= ring depth = none (the default: measured
  *                          slower)
+ *   TERN_OPT_STEP_FORM     arithmetic of the decode-step kernel for 2-bit
+ *                          slots at M = 1 and 2: 0 = default (the digit form:
+ *                          8-bit integer mma on weights unpacked four per
+ *                          instruction against activations split into four
+ *                          exact signed 8-bit digits), 1 = the fp16
+ *                          group-per-column form used for every other M
  *   TERN_OPT_TEST_STALL_US TESTS ONLY: the TMA loaders of the tensor-core and
  *                          the TMA-staged bandwidth kernels issue no loads, so
  *                          their waits can never complete, and every bounded
@@ -423,7 +429,8 @@ enum {
     TERN_OPT_TEST_STALL_US = 6,
     TERN_OPT_GEMV_VARIANT = 7,
     TERN_OPT_GEMV_GRID = 8,
-    TERN_OPT_GEMV_PREFETCH = 9
+    TERN_OPT_GEMV_PREFETCH = 9,
+    TERN_OPT_STEP_FORM = 10
 };
 tern_status tern_set_option(int option, int64_t value);
 

@@ -563,6 +563,10 @@ tern_status tern_set_option(int option, int64_t value) {
             return TERN_OK;
         case TERN_OPT_GEMV_GRID: g_opt.gemv_grid = static_cast<int>(value); return TERN_OK;
         case TERN_OPT_GEMV_PREFETCH: g_opt.gemv_prefetch = static_cast<int>(value); return TERN_OK;
+        case TERN_OPT_STEP_FORM:
+            if (value > 1) return fail(TERN_ERR_INVALID_ARG, "step form %lld", static_cast<long long>(value));
+            g_opt.step_form = static_cast<int>(value);
+            return TERN_OK;
         case TERN_OPT_TEST_STALL_US:
             g_gemm_skip_loads = value > 0 ? 1 : 0;
             g_gemm_timeout_ns = value > 0 ? static_cast<unsigned long long>(value) * 1000ull : 1000000000ull;

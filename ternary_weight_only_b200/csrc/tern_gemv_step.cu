@@ -26,7 +26,24 @@
 // several launches.  The ring runs ahead across piece boundaries: weights
 // never depend on the preceding launch or piece.
 //
-// Arithmetic: the group-per-column mma.sync form (tern_unpack_mma.cuh).
+// Arithmetic: the group-per-column mma.sync form (tern_unpack_mma.cuh), or,
+// for 2-bit slots at one or two token rows, the digit form below.
+//
+// Digit form (X8): mma.sync m16n8k32 with unsigned 8-bit weights and signed
+// 8-bit activations, exact 32-bit integer sums.  One AND of a slot word with
+// 0x03030303 << 2f leaves four bytes c * 4^f (field f of each byte: weights
+// 4b + f), so one instruction unpacks four weights and no shift is needed.
+// The activations become integers on a fixed point per 128-k group and token
+// row: X = rint(x * 2^(eC - 2f)) with eC = 29 - floor(log2 max|x|) of the
+// group, so the field factor 4^f cancels and |X| < 2^30; X is split into
+// four signed base-256 digits, and the eight mma columns carry (group or
+// token, digit) pairs.  Every X of an element within 2^13 of its group's
+// largest |x| is exact; smaller ones are off by at most 2^-24 of that largest
+// |x| (below the rounding of an fp32 sum).  A group's integer sums per digit
+// are exact, t = c - 1 is restored by starting each chain at minus the same
+// chain on the all-ones word, and the two digits a lane holds are joined as
+// d0 + 256 d1 (no overflow: |d| < 2^21) before one conversion to fp32 and
+// the multiply by the group scale and 2^(16 h - eC).
 //
 // The same kernel serves the 1-bit variant (weights in {-1, +1}, one bit
 // each, fp16 scale per 128 weights: "Bonsai 27B ternary / 1-bit
@@ -114,15 +131,23 @@ __host__ __device__ constexpr int rec_off() { return kW * kMaxNS * 8; }  // [kW]
 __host__ __device__ constexpr int rtile_off(int mt) { return rec_off() + kW * 2 * 8 * gc_lanes(mt) * 16; }  // [kW][2] int
 __host__ __device__ constexpr int wmax_off(int mt) { return rtile_off(mt) + kW * 2 * 4; }  // [kW] uint
 __host__ __device__ constexpr int d1_off(int mt) { return wmax_off(mt) + kW * 4; }
-// d1 holds one float per (set, column): kmax / 1024 * mt sets of 8 columns
-__host__ __device__ constexpr int lut_off(int kmax, int mt) { return d1_off(mt) + kmax / 32 * mt + 64; }
-__host__ __device__ constexpr int xs_off(int kmax, int mt, int f) { return lut_off(kmax, mt) + lut_bytes(f); }
-// staged x: MT token rows (M real, the rest zero)
-__host__ __device__ constexpr int ring_off(int kmax, int mt, int f) {
-    return (xs_off(kmax, mt, f) + kmax * 2 * mt + 1023) & ~1023;
+// d1 holds one float per (set, column): kmax / 1024 * mt sets of 8 columns.
+// Digit form: one 16-byte record per (set, lane q) -- minus the all-ones sums
+// of the lane's two columns and its factor 2^(16 (q & 1) - eC) -- for 4 (MT =
+// 1) or 8 (MT = 2) sets per 1024 k, then the exponents eC per (token, group).
+__host__ __device__ constexpr int d1_bytes(int kmax, int mt, bool x8) {
+    return x8 ? kmax / 4 * mt + ((kmax / 128 * mt + 15) & ~15) : kmax / 32 * mt;
 }
-size_t smem_bytes(int kmax, int mt, int ns, int f) {
-    return 1024 + static_cast<size_t>(ring_off(kmax, mt, f)) + static_cast<size_t>(kW) * ns * stage_bytes(f);
+__host__ __device__ constexpr int lut_off(int kmax, int mt, bool x8) { return d1_off(mt) + d1_bytes(kmax, mt, x8) + 64; }
+__host__ __device__ constexpr int xs_off(int kmax, int mt, int f, bool x8) { return lut_off(kmax, mt, x8) + lut_bytes(f); }
+// staged x: MT token rows (M real, the rest zero); fp16 (2 bytes per k and
+// row) or four signed digits (4 bytes per k and row)
+__host__ __device__ constexpr int xs_bytes(int k, int mt, bool x8) { return k * (x8 ? 4 : 2) * mt; }
+__host__ __device__ constexpr int ring_off(int kmax, int mt, int f, bool x8) {
+    return (xs_off(kmax, mt, f, x8) + xs_bytes(kmax, mt, x8) + 1023) & ~1023;
+}
+size_t smem_bytes(int kmax, int mt, int ns, int f, bool x8) {
+    return 1024 + static_cast<size_t>(ring_off(kmax, mt, f, x8)) + static_cast<size_t>(kW) * ns * stage_bytes(f);
 }
 
 // The 2-bit codes (c = digit, code i at bits 2i) of the five base-3 digits of
@@ -224,9 +249,14 @@ __device__ __forceinline__ void cursor_next(Cursor &c, const SParams &p, int T0,
 // MT = 8 (5..8 token rows; not for F = 1): the eight columns are the eight
 // tokens of one group, so a slice is eight sets of one group, each group's
 // eight-mma chain (group_mma) taken in turn, group by group.
-template <int MT, int F>
+// X8 (F = 0, MT = 1 or 2): the digit form; for MT = 1 set h of a 1024-k
+// unit is groups h and h + 4 (columns 4 (G / 4) + digit), for MT = 2 a set
+// is one group (columns 4 token + digit).
+template <int MT, int F, bool X8>
 __global__ void __launch_bounds__(kThreads, 1) gemv_step_kernel(const __grid_constant__ SParams p) {
+    static_assert(!X8 || (F == 0 && MT <= 2), "digit form: 2-bit slots, one or two token rows");
     constexpr int GPB = 8 / MT;  // groups per set
+    constexpr int kSPU = MT == 1 ? 4 : 8;  // digit form: sets per 1024-k unit
     constexpr int kSlotStage = slot_stage(F);
     constexpr int kStageBytes = stage_bytes(F);
     constexpr int kWords = F == 1 ? 2 : 4;  // weight words of a group a lane holds
@@ -237,8 +267,12 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_step_kernel(const __grid_con
     int *rec_tile = reinterpret_cast<int *>(base + rtile_off(MT));
     unsigned int *wmax = reinterpret_cast<unsigned int *>(base + wmax_off(MT));
     float *d1 = reinterpret_cast<float *>(base + d1_off(MT));
-    __half *xs = reinterpret_cast<__half *>(base + xs_off(p.kmax, MT, F));
-    uint32_t *lut = reinterpret_cast<uint32_t *>(base + lut_off(p.kmax, MT));
+    __half *xs = reinterpret_cast<__half *>(base + xs_off(p.kmax, MT, F, X8));
+    uint32_t *lut = reinterpret_cast<uint32_t *>(base + lut_off(p.kmax, MT, X8));
+    // digit form: staged digits, (set, q) records, exponents per (token, group)
+    uint8_t *xs8 = base + xs_off(p.kmax, MT, F, X8);
+    int4 *recs = reinterpret_cast<int4 *>(d1);
+    int8_t *egrp = reinterpret_cast<int8_t *>(base + d1_off(MT) + p.kmax / 4 * MT);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int g = lane >> 2, q = lane & 3;
@@ -282,7 +316,9 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_step_kernel(const __grid_con
     // The ring takes what this CTA's largest staged x leaves (2..4 stages).
     int kcta = 1024;
     for (int i = i0; T0 < T1 && i < p.count && p.d[i].tile0 < T1; i++) kcta = max(kcta, p.d[i].K);
-    const uint32_t roff = (static_cast<uint32_t>(xs_off(p.kmax, MT, F)) + 2u * MT * kcta + 1023u) & ~1023u;
+    const uint32_t roff =
+        (static_cast<uint32_t>(xs_off(p.kmax, MT, F, X8)) + static_cast<uint32_t>(xs_bytes(kcta, MT, X8)) + 1023u) &
+        ~1023u;
     const int ns = min(kMaxNS, static_cast<int>((p.smem_usable - roff) / (kW * kStageBytes)));
     const int M = p.M;
     uint8_t *ring = base + roff;
@@ -350,6 +386,89 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_step_kernel(const __grid_con
         const int K = d.K, N = d.N, B = K >> 10;
         // ---- stage x of matrix i: E from max |x|, pair order, all-ones sums ----
         __syncthreads();  // the previous piece is finished with xs, d1, rec
+        const __half *xlane = xs + lane * 8;
+        int E = 0;
+        if constexpr (X8) {
+            // ---- digit form: 16 consecutive k of one token row per thread ----
+            if (lane < 2) rec_tile[warp * 2 + lane] = -1;
+            const int nch = K >> 4;  // a multiple of 64: every warp runs whole iterations
+            for (int idx = threadIdx.x; idx < MT * nch; idx += nthr) {
+                const int m = idx / nch, c = idx - m * nch;
+                uint4 v0 = make_uint4(0u, 0u, 0u, 0u), v1 = v0;
+                if (m < M) {
+                    const __half *src = d.x + static_cast<size_t>(m) * d.xs + c * 16;
+                    v0 = *reinterpret_cast<const uint4 *>(src);
+                    v1 = *reinterpret_cast<const uint4 *>(src + 8);
+                }
+                const uint32_t wv[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+                // largest |x| of the 128-k group: the eight threads of a group
+                // are eight consecutive lanes (inf and NaN clamp to 65504)
+                uint32_t mx = 0;
+#pragma unroll
+                for (int e = 0; e < 8; e++) mx = __vmaxu2(mx, __vminu2(wv[e] & 0x7FFF7FFFu, 0x7BFF7BFFu));
+                mx = max(mx & 0xFFFFu, mx >> 16);
+                mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+                mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+                mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+                // eC = 29 - floor(log2 max|x|) (normal or subnormal max); 0 for an all-zero group
+                int eC = 0;
+                if (mx != 0) eC = 29 - (mx >= 0x400u ? static_cast<int>(mx >> 10) - 15 : (31 - __clz(mx)) - 24);
+                float fsc[4];
+#pragma unroll
+                for (int f = 0; f < 4; f++) fsc[f] = __int_as_float((127 + eC - 2 * f) << 23);
+                // digit words: w[s][f] holds digit s of the four x of field f
+                uint32_t w[4][4];
+#pragma unroll
+                for (int s2 = 0; s2 < 4; s2++)
+#pragma unroll
+                    for (int f = 0; f < 4; f++) w[s2][f] = 0u;
+#pragma unroll
+                for (int e = 0; e < 16; e++) {
+                    const int f = e & 3, b = e >> 2;
+                    const float xv = __half2float(__ushort_as_half(static_cast<unsigned short>(wv[e >> 1] >> (16 * (e & 1)))));
+                    int X = __float2int_rn(xv * fsc[f]);
+#pragma unroll
+                    for (int s2 = 0; s2 < 3; s2++) {
+                        const int dg = static_cast<int>(static_cast<int8_t>(X & 0xFF));
+                        w[s2][f] |= static_cast<uint32_t>(dg & 0xFF) << (8 * b);
+                        X = static_cast<int>(static_cast<uint32_t>(X) - static_cast<uint32_t>(dg)) >> 8;
+                    }
+                    w[3][f] |= static_cast<uint32_t>(X & 0xFF) << (8 * b);
+                }
+                const int k0 = c << 4, u = k0 >> 10, G8 = (k0 >> 7) & 7, qq = (k0 >> 5) & 3, r = (k0 >> 4) & 1;
+                const int set = MT == 1 ? u * 4 + (G8 & 3) : u * 8 + G8;
+                const int col0 = MT == 1 ? 4 * (G8 >> 2) : 4 * m;
+#pragma unroll
+                for (int s2 = 0; s2 < 4; s2++)
+#pragma unroll
+                    for (int f = 0; f < 4; f++)
+                        *reinterpret_cast<uint32_t *>(xs8 + ((((set * 2 + (f >> 1)) * 32 + 4 * (col0 + s2) + qq) << 4) +
+                                                              (f & 1) * 8 + r * 4)) = w[s2][f];
+                if ((lane & 7) == 0) egrp[m * (K >> 7) + (k0 >> 7)] = static_cast<int8_t>(eC);
+            }
+            __syncthreads();
+            // one all-ones chain per set (A = code 1 in every field), and the
+            // lane records: minus the sums of columns 2q, 2q + 1, and the factor
+            for (int sl = warp; sl < B * kSPU; sl += kW) {
+                int c[4] = {0, 0, 0, 0};
+#pragma unroll
+                for (int fp = 0; fp < 2; fp++) {
+                    const uint4 xq = *reinterpret_cast<const uint4 *>(xs8 + (((sl * 2 + fp) * 32 + lane) << 4));
+                    const uint32_t m0 = 0x01010101u << (4 * fp), m1 = m0 << 2;
+                    imma_acc(c, m0, m0, m0, m0, xq.x, xq.y);
+                    imma_acc(c, m1, m1, m1, m1, xq.z, xq.w);
+                }
+                if (g == 0) {
+                    const int u = sl / kSPU, hs = sl - u * kSPU;
+                    const int G8 = MT == 1 ? hs + 4 * (q >> 1) : hs;
+                    const int m = MT == 1 ? 0 : (q >> 1);
+                    const int eC = egrp[m * (K >> 7) + u * 8 + G8];
+                    const float fac = __int_as_float((127 + 16 * (q & 1) - eC) << 23);
+                    recs[sl * 4 + q] = make_int4(-c[0], -c[1], __float_as_int(fac), 0);
+                }
+            }
+            __syncthreads();
+        } else {
         {
             unsigned int mx = 0;
             const int per_row = K / 8;
@@ -371,7 +490,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_step_kernel(const __grid_con
         for (int w = 0; w < kW; w++) mx = max(mx, wmax[w]);
         const int ex = max(static_cast<int>(mx >> 10), 1) - 15;
         // the largest staged factor is 2^E: x * 2^E stays finite
-        const int E = min(F == 1 ? 7 : 8, 15 - ex);
+        E = min(F == 1 ? 7 : 8, 15 - ex);
         if constexpr (F == 1) {
             // factor of bit position p (0..15 in a half) is 2^(E - (p & 7));
             // 8 consecutive x are positions p0 .. p0 + 7, p0 = 0 or 8
@@ -427,7 +546,6 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_step_kernel(const __grid_con
             }
         }
         __syncthreads();
-        const __half *xlane = xs + lane * 8;
         // one all-ones chain per set: d1[set * 8 + column]
         for (int sl = warp; sl < B * MT; sl += kW) {
             float c[4];
@@ -438,6 +556,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_step_kernel(const __grid_con
             if (g == 0) *reinterpret_cast<float2 *>(d1 + sl * kSG + 2 * q) = make_float2(c[0], c[1]);
         }
         __syncthreads();
+        }  // fp16 staging
 
         // Lanes q < kGcLanes hold complete sums after a tile's lane
         // reduction; lane (g, q) stores v = (row g: tokens t0, t1; row g+8:
@@ -469,7 +588,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_step_kernel(const __grid_con
         // ---- this warp's units of the piece ----
         int tbeg, U, v0, v1;
         piece_range(d, T0, T1, warp, tbeg, U, v0, v1);
-        const float post = ldexpf(1.0f, 24 - E);
+        const float post = X8 ? 1.0f : ldexpf(1.0f, 24 - E);
         float acc[4] = {0.f, 0.f, 0.f, 0.f};
         // (tile, slice) of unit v, by increments
         const int tl_first = v0 / B;
@@ -510,7 +629,12 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_step_kernel(const __grid_con
                 // 2h + q/2); MT = 8: all eight groups of both rows
                 __half2 sh[MT == 1 ? 2 : (MT == 8 ? 1 : MT)];
                 uint4 s8a, s8b;
-                if constexpr (MT == 8) {
+                uint2 s4a, s4b;
+                if constexpr (X8 && MT == 1) {
+                    // digit form, one token: groups 4 (q / 2) + h of set h
+                    s4a = *reinterpret_cast<const uint2 *>(scs + row * 16 + 8 * (q >> 1));
+                    s4b = *reinterpret_cast<const uint2 *>(scs + (row + 8) * 16 + 8 * (q >> 1));
+                } else if constexpr (MT == 8 || X8) {
                     s8a = *reinterpret_cast<const uint4 *>(scs + row * 16);
                     s8b = *reinterpret_cast<const uint4 *>(scs + (row + 8) * 16);
                 } else if (MT == 1) {
@@ -533,7 +657,96 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_step_kernel(const __grid_con
                     if (lane == 0) asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
                     issue(s);
                 }
-                if constexpr (MT == 8) {
+                if constexpr (X8 && MT == 1) {
+                    // four sets of two groups (h, h + 4); lanes q < 2 keep
+                    // group h, lanes q >= 2 group h + 4.  acc[0] = row g,
+                    // acc[2] = row g + 8.
+                    int dd[kSG][4];
+                    int4 rr[4];
+#pragma unroll
+                    for (int h = 0; h < 4; h++) rr[h] = recs[(kb * 4 + h) * 4 + q];
+#pragma unroll
+                    for (int fp = 0; fp < 2; fp++) {
+                        uint4 xq[4];
+#pragma unroll
+                        for (int h = 0; h < 4; h++)
+                            xq[h] = *reinterpret_cast<const uint4 *>(xs8 + ((((kb * 4 + h) * 2 + fp) * 32 + lane) << 4));
+#pragma unroll
+                        for (int fi = 0; fi < 2; fi++) {
+                            const uint32_t mk = 0x03030303u << (2 * (2 * fp + fi));
+#pragma unroll
+                            for (int G8 = 0; G8 < kSG; G8++) {
+                                const uint4 &xv = xq[G8 & 3];
+                                const uint32_t b0 = fi ? xv.z : xv.x, b1 = fi ? xv.w : xv.y;
+                                if (fp == 0 && fi == 0)
+                                    imma_init(dd[G8], wd[G8][0] & mk, wd[G8][1] & mk, wd[G8][2] & mk, wd[G8][3] & mk,
+                                              b0, b1, rr[G8 & 3].x, rr[G8 & 3].y);
+                                else
+                                    imma_acc(dd[G8], wd[G8][0] & mk, wd[G8][1] & mk, wd[G8][2] & mk, wd[G8][3] & mk,
+                                             b0, b1);
+                            }
+                        }
+                    }
+                    const bool hi = q >= 2;
+                    const float2 a01 = __half22float2(*reinterpret_cast<const __half2 *>(&s4a.x));
+                    const float2 a23 = __half22float2(*reinterpret_cast<const __half2 *>(&s4a.y));
+                    const float2 b01 = __half22float2(*reinterpret_cast<const __half2 *>(&s4b.x));
+                    const float2 b23 = __half22float2(*reinterpret_cast<const __half2 *>(&s4b.y));
+                    const float sA[4] = {a01.x, a01.y, a23.x, a23.y}, sB[4] = {b01.x, b01.y, b23.x, b23.y};
+#pragma unroll
+                    for (int h = 0; h < 4; h++) {
+                        const int ia = dd[h][0] + dd[h][1] * 256, ib = dd[h + 4][0] + dd[h + 4][1] * 256;
+                        const int ja = dd[h][2] + dd[h][3] * 256, jb = dd[h + 4][2] + dd[h + 4][3] * 256;
+                        const float fac = __int_as_float(rr[h].z);
+                        acc[0] = fmaf(sA[h] * fac, static_cast<float>(hi ? ib : ia), acc[0]);
+                        acc[2] = fmaf(sB[h] * fac, static_cast<float>(hi ? jb : ja), acc[2]);
+                    }
+                } else if constexpr (X8) {
+                    // two tokens: one set per group, lane q holds token q / 2;
+                    // four groups at a time.  acc[0] = row g, acc[2] = row g + 8.
+                    const uint32_t sw[2][4] = {{s8a.x, s8a.y, s8a.z, s8a.w}, {s8b.x, s8b.y, s8b.z, s8b.w}};
+#pragma unroll
+                    for (int hf = 0; hf < 2; hf++) {
+                        int dd[4][4];
+                        int2 rr[4];
+#pragma unroll
+                        for (int j = 0; j < 4; j++)
+                            rr[j] = *reinterpret_cast<const int2 *>(recs + (kb * 8 + 4 * hf + j) * 4 + q);
+#pragma unroll
+                        for (int fp = 0; fp < 2; fp++) {
+                            uint4 xq[4];
+#pragma unroll
+                            for (int j = 0; j < 4; j++)
+                                xq[j] = *reinterpret_cast<const uint4 *>(
+                                    xs8 + ((((kb * 8 + 4 * hf + j) * 2 + fp) * 32 + lane) << 4));
+#pragma unroll
+                            for (int fi = 0; fi < 2; fi++) {
+                                const uint32_t mk = 0x03030303u << (2 * (2 * fp + fi));
+#pragma unroll
+                                for (int j = 0; j < 4; j++) {
+                                    const uint32_t *wg = wd[4 * hf + j];
+                                    const uint32_t b0 = fi ? xq[j].z : xq[j].x, b1 = fi ? xq[j].w : xq[j].y;
+                                    if (fp == 0 && fi == 0)
+                                        imma_init(dd[j], wg[0] & mk, wg[1] & mk, wg[2] & mk, wg[3] & mk, b0, b1,
+                                                  rr[j].x, rr[j].y);
+                                    else
+                                        imma_acc(dd[j], wg[0] & mk, wg[1] & mk, wg[2] & mk, wg[3] & mk, b0, b1);
+                                }
+                            }
+                        }
+#pragma unroll
+                        for (int j = 0; j < 4; j++) {
+                            const int G8 = 4 * hf + j;
+                            const float sa = __half2float(__ushort_as_half(
+                                static_cast<unsigned short>(sw[0][G8 >> 1] >> (16 * (G8 & 1)))));
+                            const float sb = __half2float(__ushort_as_half(
+                                static_cast<unsigned short>(sw[1][G8 >> 1] >> (16 * (G8 & 1)))));
+                            const float fac = __int_as_float(recs[(kb * 8 + G8) * 4 + q].z);
+                            acc[0] = fmaf(sa * fac, static_cast<float>(dd[j][0] + dd[j][1] * 256), acc[0]);
+                            acc[2] = fmaf(sb * fac, static_cast<float>(dd[j][2] + dd[j][3] * 256), acc[2]);
+                        }
+                    }
+                } else if constexpr (MT == 8) {
                     // group by group: acc[0..1] = row g, tokens 2q, 2q+1;
                     // acc[2..3] = row g+8
                     const uint32_t sw[2][4] = {{s8a.x, s8a.y, s8a.z, s8a.w}, {s8b.x, s8b.y, s8b.z, s8b.w}};
@@ -590,6 +803,16 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_step_kernel(const __grid_con
             if (--to_end == 0) {
                 // ---- this warp's part of a tile is complete: sum the lanes q
                 // that hold other groups of the same tokens ----
+                if constexpr (X8 && MT == 2) {
+                    // lanes q, q ^ 1 hold the two digit pairs of token q / 2:
+                    // lane 0 ends with (row g: tokens 0, 1; row g + 8: 0, 1)
+                    const float tg = acc[0] + __shfl_xor_sync(0xffffffffu, acc[0], 1);
+                    const float tg8 = acc[2] + __shfl_xor_sync(0xffffffffu, acc[2], 1);
+                    acc[1] = __shfl_xor_sync(0xffffffffu, tg, 2);
+                    acc[3] = __shfl_xor_sync(0xffffffffu, tg8, 2);
+                    acc[0] = tg;
+                    acc[2] = tg8;
+                } else {
                 if (MT == 1) {
                     acc[0] += acc[1];
                     acc[2] += acc[3];
@@ -599,6 +822,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_step_kernel(const __grid_con
                 for (int c = 0; c < 4; c++) {
                     if (MT <= 2) acc[c] += __shfl_xor_sync(0xffffffffu, acc[c], 1);
                     if (MT <= 4) acc[c] += __shfl_xor_sync(0xffffffffu, acc[c], 2);
+                }
                 }
                 const int tile = tbeg + tl;
                 const bool whole = kb == B - 1 && (tl != tl_first || !first_partial);
@@ -663,27 +887,35 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_step_kernel(const __grid_con
     if (!p.first) asm volatile("griddepcontrol.wait;" ::: "memory");
 }
 
-bool g_attr_step[64][3][4];
+bool g_attr_step[64][3][4][2];
 
 using StepKernel = void (*)(SParams);
-StepKernel step_kernel(int mt, int f) {
+StepKernel step_kernel(int mt, int f, bool x8) {
+    if (x8) return f != 0 ? nullptr : (mt == 1 ? gemv_step_kernel<1, 0, true> : (mt == 2 ? gemv_step_kernel<2, 0, true> : nullptr));
     if (f == 0)
-        return mt == 1 ? gemv_step_kernel<1, 0>
-                       : (mt == 2 ? gemv_step_kernel<2, 0> : (mt == 4 ? gemv_step_kernel<4, 0> : gemv_step_kernel<8, 0>));
+        return mt == 1 ? gemv_step_kernel<1, 0, false>
+                       : (mt == 2 ? gemv_step_kernel<2, 0, false>
+                                  : (mt == 4 ? gemv_step_kernel<4, 0, false> : gemv_step_kernel<8, 0, false>));
     if (f == 1)  // no eight-token form for the 1-bit weights
-        return mt == 1 ? gemv_step_kernel<1, 1>
-                       : (mt == 2 ? gemv_step_kernel<2, 1> : (mt == 4 ? gemv_step_kernel<4, 1> : nullptr));
-    return mt == 1 ? gemv_step_kernel<1, 2>
-                   : (mt == 2 ? gemv_step_kernel<2, 2> : (mt == 4 ? gemv_step_kernel<4, 2> : gemv_step_kernel<8, 2>));
+        return mt == 1 ? gemv_step_kernel<1, 1, false>
+                       : (mt == 2 ? gemv_step_kernel<2, 1, false> : (mt == 4 ? gemv_step_kernel<4, 1, false> : nullptr));
+    return mt == 1 ? gemv_step_kernel<1, 2, false>
+                   : (mt == 2 ? gemv_step_kernel<2, 2, false>
+                              : (mt == 4 ? gemv_step_kernel<4, 2, false> : gemv_step_kernel<8, 2, false>));
 }
 
 int step_mt(int M) { return M == 1 ? 1 : (M == 2 ? 2 : (M <= 4 ? 4 : 8)); }
 int mt_index(int mt) { return mt == 1 ? 0 : (mt == 2 ? 1 : (mt == 4 ? 2 : 3)); }
 
+// The digit form serves 2-bit slots at one and two token rows unless the
+// group-per-column fp16 form is asked for (TERN_OPT_STEP_FORM = 1).
+bool step_x8(int M, int fmt) { return fmt == 0 && M <= 2 && g_opt.step_form != 1; }
+
 }  // namespace
 
 bool gemv_step_fits(int K, int M, int fmt) {
-    return K % 1024 == 0 && M >= 1 && M <= (fmt == 1 ? 4 : 8) && smem_bytes(K, step_mt(M), 1, fmt) <= kSmemBudget;
+    return K % 1024 == 0 && M >= 1 && M <= (fmt == 1 ? 4 : 8) &&
+           smem_bytes(K, step_mt(M), 1, fmt, step_x8(M, fmt)) <= kSmemBudget;
 }
 
 bool gemv_step_supports(const MatDesc *md, int count, int M, int fmt) {
@@ -694,7 +926,7 @@ bool gemv_step_supports(const MatDesc *md, int count, int M, int fmt) {
         kmax = std::max(kmax, md[i].K);
     }
     // one ring stage per warp at least (refilled as soon as it is read)
-    return smem_bytes(kmax, step_mt(M), 1, fmt) <= kSmemBudget;
+    return smem_bytes(kmax, step_mt(M), 1, fmt, step_x8(M, fmt)) <= kSmemBudget;
 }
 
 namespace {
@@ -705,6 +937,7 @@ tern_status launch_chunk(const DeviceInfo &dev, const MatDesc *md, int count, in
     thread_local SParams p;  // large (parameter space); filled on the host for each launch, per host thread
     std::memset(&p, 0, sizeof(p));
     const int mt = step_mt(M);
+    const bool x8 = step_x8(M, fmt);
     int kmax = 0;
     long long total_units = 0;
     int tiles = 0;
@@ -754,9 +987,9 @@ tern_status launch_chunk(const DeviceInfo &dev, const MatDesc *md, int count, in
     }
     const size_t budget = std::min<size_t>(kSmemBudget, dev.max_smem_optin);
     // The whole budget: every CTA sizes its ring from what its own staged x leaves.
-    const size_t smem = std::min(budget, smem_bytes(kmax, mt, kMaxNS, fmt));
-    if (smem_bytes(kmax, mt, 1, fmt) > smem)
-        return fail(TERN_ERR_SHAPE, "step kernel needs %zu B of shared memory", smem_bytes(kmax, mt, 1, fmt));
+    const size_t smem = std::min(budget, smem_bytes(kmax, mt, kMaxNS, fmt, x8));
+    if (smem_bytes(kmax, mt, 1, fmt, x8) > smem)
+        return fail(TERN_ERR_SHAPE, "step kernel needs %zu B of shared memory", smem_bytes(kmax, mt, 1, fmt, x8));
     int grid = std::min<int>(std::min(dev.sms, kMaxCtas), tiles);
     if (g_opt.gemv_grid > 0) grid = std::min(grid, g_opt.gemv_grid);
     // Cut the flat tile list into `grid` ranges of about equal units: CTA c
@@ -798,7 +1031,7 @@ tern_status launch_chunk(const DeviceInfo &dev, const MatDesc *md, int count, in
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    cudaError_t e = cudaLaunchKernelEx(&cfg, step_kernel(mt, fmt), p);
+    cudaError_t e = cudaLaunchKernelEx(&cfg, step_kernel(mt, fmt, x8), p);
     if (e != cudaSuccess) return cuda_fail(e, "gemv step kernel launch");
     return TERN_OK;
 }
@@ -810,14 +1043,15 @@ tern_status launch_gemv_step(const MatDesc *md, int count, int M, int fmt, cudaS
     tern_status st = current_device(&dev);
     if (st != TERN_OK) return st;
     if (fmt < 0 || fmt > 2) return fail(TERN_ERR_INVALID_ARG, "step kernel: unknown weight format %d", fmt);
-    if (!gemv_step_supports(md, count, M, fmt) || step_kernel(step_mt(M), fmt) == nullptr)
+    const bool x8 = step_x8(M, fmt);
+    if (!gemv_step_supports(md, count, M, fmt) || step_kernel(step_mt(M), fmt, x8) == nullptr)
         return fail(TERN_ERR_SHAPE, "step kernel: unsupported shapes");
     const int mi = mt_index(step_mt(M));
-    if (!g_attr_step[dev.device][fmt][mi]) {
-        cudaError_t e = cudaFuncSetAttribute(step_kernel(step_mt(M), fmt), cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if (!g_attr_step[dev.device][fmt][mi][x8]) {
+        cudaError_t e = cudaFuncSetAttribute(step_kernel(step_mt(M), fmt, x8), cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              static_cast<int>(dev.max_smem_optin));
         if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(gemv step)");
-        g_attr_step[dev.device][fmt][mi] = true;
+        g_attr_step[dev.device][fmt][mi][x8] = true;
     }
     // Equal-sized launches of at most kMaxPer matrices each.
     const int launches = (count + kMaxPer - 1) / kMaxPer;

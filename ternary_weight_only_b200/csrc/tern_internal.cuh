@@ -36,6 +36,7 @@ struct Options {
     int gemv_variant = 0;
     int gemv_grid = 0;
     int gemv_prefetch = 0;
+    int step_form = 0;
 };
 extern Options g_opt;
 
