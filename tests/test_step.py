@@ -28,6 +28,15 @@ def T():
     tern.tern_set_option(tern.TERN_OPT_TEST_STALL_US, 0)
 
 
+@pytest.fixture(params=[0, 1], ids=["digit", "fp16"])
+def form(T, request):
+    """The two arithmetic forms of the 2-bit step at M <= 2: 0 = the digit
+    form (8-bit integer mma, the default), 1 = the fp16 group-per-column form."""
+    T.tern_set_option(T.TERN_OPT_STEP_FORM, request.param)
+    yield request.param
+    T.tern_set_option(T.TERN_OPT_STEP_FORM, 0)
+
+
 def make_mats(orc, shapes, seed, M=1):
     """Host inputs packed by the oracle; device copies; outputs pre-filled with NaN.
     M = 1 passes x [K] and y [N]; M > 1 passes x [M, K] and y [M, N]."""
@@ -53,7 +62,7 @@ def check_all(orc, mats, refs, what):
 
 
 @pytest.mark.parametrize("grid", [0, 1, 3, 7, 40])
-def test_mixed_shapes(T, orc, grid):
+def test_mixed_shapes(T, orc, grid, form):
     shapes = [(1024, 1), (2048, 17), (5120, 100), (1024, 16), (3072, 333), (6144, 64), (1024, 250),
               (17408, 40), (4096, 129), (2048, 7)]
     mats, refs = make_mats(orc, shapes, seed=7000 + grid)
@@ -76,7 +85,7 @@ def test_many_small_matrices(T, orc):
     check_all(orc, mats, refs, "step x300")
 
 
-def test_decode_layer_and_head(T, orc):
+def test_decode_layer_and_head(T, orc, form):
     """The seven projections of a synthetic decode layer plus the 5120x151936
     head, one launch, every output."""
     from ternary_weight_only_b200 import synth
@@ -103,7 +112,7 @@ def test_matches_single_launches(T, orc):
         check_close(y1.view(1, -1), y_ref, bound, f"single {j}")
 
 
-def test_exact_cases(T):
+def test_exact_cases(T, form):
     """All-zero codes give exactly zero; one-hot x gives s * t exactly."""
     from ternary_weight_only_b200 import synth
     N, K = 80, 3072
@@ -163,8 +172,8 @@ def test_verify_batch_mixed(T, orc, M, grid):
     check_all(orc, mats, refs, f"step M={M} grid={grid}")
 
 
-@pytest.mark.parametrize("M", [2, 4, 8])
-def test_verify_layer(T, orc, M):
+@pytest.mark.parametrize("M", [1, 2, 4, 8])
+def test_verify_layer(T, orc, M, form):
     """The seven projections of a synthetic decode layer at M token rows."""
     from ternary_weight_only_b200 import synth
     shapes = [(K, N) for _, K, N in synth.LAYER_PROJ]
@@ -224,8 +233,8 @@ def test_chained_calls_see_complete_inputs(T):
         assert torch.equal(a, b), i
 
 
-@pytest.mark.parametrize("M", [1, 4, 8])
-def test_long_rows_run_as_k_segments(T, orc, M):
+@pytest.mark.parametrize("M", [1, 2, 4, 8])
+def test_long_rows_run_as_k_segments(T, orc, M, form):
     """Rows far longer than the staged x allows (K = 65536 at M = 1 and 4,
     K = 40960 at M = 8) run as K segments; mixed with short products in one
     call; every output."""
@@ -285,3 +294,88 @@ def test_concurrent_calls_from_two_host_threads(T):
     for mats, w in zip(sets, want):
         for m, y in zip(mats, w):
             assert torch.equal(m[3], y)
+
+
+def _range_cases(M, K, seed):
+    """Activations that stress a fixed point per 128-k group: every group has
+    its own pattern (cycled): all zeros; values 2^-e with e in [0, 12]
+    (within 2^13 of the group's largest); fp16 subnormals only; values near
+    +-30000; x all +1; x all 20 (same sign); ordinary N(0,1)."""
+    gen = torch.Generator().manual_seed(seed)
+    x = torch.empty(M, K)
+    for m in range(M):
+        for gi in range(K // 128):
+            kind = (gi + 3 * m) % 7
+            sl = slice(gi * 128, (gi + 1) * 128)
+            sign = torch.where(torch.rand(128, generator=gen) < 0.5, -1.0, 1.0)
+            if kind == 0:
+                v = torch.zeros(128)
+            elif kind == 1:
+                v = sign * torch.pow(2.0, -torch.randint(0, 13, (128,), generator=gen).float())
+            elif kind == 2:
+                v = sign * torch.randint(1, 1024, (128,), generator=gen).float() * 2.0 ** -24
+            elif kind == 3:
+                v = sign * (30000.0 - torch.randint(0, 2000, (128,), generator=gen).float())
+            elif kind == 4:
+                v = torch.ones(128)
+            elif kind == 5:
+                v = torch.full((128,), 20.0)
+            else:
+                v = torch.randn(128, generator=gen)
+            x[m, sl] = v
+    return x.half()
+
+
+@pytest.mark.parametrize("M", [1, 2])
+def test_activation_range_cases(T, orc, M, form):
+    """Per-group activation patterns (zeros, a 2^12 range, subnormals, values
+    near 30000, same-sign runs) on mixed shapes; scales 1/1024 keep every sum
+    finite in fp16; every output against the oracle."""
+    from ternary_weight_only_b200 import synth
+    shapes = [(2048, 96), (5120, 40), (1024, 17)]
+    mats, refs = [], []
+    for j, (K, N) in enumerate(shapes):
+        x = _range_cases(M, K, seed=31 + j + 10 * M)
+        g = synth.gen(8100 + j + 10 * M)
+        codes = synth.codes_sparse(N, K, g)
+        if j == 0:
+            codes[: N // 2, :] = 1  # all +1 rows: no cancellation
+        scales = torch.full((N, K // 128), 1.0 / 1024).half()
+        xn, cn, sn = np_inputs(x, codes, scales)
+        slots, sc, bad, _ = orc.pack(cn, sn)
+        assert bad == 0
+        y = torch.full((M, N), float("nan"), dtype=torch.float16, device="cuda")
+        xd = x.cuda()
+        mats.append((xd[0] if M == 1 else xd, torch.from_numpy(slots).cuda(), scales.cuda(), y[0] if M == 1 else y))
+        refs.append((xn, slots, sc))
+    T.tern_gemv_step(mats, M)
+    T.tern_sync_status()
+    check_all(orc, mats, refs, f"range cases M={M}")
+
+
+@pytest.mark.parametrize("M", [1, 2, 4])
+def test_slot_value_3_is_finite_and_local(T, orc, M, form):
+    """Slot value 3 (not a valid code) in some rows: those rows give finite
+    values and every other row is still within the tolerance."""
+    from ternary_weight_only_b200 import synth
+    K, N = 3072, 160
+    x, codes, scales = synth.case(M, K, N, seed=8200 + M, codes="sparse", outlier_p=0.01)
+    xn, cn, sn = np_inputs(x, codes, scales)
+    slots, sc, bad, _ = orc.pack(cn, sn)
+    assert bad == 0
+    dirty = np.array([0, 5, 17, 18, 64, 159])
+    bad_slots = slots.copy()
+    rng = np.random.default_rng(M)
+    for r in dirty:
+        cols = rng.choice(K // 4, size=40, replace=False)
+        bad_slots[r, cols] = 0xFF  # four code-3 fields per byte
+    y = torch.full((M, N), float("nan"), dtype=torch.float16, device="cuda")
+    xd = x.cuda()
+    T.tern_gemv_step([(xd[0] if M == 1 else xd, torch.from_numpy(bad_slots).cuda(), scales.cuda(),
+                       y[0] if M == 1 else y)], M)
+    T.tern_sync_status()
+    got = y.float().cpu()
+    assert bool(torch.isfinite(got).all())
+    clean = np.setdiff1d(np.arange(N), dirty)
+    y_ref, bound = orc.matmul(xn, slots, sc, threads=NCPU)
+    check_close(got[:, clean], y_ref[:, clean], bound[:, clean], f"clean rows with slot value 3 elsewhere M={M}")
