@@ -857,7 +857,7 @@ def main():
     ap.add_argument("--profile-head", action="store_true",
                     help="profiling case: run the 5120x151936 head launch 3x instead of the layers")
     ap.add_argument("--gemv-variant", type=int, default=0,
-                    help="profiling case only: bandwidth kernel variant (0 TMA-staged, 1 register ring)")
+                    help="profiling case only: bandwidth kernel variant (TERN_OPT_GEMV_VARIANT)")
     args = ap.parse_args()
     if args.profile_layers > 0:
         return run_profile(args)

@@ -379,27 +379,25 @@ tern_status tern_sync_status(void *stream);
  *                          block cluster and distributed shared memory (1,2,4,8)
  *   TERN_OPT_GEMV_CTAS     cap on resident CTAs per SM used for the grid; for
  *                          the TMA-staged kernel 3 also selects the build with
- *                          the smaller register budget (default: 2 per SM);
- *                          for the tensor-memory kernel 1 selects one
- *                          warpgroup per CTA instead of two
+ *                          the smaller register budget (default: 2 per SM)
  *   TERN_OPT_GEMM_PATH     1 = force the bandwidth kernel (M<=8 chunks),
  *                          2 = force the tensor-core kernel
  *   TERN_OPT_GEMM_MIN_M    smallest M (> 8) sent to the tensor-core kernel
  *                          (default 32)
- *   TERN_OPT_GEMV_VARIANT  bandwidth kernel: 0 = default (variant 4 where its
- *                          shape rules hold, else variant 2),
- *                          1 = register-ring mma.sync, 2 = TMA-staged mma.sync,
+ *   TERN_OPT_GEMV_VARIANT  bandwidth kernel: 0 = default (M = 1: the
+ *                          decode-step kernel of tern_gemv_step where its
+ *                          shape rules hold; M = 2..8: variant 4 where its
+ *                          shape rules hold; else variant 2),
+ *                          2 = TMA-staged mma.sync,
  *                          3 = tcgen05 kernel for M <= 4 (splits K through the
  *                          workspace), 4 = producer/consumer mma.sync kernel
  *                          for K a multiple of 1024 (one CTA per SM, one
  *                          logic operation per weight pair; other shapes take
- *                          the default kernel), 5 = tensor-memory kernel for K
- *                          a multiple of 1024 (tcgen05, weights unpacked
- *                          into tensor memory by one thread per row),
- *                          6 = variant 4 with token rows in the mma columns
- *                          also at M = 1 (variant 4 puts the eight scale
- *                          groups of a 1024-k slice there when M = 1); all
- *                          kept for comparison
+ *                          the default kernel), 6 = variant 4 with token rows
+ *                          in the mma columns also at M = 1 (variant 4 puts
+ *                          the eight scale groups of a 1024-k slice there
+ *                          when M = 1); 1 and 5 are not accepted (kernels
+ *                          removed)
  *   TERN_OPT_GEMV_GRID     cap on the CTAs of the producer/consumer and
  *                          tensor-memory kernels
  *                          (0 = one per SM); smaller grids give every CTA

@@ -168,15 +168,21 @@ int planning_sms() {
 
 // Bandwidth kernels (M <= 8).  Default: the TMA-staged mma.sync kernel,
 // the fastest measured so far; the knob selects the others for comparison.
-enum { kVarDefault = 0, kVarRing = 1, kVarTma = 2, kVarTc = 3, kVarPc = 4, kVarTmem = 5, kVarPcTok = 6 };
+// (Values 1 and 5 named two kernels that were measured, kept for comparison
+// and then removed.)
+enum { kVarDefault = 0, kVarTma = 2, kVarTc = 3, kVarPc = 4, kVarPcTok = 6 };
 
 bool use_tc(int M) { return g_opt.gemv_variant == kVarTc && M <= 4; }
 
 tern_status launch_bandwidth(const MatDesc *d, int count, int M, void *workspace, size_t ws_bytes,
                              cudaStream_t s) {
-    if (g_opt.gemv_variant == kVarRing) return launch_gemv_mma(d, count, M, s);
+    // One token row: the persistent step kernel (digit form) where its shape
+    // rules hold -- measured faster than the per-matrix kernels on every
+    // decode shape alone and grouped (head 5120 x 151936: 38.7 us against
+    // 52.4 us; gate + up: 13.7 against 18.4 us).
+    if (g_opt.gemv_variant == kVarDefault && M == 1 && gemv_step_supports(d, count, 1, 0))
+        return launch_gemv_step(d, count, 1, 0, s);
     if (use_tc(M)) return launch_gemv_tc(d, count, M, workspace, ws_bytes, s);
-    if (g_opt.gemv_variant == kVarTmem && gemv_tmem_supports(d, count, M)) return launch_gemv_tmem(d, count, M, s);
     // Default: the producer/consumer kernel where its shape rules hold (K a
     // multiple of 1024, x fits its shared memory), else the TMA-staged one.
     if ((g_opt.gemv_variant == kVarPc || g_opt.gemv_variant == kVarDefault || g_opt.gemv_variant == kVarPcTok) &&
@@ -530,16 +536,12 @@ tern_status tern_sync_status(void *stream) {
     unsigned int z = 0;
     st = read_gemvpc_status(true, &z);
     if (st != TERN_OK) return st;
-    unsigned int t5 = 0;
-    st = read_gemvtm_status(true, &t5);
-    if (st != TERN_OK) return st;
     unsigned int t6 = 0;
     st = read_gemvstep_status(true, &t6);
     if (st != TERN_OK) return st;
     if (v == 0) v = w;
     if (v == 0) v = u;
     if (v == 0) v = z;
-    if (v == 0) v = t5;
     if (v == 0) v = t6;
     if (v != 0) return fail(static_cast<tern_status>(v), "a kernel gave up a bounded wait on the device");
     return TERN_OK;
@@ -558,7 +560,8 @@ tern_status tern_set_option(int option, int64_t value) {
             return TERN_OK;
         case TERN_OPT_GEMM_MIN_M: g_opt.gemm_min_m = static_cast<int>(value); return TERN_OK;
         case TERN_OPT_GEMV_VARIANT:
-            if (value > 6) return fail(TERN_ERR_INVALID_ARG, "gemv variant %lld", static_cast<long long>(value));
+            if (value > 6 || value == 1 || value == 5)
+                return fail(TERN_ERR_INVALID_ARG, "gemv variant %lld", static_cast<long long>(value));
             g_opt.gemv_variant = static_cast<int>(value);
             return TERN_OK;
         case TERN_OPT_GEMV_GRID: g_opt.gemv_grid = static_cast<int>(value); return TERN_OK;

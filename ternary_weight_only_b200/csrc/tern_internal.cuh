@@ -73,9 +73,6 @@ struct MatDesc {
 tern_status launch_gemv_tma(const MatDesc *d, int count, int M, cudaStream_t stream);
 // Producer/consumer form of the same kernel (K a multiple of 1024, x small).
 bool gemv_pc_supports(const MatDesc *d, int count, int M, bool token_columns);
-bool gemv_tmem_supports(const MatDesc *md, int count, int M);
-tern_status launch_gemv_tmem(const MatDesc *md, int count, int M, cudaStream_t stream);
-tern_status read_gemvtm_status(bool reset, unsigned int *out);
 // M = 1 uses the group-per-column form unless token_columns is set.
 tern_status launch_gemv_pc(const MatDesc *d, int count, int M, bool token_columns, cudaStream_t stream);
 // Tensor-core (tcgen05) bandwidth kernel for M in [1,4]; splits tiles along K
@@ -85,7 +82,6 @@ tern_status launch_gemv_tc(const MatDesc *d, int count, int M, void *workspace, 
 size_t gemv_tc_workspace_bytes(const MatDesc *d, int count, int M, int sms);
 // M = 1 product of the tcgen05 kernel with its scratch in a static device area.
 tern_status gemv_noalloc(const MatDesc &d, cudaStream_t stream);
-tern_status launch_gemv_mma(const MatDesc *d, int count, int M, cudaStream_t stream);
 // Partition of a grouped bandwidth launch: for each matrix i with ntile[i]
 // 16-row tiles and between nbmin[i] and nbc[i] k-slices per CTA, choose
 // Pout[i] warps per tile (power of two, <= nbmin[i]) and cl_out[i] CTAs (or

@@ -39,8 +39,7 @@ TERN_OPT_GEMV_VARIANT = 7
 TERN_OPT_GEMV_GRID = 8
 TERN_OPT_GEMV_PREFETCH = 9
 TERN_OPT_STEP_FORM = 10
-GEMV_VARIANT_DEFAULT, GEMV_VARIANT_RING, GEMV_VARIANT_TMA, GEMV_VARIANT_TC, GEMV_VARIANT_PC = 0, 1, 2, 3, 4
-GEMV_VARIANT_TMEM = 5
+GEMV_VARIANT_DEFAULT, GEMV_VARIANT_TMA, GEMV_VARIANT_TC, GEMV_VARIANT_PC = 0, 2, 3, 4
 TERN_MAX_GROUP = 16
 TERN_MAX_STEP = 512
 GEMV_VARIANT_PC_TOKEN_COLUMNS = 6
