@@ -406,11 +406,11 @@ tern_status tern_sync_status(void *stream);
  *                          kernel, in 16-row x 1024-k units per consumer warp;
  *                          0 or n <= ring depth = none (the default: measured
  *                          slower)
- *   TERN_OPT_STEP_FORM     arithmetic of the decode-step kernel for 2-bit
- *                          slots at M = 1 and 2: 0 = default (the digit form:
- *                          8-bit integer mma on weights unpacked four per
- *                          instruction against activations split into four
- *                          exact signed 8-bit digits), 1 = the fp16
+ *   TERN_OPT_STEP_FORM     arithmetic of the decode-step kernels (all three
+ *                          weight storages) at M = 1 and 2: 0 = default (the
+ *                          digit form: 8-bit integer mma on weights unpacked
+ *                          four per instruction against activations split
+ *                          into four exact signed 8-bit digits), 1 = the fp16
  *                          group-per-column form used for every other M
  *   TERN_OPT_TEST_STALL_US TESTS ONLY: the TMA loaders of the tensor-core and
  *                          the TMA-staged bandwidth kernels issue no loads, so

@@ -27,7 +27,7 @@
 // never depend on the preceding launch or piece.
 //
 // Arithmetic: the group-per-column mma.sync form (tern_unpack_mma.cuh), or,
-// for 2-bit slots at one or two token rows, the digit form below.
+// at one or two token rows, the digit form below (all three storages).
 //
 // Digit form (X8): mma.sync m16n8k32 with unsigned 8-bit weights and signed
 // 8-bit activations, exact 32-bit integer sums.  One AND of a slot word with
@@ -184,6 +184,36 @@ __device__ __forceinline__ void t5_words(const uint8_t *p, uint32_t sh, const ui
     hi = __funnelshift_r(s1, s2, dd);
 }
 
+// Digit form: the A registers of mma p of a group from the lane's words wg
+// (2-bit slots: fields p of words 2q and 2q + 1 of rows g, g + 8, bytes c *
+// 4^p; 1-bit: bits 2p and 2p + 1 of word q of rows g, g + 8, bytes b * 2^bit).
+template <int F>
+__device__ __forceinline__ void x8_a(const uint32_t *wg, int p, uint32_t &a0, uint32_t &a1, uint32_t &a2,
+                                     uint32_t &a3) {
+    if constexpr (F == 0) {
+        const uint32_t mk = 0x03030303u << (2 * p);
+        a0 = wg[0] & mk;
+        a1 = wg[1] & mk;
+        a2 = wg[2] & mk;
+        a3 = wg[3] & mk;
+    } else {
+        const uint32_t m0 = 0x01010101u << (2 * p), m1 = m0 << 1;
+        a0 = wg[0] & m0;
+        a1 = wg[1] & m0;
+        a2 = wg[0] & m1;
+        a3 = wg[1] & m1;
+    }
+}
+
+// The lane's two digit sums joined, t restored: 2-bit slots d0 + 256 d1
+// (the chain started at minus the all-ones sums); 1-bit 2 (d0 + 256 d1) - oc
+// with oc the all-ones sums joined the same way.
+template <int F>
+__device__ __forceinline__ int x8_join(int d0, int d1, int oc) {
+    const int j = d0 + d1 * 256;
+    return F == 0 ? j : 2 * j - oc;
+}
+
 __device__ __forceinline__ bool step_wait(uint64_t *bar, uint32_t parity, unsigned long long deadline) {
     while (!mbar_try_wait_sleep(bar, parity, 20000u)) {
         if (globaltimer() > deadline) {
@@ -254,7 +284,10 @@ __device__ __forceinline__ void cursor_next(Cursor &c, const SParams &p, int T0,
 // is one group (columns 4 token + digit).
 template <int MT, int F, bool X8>
 __global__ void __launch_bounds__(kThreads, 1) gemv_step_kernel(const __grid_constant__ SParams p) {
-    static_assert(!X8 || (F == 0 && MT <= 2), "digit form: 2-bit slots, one or two token rows");
+    static_assert(!X8 || MT <= 2, "digit form: one or two token rows");
+    // digit-form arithmetic: ternary codes (2-bit slots, and five-per-byte
+    // bytes once decoded to slot words) or 1-bit weights
+    constexpr int FA = F == 1 ? 1 : 0;
     constexpr int GPB = 8 / MT;  // groups per set
     constexpr int kSPU = MT == 1 ? 4 : 8;  // digit form: sets per 1024-k unit
     constexpr int kSlotStage = slot_stage(F);
@@ -389,23 +422,45 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_step_kernel(const __grid_con
         const __half *xlane = xs + lane * 8;
         int E = 0;
         if constexpr (X8) {
-            // ---- digit form: 16 consecutive k of one token row per thread ----
+            // ---- digit form.  Work item (token m, 32-k chunk, field half
+            // fp): the 16 x of fields 2fp, 2fp + 1 (2-bit slots: k = 16 r +
+            // 4 b + f) or of bits 4fp .. 4fp + 3 (1-bit: k = 8 i + bit) of
+            // the chunk, each as four digits, written as one 16-byte B
+            // fragment per digit.  The eight items of a 128-k group are eight
+            // consecutive lanes.
             if (lane < 2) rec_tile[warp * 2 + lane] = -1;
-            const int nch = K >> 4;  // a multiple of 64: every warp runs whole iterations
-            for (int idx = threadIdx.x; idx < MT * nch; idx += nthr) {
-                const int m = idx / nch, c = idx - m * nch;
-                uint4 v0 = make_uint4(0u, 0u, 0u, 0u), v1 = v0;
+            const int nit = K >> 4;  // a multiple of 64: every warp runs whole iterations
+            for (int idx = threadIdx.x; idx < MT * nit; idx += nthr) {
+                const int m = idx / nit, it = idx - m * nit;
+                const int c32 = it >> 1, fp = it & 1, base = c32 << 5;
+                uint32_t hv[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};  // element e = half (e & 1) of hv[e >> 1]
                 if (m < M) {
-                    const __half *src = d.x + static_cast<size_t>(m) * d.xs + c * 16;
-                    v0 = *reinterpret_cast<const uint4 *>(src);
-                    v1 = *reinterpret_cast<const uint4 *>(src + 8);
+                    const __half *src = d.x + static_cast<size_t>(m) * d.xs + base;
+                    if constexpr (FA == 0) {
+                        uint4 v[4];
+#pragma unroll
+                        for (int j = 0; j < 4; j++) v[j] = *reinterpret_cast<const uint4 *>(src + 8 * j);
+                        // hv[4 r + b] = the pair at k = 16 r + 4 b + 2 fp
+#pragma unroll
+                        for (int r = 0; r < 2; r++)
+#pragma unroll
+                            for (int b = 0; b < 4; b++) {
+                                const uint4 &vv = v[(8 * r + 2 * b) >> 2];
+                                hv[4 * r + b] = (b & 1) ? (fp ? vv.w : vv.z) : (fp ? vv.y : vv.x);
+                            }
+                    } else {
+#pragma unroll
+                        for (int i = 0; i < 4; i++) {
+                            const uint2 v = *reinterpret_cast<const uint2 *>(src + 8 * i + 4 * fp);
+                            hv[2 * i] = v.x;
+                            hv[2 * i + 1] = v.y;
+                        }
+                    }
                 }
-                const uint32_t wv[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
-                // largest |x| of the 128-k group: the eight threads of a group
-                // are eight consecutive lanes (inf and NaN clamp to 65504)
+                // largest |x| of the group (inf and NaN clamp to 65504)
                 uint32_t mx = 0;
 #pragma unroll
-                for (int e = 0; e < 8; e++) mx = __vmaxu2(mx, __vminu2(wv[e] & 0x7FFF7FFFu, 0x7BFF7BFFu));
+                for (int e = 0; e < 8; e++) mx = __vmaxu2(mx, __vminu2(hv[e] & 0x7FFF7FFFu, 0x7BFF7BFFu));
                 mx = max(mx & 0xFFFFu, mx >> 16);
                 mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
                 mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
@@ -413,50 +468,54 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_step_kernel(const __grid_con
                 // eC = 29 - floor(log2 max|x|) (normal or subnormal max); 0 for an all-zero group
                 int eC = 0;
                 if (mx != 0) eC = 29 - (mx >= 0x400u ? static_cast<int>(mx >> 10) - 15 : (31 - __clz(mx)) - 24);
-                float fsc[4];
-#pragma unroll
-                for (int f = 0; f < 4; f++) fsc[f] = __int_as_float((127 + eC - 2 * f) << 23);
-                // digit words: w[s][f] holds digit s of the four x of field f
+                const int e0 = 127 + eC - 4 * fp;  // biased exponent of 2^(eC - 4 fp)
                 uint32_t w[4][4];
 #pragma unroll
                 for (int s2 = 0; s2 < 4; s2++)
 #pragma unroll
-                    for (int f = 0; f < 4; f++) w[s2][f] = 0u;
+                    for (int j = 0; j < 4; j++) w[s2][j] = 0u;
 #pragma unroll
                 for (int e = 0; e < 16; e++) {
-                    const int f = e & 3, b = e >> 2;
-                    const float xv = __half2float(__ushort_as_half(static_cast<unsigned short>(wv[e >> 1] >> (16 * (e & 1)))));
-                    int X = __float2int_rn(xv * fsc[f]);
+                    // field shift beyond 4 fp, and the element's place in the fragment
+                    const int sh = FA == 0 ? 2 * (e & 1) : (e & 3);
+                    const int wi = FA == 0 ? (e & 1) * 2 + (e >> 3) : (e & 3);
+                    const int by = FA == 0 ? (e >> 1) & 3 : (e >> 2);
+                    const float xv = __half2float(__ushort_as_half(static_cast<unsigned short>(hv[e >> 1] >> (16 * (e & 1)))));
+                    int X = __float2int_rn(xv * __int_as_float((e0 - sh) << 23));
 #pragma unroll
                     for (int s2 = 0; s2 < 3; s2++) {
                         const int dg = static_cast<int>(static_cast<int8_t>(X & 0xFF));
-                        w[s2][f] |= static_cast<uint32_t>(dg & 0xFF) << (8 * b);
+                        w[s2][wi] |= static_cast<uint32_t>(dg & 0xFF) << (8 * by);
                         X = static_cast<int>(static_cast<uint32_t>(X) - static_cast<uint32_t>(dg)) >> 8;
                     }
-                    w[3][f] |= static_cast<uint32_t>(X & 0xFF) << (8 * b);
+                    w[3][wi] |= static_cast<uint32_t>(X & 0xFF) << (8 * by);
                 }
-                const int k0 = c << 4, u = k0 >> 10, G8 = (k0 >> 7) & 7, qq = (k0 >> 5) & 3, r = (k0 >> 4) & 1;
+                const int u = base >> 10, G8 = (base >> 7) & 7, qq = (base >> 5) & 3;
                 const int set = MT == 1 ? u * 4 + (G8 & 3) : u * 8 + G8;
                 const int col0 = MT == 1 ? 4 * (G8 >> 2) : 4 * m;
 #pragma unroll
                 for (int s2 = 0; s2 < 4; s2++)
-#pragma unroll
-                    for (int f = 0; f < 4; f++)
-                        *reinterpret_cast<uint32_t *>(xs8 + ((((set * 2 + (f >> 1)) * 32 + 4 * (col0 + s2) + qq) << 4) +
-                                                              (f & 1) * 8 + r * 4)) = w[s2][f];
-                if ((lane & 7) == 0) egrp[m * (K >> 7) + (k0 >> 7)] = static_cast<int8_t>(eC);
+                    *reinterpret_cast<uint4 *>(xs8 + (((set * 2 + fp) * 32 + 4 * (col0 + s2) + qq) << 4)) =
+                        make_uint4(w[s2][0], w[s2][1], w[s2][2], w[s2][3]);
+                if ((lane & 7) == 0) egrp[m * (K >> 7) + (base >> 7)] = static_cast<int8_t>(eC);
             }
             __syncthreads();
-            // one all-ones chain per set (A = code 1 in every field), and the
-            // lane records: minus the sums of columns 2q, 2q + 1, and the factor
+            // one all-ones chain per set (A = weight code 1, or bit 1, in every
+            // field), and the lane records: for 2-bit slots minus the sums of
+            // columns 2q, 2q + 1 (the chains start there), for 1-bit weights
+            // their sum O_2q + 256 O_2q+1 (subtracted from twice the chain);
+            // then the factor 2^(16 (q & 1) - eC)
             for (int sl = warp; sl < B * kSPU; sl += kW) {
                 int c[4] = {0, 0, 0, 0};
 #pragma unroll
                 for (int fp = 0; fp < 2; fp++) {
                     const uint4 xq = *reinterpret_cast<const uint4 *>(xs8 + (((sl * 2 + fp) * 32 + lane) << 4));
-                    const uint32_t m0 = 0x01010101u << (4 * fp), m1 = m0 << 2;
-                    imma_acc(c, m0, m0, m0, m0, xq.x, xq.y);
-                    imma_acc(c, m1, m1, m1, m1, xq.z, xq.w);
+#pragma unroll
+                    for (int pp = 0; pp < 2; pp++) {
+                        const uint32_t m0 = 0x01010101u << (2 * (2 * fp + pp));
+                        const uint32_t m1 = FA == 0 ? m0 : m0 << 1;
+                        imma_acc(c, m0, m0, m1, m1, pp ? xq.z : xq.x, pp ? xq.w : xq.y);
+                    }
                 }
                 if (g == 0) {
                     const int u = sl / kSPU, hs = sl - u * kSPU;
@@ -464,7 +523,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_step_kernel(const __grid_con
                     const int m = MT == 1 ? 0 : (q >> 1);
                     const int eC = egrp[m * (K >> 7) + u * 8 + G8];
                     const float fac = __int_as_float((127 + 16 * (q & 1) - eC) << 23);
-                    recs[sl * 4 + q] = make_int4(-c[0], -c[1], __float_as_int(fac), 0);
+                    recs[sl * 4 + q] = FA == 0 ? make_int4(-c[0], -c[1], __float_as_int(fac), 0)
+                                              : make_int4(c[0] + c[1] * 256, 0, __float_as_int(fac), 0);
                 }
             }
             __syncthreads();
@@ -673,17 +733,17 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_step_kernel(const __grid_con
                             xq[h] = *reinterpret_cast<const uint4 *>(xs8 + ((((kb * 4 + h) * 2 + fp) * 32 + lane) << 4));
 #pragma unroll
                         for (int fi = 0; fi < 2; fi++) {
-                            const uint32_t mk = 0x03030303u << (2 * (2 * fp + fi));
 #pragma unroll
                             for (int G8 = 0; G8 < kSG; G8++) {
                                 const uint4 &xv = xq[G8 & 3];
                                 const uint32_t b0 = fi ? xv.z : xv.x, b1 = fi ? xv.w : xv.y;
+                                uint32_t a0, a1, a2, a3;
+                                x8_a<FA>(wd[G8], 2 * fp + fi, a0, a1, a2, a3);
                                 if (fp == 0 && fi == 0)
-                                    imma_init(dd[G8], wd[G8][0] & mk, wd[G8][1] & mk, wd[G8][2] & mk, wd[G8][3] & mk,
-                                              b0, b1, rr[G8 & 3].x, rr[G8 & 3].y);
+                                    imma_init(dd[G8], a0, a1, a2, a3, b0, b1, FA == 0 ? rr[G8 & 3].x : 0,
+                                              FA == 0 ? rr[G8 & 3].y : 0);
                                 else
-                                    imma_acc(dd[G8], wd[G8][0] & mk, wd[G8][1] & mk, wd[G8][2] & mk, wd[G8][3] & mk,
-                                             b0, b1);
+                                    imma_acc(dd[G8], a0, a1, a2, a3, b0, b1);
                             }
                         }
                     }
@@ -695,8 +755,9 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_step_kernel(const __grid_con
                     const float sA[4] = {a01.x, a01.y, a23.x, a23.y}, sB[4] = {b01.x, b01.y, b23.x, b23.y};
 #pragma unroll
                     for (int h = 0; h < 4; h++) {
-                        const int ia = dd[h][0] + dd[h][1] * 256, ib = dd[h + 4][0] + dd[h + 4][1] * 256;
-                        const int ja = dd[h][2] + dd[h][3] * 256, jb = dd[h + 4][2] + dd[h + 4][3] * 256;
+                        const int oc = rr[h].x;
+                        const int ia = x8_join<FA>(dd[h][0], dd[h][1], oc), ib = x8_join<FA>(dd[h + 4][0], dd[h + 4][1], oc);
+                        const int ja = x8_join<FA>(dd[h][2], dd[h][3], oc), jb = x8_join<FA>(dd[h + 4][2], dd[h + 4][3], oc);
                         const float fac = __int_as_float(rr[h].z);
                         acc[0] = fmaf(sA[h] * fac, static_cast<float>(hi ? ib : ia), acc[0]);
                         acc[2] = fmaf(sB[h] * fac, static_cast<float>(hi ? jb : ja), acc[2]);
@@ -721,16 +782,16 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_step_kernel(const __grid_con
                                     xs8 + ((((kb * 8 + 4 * hf + j) * 2 + fp) * 32 + lane) << 4));
 #pragma unroll
                             for (int fi = 0; fi < 2; fi++) {
-                                const uint32_t mk = 0x03030303u << (2 * (2 * fp + fi));
 #pragma unroll
                                 for (int j = 0; j < 4; j++) {
-                                    const uint32_t *wg = wd[4 * hf + j];
                                     const uint32_t b0 = fi ? xq[j].z : xq[j].x, b1 = fi ? xq[j].w : xq[j].y;
+                                    uint32_t a0, a1, a2, a3;
+                                    x8_a<FA>(wd[4 * hf + j], 2 * fp + fi, a0, a1, a2, a3);
                                     if (fp == 0 && fi == 0)
-                                        imma_init(dd[j], wg[0] & mk, wg[1] & mk, wg[2] & mk, wg[3] & mk, b0, b1,
-                                                  rr[j].x, rr[j].y);
+                                        imma_init(dd[j], a0, a1, a2, a3, b0, b1, FA == 0 ? rr[j].x : 0,
+                                                  FA == 0 ? rr[j].y : 0);
                                     else
-                                        imma_acc(dd[j], wg[0] & mk, wg[1] & mk, wg[2] & mk, wg[3] & mk, b0, b1);
+                                        imma_acc(dd[j], a0, a1, a2, a3, b0, b1);
                                 }
                             }
                         }
@@ -742,8 +803,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_step_kernel(const __grid_con
                             const float sb = __half2float(__ushort_as_half(
                                 static_cast<unsigned short>(sw[1][G8 >> 1] >> (16 * (G8 & 1)))));
                             const float fac = __int_as_float(recs[(kb * 8 + G8) * 4 + q].z);
-                            acc[0] = fmaf(sa * fac, static_cast<float>(dd[j][0] + dd[j][1] * 256), acc[0]);
-                            acc[2] = fmaf(sb * fac, static_cast<float>(dd[j][2] + dd[j][3] * 256), acc[2]);
+                            acc[0] = fmaf(sa * fac, static_cast<float>(x8_join<FA>(dd[j][0], dd[j][1], rr[j].x)), acc[0]);
+                            acc[2] = fmaf(sb * fac, static_cast<float>(x8_join<FA>(dd[j][2], dd[j][3], rr[j].x)), acc[2]);
                         }
                     }
                 } else if constexpr (MT == 8) {
@@ -891,7 +952,11 @@ bool g_attr_step[64][3][4][2];
 
 using StepKernel = void (*)(SParams);
 StepKernel step_kernel(int mt, int f, bool x8) {
-    if (x8) return f != 0 ? nullptr : (mt == 1 ? gemv_step_kernel<1, 0, true> : (mt == 2 ? gemv_step_kernel<2, 0, true> : nullptr));
+    if (x8) {
+        if (f == 0) return mt == 1 ? gemv_step_kernel<1, 0, true> : (mt == 2 ? gemv_step_kernel<2, 0, true> : nullptr);
+        if (f == 1) return mt == 1 ? gemv_step_kernel<1, 1, true> : (mt == 2 ? gemv_step_kernel<2, 1, true> : nullptr);
+        return mt == 1 ? gemv_step_kernel<1, 2, true> : (mt == 2 ? gemv_step_kernel<2, 2, true> : nullptr);
+    }
     if (f == 0)
         return mt == 1 ? gemv_step_kernel<1, 0, false>
                        : (mt == 2 ? gemv_step_kernel<2, 0, false>
@@ -907,9 +972,9 @@ StepKernel step_kernel(int mt, int f, bool x8) {
 int step_mt(int M) { return M == 1 ? 1 : (M == 2 ? 2 : (M <= 4 ? 4 : 8)); }
 int mt_index(int mt) { return mt == 1 ? 0 : (mt == 2 ? 1 : (mt == 4 ? 2 : 3)); }
 
-// The digit form serves 2-bit slots at one and two token rows unless the
-// group-per-column fp16 form is asked for (TERN_OPT_STEP_FORM = 1).
-bool step_x8(int M, int fmt) { return fmt == 0 && M <= 2 && g_opt.step_form != 1; }
+// The digit form serves every weight storage at one and two token rows
+// unless the group-per-column fp16 form is asked for (TERN_OPT_STEP_FORM = 1).
+bool step_x8(int M, int fmt) { return M <= 2 && g_opt.step_form != 1; }
 
 }  // namespace
 

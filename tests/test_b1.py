@@ -62,6 +62,15 @@ def test_pack_counts_invalid(T, orc):
     assert np.array_equal(bits.cpu().numpy(), want_bits)
 
 
+@pytest.fixture(params=[0, 1], ids=["digit", "fp16"])
+def form(T, request):
+    """The two arithmetic forms of the 1-bit step at M <= 2: 0 = the digit
+    form (8-bit integer mma, the default), 1 = the fp16 group-per-column form."""
+    T.tern_set_option(T.TERN_OPT_STEP_FORM, request.param)
+    yield request.param
+    T.tern_set_option(T.TERN_OPT_STEP_FORM, 0)
+
+
 def make_mats(orc, shapes, seed, M=1):
     """Host inputs packed by the oracle; device copies; outputs pre-filled with NaN."""
     from ternary_weight_only_b200 import synth
@@ -90,7 +99,7 @@ SHAPES = [(1024, 1), (2048, 17), (5120, 100), (1024, 16), (3072, 333), (6144, 64
 
 
 @pytest.mark.parametrize("grid", [0, 1, 3, 40])
-def test_mixed_shapes(T, orc, grid):
+def test_mixed_shapes(T, orc, grid, form):
     mats, refs = make_mats(orc, SHAPES, seed=8000 + grid)
     T.tern_set_option(T.TERN_OPT_GEMV_GRID, grid)
     try:
@@ -110,7 +119,7 @@ def test_many_small_matrices(T, orc):
     check_all(orc, mats, refs, "b1 step x200")
 
 
-def test_decode_layer_and_head(T, orc):
+def test_decode_layer_and_head(T, orc, form):
     """The seven projections of a synthetic decode layer plus the 5120x151936
     head as 1-bit matrices, one launch, every output."""
     from ternary_weight_only_b200 import synth
@@ -123,7 +132,7 @@ def test_decode_layer_and_head(T, orc):
 
 @pytest.mark.parametrize("M", [2, 3, 4])
 @pytest.mark.parametrize("grid", [0, 5])
-def test_verify_batch_mixed(T, orc, M, grid):
+def test_verify_batch_mixed(T, orc, M, grid, form):
     shapes = [(1024, 1), (2048, 17), (5120, 100), (3072, 333), (6144, 64), (17408, 40), (4096, 129)]
     mats, refs = make_mats(orc, shapes, seed=8500 + 10 * M + grid, M=M)
     T.tern_set_option(T.TERN_OPT_GEMV_GRID, grid)
@@ -135,7 +144,7 @@ def test_verify_batch_mixed(T, orc, M, grid):
     check_all(orc, mats, refs, f"b1 step M={M} grid={grid}")
 
 
-def test_exact_cases(T):
+def test_exact_cases(T, form):
     """One-hot x gives s * t exactly, for bit positions in both halves of a
     word, both byte halves and the last group; all-(+1) weights with unit
     scales and x = 1 give exactly K."""
@@ -179,8 +188,8 @@ def test_timeout_reported_and_context_survives(T, orc):
     check_all(orc, mats, refs, "b1 step after timeout")
 
 
-@pytest.mark.parametrize("M", [1, 4])
-def test_long_rows_run_as_k_segments(T, orc, M):
+@pytest.mark.parametrize("M", [1, 2, 4])
+def test_long_rows_run_as_k_segments(T, orc, M, form):
     """Rows longer than the staged x allows run as K segments whose sums are
     added to y; mixed with a short product in one call; every output."""
     shapes = [(98304, 40), (2048, 33)]

@@ -67,6 +67,16 @@ def test_pack_counts_invalid_and_unpack_marks_bad_bytes(T, orc):
     assert np.array_equal(got, orc.t5_unpack(allb, 256))
 
 
+@pytest.fixture(params=[0, 1], ids=["digit", "fp16"])
+def form(T, request):
+    """The two arithmetic forms after the base-3 decode at M <= 2: 0 = the
+    digit form (8-bit integer mma, the default), 1 = the fp16
+    group-per-column form."""
+    T.tern_set_option(T.TERN_OPT_STEP_FORM, request.param)
+    yield request.param
+    T.tern_set_option(T.TERN_OPT_STEP_FORM, 0)
+
+
 def make_mats(orc, shapes, seed, M=1):
     from ternary_weight_only_b200 import synth
     mats, refs = [], []
@@ -94,7 +104,7 @@ SHAPES = [(1024, 1), (2048, 17), (5120, 100), (1024, 16), (3072, 333), (6144, 64
 
 
 @pytest.mark.parametrize("grid", [0, 1, 3, 40])
-def test_mixed_shapes(T, orc, grid):
+def test_mixed_shapes(T, orc, grid, form):
     mats, refs = make_mats(orc, SHAPES, seed=9000 + grid)
     T.tern_set_option(T.TERN_OPT_GEMV_GRID, grid)
     try:
@@ -114,7 +124,7 @@ def test_many_small_matrices(T, orc):
     check_all(orc, mats, refs, "t5 step x200")
 
 
-def test_decode_layer_and_head(T, orc):
+def test_decode_layer_and_head(T, orc, form):
     from ternary_weight_only_b200 import synth
     shapes = [(K, N) for _, K, N in synth.LAYER_PROJ] + [(synth.HEAD[1], synth.HEAD[2])]
     mats, refs = make_mats(orc, shapes, seed=9200)
@@ -150,7 +160,7 @@ def test_shared_memory_limit_is_a_shape_error(T):
     assert ei.value.status == T.TERN_ERR_SHAPE
 
 
-def test_exact_cases(T):
+def test_exact_cases(T, form):
     """All-zero codes give exactly zero; one-hot x gives s * t exactly, for
     positions at every lane's window start and digit offset and in the last
     byte of a group."""
@@ -193,8 +203,8 @@ def test_timeout_reported_and_context_survives(T, orc):
     check_all(orc, mats, refs, "t5 step after timeout")
 
 
-@pytest.mark.parametrize("M", [1, 8])
-def test_long_rows_run_as_k_segments(T, orc, M):
+@pytest.mark.parametrize("M", [1, 2, 8])
+def test_long_rows_run_as_k_segments(T, orc, M, form):
     """Rows longer than the staged x and the decode table allow run as K
     segments whose sums are added to y; every output."""
     K = 65536 if M == 1 else 24576
@@ -205,7 +215,7 @@ def test_long_rows_run_as_k_segments(T, orc, M):
     check_all(orc, mats, refs, f"t5 step K segments M={M}")
 
 
-def test_invalid_bytes_give_finite_values_and_spare_other_rows(T, orc):
+def test_invalid_bytes_give_finite_values_and_spare_other_rows(T, orc, form):
     """Bytes 243..255 are invalid: the rows holding them get some finite
     value, every other row is computed as the oracle computes it."""
     from ternary_weight_only_b200 import synth
