@@ -692,6 +692,25 @@ def run_profile(args):
     return 0
 
 
+def run_profile_prefill(args):
+    """Small case for ncu captures of the tensor-core prefill kernel: one
+    K = 5120 -> N = 17408 product at M token rows (the prefill workload's
+    first shape), run three times."""
+    torch.cuda.set_device(0)
+    from ternary_weight_only_b200 import tern as T
+    M, (K, N) = args.profile_prefill, synth.PREFILL[0]
+    g = synth.gen(3000, "cuda")
+    slots, sc = T.tern_pack_g128(synth.codes_uniform(N, K, g, device="cuda"),
+                                 synth.scales_uniform(N, K, g, device="cuda"))
+    x = synth.activations(M, K, g, device="cuda")
+    y = torch.empty(M, N, dtype=torch.float16, device="cuda")
+    for _ in range(3):
+        T.tern_gemm(x, slots, sc, y)
+    torch.cuda.synchronize()
+    print(json.dumps({"profile_prefill": M, "K": K, "N": N, "flops_per_launch": 2 * M * N * K}))
+    return 0
+
+
 def run_tern(args):
     ws, rank, local = dist_setup(args)
     from ternary_weight_only_b200 import tern as T
@@ -856,9 +875,13 @@ def main():
                          "matrices in one step call (run 3x)")
     ap.add_argument("--profile-head", action="store_true",
                     help="profiling case: run the 5120x151936 head launch 3x instead of the layers")
+    ap.add_argument("--profile-prefill", type=int, default=0, metavar="M",
+                    help="profiling case: the prefill GEMM K=5120 -> N=17408 at M token rows, run 3x, exit")
     ap.add_argument("--gemv-variant", type=int, default=0,
                     help="profiling case only: bandwidth kernel variant (TERN_OPT_GEMV_VARIANT)")
     args = ap.parse_args()
+    if args.profile_prefill > 0:
+        return run_profile_prefill(args)
     if args.profile_layers > 0:
         return run_profile(args)
     if args.warmup < 3:
