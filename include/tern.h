@@ -38,8 +38,14 @@
  *     Errors raised while kernels run surface on the caller's next
  *     synchronisation, as for any CUDA work.
  *   - K must be a positive multiple of 128; M and N must be >= 1.
- *   - x, slots, codes and y must be 16-byte aligned; scales 16-byte aligned.
- *     (Allocations from cudaMalloc / PyTorch are 256-byte aligned.)
+ *   - x, slots, codes and y must be 16-byte aligned.  scales must be 16-byte
+ *     aligned for the products (tern_gemv, tern_gemm, tern_gemv_grouped, the
+ *     step calls and tern_gemv_noalloc) and 2-byte aligned for pack, unpack
+ *     and the embedding gather.  The products bring the scale rows on chip
+ *     with the tensor memory accelerator, whose global addresses must be
+ *     16-byte aligned; a misaligned scales pointer returns TERN_ERR_ALIGN
+ *     before any launch.  (Allocations from cudaMalloc / PyTorch are 256-byte
+ *     aligned, and a scale row is K/64 bytes.)
  *   - An invalid slot value (3) in tern_gemv / tern_gemm contributes an
  *     unspecified finite value for that weight; it never faults.  Validation
  *     is the job of tern_pack_g128.
@@ -116,6 +122,11 @@ size_t tern_workspace_bytes(int64_t M, int64_t N, int64_t K);
  *              slot value 3.  NULL to skip counting.
  * Alignment: codes and slots_out 16 bytes; scales 2 bytes.  Any N >= 1.
  * Result is bit-exact and independent of launch configuration.
+ * Format: ternary weights with one FP16 scale per 128-weight group ("Bonsai
+ * 27B ternary / 1-bit quantization", ThakiCloud blog, section "How
+ * compression works"), stored in 2-bit slots ("Ternary quantization: 27B in
+ * 7 GB", devnsb blog, section "Limits"); the code and bit order are this
+ * library's (see the top of this file).
  */
 tern_status tern_pack_g128(const int8_t *codes, const uint16_t *scales_in, int64_t N, int64_t K,
                            uint8_t *slots_out, uint16_t *scales_out, int32_t *invalid_count,
@@ -139,7 +150,13 @@ tern_status tern_unpack_g128(const uint8_t *slots, int64_t N, int64_t K, int8_t 
  *   y       fp16 [N]        (device, written)
  *   workspace / ws_bytes: optional, see tern_workspace_bytes.
  * Bandwidth-bound: the weights are streamed from HBM once, unpacked on chip
- * and never written back in any other precision.
+ * and never written back in any other precision.  Generation is bound by the
+ * weight bytes read per token ("Bonsai 27B ternary / 1-bit quantization",
+ * ThakiCloud blog, section "Throughput and speculative decoding"); the kernels
+ * read the packed slots directly and apply the group scale inside the
+ * product ("Ternary-Bonsai-27B" model summary, aitrends.kr, section
+ * "Technical features").  With K a multiple of 1024 it runs the decode-step
+ * kernel of tern_gemv_step (one product).
  */
 tern_status tern_gemv(const uint16_t *x, const uint8_t *slots, const uint16_t *scales, uint16_t *y,
                       int64_t N, int64_t K, void *workspace, size_t ws_bytes, void *stream);
@@ -151,7 +168,11 @@ tern_status tern_gemv(const uint16_t *x, const uint8_t *slots, const uint16_t *s
  * tern_gemv, reading the weights once for all rows.  M >= 32 runs the
  * tensor-core prefill kernel (tcgen05), which unpacks weight tiles on chip to
  * s*t (exact in fp16) straight into tensor memory and accumulates in fp32;
- * 8 < M < 32 runs the bandwidth kernel once per eight rows.
+ * 8 < M < 32 runs the bandwidth kernel once per eight rows.  Small M is the
+ * verification pass of speculative decoding (several drafted tokens checked
+ * in one pass of the target) and large M the compute-bound prompt
+ * processing ("Bonsai 27B ternary / 1-bit quantization", ThakiCloud blog,
+ * section "Throughput and speculative decoding").
  */
 tern_status tern_gemm(const uint16_t *x, const uint8_t *slots, const uint16_t *scales, uint16_t *y,
                       int64_t M, int64_t N, int64_t K, void *workspace, size_t ws_bytes,
