@@ -71,7 +71,8 @@ typedef enum tern_status {
     TERN_ERR_WORKSPACE = 4,   /* workspace smaller than tern_workspace_bytes() */
     TERN_ERR_CUDA = 5,        /* a CUDA runtime call or launch failed */
     TERN_ERR_TIMEOUT = 6,     /* a bounded on-device wait gave up (see tern_gemm) */
-    TERN_ERR_DEVICE = 7       /* current device is not compute capability 10.0 */
+    TERN_ERR_DEVICE = 7,      /* current device is not compute capability 10.0 */
+    TERN_ERR_GUARD = 8        /* an in-kernel index check failed (debug build only; see tern_sync_status) */
 } tern_status;
 
 /* Library version, e.g. 100 for 0.1.0. */
@@ -387,7 +388,10 @@ tern_status tern_t5_gemv_step(const tern_gemv_desc *descs, int32_t count, int64_
  * the previous call (TERN_ERR_TIMEOUT), clearing that record.  No kernel of
  * this library spins without a limit: a wait that exceeds it (1 s by default)
  * makes the kernel stop, release its resources and return, leaving its output
- * undefined and the CUDA context usable.
+ * undefined and the CUDA context usable.  A library built with in-kernel
+ * index checks (build.py: debug) also reports TERN_ERR_GUARD when a check in
+ * the decode-step kernels failed since the previous call (the access was
+ * skipped, nothing trapped); the normal build has no such checks.
  */
 tern_status tern_sync_status(void *stream);
 

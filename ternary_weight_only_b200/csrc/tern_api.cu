@@ -240,6 +240,7 @@ const char *tern_status_string(int status) {
         case TERN_ERR_CUDA: return "CUDA error";
         case TERN_ERR_TIMEOUT: return "device wait timed out";
         case TERN_ERR_DEVICE: return "unsupported device";
+        case TERN_ERR_GUARD: return "in-kernel index check failed";
         default: return "unknown status";
     }
 }
@@ -544,6 +545,10 @@ tern_status tern_sync_status(void *stream) {
     if (v == 0) v = z;
     if (v == 0) v = t6;
     if (v != 0) return fail(static_cast<tern_status>(v), "a kernel gave up a bounded wait on the device");
+    unsigned int guard = 0;
+    st = read_gemvstep_guard(true, &guard);
+    if (st != TERN_OK) return st;
+    if (guard != 0) return fail(TERN_ERR_GUARD, "%u in-kernel index checks failed (debug build)", guard);
     return TERN_OK;
 }
 

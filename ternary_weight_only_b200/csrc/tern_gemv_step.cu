@@ -71,6 +71,8 @@ namespace tern {
 
 // Device-side record of a bounded wait in this kernel that gave up.
 __device__ unsigned int g_tern_gemvstep_status;
+// Failed in-kernel index checks (debug build; see TERN_GUARD).
+__device__ unsigned int g_tern_gemvstep_guard;
 
 namespace {
 
@@ -434,7 +436,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_step_kernel(const __grid_con
                 const int m = idx / nit, it = idx - m * nit;
                 const int c32 = it >> 1, fp = it & 1, base = c32 << 5;
                 uint32_t hv[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};  // element e = half (e & 1) of hv[e >> 1]
-                if (m < M) {
+                if (m < M && TERN_GUARD(base + 32 <= K, g_tern_gemvstep_guard)) {
                     const __half *src = d.x + static_cast<size_t>(m) * d.xs + base;
                     if constexpr (FA == 0) {
                         uint4 v[4];
@@ -494,10 +496,14 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_step_kernel(const __grid_con
                 const int set = MT == 1 ? u * 4 + (G8 & 3) : u * 8 + G8;
                 const int col0 = MT == 1 ? 4 * (G8 >> 2) : 4 * m;
 #pragma unroll
-                for (int s2 = 0; s2 < 4; s2++)
-                    *reinterpret_cast<uint4 *>(xs8 + (((set * 2 + fp) * 32 + 4 * (col0 + s2) + qq) << 4)) =
-                        make_uint4(w[s2][0], w[s2][1], w[s2][2], w[s2][3]);
-                if ((lane & 7) == 0) egrp[m * (K >> 7) + (base >> 7)] = static_cast<int8_t>(eC);
+                for (int s2 = 0; s2 < 4; s2++) {
+                    const int xo = ((set * 2 + fp) * 32 + 4 * (col0 + s2) + qq) << 4;
+                    if (TERN_GUARD(xo + 16 <= xs_bytes(kcta, MT, X8), g_tern_gemvstep_guard))
+                        *reinterpret_cast<uint4 *>(xs8 + xo) = make_uint4(w[s2][0], w[s2][1], w[s2][2], w[s2][3]);
+                }
+                const int eo = m * (K >> 7) + (base >> 7);
+                if ((lane & 7) == 0 && TERN_GUARD(eo < MT * (p.kmax >> 7), g_tern_gemvstep_guard))
+                    egrp[eo] = static_cast<int8_t>(eC);
             }
             __syncthreads();
             // one all-ones chain per set (A = weight code 1, or bit 1, in every
@@ -523,8 +529,9 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_step_kernel(const __grid_con
                     const int m = MT == 1 ? 0 : (q >> 1);
                     const int eC = egrp[m * (K >> 7) + u * 8 + G8];
                     const float fac = __int_as_float((127 + 16 * (q & 1) - eC) << 23);
-                    recs[sl * 4 + q] = FA == 0 ? make_int4(-c[0], -c[1], __float_as_int(fac), 0)
-                                              : make_int4(c[0] + c[1] * 256, 0, __float_as_int(fac), 0);
+                    if (TERN_GUARD(sl * 4 + q < p.kmax / 64 * MT, g_tern_gemvstep_guard))
+                        recs[sl * 4 + q] = FA == 0 ? make_int4(-c[0], -c[1], __float_as_int(fac), 0)
+                                                   : make_int4(c[0] + c[1] * 256, 0, __float_as_int(fac), 0);
                 }
             }
             __syncthreads();
@@ -567,8 +574,9 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_step_kernel(const __grid_con
                 const uint32_t pr[4] = {v.x, v.y, v.z, v.w};
                 const int kl = c8 * 8;
                 const int gk = kl >> 7;
-                unsigned short *dst = reinterpret_cast<unsigned short *>(
-                    xs + (gk / GPB) * 1024 + b1_xs_index((gk % GPB) * MT + m, kl & 127));
+                const int bi = (gk / GPB) * 1024 + b1_xs_index((gk % GPB) * MT + m, kl & 127);
+                unsigned short *dst = reinterpret_cast<unsigned short *>(xs + bi);
+                if (!TERN_GUARD((bi + 263) * 2 <= xs_bytes(kcta, MT, X8), g_tern_gemvstep_guard)) continue;
 #pragma unroll
                 for (int c = 0; c < 4; c++) {
                     uint32_t h2;
@@ -594,8 +602,9 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_step_kernel(const __grid_con
                 const uint32_t pr[4] = {v.x, v.y, v.z, v.w};
                 const int kl = c8 * 8;
                 const int gk = kl >> 7;
-                unsigned short *dst = reinterpret_cast<unsigned short *>(
-                    xs + xs_pair_index<8>((gk % GPB) * MT + m, ((gk / GPB) << 7) | (kl & 127)));
+                const int bi = xs_pair_index<8>((gk % GPB) * MT + m, ((gk / GPB) << 7) | (kl & 127));
+                unsigned short *dst = reinterpret_cast<unsigned short *>(xs + bi);
+                if (!TERN_GUARD((bi + 773) * 2 <= xs_bytes(kcta, MT, X8), g_tern_gemvstep_guard)) continue;
 #pragma unroll
                 for (int c = 0; c < 4; c++) {
                     uint32_t h2;
@@ -730,7 +739,12 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_step_kernel(const __grid_con
                         uint4 xq[4];
 #pragma unroll
                         for (int h = 0; h < 4; h++)
-                            xq[h] = *reinterpret_cast<const uint4 *>(xs8 + ((((kb * 4 + h) * 2 + fp) * 32 + lane) << 4));
+                        {
+                            const int xo = (((kb * 4 + h) * 2 + fp) * 32 + lane) << 4;
+                            xq[h] = TERN_GUARD(xo + 16 <= xs_bytes(kcta, MT, X8), g_tern_gemvstep_guard)
+                                        ? *reinterpret_cast<const uint4 *>(xs8 + xo)
+                                        : make_uint4(0u, 0u, 0u, 0u);
+                        }
 #pragma unroll
                         for (int fi = 0; fi < 2; fi++) {
 #pragma unroll
@@ -778,8 +792,12 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_step_kernel(const __grid_con
                             uint4 xq[4];
 #pragma unroll
                             for (int j = 0; j < 4; j++)
-                                xq[j] = *reinterpret_cast<const uint4 *>(
-                                    xs8 + ((((kb * 8 + 4 * hf + j) * 2 + fp) * 32 + lane) << 4));
+                            {
+                                const int xo = (((kb * 8 + 4 * hf + j) * 2 + fp) * 32 + lane) << 4;
+                                xq[j] = TERN_GUARD(xo + 16 <= xs_bytes(kcta, MT, X8), g_tern_gemvstep_guard)
+                                            ? *reinterpret_cast<const uint4 *>(xs8 + xo)
+                                            : make_uint4(0u, 0u, 0u, 0u);
+                            }
 #pragma unroll
                             for (int fi = 0; fi < 2; fi++) {
 #pragma unroll
@@ -1127,6 +1145,19 @@ tern_status launch_gemv_step(const MatDesc *md, int count, int M, int fmt, cudaS
         if (st != TERN_OK) return st;
         done += n;
     }
+    return TERN_OK;
+}
+
+tern_status read_gemvstep_guard(bool reset, unsigned int *out) {
+    unsigned int v = 0;
+    cudaError_t e = cudaMemcpyFromSymbol(&v, g_tern_gemvstep_guard, sizeof(v));
+    if (e != cudaSuccess) return cuda_fail(e, "reading device guard count");
+    if (reset && v != 0) {
+        const unsigned int zero = 0;
+        e = cudaMemcpyToSymbol(g_tern_gemvstep_guard, &zero, sizeof(zero));
+        if (e != cudaSuccess) return cuda_fail(e, "clearing device guard count");
+    }
+    *out = v;
     return TERN_OK;
 }
 

@@ -119,6 +119,23 @@ tern_status read_gemvstep_status(bool reset, unsigned int *out);
 extern unsigned long long g_gemm_timeout_ns;
 extern int g_gemm_skip_loads;
 
+// ---- debug build: in-kernel index checks -----------------------------------
+// Compiled with -DTERN_DEBUG_GUARDS, TERN_GUARD(ok, counter) counts a failed
+// check in the device word `counter` and yields false, so that the access it
+// protects is skipped (no trap, the context stays usable); in the normal
+// build it is the constant true and costs nothing.
+#ifdef TERN_DEBUG_GUARDS
+#define TERN_GUARD(ok, counter) (tern::guard_check((ok), &(counter)))
+#else
+#define TERN_GUARD(ok, counter) true
+#endif
+__device__ __forceinline__ bool guard_check(bool ok, unsigned int *counter) {
+    if (!ok) atomicAdd(counter, 1u);
+    return ok;
+}
+// Failed index checks of the step kernel since the last read (0 in the normal build).
+tern_status read_gemvstep_guard(bool reset, unsigned int *out);
+
 // ---- device helpers -------------------------------------------------------
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));

@@ -28,6 +28,7 @@ TERN_ERR_WORKSPACE = 4
 TERN_ERR_CUDA = 5
 TERN_ERR_TIMEOUT = 6
 TERN_ERR_DEVICE = 7
+TERN_ERR_GUARD = 8
 
 TERN_OPT_GEMV_KSPLIT = 1
 TERN_OPT_GEMV_CLUSTER = 2

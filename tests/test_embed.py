@@ -62,12 +62,38 @@ def test_invalid_ids_zero_rows_and_counted(T, orc):
 
 
 def test_many_rows_and_single_row(T, orc):
-    """70000 rows (more than one grid row per block) and a single row."""
+    """70000 rows at K = 256 and a single row."""
     V, K = 200, 256
     slots, sc = table(orc, V, K, seed=5)
     rng = np.random.default_rng(9)
     check(T, orc, slots, sc, K, rng.integers(-2, V + 2, size=70000).astype(np.int32))
     check(T, orc, slots, sc, K, np.array([123], dtype=np.int32))
+
+
+def test_grid_stride_reuse_and_tail_guard(T, orc):
+    """More 64-weight items than the capped grid holds (70000 rows x K = 512
+    -> 560000 items against 148 SMs x 16 blocks x 4 warps x 32 = 303104), so
+    every warp takes a second pass and reuses its shared-memory stage; the
+    row count leaves a ragged last warp item; a canary written after the
+    output must be untouched."""
+    V, K = 300, 512
+    slots, sc = table(orc, V, K, seed=6, neg=True)
+    rng = np.random.default_rng(10)
+    ids = rng.integers(-2, V + 2, size=70001).astype(np.int32)
+    M = ids.size
+    canary = 4096
+    buf = torch.full((M * K + canary,), -7.0, dtype=torch.float16, device="cuda")
+    out = buf[: M * K].view(M, K)
+    bad = torch.zeros(1, dtype=torch.int32, device="cuda")
+    T.tern_embed_gather(torch.from_numpy(ids).cuda(), torch.from_numpy(slots).cuda(),
+                        torch.from_numpy(sc.view(np.int16)).cuda().view(torch.float16), K, out=out, bad_count=bad)
+    T.tern_sync_status()
+    want, nbad = orc.embed(slots, sc, K, ids)
+    got = out.cpu().float().double().numpy()
+    assert int(bad.item()) == nbad
+    assert np.array_equal(got, want)
+    assert np.array_equal(np.signbit(got), np.signbit(want))
+    assert bool(torch.all(buf[M * K:] == -7.0)), "the gather wrote past its output"
 
 
 def test_tied_head_table(T, orc):
