@@ -471,26 +471,32 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_step_kernel(const __grid_con
                 int eC = 0;
                 if (mx != 0) eC = 29 - (mx >= 0x400u ? static_cast<int>(mx >> 10) - 15 : (31 - __clz(mx)) - 24);
                 const int e0 = 127 + eC - 4 * fp;  // biased exponent of 2^(eC - 4 fp)
+                // w[s][j]: fragment word j of digit s.  The four x of one word
+                // (2-bit slots: word (e & 1) * 2 + (e >> 3), byte (e >> 1) & 3;
+                // 1-bit: word e & 3, byte e >> 2) are converted together: the
+                // signed base-256 digits of X are the bytes of
+                // (X + 0x80808080) ^ 0x80808080 (exact for |X| < 2^31 - 2^24), and a
+                // 4 x 4 byte transpose puts digit s of the four x into word s.
                 uint32_t w[4][4];
 #pragma unroll
-                for (int s2 = 0; s2 < 4; s2++)
+                for (int j = 0; j < 4; j++) {
+                    uint32_t D[4];
 #pragma unroll
-                    for (int j = 0; j < 4; j++) w[s2][j] = 0u;
-#pragma unroll
-                for (int e = 0; e < 16; e++) {
-                    // field shift beyond 4 fp, and the element's place in the fragment
-                    const int sh = FA == 0 ? 2 * (e & 1) : (e & 3);
-                    const int wi = FA == 0 ? (e & 1) * 2 + (e >> 3) : (e & 3);
-                    const int by = FA == 0 ? (e >> 1) & 3 : (e >> 2);
-                    const float xv = __half2float(__ushort_as_half(static_cast<unsigned short>(hv[e >> 1] >> (16 * (e & 1)))));
-                    int X = __float2int_rn(xv * __int_as_float((e0 - sh) << 23));
-#pragma unroll
-                    for (int s2 = 0; s2 < 3; s2++) {
-                        const int dg = static_cast<int>(static_cast<int8_t>(X & 0xFF));
-                        w[s2][wi] |= static_cast<uint32_t>(dg & 0xFF) << (8 * by);
-                        X = static_cast<int>(static_cast<uint32_t>(X) - static_cast<uint32_t>(dg)) >> 8;
+                    for (int b4 = 0; b4 < 4; b4++) {
+                        // element e holding byte b4 of word j
+                        const int e = FA == 0 ? (j >> 1) + ((j & 1) << 3) + (b4 << 1) : (b4 << 2) + j;
+                        const int sh = FA == 0 ? 2 * (e & 1) : (e & 3);
+                        const float xv =
+                            __half2float(__ushort_as_half(static_cast<unsigned short>(hv[e >> 1] >> (16 * (e & 1)))));
+                        const int X = __float2int_rn(xv * __int_as_float((e0 - sh) << 23));
+                        D[b4] = (static_cast<uint32_t>(X) + 0x80808080u) ^ 0x80808080u;
                     }
-                    w[3][wi] |= static_cast<uint32_t>(X & 0xFF) << (8 * by);
+                    const uint32_t t0 = __byte_perm(D[0], D[1], 0x5140), t1 = __byte_perm(D[0], D[1], 0x7362);
+                    const uint32_t t2 = __byte_perm(D[2], D[3], 0x5140), t3 = __byte_perm(D[2], D[3], 0x7362);
+                    w[0][j] = __byte_perm(t0, t2, 0x5410);
+                    w[1][j] = __byte_perm(t0, t2, 0x7632);
+                    w[2][j] = __byte_perm(t1, t3, 0x5410);
+                    w[3][j] = __byte_perm(t1, t3, 0x7632);
                 }
                 const int u = base >> 10, G8 = (base >> 7) & 7, qq = (base >> 5) & 3;
                 const int set = MT == 1 ? u * 4 + (G8 & 3) : u * 8 + G8;
@@ -673,8 +679,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_step_kernel(const __grid_con
             dead = dead || !ok;
             if (ok) {
                 uint32_t wd[kSG][kWords];
-#pragma unroll
-                for (int G8 = 0; G8 < kSG; G8++) {
+                // the lane's words of group G8 of the stage
+                auto load_wd = [&](int G8) {
                     if constexpr (F == 2) {
                         const uint8_t *pw = stage + off[G8 & 1] + 52 * (G8 >> 1);
                         const uint32_t sh = off[2 + (G8 & 1)];
@@ -692,7 +698,13 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_step_kernel(const __grid_con
                         wd[G8][0] = *reinterpret_cast<const uint32_t *>(stage + off[G8]);
                         wd[G8][1] = *reinterpret_cast<const uint32_t *>(stage + off[G8] + 8 * kBox);
                     }
-                }
+                };
+                // The digit form at two token rows reads the second half of
+                // the stage after the first half's mmas (fewer live registers)
+                // and refills the stage only then.
+                constexpr bool kLate = X8 && MT == 2;
+#pragma unroll
+                for (int G8 = 0; G8 < (kLate ? kSG / 2 : kSG); G8++) load_wd(G8);
                 // scales of the lane's groups (rows `row`, `row` + 8): MT = 1
                 // groups 2q, 2q+1; MT = 2, 4: one group per set h (4h + q, or
                 // 2h + q/2); MT = 8: all eight groups of both rows
@@ -720,12 +732,15 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_step_kernel(const __grid_con
                 // The stage is in registers: refill it with this warp's next
                 // unit (the warp barrier and the proxy fence order the reads
                 // before the copy that overwrites it).
-                __syncwarp();
-                consumed++;
-                if (ic.i >= 0) {
-                    if (lane == 0) asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-                    issue(s);
-                }
+                auto refill = [&]() {
+                    __syncwarp();
+                    consumed++;
+                    if (ic.i >= 0) {
+                        if (lane == 0) asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                        issue(s);
+                    }
+                };
+                if constexpr (!kLate) refill();
                 if constexpr (X8 && MT == 1) {
                     // four sets of two groups (h, h + 4); lanes q < 2 keep
                     // group h, lanes q >= 2 group h + 4.  acc[0] = row g,
@@ -782,6 +797,11 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_step_kernel(const __grid_con
                     const uint32_t sw[2][4] = {{s8a.x, s8a.y, s8a.z, s8a.w}, {s8b.x, s8b.y, s8b.z, s8b.w}};
 #pragma unroll
                     for (int hf = 0; hf < 2; hf++) {
+                        if (hf == 1) {
+#pragma unroll
+                            for (int G8 = kSG / 2; G8 < kSG; G8++) load_wd(G8);
+                            refill();
+                        }
                         int dd[4][4];
                         int2 rr[4];
 #pragma unroll
