@@ -432,11 +432,14 @@ tern_status tern_sync_status(void *stream);
  *                          0 or n <= ring depth = none (the default: measured
  *                          slower)
  *   TERN_OPT_STEP_FORM     arithmetic of the decode-step kernels (all three
- *                          weight storages) at M = 1 and 2: 0 = default (the
- *                          digit form: 8-bit integer mma on weights unpacked
- *                          four per instruction against activations split
- *                          into four exact signed 8-bit digits), 1 = the fp16
- *                          group-per-column form used for every other M
+ *                          weight storages): 0 = default (M = 1, 2: the digit
+ *                          form -- 8-bit integer mma on weights unpacked four
+ *                          per instruction against activations split into
+ *                          four exact signed 8-bit digits; M = 3..8: the fp16
+ *                          group-per-column form), 1 = the fp16 form at every
+ *                          M, 2 = the digit form also at M = 3, 4 (measured
+ *                          slower there: its staged activations leave one ring
+ *                          stage per warp)
  *   TERN_OPT_TEST_STALL_US TESTS ONLY: the TMA loaders of the tensor-core and
  *                          the TMA-staged bandwidth kernels issue no loads, so
  *                          their waits can never complete, and every bounded

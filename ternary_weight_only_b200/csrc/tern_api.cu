@@ -180,8 +180,8 @@ tern_status launch_bandwidth(const MatDesc *d, int count, int M, void *workspace
     // rules hold -- measured faster than the per-matrix kernels on every
     // decode shape alone and grouped (head 5120 x 151936: 38.7 us against
     // 52.4 us; gate + up: 13.7 against 18.4 us).
-    if (g_opt.gemv_variant == kVarDefault && M == 1 && gemv_step_supports(d, count, 1, 0))
-        return launch_gemv_step(d, count, 1, 0, s);
+    if (g_opt.gemv_variant == kVarDefault && M == 1 && gemv_step_supports(d, count, 1, 0, gemv_step_digit_form(1, 0)))
+        return launch_gemv_step(d, count, 1, 0, gemv_step_digit_form(1, 0), s);
     if (use_tc(M)) return launch_gemv_tc(d, count, M, workspace, ws_bytes, s);
     // Default: the producer/consumer kernel where its shape rules hold (K a
     // multiple of 1024, x fits its shared memory), else the TMA-staged one.
@@ -369,6 +369,48 @@ tern_status tern_embed_gather(const int32_t *ids, int64_t M, const uint8_t *slot
 }
 
 namespace {
+// Products whose M rows of x do not fit in shared memory beside the rings run
+// as K segments of whole 1024-k units that do, in calls of their own: segment
+// 0 (with every product that fits) writes y, each later segment adds its sum
+// to y.  Each weight is still read once.  Fills seg[s][0..n[s]) for segments
+// s < nseg_max (everything in segment 0 when every product fits).
+tern_status plan_step_segments(const MatDesc *d, int count, int m, int fmt, bool x8, const char *name,
+                               MatDesc (&seg)[8][TERN_MAX_STEP], int (&n)[8], int &nseg_max) {
+    nseg_max = 1;
+    for (int s = 0; s < 8; s++) n[s] = 0;
+    const int unit_bytes = fmt == 0 ? 256 : (fmt == 1 ? 128 : 208);  // weight bytes of one 1024-k row unit
+    for (int i = 0; i < count; i++) {
+        if (gemv_step_fits(d[i].K, m, fmt, x8)) {
+            seg[0][n[0]++] = d[i];
+            continue;
+        }
+        const int B = d[i].K / 1024;
+        int bfit = B - 1;
+        while (bfit > 0 && !gemv_step_fits(bfit * 1024, m, fmt, x8)) bfit--;
+        if (bfit == 0) return fail(TERN_ERR_SHAPE, "%s: M x 1024 too large for shared memory", name);
+        const int nseg = (B + bfit - 1) / bfit;
+        if (nseg > 8) return fail(TERN_ERR_SHAPE, "%s: K=%d needs more than 8 segments at M=%d", name, d[i].K, m);
+        nseg_max = std::max(nseg_max, nseg);
+        for (int sgi = 0; sgi < nseg; sgi++) {
+            const int u0 = sgi * B / nseg, u1 = (sgi + 1) * B / nseg;
+            MatDesc e = d[i];
+            e.x = d[i].x + static_cast<size_t>(u0) * 1024;
+            e.slots = d[i].slots + static_cast<size_t>(u0) * unit_bytes;
+            e.scales = d[i].scales + static_cast<size_t>(u0) * (1024 / kGroup);
+            e.K = (u1 - u0) * 1024;
+            e.kfull = d[i].K;
+            e.accum = sgi > 0;
+            seg[sgi][n[sgi]++] = e;
+        }
+    }
+    for (int sgi = 0; sgi < nseg_max; sgi++) {
+        if (n[sgi] == 0) continue;
+        if (!gemv_step_supports(seg[sgi], n[sgi], m, fmt, x8))
+            return fail(TERN_ERR_SHAPE, "%s: M x K too large for shared memory", name);
+    }
+    return TERN_OK;
+}
+
 tern_status gemv_step_api(const tern_gemv_desc *descs, int32_t count, int64_t M, int fmt, const char *name,
                           void *stream) {
     clear_error();
@@ -391,46 +433,21 @@ tern_status gemv_step_api(const tern_gemv_desc *descs, int32_t count, int64_t M,
     }
     const int m = static_cast<int>(M);
     cudaStream_t st_ = static_cast<cudaStream_t>(stream);
-    if (gemv_step_supports(d, count, m, fmt)) return launch_gemv_step(d, count, m, fmt, st_);
-    // Products whose M rows of x do not fit in shared memory beside the
-    // rings run as K segments of whole 1024-k units that do, in calls of
-    // their own: segment 0 (with every product that fits) writes y, each
-    // later segment adds its sum to y.  Each weight is still read once.
+    // The digit form by default (M <= 4); a call whose products the digit
+    // form cannot cut into at most eight K segments (its staged x takes twice
+    // the room) runs in the fp16 form instead.
+    bool x8 = gemv_step_digit_form(m, fmt);
     thread_local MatDesc seg[8][TERN_MAX_STEP];
     int nseg_max = 1, n[8] = {0};
-    const int unit_bytes = fmt == 0 ? 256 : (fmt == 1 ? 128 : 208);  // weight bytes of one 1024-k row unit
-    for (int i = 0; i < count; i++) {
-        if (gemv_step_fits(d[i].K, m, fmt)) {
-            seg[0][n[0]++] = d[i];
-            continue;
-        }
-        const int B = d[i].K / 1024;
-        int bfit = B - 1;
-        while (bfit > 0 && !gemv_step_fits(bfit * 1024, m, fmt)) bfit--;
-        if (bfit == 0) return fail(TERN_ERR_SHAPE, "%s: M x 1024 too large for shared memory", name);
-        const int nseg = (B + bfit - 1) / bfit;
-        if (nseg > 8) return fail(TERN_ERR_SHAPE, "%s: K=%d needs more than 8 segments at M=%d", name, d[i].K, m);
-        nseg_max = std::max(nseg_max, nseg);
-        for (int sgi = 0; sgi < nseg; sgi++) {
-            const int u0 = sgi * B / nseg, u1 = (sgi + 1) * B / nseg;
-            MatDesc e = d[i];
-            e.x = d[i].x + static_cast<size_t>(u0) * 1024;
-            e.slots = d[i].slots + static_cast<size_t>(u0) * unit_bytes;
-            e.scales = d[i].scales + static_cast<size_t>(u0) * (1024 / kGroup);
-            e.K = (u1 - u0) * 1024;
-            e.kfull = d[i].K;
-            e.accum = sgi > 0;
-            seg[sgi][n[sgi]++] = e;
-        }
+    tern_status st = plan_step_segments(d, count, m, fmt, x8, name, seg, n, nseg_max);
+    if (st == TERN_ERR_SHAPE && x8) {
+        x8 = false;
+        st = plan_step_segments(d, count, m, fmt, x8, name, seg, n, nseg_max);
     }
+    if (st != TERN_OK) return st;
     for (int sgi = 0; sgi < nseg_max; sgi++) {
         if (n[sgi] == 0) continue;
-        if (!gemv_step_supports(seg[sgi], n[sgi], m, fmt))
-            return fail(TERN_ERR_SHAPE, "%s: M x K too large for shared memory", name);
-    }
-    for (int sgi = 0; sgi < nseg_max; sgi++) {
-        if (n[sgi] == 0) continue;
-        tern_status st = launch_gemv_step(seg[sgi], n[sgi], m, fmt, st_);
+        st = launch_gemv_step(seg[sgi], n[sgi], m, fmt, x8, st_);
         if (st != TERN_OK) return st;
     }
     return TERN_OK;
@@ -572,7 +589,7 @@ tern_status tern_set_option(int option, int64_t value) {
         case TERN_OPT_GEMV_GRID: g_opt.gemv_grid = static_cast<int>(value); return TERN_OK;
         case TERN_OPT_GEMV_PREFETCH: g_opt.gemv_prefetch = static_cast<int>(value); return TERN_OK;
         case TERN_OPT_STEP_FORM:
-            if (value > 1) return fail(TERN_ERR_INVALID_ARG, "step form %lld", static_cast<long long>(value));
+            if (value > 2) return fail(TERN_ERR_INVALID_ARG, "step form %lld", static_cast<long long>(value));
             g_opt.step_form = static_cast<int>(value);
             return TERN_OK;
         case TERN_OPT_TEST_STALL_US:

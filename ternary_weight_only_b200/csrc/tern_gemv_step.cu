@@ -27,7 +27,7 @@
 // never depend on the preceding launch or piece.
 //
 // Arithmetic: the group-per-column mma.sync form (tern_unpack_mma.cuh), or,
-// at one or two token rows, the digit form below (all three storages).
+// at one to four token rows, the digit form below (all three storages).
 //
 // Digit form (X8): mma.sync m16n8k32 with unsigned 8-bit weights and signed
 // 8-bit activations, exact 32-bit integer sums.  One AND of a slot word with
@@ -37,7 +37,8 @@
 // row: X = rint(x * 2^(eC - 2f)) with eC = 29 - floor(log2 max|x|) of the
 // group, so the field factor 4^f cancels and |X| < 2^30; X is split into
 // four signed base-256 digits, and the eight mma columns carry (group or
-// token, digit) pairs.  Every X of an element within 2^13 of its group's
+// token, digit) pairs (four token rows: two column sets of two tokens, fed
+// by the same unpacked weights).  Every X of an element within 2^13 of its group's
 // largest |x| is exact; smaller ones are off by at most 2^-24 of that largest
 // |x| (below the rounding of an fp32 sum).  A group's integer sums per digit
 // are exact, t = c - 1 is restored by starting each chain at minus the same
@@ -286,12 +287,14 @@ __device__ __forceinline__ void cursor_next(Cursor &c, const SParams &p, int T0,
 // is one group (columns 4 token + digit).
 template <int MT, int F, bool X8>
 __global__ void __launch_bounds__(kThreads, 1) gemv_step_kernel(const __grid_constant__ SParams p) {
-    static_assert(!X8 || MT <= 2, "digit form: one or two token rows");
+    static_assert(!X8 || MT <= 4, "digit form: one to four token rows");
     // digit-form arithmetic: ternary codes (2-bit slots, and five-per-byte
     // bytes once decoded to slot words) or 1-bit weights
     constexpr int FA = F == 1 ? 1 : 0;
     constexpr int GPB = 8 / MT;  // groups per set
-    constexpr int kSPU = MT == 1 ? 4 : 8;  // digit form: sets per 1024-k unit
+    // digit form: sets per 1024-k unit (MT = 4: two column sets per group,
+    // tokens 0, 1 and 2, 3)
+    constexpr int kSPU = MT == 1 ? 4 : (MT == 2 ? 8 : 16);
     constexpr int kSlotStage = slot_stage(F);
     constexpr int kStageBytes = stage_bytes(F);
     constexpr int kWords = F == 1 ? 2 : 4;  // weight words of a group a lane holds
@@ -499,8 +502,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_step_kernel(const __grid_con
                     w[3][j] = __byte_perm(t1, t3, 0x7632);
                 }
                 const int u = base >> 10, G8 = (base >> 7) & 7, qq = (base >> 5) & 3;
-                const int set = MT == 1 ? u * 4 + (G8 & 3) : u * 8 + G8;
-                const int col0 = MT == 1 ? 4 * (G8 >> 2) : 4 * m;
+                const int set = MT == 1 ? u * 4 + (G8 & 3) : (MT == 2 ? u * 8 + G8 : (u * 8 + G8) * 2 + (m >> 1));
+                const int col0 = MT == 1 ? 4 * (G8 >> 2) : (MT == 2 ? 4 * m : 4 * (m & 1));
 #pragma unroll
                 for (int s2 = 0; s2 < 4; s2++) {
                     const int xo = ((set * 2 + fp) * 32 + 4 * (col0 + s2) + qq) << 4;
@@ -531,8 +534,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_step_kernel(const __grid_con
                 }
                 if (g == 0) {
                     const int u = sl / kSPU, hs = sl - u * kSPU;
-                    const int G8 = MT == 1 ? hs + 4 * (q >> 1) : hs;
-                    const int m = MT == 1 ? 0 : (q >> 1);
+                    const int G8 = MT == 1 ? hs + 4 * (q >> 1) : (MT == 2 ? hs : hs >> 1);
+                    const int m = MT == 1 ? 0 : (MT == 2 ? (q >> 1) : 2 * (hs & 1) + (q >> 1));
                     const int eC = egrp[m * (K >> 7) + u * 8 + G8];
                     const float fac = __int_as_float((127 + 16 * (q & 1) - eC) << 23);
                     if (TERN_GUARD(sl * 4 + q < p.kmax / 64 * MT, g_tern_gemvstep_guard))
@@ -791,7 +794,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_step_kernel(const __grid_con
                         acc[0] = fmaf(sA[h] * fac, static_cast<float>(hi ? ib : ia), acc[0]);
                         acc[2] = fmaf(sB[h] * fac, static_cast<float>(hi ? jb : ja), acc[2]);
                     }
-                } else if constexpr (X8) {
+                } else if constexpr (X8 && MT == 2) {
                     // two tokens: one set per group, lane q holds token q / 2;
                     // four groups at a time.  acc[0] = row g, acc[2] = row g + 8.
                     const uint32_t sw[2][4] = {{s8a.x, s8a.y, s8a.z, s8a.w}, {s8b.x, s8b.y, s8b.z, s8b.w}};
@@ -843,6 +846,72 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_step_kernel(const __grid_con
                             const float fac = __int_as_float(recs[(kb * 8 + G8) * 4 + q].z);
                             acc[0] = fmaf(sa * fac, static_cast<float>(x8_join<FA>(dd[j][0], dd[j][1], rr[j].x)), acc[0]);
                             acc[2] = fmaf(sb * fac, static_cast<float>(x8_join<FA>(dd[j][2], dd[j][3], rr[j].x)), acc[2]);
+                        }
+                    }
+                } else if constexpr (X8 && MT == 4) {
+                    // two column sets per group (tokens 0, 1 and 2, 3), both
+                    // fed by the same A registers; two groups at a time.
+                    // acc[0] / acc[1] = row g, tokens q/2 and 2 + q/2;
+                    // acc[2] / acc[3] = row g + 8.
+                    const uint32_t sw[2][4] = {{s8a.x, s8a.y, s8a.z, s8a.w}, {s8b.x, s8b.y, s8b.z, s8b.w}};
+#pragma unroll
+                    for (int qt = 0; qt < 4; qt++) {
+                        int dd[2][2][4];
+                        int2 rr[2][2];
+#pragma unroll
+                        for (int j = 0; j < 2; j++)
+#pragma unroll
+                            for (int cs = 0; cs < 2; cs++)
+                                rr[j][cs] = *reinterpret_cast<const int2 *>(
+                                    recs + ((kb * 8 + 2 * qt + j) * 2 + cs) * 4 + q);
+#pragma unroll
+                        for (int fp = 0; fp < 2; fp++) {
+                            uint4 xq[2][2];
+#pragma unroll
+                            for (int j = 0; j < 2; j++)
+#pragma unroll
+                                for (int cs = 0; cs < 2; cs++) {
+                                    const int xo = ((((kb * 8 + 2 * qt + j) * 2 + cs) * 2 + fp) * 32 + lane) << 4;
+                                    xq[j][cs] = TERN_GUARD(xo + 16 <= xs_bytes(kcta, MT, X8), g_tern_gemvstep_guard)
+                                                    ? *reinterpret_cast<const uint4 *>(xs8 + xo)
+                                                    : make_uint4(0u, 0u, 0u, 0u);
+                                }
+#pragma unroll
+                            for (int fi = 0; fi < 2; fi++) {
+#pragma unroll
+                                for (int j = 0; j < 2; j++) {
+                                    uint32_t a0, a1, a2, a3;
+                                    x8_a<FA>(wd[2 * qt + j], 2 * fp + fi, a0, a1, a2, a3);
+#pragma unroll
+                                    for (int cs = 0; cs < 2; cs++) {
+                                        const uint4 &xv = xq[j][cs];
+                                        const uint32_t b0 = fi ? xv.z : xv.x, b1 = fi ? xv.w : xv.y;
+                                        if (fp == 0 && fi == 0)
+                                            imma_init(dd[j][cs], a0, a1, a2, a3, b0, b1, FA == 0 ? rr[j][cs].x : 0,
+                                                      FA == 0 ? rr[j][cs].y : 0);
+                                        else
+                                            imma_acc(dd[j][cs], a0, a1, a2, a3, b0, b1);
+                                    }
+                                }
+                            }
+                        }
+#pragma unroll
+                        for (int j = 0; j < 2; j++) {
+                            const int G8 = 2 * qt + j;
+                            const float sa = __half2float(__ushort_as_half(
+                                static_cast<unsigned short>(sw[0][G8 >> 1] >> (16 * (G8 & 1)))));
+                            const float sb = __half2float(__ushort_as_half(
+                                static_cast<unsigned short>(sw[1][G8 >> 1] >> (16 * (G8 & 1)))));
+#pragma unroll
+                            for (int cs = 0; cs < 2; cs++) {
+                                const float fac = __int_as_float(recs[((kb * 8 + G8) * 2 + cs) * 4 + q].z);
+                                acc[cs] = fmaf(sa * fac,
+                                               static_cast<float>(x8_join<FA>(dd[j][cs][0], dd[j][cs][1], rr[j][cs].x)),
+                                               acc[cs]);
+                                acc[2 + cs] = fmaf(sb * fac,
+                                                   static_cast<float>(x8_join<FA>(dd[j][cs][2], dd[j][cs][3], rr[j][cs].x)),
+                                                   acc[2 + cs]);
+                            }
                         }
                     }
                 } else if constexpr (MT == 8) {
@@ -902,7 +971,22 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_step_kernel(const __grid_con
             if (--to_end == 0) {
                 // ---- this warp's part of a tile is complete: sum the lanes q
                 // that hold other groups of the same tokens ----
-                if constexpr (X8 && MT == 2) {
+                if constexpr (X8 && MT == 4) {
+                    // lanes q, q ^ 1 hold the two digit pairs of tokens q / 2
+                    // (acc[0], acc[2]) and 2 + q / 2 (acc[1], acc[3]); lane 0
+                    // ends with tokens 0, 1 and lane 1 with tokens 2, 3 (rows g, g + 8)
+                    float o[4];
+#pragma unroll
+                    for (int c = 0; c < 4; c++) acc[c] += __shfl_xor_sync(0xffffffffu, acc[c], 1);
+#pragma unroll
+                    for (int c = 0; c < 4; c++) o[c] = __shfl_xor_sync(0xffffffffu, acc[c], 2);
+                    const bool odd = (q & 1) != 0;
+                    const float v0 = odd ? acc[1] : acc[0], v2 = odd ? acc[3] : acc[2];
+                    acc[0] = v0;
+                    acc[1] = odd ? o[1] : o[0];
+                    acc[2] = v2;
+                    acc[3] = odd ? o[3] : o[2];
+                } else if constexpr (X8 && MT == 2) {
                     // lanes q, q ^ 1 hold the two digit pairs of token q / 2:
                     // lane 0 ends with (row g: tokens 0, 1; row g + 8: 0, 1)
                     const float tg = acc[0] + __shfl_xor_sync(0xffffffffu, acc[0], 1);
@@ -991,9 +1075,14 @@ bool g_attr_step[64][3][4][2];
 using StepKernel = void (*)(SParams);
 StepKernel step_kernel(int mt, int f, bool x8) {
     if (x8) {
-        if (f == 0) return mt == 1 ? gemv_step_kernel<1, 0, true> : (mt == 2 ? gemv_step_kernel<2, 0, true> : nullptr);
-        if (f == 1) return mt == 1 ? gemv_step_kernel<1, 1, true> : (mt == 2 ? gemv_step_kernel<2, 1, true> : nullptr);
-        return mt == 1 ? gemv_step_kernel<1, 2, true> : (mt == 2 ? gemv_step_kernel<2, 2, true> : nullptr);
+        if (f == 0)
+            return mt == 1 ? gemv_step_kernel<1, 0, true>
+                           : (mt == 2 ? gemv_step_kernel<2, 0, true> : (mt == 4 ? gemv_step_kernel<4, 0, true> : nullptr));
+        if (f == 1)
+            return mt == 1 ? gemv_step_kernel<1, 1, true>
+                           : (mt == 2 ? gemv_step_kernel<2, 1, true> : (mt == 4 ? gemv_step_kernel<4, 1, true> : nullptr));
+        return mt == 1 ? gemv_step_kernel<1, 2, true>
+                       : (mt == 2 ? gemv_step_kernel<2, 2, true> : (mt == 4 ? gemv_step_kernel<4, 2, true> : nullptr));
     }
     if (f == 0)
         return mt == 1 ? gemv_step_kernel<1, 0, false>
@@ -1011,17 +1100,22 @@ int step_mt(int M) { return M == 1 ? 1 : (M == 2 ? 2 : (M <= 4 ? 4 : 8)); }
 int mt_index(int mt) { return mt == 1 ? 0 : (mt == 2 ? 1 : (mt == 4 ? 2 : 3)); }
 
 // The digit form serves every weight storage at one and two token rows
-// unless the group-per-column fp16 form is asked for (TERN_OPT_STEP_FORM = 1).
-bool step_x8(int M, int fmt) { return M <= 2 && g_opt.step_form != 1; }
+// unless the group-per-column fp16 form is asked for (TERN_OPT_STEP_FORM =
+// 1); at three and four rows only when asked for (= 2): its 16 bytes of
+// staged x per k leave one ring stage per warp at K = 5120 and 6144, and the
+// verify step at M = 4 measured 2.25 ms against 1.41 ms in the fp16 form.
+bool step_x8(int M, int fmt) { return g_opt.step_form == 1 ? false : M <= (g_opt.step_form == 2 ? 4 : 2); }
 
 }  // namespace
 
-bool gemv_step_fits(int K, int M, int fmt) {
-    return K % 1024 == 0 && M >= 1 && M <= (fmt == 1 ? 4 : 8) &&
-           smem_bytes(K, step_mt(M), 1, fmt, step_x8(M, fmt)) <= kSmemBudget;
+bool gemv_step_digit_form(int M, int fmt) { return step_x8(M, fmt); }
+
+bool gemv_step_fits(int K, int M, int fmt, bool x8) {
+    return K % 1024 == 0 && M >= 1 && M <= (fmt == 1 ? 4 : 8) && (!x8 || M <= 4) &&
+           smem_bytes(K, step_mt(M), 1, fmt, x8) <= kSmemBudget;
 }
 
-bool gemv_step_supports(const MatDesc *md, int count, int M, int fmt) {
+bool gemv_step_supports(const MatDesc *md, int count, int M, int fmt, bool x8) {
     if (count < 1 || count > TERN_MAX_STEP || M < 1 || M > (fmt == 1 ? 4 : 8)) return false;
     int kmax = 0;
     for (int i = 0; i < count; i++) {
@@ -1029,18 +1123,17 @@ bool gemv_step_supports(const MatDesc *md, int count, int M, int fmt) {
         kmax = std::max(kmax, md[i].K);
     }
     // one ring stage per warp at least (refilled as soon as it is read)
-    return smem_bytes(kmax, step_mt(M), 1, fmt, step_x8(M, fmt)) <= kSmemBudget;
+    return (!x8 || M <= 4) && smem_bytes(kmax, step_mt(M), 1, fmt, x8) <= kSmemBudget;
 }
 
 namespace {
 
 // One launch over md[0..count) (count <= kMaxPer).
-tern_status launch_chunk(const DeviceInfo &dev, const MatDesc *md, int count, int M, int fmt, bool first,
+tern_status launch_chunk(const DeviceInfo &dev, const MatDesc *md, int count, int M, int fmt, bool x8, bool first,
                          cudaStream_t stream) {
     thread_local SParams p;  // large (parameter space); filled on the host for each launch, per host thread
     std::memset(&p, 0, sizeof(p));
     const int mt = step_mt(M);
-    const bool x8 = step_x8(M, fmt);
     int kmax = 0;
     long long total_units = 0;
     int tiles = 0;
@@ -1141,13 +1234,12 @@ tern_status launch_chunk(const DeviceInfo &dev, const MatDesc *md, int count, in
 
 }  // namespace
 
-tern_status launch_gemv_step(const MatDesc *md, int count, int M, int fmt, cudaStream_t stream) {
+tern_status launch_gemv_step(const MatDesc *md, int count, int M, int fmt, bool x8, cudaStream_t stream) {
     DeviceInfo dev;
     tern_status st = current_device(&dev);
     if (st != TERN_OK) return st;
     if (fmt < 0 || fmt > 2) return fail(TERN_ERR_INVALID_ARG, "step kernel: unknown weight format %d", fmt);
-    const bool x8 = step_x8(M, fmt);
-    if (!gemv_step_supports(md, count, M, fmt) || step_kernel(step_mt(M), fmt, x8) == nullptr)
+    if (!gemv_step_supports(md, count, M, fmt, x8) || step_kernel(step_mt(M), fmt, x8) == nullptr)
         return fail(TERN_ERR_SHAPE, "step kernel: unsupported shapes");
     const int mi = mt_index(step_mt(M));
     if (!g_attr_step[dev.device][fmt][mi][x8]) {
@@ -1161,7 +1253,7 @@ tern_status launch_gemv_step(const MatDesc *md, int count, int M, int fmt, cudaS
     int done = 0;
     for (int l = 0; l < launches; l++) {
         const int n = (count - done) / (launches - l);
-        st = launch_chunk(dev, md + done, n, M, fmt, l == 0, stream);
+        st = launch_chunk(dev, md + done, n, M, fmt, x8, l == 0, stream);
         if (st != TERN_OK) return st;
         done += n;
     }

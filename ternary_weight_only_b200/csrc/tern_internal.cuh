@@ -111,10 +111,13 @@ tern_status launch_embed(const int32_t *ids, int64_t M, const uint8_t *slots, co
 // Persistent launch over many matrices (M = 1..8, 1..4 for fmt 1; K multiples of 1024); fmt 0
 // = ternary slots, 1 = the 1-bit variant (MatDesc::slots holds the bits), 2 =
 // five trits per byte (MatDesc::slots holds the base-3 bytes).
-bool gemv_step_supports(const MatDesc *d, int count, int M, int fmt);
+// x8: the digit form (M <= 4) or the fp16 group-per-column form.
+bool gemv_step_supports(const MatDesc *d, int count, int M, int fmt, bool x8);
 // whether one product of depth K at M token rows fits the step kernel
-bool gemv_step_fits(int K, int M, int fmt);
-tern_status launch_gemv_step(const MatDesc *d, int count, int M, int fmt, cudaStream_t stream);
+bool gemv_step_fits(int K, int M, int fmt, bool x8);
+// the form the step kernels use by default for M token rows (TERN_OPT_STEP_FORM)
+bool gemv_step_digit_form(int M, int fmt);
+tern_status launch_gemv_step(const MatDesc *d, int count, int M, int fmt, bool x8, cudaStream_t stream);
 tern_status read_gemvstep_status(bool reset, unsigned int *out);
 extern unsigned long long g_gemm_timeout_ns;
 extern int g_gemm_skip_loads;

@@ -236,12 +236,13 @@ def test_valid_call_without_gpu_reports_cuda_error(lib):
 
 def test_option_values(lib):
     """Kernel variants 1 and 5 were removed and are refused; the step form
-    takes 0 and 1 only; 0 restores every default."""
+    takes 0, 1 and 2 only; 0 restores every default."""
     from ternary_weight_only_b200 import tern as T
     for v in (1, 5, 7):
         assert lib.tern_set_option(T.TERN_OPT_GEMV_VARIANT, v) == T.TERN_ERR_INVALID_ARG
     for v in (0, 2, 3, 4, 6, 0):
         assert lib.tern_set_option(T.TERN_OPT_GEMV_VARIANT, v) == T.TERN_OK
-    assert lib.tern_set_option(T.TERN_OPT_STEP_FORM, 2) == T.TERN_ERR_INVALID_ARG
+    assert lib.tern_set_option(T.TERN_OPT_STEP_FORM, 3) == T.TERN_ERR_INVALID_ARG
+    assert lib.tern_set_option(T.TERN_OPT_STEP_FORM, 2) == T.TERN_OK
     assert lib.tern_set_option(T.TERN_OPT_STEP_FORM, 1) == T.TERN_OK
     assert lib.tern_set_option(T.TERN_OPT_STEP_FORM, 0) == T.TERN_OK

@@ -197,3 +197,18 @@ def test_long_rows_run_as_k_segments(T, orc, M, form):
     T.tern_b1_gemv_step(mats, M)
     T.tern_sync_status()
     check_all(orc, mats, refs, f"b1 step K segments M={M}")
+
+
+@pytest.mark.parametrize("M", [3, 4])
+def test_digit_form_at_three_and_four_rows(T, orc, M):
+    """The digit form at three and four token rows (TERN_OPT_STEP_FORM = 2);
+    mixed shapes and a row run as K segments; every output."""
+    shapes = [(1024, 40), (5120, 100), (17408, 48), (2048, 17), (40960, 20)]
+    mats, refs = make_mats(orc, shapes, seed=8400 + M, M=M)
+    T.tern_set_option(T.TERN_OPT_STEP_FORM, 2)
+    try:
+        T.tern_b1_gemv_step(mats, M)
+        T.tern_sync_status()
+    finally:
+        T.tern_set_option(T.TERN_OPT_STEP_FORM, 0)
+    check_all(orc, mats, refs, f"b1 digit form M={M}")

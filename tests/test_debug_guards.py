@@ -1,7 +1,7 @@
 """The debug build (libtern_debug.so: in-kernel index checks in the
 decode-step kernels, failed checks counted in a device word and reported by
 tern_sync_status as TERN_ERR_GUARD, no trap) on legal shapes: every form the
-step kernels take -- the three weight storages, one and two token rows in the
+step kernels take -- the three weight storages, one, two and four token rows in the
 digit form, the fp16 group-per-column form at 1, 2, 4 and 8 rows, products
 cut into K segments, several matrices per CTA -- reports no failed check and
 still matches the oracle.  This stands in for a memory checker, which cannot
@@ -35,7 +35,7 @@ def D():
 
 
 @pytest.mark.parametrize("fmt", ["tern", "b1", "t5"])
-@pytest.mark.parametrize("M,form", [(1, 0), (2, 0), (1, 1), (2, 1), (4, 1), (8, 1)])
+@pytest.mark.parametrize("M,form", [(1, 0), (2, 0), (3, 2), (4, 2), (1, 1), (2, 1), (4, 1), (8, 1)])
 def test_no_index_check_fails(D, orc, fmt, M, form):
     lib, T = D
     if fmt == "b1" and M > 4:
@@ -43,7 +43,7 @@ def test_no_index_check_fails(D, orc, fmt, M, form):
     from ternary_weight_only_b200 import synth
     # the last row is long enough to run as K segments (five-per-byte at
     # M = 8 takes at most eight segments of its shorter x room)
-    shapes = [(1024, 40), (3072, 333), (17408, 48), (2048, 17), (65536 if M < 8 else 24576, 20)]
+    shapes = [(1024, 40), (3072, 333), (17408, 48), (2048, 17), (65536 if M <= 2 else 24576, 20)]
     kind = "sign" if fmt == "b1" else "sparse"
     pack = {"tern": T.tern_pack_g128, "b1": T.tern_b1_pack, "t5": T.tern_t5_pack}[fmt]
     orc_pack = {"tern": orc.pack, "b1": orc.b1_pack, "t5": orc.t5_pack}[fmt]

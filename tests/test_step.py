@@ -379,3 +379,21 @@ def test_slot_value_3_is_finite_and_local(T, orc, M, form):
     clean = np.setdiff1d(np.arange(N), dirty)
     y_ref, bound = orc.matmul(xn, slots, sc, threads=NCPU)
     check_close(got[:, clean], y_ref[:, clean], bound[:, clean], f"clean rows with slot value 3 elsewhere M={M}")
+
+
+@pytest.mark.parametrize("M", [3, 4])
+def test_digit_form_at_three_and_four_rows(T, orc, M):
+    """The digit form at three and four token rows (TERN_OPT_STEP_FORM = 2:
+    two column sets of two tokens per group): mixed shapes, a decode layer,
+    and a row long enough to run as K segments; every output."""
+    from ternary_weight_only_b200 import synth
+    shapes = [(1024, 1), (2048, 17), (5120, 100), (3072, 333), (17408, 40)]
+    shapes += [(K, N) for _, K, N in synth.LAYER_PROJ] + [(40960, 24)]
+    mats, refs = make_mats(orc, shapes, seed=8300 + M, M=M)
+    T.tern_set_option(T.TERN_OPT_STEP_FORM, 2)
+    try:
+        T.tern_gemv_step(mats, M)
+        T.tern_sync_status()
+    finally:
+        T.tern_set_option(T.TERN_OPT_STEP_FORM, 0)
+    check_all(orc, mats, refs, f"digit form M={M}")

@@ -235,3 +235,18 @@ def test_invalid_bytes_give_finite_values_and_spare_other_rows(T, orc, form):
     good = [n for n in range(N) if n not in bad_rows]
     y_ref, bound = orc.t5_matmul(xn, packed[good], sc[good], threads=NCPU)
     check_close(y[good].view(1, -1), y_ref, bound, "t5 rows without invalid bytes")
+
+
+@pytest.mark.parametrize("M", [3, 4])
+def test_digit_form_at_three_and_four_rows(T, orc, M):
+    """The digit form at three and four token rows (TERN_OPT_STEP_FORM = 2);
+    mixed shapes and a row run as K segments; every output."""
+    shapes = [(1024, 40), (5120, 100), (17408, 48), (2048, 17), (24576, 20)]
+    mats, refs = make_mats(orc, shapes, seed=8400 + M, M=M)
+    T.tern_set_option(T.TERN_OPT_STEP_FORM, 2)
+    try:
+        T.tern_t5_gemv_step(mats, M)
+        T.tern_sync_status()
+    finally:
+        T.tern_set_option(T.TERN_OPT_STEP_FORM, 0)
+    check_all(orc, mats, refs, f"t5 digit form M={M}")
