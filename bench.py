@@ -6,9 +6,9 @@ q 5120->6144, k/v 5120->1024, o 6144->5120, gate/up 5120->17408,
 down 17408->5120, plus a 5120->151936 output head; M = 1; all weights
 ternary-g128 in 2-bit slots (6,000,015,360 bytes resident, far larger than
 the 126 MB L2, so every step streams cold weights from HBM).  Every projection
-gets its own fresh N(0,1) fp16 input, so the seven projections of a layer are
-independent and run as one grouped launch; the step is 65 launches captured
-in one CUDA graph.
+gets its own fresh N(0,1) fp16 input, so all 449 products of a step are
+independent and run as one tern_gemv_step call (five launches of at most 96
+products, overlapped), captured in one CUDA graph.
 
 Prints ONE JSON line (rank 0).  `--impl reference` times the fp64 CPU oracle
 on a bounded sample of the same workload instead.
