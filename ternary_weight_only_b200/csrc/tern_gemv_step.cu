@@ -407,7 +407,14 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_step_kernel(const __grid_con
         cursor_next(ic, p, T0, T1, warp);
         issued++;
     };
-    for (int st = 0; st < ns && ic.i >= 0; st++) issue(st);
+    // Only the first stage of every ring goes out before the first piece's
+    // activations are staged: the staging's small loads of x would otherwise
+    // queue in DRAM behind every SM's whole ring (~20 MB, ~3 us); one stage
+    // per warp (~10 MB in flight) still covers the staging.  The other stages
+    // follow right after it, before any stage is consumed and refilled, so
+    // stage st still holds the warp's unit st.
+    if (ns > 0 && ic.i >= 0) issue(0);
+    bool topped = false;
 
     if (p.first) {
         asm volatile("griddepcontrol.wait;" ::: "memory");
@@ -636,6 +643,10 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_step_kernel(const __grid_con
         __syncthreads();
         }  // fp16 staging
 
+        if (!topped) {
+            for (int st = 1; st < ns && ic.i >= 0; st++) issue(st);
+            topped = true;
+        }
         // Lanes q < kGcLanes hold complete sums after a tile's lane
         // reduction; lane (g, q) stores v = (row g: tokens t0, t1; row g+8:
         // tokens t0, t1), t0 = 2q, t1 = 2q + 1 (MT = 4), 0, 1 (MT = 2), or
