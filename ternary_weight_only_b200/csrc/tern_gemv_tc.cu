@@ -762,6 +762,9 @@ tern_status gemv_noalloc(const MatDesc &d, cudaStream_t stream) {
     DeviceInfo dev;
     tern_status st = current_device(&dev);
     if (st != TERN_OK) return st;
+    // (current_device refuses ordinals outside [0, 64); checked again here,
+    // where the per-device table is indexed)
+    if (dev.device < 0 || dev.device >= 64) return fail(TERN_ERR_DEVICE, "device ordinal %d out of range", dev.device);
     void *scratch = nullptr;
     {
         // One-time set-up per device, with that device current: the host can
