@@ -552,15 +552,35 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_step_kernel(const __grid_con
             }
             __syncthreads();
         } else {
+        // x of token m, elements 8 c8 .. 8 c8 + 7, for the staging items
+        // idx0 + u * nthr (u < kLd; idx = m * K / 8 + c8; zeros past tot or for
+        // padding tokens m >= M): at eight token rows (ten or more items per
+        // thread) loaded four at a time, so that a thread's global loads
+        // overlap instead of queueing one round trip per item.
+        constexpr int kLd = MT == 8 ? 4 : 1;
+        auto load_items = [&](int idx0, int tot, uint4 (&v)[kLd]) {
+            const int per_m = K / 8;
+#pragma unroll
+            for (int u = 0; u < kLd; u++) {
+                const int idx = idx0 + u * nthr;
+                const int m = idx / per_m, c8 = idx - m * per_m;
+                v[u] = make_uint4(0u, 0u, 0u, 0u);
+                if (idx < tot && m < M)
+                    v[u] = *reinterpret_cast<const uint4 *>(d.x + static_cast<size_t>(m) * d.xs + c8 * 8);
+            }
+        };
         {
             unsigned int mx = 0;
-            const int per_row = K / 8;
-            for (int idx = threadIdx.x; idx < M * per_row; idx += nthr) {
-                const int m = idx / per_row, c8 = idx - m * per_row;
-                const uint4 v = *reinterpret_cast<const uint4 *>(d.x + static_cast<size_t>(m) * d.xs + c8 * 8);
-                const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
+            const int tot = M * (K / 8);
+            for (int idx0 = threadIdx.x; idx0 < tot; idx0 += kLd * nthr) {
+                uint4 v[kLd];
+                load_items(idx0, tot, v);
 #pragma unroll
-                for (int e = 0; e < 4; e++) mx = __vmaxu2(mx, __vminu2(wv[e] & 0x7FFF7FFFu, 0x7BFF7BFFu));
+                for (int u = 0; u < kLd; u++) {
+                    const uint32_t wv[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+#pragma unroll
+                    for (int e = 0; e < 4; e++) mx = __vmaxu2(mx, __vminu2(wv[e] & 0x7FFF7FFFu, 0x7BFF7BFFu));
+                }
             }
             mx = max(mx & 0xFFFFu, mx >> 16);
             mx = __reduce_max_sync(0xffffffffu, mx);
@@ -582,23 +602,28 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_step_kernel(const __grid_con
             for (int c = 0; c < 4; c++)
                 fac2[c] = (static_cast<uint32_t>(15 + E - 2 * c) << 10) |
                           (static_cast<uint32_t>(15 + E - 2 * c - 1) << 26);
-            const int per_m = K / 8;
-            for (int idx = threadIdx.x; idx < MT * per_m; idx += nthr) {
-                const int m = idx / per_m, c8 = idx - m * per_m;
-                uint4 v = make_uint4(0u, 0u, 0u, 0u);
-                if (m < M) v = *reinterpret_cast<const uint4 *>(d.x + static_cast<size_t>(m) * d.xs + c8 * 8);
-                const uint32_t pr[4] = {v.x, v.y, v.z, v.w};
-                const int kl = c8 * 8;
-                const int gk = kl >> 7;
-                const int bi = (gk / GPB) * 1024 + b1_xs_index((gk % GPB) * MT + m, kl & 127);
-                unsigned short *dst = reinterpret_cast<unsigned short *>(xs + bi);
-                if (!TERN_GUARD((bi + 263) * 2 <= xs_bytes(kcta, MT, X8), g_tern_gemvstep_guard)) continue;
+            const int per_m = K / 8, tot = MT * per_m;
+            for (int idx0 = threadIdx.x; idx0 < tot; idx0 += kLd * nthr) {
+                uint4 v[kLd];
+                load_items(idx0, tot, v);
 #pragma unroll
-                for (int c = 0; c < 4; c++) {
-                    uint32_t h2;
-                    asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(h2) : "r"(pr[c]), "r"(fac2[c]));
-                    dst[(c >> 1) * 256 + (c & 1) * 4] = static_cast<unsigned short>(h2);
-                    dst[(c >> 1) * 256 + (c & 1) * 4 + 2] = static_cast<unsigned short>(h2 >> 16);
+                for (int u = 0; u < kLd; u++) {
+                    const int idx = idx0 + u * nthr;
+                    if (idx >= tot) break;
+                    const int m = idx / per_m, c8 = idx - m * per_m;
+                    const uint32_t pr[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+                    const int kl = c8 * 8;
+                    const int gk = kl >> 7;
+                    const int bi = (gk / GPB) * 1024 + b1_xs_index((gk % GPB) * MT + m, kl & 127);
+                    unsigned short *dst = reinterpret_cast<unsigned short *>(xs + bi);
+                    if (!TERN_GUARD((bi + 263) * 2 <= xs_bytes(kcta, MT, X8), g_tern_gemvstep_guard)) continue;
+#pragma unroll
+                    for (int c = 0; c < 4; c++) {
+                        uint32_t h2;
+                        asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(h2) : "r"(pr[c]), "r"(fac2[c]));
+                        dst[(c >> 1) * 256 + (c & 1) * 4] = static_cast<unsigned short>(h2);
+                        dst[(c >> 1) * 256 + (c & 1) * 4 + 2] = static_cast<unsigned short>(h2 >> 16);
+                    }
                 }
             }
         } else {
@@ -610,23 +635,28 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_step_kernel(const __grid_con
                 fac2[c] = (static_cast<uint32_t>(15 + e0) << 10) | (static_cast<uint32_t>(15 + e1) << 26);
             }
             // token m of group G sits in column (G % GPB) * MT + m of set G / GPB
-            const int per_m = K / 8;
-            for (int idx = threadIdx.x; idx < MT * per_m; idx += nthr) {
-                const int m = idx / per_m, c8 = idx - m * per_m;
-                uint4 v = make_uint4(0u, 0u, 0u, 0u);
-                if (m < M) v = *reinterpret_cast<const uint4 *>(d.x + static_cast<size_t>(m) * d.xs + c8 * 8);
-                const uint32_t pr[4] = {v.x, v.y, v.z, v.w};
-                const int kl = c8 * 8;
-                const int gk = kl >> 7;
-                const int bi = xs_pair_index<8>((gk % GPB) * MT + m, ((gk / GPB) << 7) | (kl & 127));
-                unsigned short *dst = reinterpret_cast<unsigned short *>(xs + bi);
-                if (!TERN_GUARD((bi + 773) * 2 <= xs_bytes(kcta, MT, X8), g_tern_gemvstep_guard)) continue;
+            const int per_m = K / 8, tot = MT * per_m;
+            for (int idx0 = threadIdx.x; idx0 < tot; idx0 += kLd * nthr) {
+                uint4 v[kLd];
+                load_items(idx0, tot, v);
 #pragma unroll
-                for (int c = 0; c < 4; c++) {
-                    uint32_t h2;
-                    asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(h2) : "r"(pr[c]), "r"(fac2[c]));
-                    dst[c * 256] = static_cast<unsigned short>(h2);
-                    dst[c * 256 + 4] = static_cast<unsigned short>(h2 >> 16);
+                for (int u = 0; u < kLd; u++) {
+                    const int idx = idx0 + u * nthr;
+                    if (idx >= tot) break;
+                    const int m = idx / per_m, c8 = idx - m * per_m;
+                    const uint32_t pr[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+                    const int kl = c8 * 8;
+                    const int gk = kl >> 7;
+                    const int bi = xs_pair_index<8>((gk % GPB) * MT + m, ((gk / GPB) << 7) | (kl & 127));
+                    unsigned short *dst = reinterpret_cast<unsigned short *>(xs + bi);
+                    if (!TERN_GUARD((bi + 773) * 2 <= xs_bytes(kcta, MT, X8), g_tern_gemvstep_guard)) continue;
+#pragma unroll
+                    for (int c = 0; c < 4; c++) {
+                        uint32_t h2;
+                        asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(h2) : "r"(pr[c]), "r"(fac2[c]));
+                        dst[c * 256] = static_cast<unsigned short>(h2);
+                        dst[c * 256 + 4] = static_cast<unsigned short>(h2 >> 16);
+                    }
                 }
             }
         }
@@ -677,6 +707,12 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_step_kernel(const __grid_con
         // ---- this warp's units of the piece ----
         int tbeg, U, v0, v1;
         piece_range(d, T0, T1, warp, tbeg, U, v0, v1);
+        // (the staging is done with wmax: it keeps the piece's first tile and
+        // unit count for the combine below)
+        if (threadIdx.x == 0) {
+            wmax[0] = static_cast<unsigned int>(tbeg);
+            wmax[1] = static_cast<unsigned int>(U);
+        }
         const float post = X8 ? 1.0f : ldexpf(1.0f, 24 - E);
         float acc[4] = {0.f, 0.f, 0.f, 0.f};
         // (tile, slice) of unit v, by increments
@@ -1039,33 +1075,38 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_step_kernel(const __grid_con
         }
         // ---- tiles of this piece split over several warps: summed in warp
         // order by the first warp that holds a part ----
-        __syncthreads();
+        // (no partial tile is stored once any warp of the CTA has given up)
+        if (__syncthreads_or(dead ? 1 : 0) == 0) {
+            // warp w2 holds units [PU w2 / kW, PU (w2 + 1) / kW) of the piece
+            const int pbeg = static_cast<int>(wmax[0]), PU = static_cast<int>(wmax[1]);
+            const int pv0 = static_cast<int>((static_cast<long long>(PU) * warp) / kW);
 #pragma unroll 1
-        for (int slot = 0; slot < 2; slot++) {
-            const int tile = rec_tile[warp * 2 + slot];
-            if (tile < 0) continue;
-            bool owner = true;
-            for (int w2 = 0; w2 < warp; w2++)
-                if (rec_tile[w2 * 2] == tile || rec_tile[w2 * 2 + 1] == tile) owner = false;
-            if (!owner) continue;
-            bool bad = false;
-            for (int w2 = 0; w2 < kW; w2++)
-                if (rec_tile[w2 * 2] == -2 || rec_tile[w2 * 2 + 1] == -2) bad = true;
-            if (bad) continue;
-            float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (q < kGcLanes) {
-                for (int w2 = warp; w2 < kW; w2++)
-                    for (int s2i = 0; s2i < 2; s2i++) {
-                        if (rec_tile[w2 * 2 + s2i] != tile) continue;
-                        const float4 o =
-                            *reinterpret_cast<const float4 *>(rec + (((w2 * 2 + s2i) * 8 + g) * kGcLanes + q) * 4);
+            for (int slot = 0; slot < 2; slot++) {
+                const int tile = rec_tile[warp * 2 + slot];
+                if (tile < 0) continue;
+                // The first warp holding a part holds the tile's first unit:
+                // slot 1 always, slot 0 when this warp's range starts there.
+                if (slot == 0 && pv0 % B != 0) continue;
+                // The other parts are the slot-0 parts of the following warps
+                // whose ranges start inside the tile, up to warp wl (the last
+                // with PU w / kW < tend); warps with empty ranges hold none.
+                const int tend = (tile - pbeg + 1) * B;
+                const int wl = static_cast<int>(
+                    min(static_cast<long long>(kW - 1), (static_cast<long long>(kW) * tend - 1) / PU));
+                float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
+                if (q < kGcLanes) {
+                    sum = *reinterpret_cast<const float4 *>(rec + (((warp * 2 + slot) * 8 + g) * kGcLanes + q) * 4);
+                    for (int w2 = warp + 1; w2 <= wl; w2++) {
+                        if (PU < kW && (PU * (w2 + 1)) / kW == (PU * w2) / kW) continue;
+                        const float4 o = *reinterpret_cast<const float4 *>(rec + (((w2 * 2) * 8 + g) * kGcLanes + q) * 4);
                         sum.x += o.x;
                         sum.y += o.y;
                         sum.z += o.z;
                         sum.w += o.w;
                     }
+                }
+                gc_store(tile, sum);
             }
-            gc_store(tile, sum);
         }
     }
     // A warp that gave up may still have copies of its own in flight: they
