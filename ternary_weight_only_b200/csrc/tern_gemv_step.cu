@@ -63,6 +63,7 @@
 // 10-bit results joined and shifted by the digit offset -- after which the
 // ternary arithmetic runs unchanged.
 #include <algorithm>
+#include <cmath>
 #include <cstring>
 
 #include "tern_internal.cuh"
@@ -1149,6 +1150,99 @@ StepKernel step_kernel(int mt, int f, bool x8) {
 }
 
 int step_mt(int M) { return M == 1 ? 1 : (M == 2 ? 2 : (M <= 4 ? 4 : 8)); }
+
+// What staging one piece's x costs a CTA, in 1024-k units of streaming
+// (measured on B200: a piece's staging takes ~1.5-5 us at one token row,
+// ~3.5-8.5 us at four and ~5.5-6.5 us at eight, against ~10, ~6.5 and ~6
+// units streamed per microsecond and CTA).
+int piece_cost(int K, int M) {
+    const int B = K / 1024;
+    if (M == 1) return 5 + (12 * B) / 5;
+    if (M == 2) return 6 + (5 * B) / 2;
+    if (M <= 4) return 10 + (13 * B) / 5;
+    return 20 + 3 * B;
+}
+
+// Greedy cut of the flat tile list into CTA ranges whose units plus piece
+// costs stay within C (each range that starts or continues a matrix pays that
+// matrix's piece cost).  Returns the number of ranges; with `cut` non-null
+// writes their first tiles cut[1..].
+int cut_ranges(const SDesc *d, const int *pc, int count, long long C, int *cut) {
+    int n = 0;
+    long long acc = 0;
+    bool open = false;
+    for (int i = 0; i < count; i++) {
+        const int B = d[i].K / 1024;
+        int left = d[i].ntile, t = d[i].tile0;
+        while (left > 0) {
+            if (open && acc + pc[i] + B > C) {
+                n++;
+                if (cut) cut[n] = t;
+                acc = 0;
+            }
+            open = true;
+            acc += pc[i];
+            long long take = (C - acc) / B;
+            if (take < 1) take = 1;
+            if (take > left) take = left;
+            acc += take * B;
+            left -= static_cast<int>(take);
+            t += static_cast<int>(take);
+            if (left > 0) {
+                n++;
+                if (cut) cut[n] = t;
+                acc = 0;
+                open = false;
+            }
+        }
+    }
+    return open ? n + 1 : n;
+}
+
+// Cuts at the multiples of total / grid along the same cost axis (so that
+// every CTA gets a range), each range kept within Cmax.  Returns the number
+// of ranges (above grid: unusable); writes the first tiles of ranges
+// 1 .. grid - 1 to cut[] and the axis length to *end.
+int cut_even(const SDesc *d, const int *pc, int count, double total, int grid, long long Cmax, int *cut,
+             long long *end) {
+    const double target = total / grid;
+    int n = 1;
+    long long acc = 0, pos = 0;
+    for (int i = 0; i < count; i++) {
+        const long long B = d[i].K / 1024;
+        long long left = d[i].ntile;
+        int t = d[i].tile0;
+        bool pending = true;  // the range has not paid matrix i's piece cost yet
+        while (left > 0) {
+            long long add = (pending ? pc[i] : 0) + B;
+            if (acc > 0 && (acc + add > Cmax || (n < grid && pos + 0.5 * add > n * target))) {
+                if (n < grid) cut[n] = t;
+                n++;
+                acc = 0;
+                add = pc[i] + B;
+            }
+            pos += add;
+            acc += add;
+            pending = false;
+            t++;
+            left--;
+            // tiles that can follow before the next cut: within Cmax, and
+            // before the axis passes the next multiple of the target
+            long long k = std::max<long long>(0, (Cmax - acc) / B);
+            if (n < grid) {
+                const double r = n * target - static_cast<double>(pos) - 0.5 * static_cast<double>(B);
+                k = std::min<long long>(k, r >= 0 ? static_cast<long long>(std::floor(r / static_cast<double>(B))) + 1 : 0);
+            }
+            k = std::min(k, left);
+            pos += k * B;
+            acc += k * B;
+            t += static_cast<int>(k);
+            left -= k;
+        }
+    }
+    *end = pos;
+    return n;
+}
 int mt_index(int mt) { return mt == 1 ? 0 : (mt == 2 ? 1 : (mt == 4 ? 2 : 3)); }
 
 // The digit form serves every weight storage at one and two token rows
@@ -1240,26 +1334,40 @@ tern_status launch_chunk(const DeviceInfo &dev, const MatDesc *md, int count, in
         return fail(TERN_ERR_SHAPE, "step kernel needs %zu B of shared memory", smem_bytes(kmax, mt, 1, fmt, x8));
     int grid = std::min<int>(std::min(dev.sms, kMaxCtas), tiles);
     if (g_opt.gemv_grid > 0) grid = std::min(grid, g_opt.gemv_grid);
-    // Cut the flat tile list into `grid` ranges of about equal units: CTA c
-    // starts at the first tile boundary at or after c * total / grid units.
-    p.cta_tile[0] = 0;
+    // Cut the flat tile list into at most `grid` CTA ranges of about equal
+    // cost (units plus the staging of each piece).  The smallest bound C
+    // whose greedy cut needs no more ranges than CTAs is the best possible
+    // largest range; cuts at even steps of the cost axis within that bound
+    // give every CTA a range (the axis length, which depends on where the cuts
+    // fall, is refined over a few passes); where they need more ranges than
+    // CTAs, the greedy cut stands.
     {
-        int i = 0;
-        long long ubase = 0;  // units before matrix i
-        for (int c = 1; c < grid; c++) {
-            const long long target = (total_units * c) / grid;
-            while (i < count && ubase + static_cast<long long>(p.d[i].ntile) * (p.d[i].K / 1024) <= target) {
-                ubase += static_cast<long long>(p.d[i].ntile) * (p.d[i].K / 1024);
-                i++;
-            }
-            int t = tiles;
-            if (i < count) {
-                const long long B = p.d[i].K / 1024;
-                t = p.d[i].tile0 + static_cast<int>((target - ubase + B - 1) / B);
-            }
-            p.cta_tile[c] = std::max(p.cta_tile[c - 1], std::min(t, tiles));
+        int pc[TERN_MAX_STEP];
+        long long hi = 0, pcsum = 0;
+        for (int i = 0; i < count; i++) {
+            pc[i] = piece_cost(p.d[i].K, M);
+            pcsum += pc[i];
+            hi += static_cast<long long>(p.d[i].ntile) * (p.d[i].K / 1024) + static_cast<long long>(pc[i]) * p.d[i].ntile;
         }
-        p.cta_tile[grid] = tiles;
+        long long lo = std::max<long long>(1, total_units / grid);
+        while (lo < hi) {
+            const long long mid = (lo + hi) / 2;
+            if (cut_ranges(p.d, pc, count, mid, nullptr) <= grid) hi = mid; else lo = mid + 1;
+        }
+        int used = cut_ranges(p.d, pc, count, lo, p.cta_tile);
+        int cut[kMaxCtas + 1];
+        double total = static_cast<double>(total_units + pcsum) + static_cast<double>(grid - 1) * pcsum / count;
+        for (int pass = 0; pass < 4; pass++) {
+            long long end = 0;
+            const int n = cut_even(p.d, pc, count, total, grid, lo, cut, &end);
+            if (n <= grid && n > used) {
+                used = n;
+                for (int c = 1; c < n; c++) p.cta_tile[c] = cut[c];
+            }
+            total = static_cast<double>(end);
+        }
+        p.cta_tile[0] = 0;
+        for (int c = used; c <= grid; c++) p.cta_tile[c] = tiles;
     }
     p.count = count;
     p.M = M;
