@@ -362,8 +362,11 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_step_kernel(const __grid_con
     const int M = p.M;
     uint8_t *ring = base + roff;
 
-    if (threadIdx.x == 0) {
-        for (int i = 0; i < kW * kMaxNS; i++) mbar_init(&full[i], 1);
+    // one barrier per thread of the first warps (the fence orders this
+    // thread's initialisation before the copies that arrive on it)
+    static_assert(kW * kMaxNS <= kThreads, "one thread per ring barrier");
+    if (threadIdx.x < kW * kMaxNS) {
+        mbar_init(&full[threadIdx.x], 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     if constexpr (F == 2) {
@@ -1079,26 +1082,27 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_step_kernel(const __grid_con
         // (no partial tile is stored once any warp of the CTA has given up)
         if (__syncthreads_or(dead ? 1 : 0) == 0) {
             // warp w2 holds units [PU w2 / kW, PU (w2 + 1) / kW) of the piece
-            const int pbeg = static_cast<int>(wmax[0]), PU = static_cast<int>(wmax[1]);
-            const int pv0 = static_cast<int>((static_cast<long long>(PU) * warp) / kW);
+            // (32-bit: a piece has far fewer than 2^27 units)
+            const int pbeg = static_cast<int>(wmax[0]);
+            const unsigned int PU = wmax[1], UB = static_cast<unsigned int>(B);
+            const unsigned int pv0 = (PU * static_cast<unsigned int>(warp)) / kW;
 #pragma unroll 1
             for (int slot = 0; slot < 2; slot++) {
                 const int tile = rec_tile[warp * 2 + slot];
                 if (tile < 0) continue;
                 // The first warp holding a part holds the tile's first unit:
                 // slot 1 always, slot 0 when this warp's range starts there.
-                if (slot == 0 && pv0 % B != 0) continue;
+                if (slot == 0 && pv0 % UB != 0u) continue;
                 // The other parts are the slot-0 parts of the following warps
                 // whose ranges start inside the tile, up to warp wl (the last
                 // with PU w / kW < tend); warps with empty ranges hold none.
-                const int tend = (tile - pbeg + 1) * B;
-                const int wl = static_cast<int>(
-                    min(static_cast<long long>(kW - 1), (static_cast<long long>(kW) * tend - 1) / PU));
+                const unsigned int tend = static_cast<unsigned int>(tile - pbeg + 1) * UB;
+                const int wl = static_cast<int>(min(static_cast<unsigned int>(kW - 1), (kW * tend - 1u) / PU));
                 float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
                 if (q < kGcLanes) {
                     sum = *reinterpret_cast<const float4 *>(rec + (((warp * 2 + slot) * 8 + g) * kGcLanes + q) * 4);
                     for (int w2 = warp + 1; w2 <= wl; w2++) {
-                        if (PU < kW && (PU * (w2 + 1)) / kW == (PU * w2) / kW) continue;
+                        if (PU < kW && (PU * (w2 + 1u)) / kW == (PU * w2) / kW) continue;
                         const float4 o = *reinterpret_cast<const float4 *>(rec + (((w2 * 2) * 8 + g) * kGcLanes + q) * 4);
                         sum.x += o.x;
                         sum.y += o.y;
