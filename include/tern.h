@@ -166,7 +166,10 @@ tern_status tern_gemv(const uint16_t *x, const uint8_t *slots, const uint16_t *s
  * tern_gemm -- y[M][N] = x[M][K] * W^T for any M >= 1.
  *   x  fp16 [M][K] row-major (device, read);  y  fp16 [M][N] row-major (device, written).
  * M <= 8 (speculative-verify batches) runs the same bandwidth-bound kernels as
- * tern_gemv, reading the weights once for all rows.  M >= 32 runs the
+ * tern_gemv (M = 2 with K a multiple of 1024: the step kernel's two-row
+ * form), reading the weights once for all rows wherever the M rows of x fit
+ * on chip (M = 5..8 with K above ~7000: two passes of up to four rows).
+ * M >= 32 runs the
  * tensor-core prefill kernel (tcgen05), which unpacks weight tiles on chip to
  * s*t (exact in fp16) straight into tensor memory and accumulates in fp32;
  * 8 < M < 32 runs the bandwidth kernel once per eight rows.  Small M is the
@@ -218,8 +221,9 @@ typedef struct tern_gemv_desc {
 
 /*
  * tern_gemv_grouped -- up to TERN_MAX_GROUP independent products with the same
- * M (1..8) in ONE kernel launch, e.g. the q/k/v projections of a layer, or
- * all seven projections of one synthetic decode layer.  Descriptors are read
+ * M (1..8) in ONE kernel launch (two at M = 5..8 when some x does not fit on
+ * chip), e.g. the q/k/v projections of a layer, or all seven projections of
+ * one synthetic decode layer.  Descriptors are read
  * on the host during the call (the array need not outlive it).  Outputs must
  * not overlap inputs or each other.
  */

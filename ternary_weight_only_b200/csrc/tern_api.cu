@@ -176,12 +176,17 @@ bool use_tc(int M) { return g_opt.gemv_variant == kVarTc && M <= 4; }
 
 tern_status launch_bandwidth(const MatDesc *d, int count, int M, void *workspace, size_t ws_bytes,
                              cudaStream_t s) {
-    // One token row: the persistent step kernel (digit form) where its shape
-    // rules hold -- measured faster than the per-matrix kernels on every
-    // decode shape alone and grouped (head 5120 x 151936: 38.7 us against
-    // 52.4 us; gate + up: 13.7 against 18.4 us).
-    if (g_opt.gemv_variant == kVarDefault && M == 1 && gemv_step_supports(d, count, 1, 0, gemv_step_digit_form(1, 0)))
-        return launch_gemv_step(d, count, 1, 0, gemv_step_digit_form(1, 0), s);
+    // The persistent step kernel where its shape rules hold, as measured on
+    // B200 against the per-matrix kernels: at one and two token rows (digit
+    // form) for every decode shape alone and grouped (M = 1: head 5120 x
+    // 151936 39 against 52 us; M = 2: gate 9.8 against 13.1 us, a decode
+    // layer 22.9 against 28.1 us), and at five to eight rows for groups of
+    // four products or more, which it reads once where the per-matrix kernel
+    // takes two passes of four rows (a decode layer at M = 8: 56.7 against
+    // 64.2 us; single products stay on the per-matrix kernels, 5-10 % faster).
+    const bool step_m = M <= 2 || (M >= 5 && count >= 4);
+    if (g_opt.gemv_variant == kVarDefault && step_m && gemv_step_supports(d, count, M, 0, gemv_step_digit_form(M, 0)))
+        return launch_gemv_step(d, count, M, 0, gemv_step_digit_form(M, 0), s);
     if (use_tc(M)) return launch_gemv_tc(d, count, M, workspace, ws_bytes, s);
     // Default: the producer/consumer kernel where its shape rules hold (K a
     // multiple of 1024, x fits its shared memory), else the TMA-staged one.
