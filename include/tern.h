@@ -269,6 +269,28 @@ size_t tern_gemv_grouped_workspace_bytes(const tern_gemv_desc *descs, int32_t co
 tern_status tern_gemv_step(const tern_gemv_desc *descs, int32_t count, int64_t M, void *stream);
 
 /*
+ * tern_step_plan -- the split of one step-kernel launch over CTAs, for
+ * inspection and tests; host only (no device is touched).  The pages have no
+ * counterpart: it states how the bytes a step streams are shared out.
+ *   N, K        count row counts and depths (host arrays), in launch order;
+ *               every K a multiple of 1024
+ *   count       1..96 (the products of one launch; tern_gemv_step cuts longer
+ *               lists into launches of at most 96)
+ *   M           1..8 token rows
+ *   grid        1..160 CTAs (one per SM on B200: 148)
+ *   first_tile  int32 [grid + 1] (host, written): CTA c streams the 16-row
+ *               tiles first_tile[c] .. first_tile[c + 1] - 1 of the flat list
+ *               (tiles of product 0 first); first_tile[0] = 0 and
+ *               first_tile[grid] = all tiles; trailing CTAs may get empty
+ *               ranges (always when there are fewer tiles than CTAs).
+ * Ranges are cut so that each CTA's streaming (1024-k units) plus the
+ * staging of every product it starts is about equal.  Returns TERN_OK, or
+ * TERN_ERR_SHAPE / TERN_ERR_INVALID_ARG for arguments out of range.
+ */
+tern_status tern_step_plan(const int64_t *N, const int64_t *K, int32_t count, int64_t M, int32_t grid,
+                           int32_t *first_tile);
+
+/*
  * tern_embed_gather -- ternary embedding lookup: rows of a ternary-g128
  * matrix gathered by token id, written as fp16.  The pages count the
  * embeddings among the ternary matrices ("Ternary-Bonsai-27B" model summary,

@@ -463,6 +463,13 @@ tern_status tern_gemv_step(const tern_gemv_desc *descs, int32_t count, int64_t M
     return gemv_step_api(descs, count, M, 0, "tern_gemv_step", stream);
 }
 
+tern_status tern_step_plan(const int64_t *N, const int64_t *K, int32_t count, int64_t M, int32_t grid,
+                           int32_t *first_tile) {
+    clear_error();
+    if (M < 1 || M > 8) return fail(TERN_ERR_SHAPE, "M must be in [1, 8] (got %lld)", static_cast<long long>(M));
+    return gemv_step_plan(N, K, count, static_cast<int>(M), grid, first_tile);
+}
+
 tern_status tern_b1_gemv_step(const tern_gemv_desc *descs, int32_t count, int64_t M, void *stream) {
     return gemv_step_api(descs, count, M, 1, "tern_b1_gemv_step", stream);
 }

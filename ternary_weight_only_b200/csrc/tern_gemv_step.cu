@@ -1247,6 +1247,47 @@ int cut_even(const SDesc *d, const int *pc, int count, double total, int grid, l
     *end = pos;
     return n;
 }
+
+// Cut the flat tile list of one launch (d[i].tile0, ntile, K; tiles in
+// descriptor order) into at most `grid` CTA ranges of about equal cost
+// (units plus the staging of each piece): cta_tile[c] .. cta_tile[c + 1] is
+// CTA c's range, cta_tile[0] = 0, cta_tile[grid] = all tiles; trailing CTAs
+// may get empty ranges.  The smallest bound C whose greedy cut needs no more
+// ranges than CTAs is the best possible largest range; cuts at even steps of
+// the cost axis within that bound give every CTA a range (the axis length,
+// which depends on where the cuts fall, is refined over a few passes); where
+// they need more ranges than CTAs, the greedy cut stands.
+void plan_ranges(const SDesc *d, int count, int M, int grid, int *cta_tile) {
+    int pc[TERN_MAX_STEP];
+    long long hi = 0, pcsum = 0, total_units = 0;
+    int tiles = 0;
+    for (int i = 0; i < count; i++) {
+        pc[i] = piece_cost(d[i].K, M);
+        pcsum += pc[i];
+        total_units += static_cast<long long>(d[i].ntile) * (d[i].K / 1024);
+        hi += static_cast<long long>(d[i].ntile) * (d[i].K / 1024) + static_cast<long long>(pc[i]) * d[i].ntile;
+        tiles = std::max(tiles, d[i].tile0 + d[i].ntile);
+    }
+    long long lo = std::max<long long>(1, total_units / grid);
+    while (lo < hi) {
+        const long long mid = (lo + hi) / 2;
+        if (cut_ranges(d, pc, count, mid, nullptr) <= grid) hi = mid; else lo = mid + 1;
+    }
+    int used = cut_ranges(d, pc, count, lo, cta_tile);
+    int cut[kMaxCtas + 1];
+    double total = static_cast<double>(total_units + pcsum) + static_cast<double>(grid - 1) * pcsum / count;
+    for (int pass = 0; pass < 4; pass++) {
+        long long end = 0;
+        const int n = cut_even(d, pc, count, total, grid, lo, cut, &end);
+        if (n <= grid && n > used) {
+            used = n;
+            for (int c = 1; c < n; c++) cta_tile[c] = cut[c];
+        }
+        total = static_cast<double>(end);
+    }
+    cta_tile[0] = 0;
+    for (int c = used; c <= grid; c++) cta_tile[c] = tiles;
+}
 int mt_index(int mt) { return mt == 1 ? 0 : (mt == 2 ? 1 : (mt == 4 ? 2 : 3)); }
 
 // The digit form serves every weight storage at one and two token rows
@@ -1338,41 +1379,7 @@ tern_status launch_chunk(const DeviceInfo &dev, const MatDesc *md, int count, in
         return fail(TERN_ERR_SHAPE, "step kernel needs %zu B of shared memory", smem_bytes(kmax, mt, 1, fmt, x8));
     int grid = std::min<int>(std::min(dev.sms, kMaxCtas), tiles);
     if (g_opt.gemv_grid > 0) grid = std::min(grid, g_opt.gemv_grid);
-    // Cut the flat tile list into at most `grid` CTA ranges of about equal
-    // cost (units plus the staging of each piece).  The smallest bound C
-    // whose greedy cut needs no more ranges than CTAs is the best possible
-    // largest range; cuts at even steps of the cost axis within that bound
-    // give every CTA a range (the axis length, which depends on where the cuts
-    // fall, is refined over a few passes); where they need more ranges than
-    // CTAs, the greedy cut stands.
-    {
-        int pc[TERN_MAX_STEP];
-        long long hi = 0, pcsum = 0;
-        for (int i = 0; i < count; i++) {
-            pc[i] = piece_cost(p.d[i].K, M);
-            pcsum += pc[i];
-            hi += static_cast<long long>(p.d[i].ntile) * (p.d[i].K / 1024) + static_cast<long long>(pc[i]) * p.d[i].ntile;
-        }
-        long long lo = std::max<long long>(1, total_units / grid);
-        while (lo < hi) {
-            const long long mid = (lo + hi) / 2;
-            if (cut_ranges(p.d, pc, count, mid, nullptr) <= grid) hi = mid; else lo = mid + 1;
-        }
-        int used = cut_ranges(p.d, pc, count, lo, p.cta_tile);
-        int cut[kMaxCtas + 1];
-        double total = static_cast<double>(total_units + pcsum) + static_cast<double>(grid - 1) * pcsum / count;
-        for (int pass = 0; pass < 4; pass++) {
-            long long end = 0;
-            const int n = cut_even(p.d, pc, count, total, grid, lo, cut, &end);
-            if (n <= grid && n > used) {
-                used = n;
-                for (int c = 1; c < n; c++) p.cta_tile[c] = cut[c];
-            }
-            total = static_cast<double>(end);
-        }
-        p.cta_tile[0] = 0;
-        for (int c = used; c <= grid; c++) p.cta_tile[c] = tiles;
-    }
+    plan_ranges(p.d, count, M, grid, p.cta_tile);
     p.count = count;
     p.M = M;
     p.smem_usable = static_cast<unsigned int>(smem - 1024);
@@ -1447,6 +1454,33 @@ tern_status read_gemvstep_status(bool reset, unsigned int *out) {
         if (e != cudaSuccess) return cuda_fail(e, "clearing device status");
     }
     *out = v;
+    return TERN_OK;
+}
+
+// The CTA ranges one launch of the step kernel would use (see plan_ranges).
+tern_status gemv_step_plan(const int64_t *N, const int64_t *K, int count, int M, int grid, int32_t *first_tile) {
+    if (!N || !K || !first_tile) return fail(TERN_ERR_INVALID_ARG, "null pointer");
+    if (count < 1 || count > kMaxPer) return fail(TERN_ERR_SHAPE, "count must be in [1, %d] (got %d)", kMaxPer, count);
+    if (M < 1 || M > 8) return fail(TERN_ERR_SHAPE, "M must be in [1, 8] (got %d)", M);
+    if (grid < 1 || grid > kMaxCtas) return fail(TERN_ERR_SHAPE, "grid must be in [1, %d] (got %d)", kMaxCtas, grid);
+    SDesc d[kMaxPer];
+    int tiles = 0;
+    for (int i = 0; i < count; i++) {
+        if (N[i] < 1 || N[i] > 0x7FFFFFF0ll || K[i] < 1024 || K[i] % 1024 != 0 || K[i] > (1 << 20))
+            return fail(TERN_ERR_SHAPE, "descriptor %d: N >= 1 and K a positive multiple of 1024 required", i);
+        std::memset(&d[i], 0, sizeof(SDesc));
+        d[i].N = static_cast<int>(N[i]);
+        d[i].K = static_cast<int>(K[i]);
+        d[i].tile0 = tiles;
+        d[i].ntile = static_cast<int>((N[i] + kRows - 1) / kRows);
+        if (tiles > 0x7FFFFFFF - d[i].ntile) return fail(TERN_ERR_SHAPE, "too many rows");
+        tiles += d[i].ntile;
+    }
+    const int g = std::min(grid, tiles);
+    int cta_tile[kMaxCtas + 1];
+    plan_ranges(d, count, M, g, cta_tile);
+    for (int c = 0; c <= g; c++) first_tile[c] = cta_tile[c];
+    for (int c = g + 1; c <= grid; c++) first_tile[c] = tiles;
     return TERN_OK;
 }
 

@@ -118,6 +118,9 @@ bool gemv_step_fits(int K, int M, int fmt, bool x8);
 // the form the step kernels use by default for M token rows (TERN_OPT_STEP_FORM)
 bool gemv_step_digit_form(int M, int fmt);
 tern_status launch_gemv_step(const MatDesc *d, int count, int M, int fmt, bool x8, cudaStream_t stream);
+// The CTA ranges one launch of the step kernel uses for these shapes on
+// `grid` CTAs: first_tile[0..grid] (host only).
+tern_status gemv_step_plan(const int64_t *N, const int64_t *K, int count, int M, int grid, int32_t *first_tile);
 tern_status read_gemvstep_status(bool reset, unsigned int *out);
 extern unsigned long long g_gemm_timeout_ns;
 extern int g_gemm_skip_loads;

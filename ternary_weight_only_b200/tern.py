@@ -11,6 +11,7 @@ import ctypes
 import os
 from typing import Optional, Sequence
 
+import numpy as np
 import torch
 
 _LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libtern.so")
@@ -77,6 +78,7 @@ _SIGS = {
     "tern_t5_pack": ([_vp, _vp, _i64, _i64, _vp, _vp, _vp, _vp], _int),
     "tern_t5_unpack": ([_vp, _i64, _i64, _vp, _vp], _int),
     "tern_t5_gemv_step": ([ctypes.POINTER(tern_gemv_desc), _i32, _i64, _vp], _int),
+    "tern_step_plan": ([_vp, _vp, _i32, _i64, _i32, _vp], _int),
 }
 for _name, (_args, _res) in _SIGS.items():
     _f = getattr(_L, _name)
@@ -288,6 +290,17 @@ def _step_descs(mats: Sequence):
         arr[i].N = s.shape[0]
         arr[i].K = x.shape[-1]
     return arr
+
+
+def tern_step_plan(shapes: Sequence, M: int = 1, grid: int = 148):
+    """shapes: sequence of (N, K) of one launch's products (host only).
+    Returns the grid + 1 tile boundaries: CTA c streams the 16-row tiles
+    [first[c], first[c + 1]) of the flat list."""
+    n = np.ascontiguousarray([int(a) for a, _ in shapes], dtype=np.int64)
+    k = np.ascontiguousarray([int(b) for _, b in shapes], dtype=np.int64)
+    out = np.zeros(grid + 1, dtype=np.int32)
+    _check(_L.tern_step_plan(n.ctypes.data, k.ctypes.data, len(shapes), M, grid, out.ctypes.data), "tern_step_plan")
+    return out.tolist()
 
 
 def tern_gemv_step(mats: Sequence, M: int = 1, stream=None):
