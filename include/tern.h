@@ -255,10 +255,11 @@ size_t tern_gemv_grouped_workspace_bytes(const tern_gemv_desc *descs, int32_t co
  * Every K must be a multiple of 1024.  The M rows of a product's x are
  * staged in shared memory beside the weight rings; a product whose x does
  * not fit (at M = 8 above K ~ 8900, at M = 4 above K ~ 17900) runs as up to
- * eight K segments of whole 1024-k units, in launches of their own after the
- * others: the first writes y, each later one adds its fp16-rounded partial
- * sum to y (one extra rounding, within the tolerance below); beyond eight
- * segments TERN_ERR_SHAPE.  Each weight is read once either way.  Results are
+ * four K segments of whole 1024-k units, in launches of their own after the
+ * others: the first writes y, each later one adds its partial sum to the
+ * fp16 y (one more fp16 rounding each, at most 2^-11 of sum_k |x_k w_k|; four
+ * stay within the tolerance below); beyond four segments TERN_ERR_SHAPE
+ * (at M = 8, K above ~36000).  Each weight is read once either way.  Results are
  * within |y - y_ref| <= 2e-3 sum_k |x_k w_k| + 1e-5 of the exact product, as
  * for tern_gemv / tern_gemm (fixed summation order per tile);
  * outputs must not overlap inputs or each other.  Argument errors return

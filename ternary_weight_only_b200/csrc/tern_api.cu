@@ -377,8 +377,12 @@ namespace {
 // Products whose M rows of x do not fit in shared memory beside the rings run
 // as K segments of whole 1024-k units that do, in calls of their own: segment
 // 0 (with every product that fits) writes y, each later segment adds its sum
-// to y.  Each weight is still read once.  Fills seg[s][0..n[s]) for segments
-// s < nseg_max (everything in segment 0 when every product fits).
+// to y.  Each weight is still read once.  At most kMaxSeg segments: each one
+// rounds the running sum to fp16 once more (at most 2^-11 of sum |x w| each),
+// and four roundings, 1.95e-3 of sum |x w|, stay within the 2e-3 tolerance.
+// Fills seg[s][0..n[s]) for segments s < nseg_max (everything in segment 0
+// when every product fits).
+constexpr int kMaxSeg = 4;
 tern_status plan_step_segments(const MatDesc *d, int count, int m, int fmt, bool x8, const char *name,
                                MatDesc (&seg)[8][TERN_MAX_STEP], int (&n)[8], int &nseg_max) {
     nseg_max = 1;
@@ -394,7 +398,8 @@ tern_status plan_step_segments(const MatDesc *d, int count, int m, int fmt, bool
         while (bfit > 0 && !gemv_step_fits(bfit * 1024, m, fmt, x8)) bfit--;
         if (bfit == 0) return fail(TERN_ERR_SHAPE, "%s: M x 1024 too large for shared memory", name);
         const int nseg = (B + bfit - 1) / bfit;
-        if (nseg > 8) return fail(TERN_ERR_SHAPE, "%s: K=%d needs more than 8 segments at M=%d", name, d[i].K, m);
+        if (nseg > kMaxSeg)
+            return fail(TERN_ERR_SHAPE, "%s: K=%d needs more than %d segments at M=%d", name, d[i].K, kMaxSeg, m);
         nseg_max = std::max(nseg_max, nseg);
         for (int sgi = 0; sgi < nseg; sgi++) {
             const int u0 = sgi * B / nseg, u1 = (sgi + 1) * B / nseg;
@@ -439,8 +444,8 @@ tern_status gemv_step_api(const tern_gemv_desc *descs, int32_t count, int64_t M,
     const int m = static_cast<int>(M);
     cudaStream_t st_ = static_cast<cudaStream_t>(stream);
     // The digit form by default (M <= 4); a call whose products the digit
-    // form cannot cut into at most eight K segments (its staged x takes twice
-    // the room) runs in the fp16 form instead.
+    // form cannot cut into at most kMaxSeg K segments (its staged x takes
+    // twice the room) runs in the fp16 form instead.
     bool x8 = gemv_step_digit_form(m, fmt);
     thread_local MatDesc seg[8][TERN_MAX_STEP];
     int nseg_max = 1, n[8] = {0};

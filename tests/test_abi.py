@@ -167,7 +167,7 @@ def test_step_rejects(lib, fn):
     arr[0].x = None
     assert lib.tern_gemv_step(arr, 3, 1, None) == 1
     arr[0].x = A
-    arr[1].K = 204800                    # x beyond eight K segments that fit shared memory
+    arr[1].K = 204800                    # x beyond four K segments that fit shared memory
     assert lib.tern_gemv_step(arr, 3, mmax, None) == 3
 
 

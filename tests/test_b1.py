@@ -192,7 +192,7 @@ def test_timeout_reported_and_context_survives(T, orc):
 def test_long_rows_run_as_k_segments(T, orc, M, form):
     """Rows longer than the staged x allows run as K segments whose sums are
     added to y; mixed with a short product in one call; every output."""
-    shapes = [(98304, 40), (2048, 33)]
+    shapes = [(65536, 40), (2048, 33)]
     mats, refs = make_mats(orc, shapes, seed=8700 + M, M=M)
     T.tern_b1_gemv_step(mats, M)
     T.tern_sync_status()
@@ -203,7 +203,7 @@ def test_long_rows_run_as_k_segments(T, orc, M, form):
 def test_digit_form_at_three_and_four_rows(T, orc, M):
     """The digit form at three and four token rows (TERN_OPT_STEP_FORM = 2);
     mixed shapes and a row run as K segments; every output."""
-    shapes = [(1024, 40), (5120, 100), (17408, 48), (2048, 17), (40960, 20)]
+    shapes = [(1024, 40), (5120, 100), (17408, 48), (2048, 17), (32768, 20)]
     mats, refs = make_mats(orc, shapes, seed=8400 + M, M=M)
     T.tern_set_option(T.TERN_OPT_STEP_FORM, 2)
     try:

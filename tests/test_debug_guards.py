@@ -42,7 +42,8 @@ def test_no_index_check_fails(D, orc, fmt, M, form):
         pytest.skip("the 1-bit step takes M <= 4")
     from ternary_weight_only_b200 import synth
     # the last row is long enough to run as K segments (five-per-byte at
-    # M = 8 takes at most eight segments of its shorter x room)
+    # M = 8 fits K = 24576 in four segments of its shorter x room, the most
+    # a call takes)
     shapes = [(1024, 40), (3072, 333), (17408, 48), (2048, 17), (65536 if M <= 2 else 24576, 20)]
     kind = "sign" if fmt == "b1" else "sparse"
     pack = {"tern": T.tern_pack_g128, "b1": T.tern_b1_pack, "t5": T.tern_t5_pack}[fmt]

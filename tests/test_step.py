@@ -236,9 +236,9 @@ def test_chained_calls_see_complete_inputs(T):
 @pytest.mark.parametrize("M", [1, 2, 4, 8])
 def test_long_rows_run_as_k_segments(T, orc, M, form):
     """Rows far longer than the staged x allows (K = 65536 at M = 1 and 4,
-    K = 40960 at M = 8) run as K segments; mixed with short products in one
-    call; every output."""
-    K = 65536 if M < 8 else 40960
+    K = 32768 at M = 8: four segments, the most a call takes) run as K
+    segments; mixed with short products in one call; every output."""
+    K = 65536 if M < 8 else 32768
     shapes = [(K, 48), (2048, 33), (K, 17)]
     mats, refs = make_mats(orc, shapes, seed=7800 + M, M=M)
     T.tern_gemv_step(mats, M)
@@ -388,7 +388,7 @@ def test_digit_form_at_three_and_four_rows(T, orc, M):
     and a row long enough to run as K segments; every output."""
     from ternary_weight_only_b200 import synth
     shapes = [(1024, 1), (2048, 17), (5120, 100), (3072, 333), (17408, 40)]
-    shapes += [(K, N) for _, K, N in synth.LAYER_PROJ] + [(40960, 24)]
+    shapes += [(K, N) for _, K, N in synth.LAYER_PROJ] + [(32768, 24)]
     mats, refs = make_mats(orc, shapes, seed=8300 + M, M=M)
     T.tern_set_option(T.TERN_OPT_STEP_FORM, 2)
     try:

@@ -148,7 +148,7 @@ def test_verify_batch_mixed(T, orc, M, grid):
 
 
 def test_shared_memory_limit_is_a_shape_error(T):
-    """A row so long that even eight K segments leave x too large for the
+    """A row so long that even four K segments leave x too large for the
     room beside the decode table is refused before any launch."""
     K, N = 204800, 16
     x = torch.zeros(8, K, dtype=torch.float16, device="cuda")
