@@ -246,6 +246,28 @@ def test_long_rows_run_as_k_segments(T, orc, M, form):
     check_all(orc, mats, refs, f"step K segments M={M}")
 
 
+@pytest.mark.parametrize("M", [2, 8])
+def test_same_sign_rows_over_four_segments(T, orc, M):
+    """The worst case for the K segments' fp16 roundings: every weight +1 with
+    a positive scale and every x positive, so the running sum only grows and
+    each segment's rounding of it can add up to 2^-11 of sum |x w|.  A row cut
+    into four segments (the most a call takes: K = 65536 at M = 2, 32768 at
+    M = 8) stays within the tolerance; every output."""
+    K, N = (65536 if M == 2 else 32768), 40
+    rng = np.random.default_rng(9100 + M)
+    x = torch.from_numpy(rng.uniform(0.5, 1.0, size=(M, K)).astype(np.float16))
+    codes = torch.ones((N, K), dtype=torch.int8)
+    scales = torch.from_numpy(rng.uniform(0.005, 0.05, size=(N, K // 128)).astype(np.float16))
+    xn, cn, sn = np_inputs(x, codes, scales)
+    slots, sc, bad, _ = orc.pack(cn, sn)
+    assert bad == 0
+    y = torch.full((M, N), float("nan"), dtype=torch.float16, device="cuda")
+    mats = [(x.cuda(), torch.from_numpy(slots).cuda(), scales.cuda(), y)]
+    T.tern_gemv_step(mats, M)
+    T.tern_sync_status()
+    check_all(orc, mats, [(xn, slots, sc)], f"same-sign four segments M={M}")
+
+
 def test_concurrent_calls_from_two_host_threads(T):
     """Two host threads call tern_gemv_step at the same time on their own
     streams (120 products each, two launches per call); every output equals
