@@ -792,8 +792,8 @@ def run_tern(args):
         graph = torch.cuda.CUDAGraph()
         with torch.cuda.graph(graph, stream=stream):
             model.step()
-        # The weight packing above streams HBM for seconds.  On these B200s a
-        # sustained HBM stream is power-capped after ~60 ms (SM clock down to
+        # The weight packing above streams HBM for seconds.  On B200 the step
+        # held back to back trips the power cap after ~60 ms (SM clock down to
         # ~1.55 GHz, the step ~1.07 ms instead of ~0.93 ms), so the timed steps
         # start from a rested GPU, as the burst copy that the roofline peak
         # comes from does; the back-to-back rate is reported as "sustained".
