@@ -4,8 +4,8 @@ tern_sync_status as TERN_ERR_GUARD, no trap) on legal shapes: every form the
 step kernels take -- the three weight storages, one, two and four token rows in the
 digit form, the fp16 group-per-column form at 1, 2, 4 and 8 rows, products
 cut into K segments, several matrices per CTA -- reports no failed check and
-still matches the oracle.  This stands in for a memory checker, which cannot
-run on the test machines.
+still matches the oracle.  This stands in for a memory checker where none
+can be run.
 """
 import ctypes
 import os
