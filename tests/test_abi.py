@@ -171,6 +171,23 @@ def test_step_rejects(lib, fn):
     assert lib.tern_gemv_step(arr, 3, mmax, None) == 3
 
 
+def test_step_takes_at_most_four_k_segments(lib):
+    """At M = 8 a row of K = 40960 would need five K segments, each rounding
+    the running sum to fp16 once more, and is refused before any launch;
+    K = 32768 (four segments) passes the planning and, with no usable device,
+    fails later with a CUDA status instead."""
+    import torch
+    from ternary_weight_only_b200 import tern
+    arr = (tern.tern_gemv_desc * 1)()
+    arr[0].x, arr[0].slots, arr[0].scales, arr[0].y, arr[0].N = A, A, A, A, 16
+    arr[0].K = 40960
+    assert lib.tern_gemv_step(arr, 1, 8, None) == 3
+    if torch.cuda.is_available():
+        return
+    arr[0].K = 32768
+    assert lib.tern_gemv_step(arr, 1, 8, None) in (5, 7)
+
+
 def test_b1_pack_rejects(lib):
     """tern_b1_pack / tern_b1_unpack: argument errors return before any launch."""
     assert lib.tern_b1_pack(None, A, 4, 256, A, A, None, None) == 1
